@@ -1,0 +1,768 @@
+// C ABI of libqwen3blk: argument validation, workspace carving and the kernel
+// sequences of the block, MoE block and stack calls. Host code only launches
+// kernels on the caller's stream; it never allocates device memory.
+//
+// Pages cited:
+//   [P-Mini] "从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构" (quarkcode.cn)
+//   [P-Hand] "手搓一个Qwen3" (news.43b.com.cn)
+//   [P-SGL]  "从0实现SGLang 3: Qwen3-0.6B" (wmrh.cn)
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+#include "../../include/qwen3blk.h"
+#include "common.cuh"
+#include "internal.h"
+
+namespace q3 {
+
+int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
+                   int rows, int n, float eps, cudaStream_t s);
+int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv, const int* pos_base,
+                        const uint16_t* qw, const uint16_t* kw, const float* rope, uint16_t* ck, uint16_t* cv,
+                        int s_max, int max_pos, float eps, int* err, cudaStream_t s);
+int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, void* out, bool out_f32, int* err,
+                 cudaStream_t s);
+int launch_pack_gate_up(const uint16_t* gate, const uint16_t* up, long long mat_stride, int n_mats, int I, int H,
+                        uint16_t* out, cudaStream_t s);
+int launch_advance_lengths(int* len, int B, cudaStream_t s);
+int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv,
+                             const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
+                             long long ldo, int* err, cudaStream_t s);
+int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
+                            const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
+                            long long ldo, int* err, cudaStream_t s);
+size_t decode_partial_bytes(int B, int Hq, int s_max);
+int launch_moe_route(const float* logits, int T, int E, int k, int renorm, int* idx, float* w, int* counts,
+                     cudaStream_t s);
+int launch_moe_permute(const int* idx, int T, int k, int E, const int* counts, int* offsets, int* perm_token,
+                       int* perm_slot, int* inv_pos, const uint16_t* h, int H, uint16_t* a_perm, cudaStream_t s);
+int launch_moe_combine(const float* x1, const uint16_t* Y, const float* w, const int* inv_pos, int T, int k, int H,
+                       void* out, bool out_f32, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- errors
+static thread_local std::string g_last_error;
+
+void set_last_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+// The device error word (first failure wins; cleared by qwen3_check_device_error).
+__device__ int g_device_error;
+
+static int g_sm_count[64];
+static int* g_err_ptr[64];
+static std::mutex g_dev_mu;
+
+static int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d < 0 || d >= 64 ? 0 : d;
+}
+
+int num_sms() {
+  const int d = current_device();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_sm_count[d] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sm_count[d] = n > 0 ? n : 148;
+  }
+  return g_sm_count[d];
+}
+
+int* device_error_word() {
+  const int d = current_device();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_err_ptr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess) g_err_ptr[d] = static_cast<int*>(p);
+  }
+  return g_err_ptr[d];
+}
+
+// ----------------------------------------------------------------------------- validation
+#define Q3_CHECK(cond, code, ...)  \
+  do {                             \
+    if (!(cond)) {                 \
+      set_last_error(__VA_ARGS__); \
+      return (code);               \
+    }                              \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_device() {
+  static int ok[64] = {0};
+  const int d = current_device();
+  if (ok[d] == 1) return 0;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, d) != cudaSuccess) {
+    set_last_error("no CUDA device available");
+    return QWEN3_EDEVICE;
+  }
+  if (prop.major != 10) {
+    set_last_error("device %d is sm_%d%d; libqwen3blk needs an sm_100 (B200) GPU", d, prop.major, prop.minor);
+    return QWEN3_EDEVICE;
+  }
+  ok[d] = 1;
+  return 0;
+}
+
+static int validate_cfg(const qwen3_config* c) {
+  Q3_CHECK(c, QWEN3_EINVAL, "cfg is NULL");
+  Q3_CHECK(c->head_dim == 128, QWEN3_ESHAPE, "head_dim must be 128 (got %d)", c->head_dim);
+  Q3_CHECK(c->n_q_heads > 0 && c->n_kv_heads > 0, QWEN3_ESHAPE, "head counts must be positive");
+  // [P-Hand] section GroupedQueryAttention: num_heads must be divisible by the number of KV groups
+  Q3_CHECK(c->n_q_heads % c->n_kv_heads == 0, QWEN3_ESHAPE, "n_q_heads (%d) %% n_kv_heads (%d) != 0", c->n_q_heads,
+           c->n_kv_heads);
+  const int G = c->n_q_heads / c->n_kv_heads;
+  Q3_CHECK(128 % G == 0, QWEN3_ESHAPE, "query heads per KV group (%d) must divide 128", G);
+  Q3_CHECK(c->hidden > 0 && c->hidden % 256 == 0 && c->hidden <= 2048, QWEN3_ESHAPE,
+           "hidden (%d) must be a multiple of 256 and at most 2048", c->hidden);
+  Q3_CHECK(c->max_pos > 0, QWEN3_ESHAPE, "max_pos must be positive");
+  Q3_CHECK(c->rms_eps >= 0.f, QWEN3_ESHAPE, "rms_eps must be non-negative");
+  if (c->intermediate > 0)
+    Q3_CHECK(c->intermediate % 64 == 0, QWEN3_ESHAPE, "intermediate (%d) must be a multiple of 64", c->intermediate);
+  if (c->vocab > 0) Q3_CHECK(c->vocab % 32 == 0, QWEN3_ESHAPE, "vocab (%d) must be a multiple of 32", c->vocab);
+  if (c->n_experts > 0) {
+    Q3_CHECK(c->n_experts <= 256 && c->n_experts % 32 == 0, QWEN3_ESHAPE,
+             "n_experts (%d) must be a multiple of 32 and at most 256", c->n_experts);
+    Q3_CHECK(c->top_k >= 1 && c->top_k <= c->n_experts && c->top_k <= 32, QWEN3_ESHAPE,
+             "top_k (%d) must be in [1, min(n_experts, 32)]", c->top_k);
+    Q3_CHECK(c->moe_intermediate > 0 && c->moe_intermediate % 64 == 0, QWEN3_ESHAPE,
+             "moe_intermediate (%d) must be a positive multiple of 64", c->moe_intermediate);
+  }
+  return 0;
+}
+
+// ----------------------------------------------------------------------------- workspace
+struct Carver {
+  char* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t count) {
+    used = (used + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+struct Buffers {
+  uint16_t* h = nullptr;     // [M, H] normed activations
+  uint16_t* qkv = nullptr;   // [M, Nqkv]
+  uint16_t* o = nullptr;     // [M, Hq*D]
+  float* x1 = nullptr;       // [M, H] residual after attention (fp32)
+  uint16_t* act = nullptr;   // [M, I] SwiGLU output
+  float* part = nullptr;     // decode partials
+  // MoE
+  float* logits = nullptr;   // [M, E]
+  int* idx = nullptr;        // [M, k]
+  float* w = nullptr;        // [M, k]
+  int* counts = nullptr;     // [E]
+  int* offsets = nullptr;    // [E+1]
+  int* perm_token = nullptr; // [M*k]
+  int* perm_slot = nullptr;  // [M*k]
+  int* inv_pos = nullptr;    // [M*k]
+  uint16_t* a_perm = nullptr;   // [M*k, H]
+  uint16_t* act_perm = nullptr; // [M*k, Im]
+  uint16_t* y = nullptr;        // [M*k, H]
+  // stack
+  float* xs = nullptr;       // [M, H] fp32 residual stream
+  uint16_t* hf = nullptr;    // [rows, H] final-normed
+};
+
+static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void* ws, Buffers* out) {
+  Carver cv(ws);
+  Buffers b;
+  const bool decode = op == QWEN3_OP_BLOCK_DECODE || op == QWEN3_OP_STACK_DECODE;
+  const long long M = (long long)B * (decode ? 1 : T);
+  const int D = c.head_dim, H = c.hidden;
+  const long long nqkv = (long long)(c.n_q_heads + 2 * c.n_kv_heads) * D;
+  b.h = cv.take<uint16_t>(M * H);
+  b.qkv = cv.take<uint16_t>(M * nqkv);
+  b.o = cv.take<uint16_t>(M * c.n_q_heads * D);
+  b.x1 = cv.take<float>(M * H);
+  if (decode) b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, s_max) / sizeof(float));
+  if (op == QWEN3_OP_MOE_BLOCK) {
+    const int E = c.n_experts, k = c.top_k;
+    b.logits = cv.take<float>(M * E);
+    b.idx = cv.take<int>(M * k);
+    b.w = cv.take<float>(M * k);
+    b.counts = cv.take<int>(E);
+    b.offsets = cv.take<int>(E + 1);
+    b.perm_token = cv.take<int>(M * k);
+    b.perm_slot = cv.take<int>(M * k);
+    b.inv_pos = cv.take<int>(M * k);
+    b.a_perm = cv.take<uint16_t>(M * k * H);
+    b.act_perm = cv.take<uint16_t>(M * k * c.moe_intermediate);
+    b.y = cv.take<uint16_t>(M * k * H);
+  } else {
+    b.act = cv.take<uint16_t>(M * c.intermediate);
+  }
+  if (op == QWEN3_OP_STACK_PREFILL || op == QWEN3_OP_STACK_DECODE) {
+    b.xs = cv.take<float>(M * H);
+    b.hf = cv.take<uint16_t>(M * H);
+  }
+  if (out) *out = b;
+  return cv.used + 256;
+}
+
+// ----------------------------------------------------------------------------- layer pieces
+struct Ctx {
+  const qwen3_config& c;
+  cudaStream_t s;
+  int* err;
+};
+
+static inline bool swap_for(long long M) { return M <= 256; }
+
+// x1 = x + o_proj(attn(norm1(x)))   ([P-Mini] section TransformerBlock, first half)
+static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void* x, bool x_f32, int B, int T,
+                          bool decode, const int* pos, const qwen3_kv_layer& kv, const float* rope, Buffers& b) {
+  const qwen3_config& c = k.c;
+  const int H = c.hidden, D = c.head_dim;
+  const long long M = (long long)B * T;
+  const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * D;
+  int rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  if (rc) return rc;
+  GemmDesc g;
+  g.swap = swap_for(M);
+  g.K = H;
+  const void* act = b.h;
+  if (g.swap) { g.P = w.w_qkv; g.p_rows = nqkv; g.ldp = H; g.Q = act; g.q_rows = (int)M; g.ldq = H; }
+  else        { g.P = act; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_qkv; g.q_rows = nqkv; g.ldq = H; }
+  g.epi = kEpiStore;
+  g.out = b.qkv;
+  g.ldo = nqkv;
+  if ((rc = launch_gemm(g, k.s, k.err))) return rc;
+  if ((rc = launch_qk_norm_rope(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, w.q_norm, w.k_norm, rope, kv.k,
+                                kv.v, kv.s_max, c.max_pos, c.rms_eps, k.err, k.s)))
+    return rc;
+  if (decode)
+    rc = launch_attention_decode(b.qkv, nqkv, B, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part, b.o,
+                                 (long long)c.n_q_heads * D, k.err, k.s);
+  else
+    rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
+                                  (long long)c.n_q_heads * D, k.err, k.s);
+  if (rc) return rc;
+  GemmDesc o;
+  o.swap = swap_for(M);
+  o.K = c.n_q_heads * D;
+  if (o.swap) { o.P = w.w_o; o.p_rows = H; o.ldp = o.K; o.Q = b.o; o.q_rows = (int)M; o.ldq = o.K; }
+  else        { o.P = b.o; o.p_rows = (int)M; o.ldp = o.K; o.Q = w.w_o; o.q_rows = H; o.ldq = o.K; }
+  o.epi = kEpiResid;
+  o.resid = x;
+  o.resid_f32 = x_f32;
+  o.ldr = H;
+  o.out = b.x1;
+  o.out_f32 = true;
+  o.ldo = H;
+  return launch_gemm(o, k.s, k.err);
+}
+
+// out = x1 + down(silu(gate(norm2(x1))) * up(norm2(x1)))   ([P-Mini] sections SwiGLU FFN, TransformerBlock)
+static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
+  const qwen3_config& c = k.c;
+  const int H = c.hidden, I = c.intermediate;
+  int rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  if (rc) return rc;
+  GemmDesc g;
+  g.swap = swap_for(M);
+  g.K = H;
+  if (g.swap) { g.P = w.w_gate_up; g.p_rows = 2 * I; g.ldp = H; g.Q = b.h; g.q_rows = (int)M; g.ldq = H; }
+  else        { g.P = b.h; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_gate_up; g.q_rows = 2 * I; g.ldq = H; }
+  g.epi = kEpiSwiglu;
+  g.out = b.act;
+  g.ldo = I;
+  if ((rc = launch_gemm(g, k.s, k.err))) return rc;
+  GemmDesc d;
+  d.swap = swap_for(M);
+  d.K = I;
+  if (d.swap) { d.P = w.w_down; d.p_rows = H; d.ldp = I; d.Q = b.act; d.q_rows = (int)M; d.ldq = I; }
+  else        { d.P = b.act; d.p_rows = (int)M; d.ldp = I; d.Q = w.w_down; d.q_rows = H; d.ldq = I; }
+  d.epi = kEpiResid;
+  d.resid = b.x1;
+  d.resid_f32 = true;
+  d.ldr = H;
+  d.out = out;
+  d.out_f32 = out_f32;
+  d.ldo = H;
+  return launch_gemm(d, k.s, k.err);
+}
+
+// out = x1 + sum_j w_j Expert_{e_j}(norm2(x1))   ([P-Mini] section MoE)
+static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
+  const qwen3_config& c = k.c;
+  const int H = c.hidden, E = c.n_experts, kk = c.top_k, Im = c.moe_intermediate;
+  int rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  if (rc) return rc;
+  // router logits in fp32 (no bf16 rounding before the softmax)
+  GemmDesc r;
+  r.swap = swap_for(M);
+  r.K = H;
+  if (r.swap) { r.P = w.router; r.p_rows = E; r.ldp = H; r.Q = b.h; r.q_rows = (int)M; r.ldq = H; }
+  else        { r.P = b.h; r.p_rows = (int)M; r.ldp = H; r.Q = w.router; r.q_rows = E; r.ldq = H; r.force_bn = 128; }
+  r.epi = kEpiStore;
+  r.out = b.logits;
+  r.out_f32 = true;
+  r.ldo = E;
+  if ((rc = launch_gemm(r, k.s, k.err))) return rc;
+  if ((rc = launch_moe_route(b.logits, (int)M, E, kk, c.norm_topk_prob, b.idx, b.w, b.counts, k.s))) return rc;
+  if ((rc = launch_moe_permute(b.idx, (int)M, kk, E, b.counts, b.offsets, b.perm_token, b.perm_slot, b.inv_pos, b.h,
+                               H, b.a_perm, k.s)))
+    return rc;
+  const long long rows = M * kk;
+  GemmDesc gu;
+  gu.P = b.a_perm; gu.p_rows = (int)rows; gu.ldp = H;
+  gu.Q = w.moe_gate_up; gu.q_rows = 2 * Im; gu.ldq = H; gu.q_rows_total = (long long)E * 2 * Im;
+  gu.K = H;
+  gu.epi = kEpiSwiglu;
+  gu.out = b.act_perm; gu.ldo = Im;
+  gu.n_groups = E; gu.group_offsets = b.offsets;
+  if ((rc = launch_gemm(gu, k.s, k.err))) return rc;
+  GemmDesc dn;
+  dn.P = b.act_perm; dn.p_rows = (int)rows; dn.ldp = Im;
+  dn.Q = w.moe_down; dn.q_rows = H; dn.ldq = Im; dn.q_rows_total = (long long)E * H;
+  dn.K = Im;
+  dn.epi = kEpiStore;
+  dn.out = b.y; dn.ldo = H;
+  dn.n_groups = E; dn.group_offsets = b.offsets;
+  if ((rc = launch_gemm(dn, k.s, k.err))) return rc;
+  return launch_moe_combine(b.x1, b.y, b.w, b.inv_pos, (int)M, kk, H, out, out_f32, k.s);
+}
+
+static int check_weights(const qwen3_config& c, const qwen3_layer_weights* w, bool moe) {
+  Q3_CHECK(w, QWEN3_EINVAL, "layer weights pointer is NULL");
+  const void* need[] = {w->in_norm, w->w_qkv, w->q_norm, w->k_norm, w->w_o, w->post_norm};
+  const char* names[] = {"in_norm", "w_qkv", "q_norm", "k_norm", "w_o", "post_norm"};
+  for (int i = 0; i < 6; ++i) {
+    Q3_CHECK(need[i], QWEN3_EINVAL, "weights.%s is NULL", names[i]);
+    Q3_CHECK(aligned16(need[i]), QWEN3_EALIGN, "weights.%s is not 16-byte aligned", names[i]);
+  }
+  if (moe) {
+    Q3_CHECK(c.n_experts > 0, QWEN3_ESHAPE, "MoE block needs n_experts > 0");
+    const void* m[] = {w->router, w->moe_gate_up, w->moe_down};
+    const char* mn[] = {"router", "moe_gate_up", "moe_down"};
+    for (int i = 0; i < 3; ++i) {
+      Q3_CHECK(m[i], QWEN3_EINVAL, "weights.%s is NULL", mn[i]);
+      Q3_CHECK(aligned16(m[i]), QWEN3_EALIGN, "weights.%s is not 16-byte aligned", mn[i]);
+    }
+  } else {
+    Q3_CHECK(c.intermediate > 0, QWEN3_ESHAPE, "dense block needs intermediate > 0");
+    Q3_CHECK(w->w_gate_up && w->w_down, QWEN3_EINVAL, "weights.w_gate_up / w_down is NULL");
+    Q3_CHECK(aligned16(w->w_gate_up) && aligned16(w->w_down), QWEN3_EALIGN, "FFN weights not 16-byte aligned");
+  }
+  return 0;
+}
+
+static int check_kv(const qwen3_config& c, const qwen3_kv_layer* kv, int T) {
+  Q3_CHECK(kv, QWEN3_EINVAL, "kv descriptor is NULL");
+  Q3_CHECK(kv->k && kv->v, QWEN3_EINVAL, "kv->k / kv->v is NULL");
+  Q3_CHECK(aligned16(kv->k) && aligned16(kv->v), QWEN3_EALIGN, "kv buffers are not 16-byte aligned");
+  Q3_CHECK(kv->s_max > 0, QWEN3_EINVAL, "kv->s_max must be positive");
+  Q3_CHECK(T <= kv->s_max && T <= c.max_pos, QWEN3_ECAPACITY, "T (%d) exceeds the cache capacity (%d) or max_pos (%d)",
+           T, kv->s_max, c.max_pos);
+  return 0;
+}
+
+static int finish(int rc) {
+  if (rc == -6 && g_last_error.empty()) set_last_error("CUDA error: %s", cudaGetErrorString(cudaGetLastError()));
+  return rc;
+}
+
+}  // namespace q3
+
+using namespace q3;
+
+// ============================================================================= C ABI
+extern "C" {
+
+const char* qwen3_last_error(void) { return g_last_error.c_str(); }
+
+const char* qwen3_status_string(int s) {
+  switch (s) {
+    case QWEN3_OK: return "ok";
+    case QWEN3_EINVAL: return "invalid argument";
+    case QWEN3_ESHAPE: return "unsupported shape";
+    case QWEN3_EALIGN: return "misaligned pointer";
+    case QWEN3_ECAPACITY: return "capacity exceeded";
+    case QWEN3_EWORKSPACE: return "workspace too small";
+    case QWEN3_ECUDA: return "CUDA error";
+    case QWEN3_ETIMEOUT: return "device wait timed out";
+    case QWEN3_EDEVICE: return "unsupported device";
+    default: return "unknown status";
+  }
+}
+
+int qwen3_config_qwen3_0_6b(qwen3_config* c) {
+  Q3_CHECK(c, QWEN3_EINVAL, "cfg is NULL");
+  memset(c, 0, sizeof(*c));
+  c->hidden = 1024;
+  c->n_q_heads = 16;
+  c->n_kv_heads = 8;
+  c->head_dim = 128;
+  c->intermediate = 3072;
+  c->vocab = 151936;
+  c->n_layers = 28;
+  c->max_pos = 40960;
+  c->norm_topk_prob = 1;
+  c->rms_eps = 1e-6f;
+  c->rope_theta = 1e6;
+  return 0;
+}
+
+int qwen3_validate_config(const qwen3_config* c) {
+  g_last_error.clear();
+  return validate_cfg(c);
+}
+
+size_t qwen3_rope_table_bytes(const qwen3_config* c) {
+  if (!c || c->max_pos <= 0 || c->head_dim <= 0) return 0;
+  return (size_t)c->max_pos * (c->head_dim / 2) * 2 * sizeof(float);
+}
+
+int qwen3_rope_table(const qwen3_config* c, float* rope, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(rope && aligned16(rope), rope ? QWEN3_EALIGN : QWEN3_EINVAL, "rope table pointer NULL or misaligned");
+  if ((rc = check_device())) return rc;
+  const int half = c->head_dim / 2;
+  std::vector<float> host((size_t)c->max_pos * half * 2);
+  std::vector<double> inv_freq(half);
+  // theta_i = theta^(-2i/D)   ([P-Mini] section RoPE)
+  for (int i = 0; i < half; ++i) inv_freq[i] = std::pow(c->rope_theta, -2.0 * i / c->head_dim);
+  for (int m = 0; m < c->max_pos; ++m)
+    for (int i = 0; i < half; ++i) {
+      const double a = (double)m * inv_freq[i];
+      host[((size_t)m * half + i) * 2 + 0] = (float)std::cos(a);
+      host[((size_t)m * half + i) * 2 + 1] = (float)std::sin(a);
+    }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(rope, host.data(), host.size() * sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    set_last_error("rope table copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return QWEN3_ECUDA;
+  }
+  return 0;
+}
+
+size_t qwen3_workspace_size(const qwen3_config* c, int op, int B, int T, int s_max) {
+  if (!c || validate_cfg(c) != 0 || B <= 0 || s_max <= 0) return 0;
+  if (op < QWEN3_OP_BLOCK_PREFILL || op > QWEN3_OP_STACK_DECODE) return 0;
+  if (op != QWEN3_OP_BLOCK_DECODE && op != QWEN3_OP_STACK_DECODE && T <= 0) return 0;
+  return carve(*c, op, B, T, s_max, nullptr, nullptr);
+}
+
+int qwen3_pack_qkv(const qwen3_config* c, const qwen3_bf16* wq, const qwen3_bf16* wk, const qwen3_bf16* wv,
+                   qwen3_bf16* out, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(wq && wk && wv && out, QWEN3_EINVAL, "pack_qkv: NULL pointer");
+  const size_t H = c->hidden, D = c->head_dim;
+  const size_t nq = (size_t)c->n_q_heads * D * H, nk = (size_t)c->n_kv_heads * D * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(out, wq, nq * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(out + nq, wk, nk * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(out + nq + nk, wv, nk * 2, cudaMemcpyDeviceToDevice, s) != cudaSuccess) {
+    set_last_error("pack_qkv copy failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return QWEN3_ECUDA;
+  }
+  return 0;
+}
+
+int qwen3_pack_gate_up(int I, int H, const qwen3_bf16* gate, const qwen3_bf16* up, qwen3_bf16* out, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(gate && up && out, QWEN3_EINVAL, "pack_gate_up: NULL pointer");
+  Q3_CHECK(I > 0 && I % 16 == 0 && H > 0 && H % 8 == 0, QWEN3_ESHAPE, "pack_gate_up: I %% 16 and H %% 8 required");
+  Q3_CHECK(aligned16(gate) && aligned16(up) && aligned16(out), QWEN3_EALIGN, "pack_gate_up: misaligned pointer");
+  return finish(launch_pack_gate_up(gate, up, (long long)I * H, 1, I, H, out, static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_pack_moe_gate_up(int E, int Im, int H, const qwen3_bf16* gate_up, qwen3_bf16* out, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(gate_up && out, QWEN3_EINVAL, "pack_moe_gate_up: NULL pointer");
+  Q3_CHECK(E > 0 && Im > 0 && Im % 16 == 0 && H > 0 && H % 8 == 0, QWEN3_ESHAPE,
+           "pack_moe_gate_up: Im %% 16 and H %% 8 required");
+  Q3_CHECK(aligned16(gate_up) && aligned16(out), QWEN3_EALIGN, "pack_moe_gate_up: misaligned pointer");
+  return finish(launch_pack_gate_up(gate_up, gate_up + (size_t)Im * H, (long long)2 * Im * H, E, Im, H, out,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_check_device_error(void* stream) {
+  g_last_error.clear();
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_last_error("stream error: %s", cudaGetErrorString(e));
+    return QWEN3_ECUDA;
+  }
+  int* p = device_error_word();
+  if (!p) {
+    set_last_error("device error word unavailable");
+    return QWEN3_ECUDA;
+  }
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QWEN3_ECUDA;
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    set_last_error("device reported: %s", qwen3_status_string(v));
+  }
+  return v;
+}
+
+static int common_block_checks(const qwen3_config* c, const qwen3_layer_weights* w, const void* x, int B, int T,
+                               const int* pos, const qwen3_kv_layer* kv, const float* rope, void* ws, size_t ws_bytes,
+                               int op, bool moe) {
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  if ((rc = check_weights(*c, w, moe))) return rc;
+  Q3_CHECK(x && pos && rope && ws, QWEN3_EINVAL, "x, positions, rope and ws must be non-NULL");
+  Q3_CHECK(aligned16(x) && aligned16(rope) && aligned16(ws), QWEN3_EALIGN, "x, rope or ws not 16-byte aligned");
+  Q3_CHECK(B > 0 && T > 0, QWEN3_EINVAL, "B (%d) and T (%d) must be positive", B, T);
+  if ((rc = check_kv(*c, kv, T))) return rc;
+  const size_t need = qwen3_workspace_size(c, op, B, T, kv->s_max);
+  Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return check_device();
+}
+
+int qwen3_block_prefill(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_bf16* x, int B, int T,
+                        const int* start_pos, const qwen3_kv_layer* kv, const float* rope, void* ws, size_t ws_bytes,
+                        void* stream) {
+  g_last_error.clear();
+  int rc = common_block_checks(c, w, x, B, T, start_pos, kv, rope, ws, ws_bytes, QWEN3_OP_BLOCK_PREFILL, false);
+  if (rc) return rc;
+  Buffers b;
+  carve(*c, QWEN3_OP_BLOCK_PREFILL, B, T, kv->s_max, ws, &b);
+  Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
+  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b))) return finish(rc);
+  return finish(dense_ffn(k, *w, (long long)B * T, x, false, b));
+}
+
+int qwen3_block_decode(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_bf16* x, int B,
+                       const int* cache_len, const qwen3_kv_layer* kv, const float* rope, void* ws, size_t ws_bytes,
+                       void* stream) {
+  g_last_error.clear();
+  int rc = common_block_checks(c, w, x, B, 1, cache_len, kv, rope, ws, ws_bytes, QWEN3_OP_BLOCK_DECODE, false);
+  if (rc) return rc;
+  Buffers b;
+  carve(*c, QWEN3_OP_BLOCK_DECODE, B, 1, kv->s_max, ws, &b);
+  Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
+  if ((rc = attention_half(k, *w, x, false, B, 1, true, cache_len, *kv, rope, b))) return finish(rc);
+  return finish(dense_ffn(k, *w, B, x, false, b));
+}
+
+int qwen3_moe_block(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_bf16* x, int B, int T,
+                    const int* start_pos, const qwen3_kv_layer* kv, const float* rope, int* topk_idx, float* topk_w,
+                    int* expert_offsets, int* perm_token, void* ws, size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = common_block_checks(c, w, x, B, T, start_pos, kv, rope, ws, ws_bytes, QWEN3_OP_MOE_BLOCK, true);
+  if (rc) return rc;
+  Buffers b;
+  carve(*c, QWEN3_OP_MOE_BLOCK, B, T, kv->s_max, ws, &b);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Ctx k{*c, s, device_error_word()};
+  const long long M = (long long)B * T;
+  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b))) return finish(rc);
+  if ((rc = moe_ffn(k, *w, M, x, false, b))) return finish(rc);
+  const size_t mk = (size_t)M * c->top_k;
+  if (topk_idx && cudaMemcpyAsync(topk_idx, b.idx, mk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) rc = -6;
+  if (topk_w && cudaMemcpyAsync(topk_w, b.w, mk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) rc = -6;
+  if (expert_offsets &&
+      cudaMemcpyAsync(expert_offsets, b.offsets, (c->n_experts + 1) * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    rc = -6;
+  if (perm_token && cudaMemcpyAsync(perm_token, b.perm_token, mk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    rc = -6;
+  return finish(rc);
+}
+
+int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qwen3_layer_weights* layers,
+                        const qwen3_bf16* final_norm, const int* ids, int B, int T, int mode, int* pos_or_len,
+                        const qwen3_kv_layer* kv, const float* rope, float* logits, int last_only, void* ws,
+                        size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(c->n_layers > 0 && c->vocab > 0, QWEN3_ESHAPE, "stack needs n_layers > 0 and vocab > 0");
+  Q3_CHECK(mode == QWEN3_MODE_PREFILL || mode == QWEN3_MODE_DECODE, QWEN3_EINVAL, "mode must be PREFILL or DECODE");
+  const bool decode = mode == QWEN3_MODE_DECODE;
+  Q3_CHECK(!decode || T == 1, QWEN3_EINVAL, "decode mode needs T == 1 (got %d)", T);
+  Q3_CHECK(embed && layers && final_norm && ids && pos_or_len && kv && rope && logits && ws, QWEN3_EINVAL,
+           "stack_forward: NULL argument");
+  Q3_CHECK(aligned16(embed) && aligned16(final_norm) && aligned16(rope) && aligned16(logits) && aligned16(ws),
+           QWEN3_EALIGN, "stack_forward: misaligned pointer");
+  Q3_CHECK(B > 0 && T > 0, QWEN3_EINVAL, "B (%d) and T (%d) must be positive", B, T);
+  for (int l = 0; l < c->n_layers; ++l) {
+    if ((rc = check_weights(*c, &layers[l], false))) {
+      set_last_error("layer %d: %s", l, g_last_error.c_str());
+      return rc;
+    }
+    if ((rc = check_kv(*c, &kv[l], T))) {
+      set_last_error("layer %d: %s", l, g_last_error.c_str());
+      return rc;
+    }
+    Q3_CHECK(kv[l].s_max == kv[0].s_max, QWEN3_EINVAL, "all layers' caches must share s_max");
+  }
+  const int op = decode ? QWEN3_OP_STACK_DECODE : QWEN3_OP_STACK_PREFILL;
+  const size_t need = qwen3_workspace_size(c, op, B, T, kv[0].s_max);
+  Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  if ((rc = check_device())) return rc;
+  Buffers b;
+  carve(*c, op, B, T, kv[0].s_max, ws, &b);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Ctx k{*c, s, device_error_word()};
+  const int H = c->hidden;
+  const long long M = (long long)B * T;
+  if ((rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s))) return finish(rc);
+  for (int l = 0; l < c->n_layers; ++l) {
+    if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b))) return finish(rc);
+    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b))) return finish(rc);
+  }
+  // final RMSNorm and tied LM head ([P-Mini] section 骨架; [P-SGL] section 一)
+  const int rows = last_only ? B : (int)M;
+  const float* xf = last_only ? b.xs + (long long)(T - 1) * H : b.xs;
+  const long long ldx = last_only ? (long long)T * H : H;
+  if ((rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s))) return finish(rc);
+  GemmDesc g;
+  g.swap = swap_for(rows);
+  g.K = H;
+  if (g.swap) { g.P = embed; g.p_rows = c->vocab; g.ldp = H; g.Q = b.hf; g.q_rows = rows; g.ldq = H; }
+  else        { g.P = b.hf; g.p_rows = rows; g.ldp = H; g.Q = embed; g.q_rows = c->vocab; g.ldq = H; }
+  g.epi = kEpiStore;
+  g.out = logits;
+  g.out_f32 = true;
+  g.ldo = c->vocab;
+  if ((rc = launch_gemm(g, s, k.err))) return finish(rc);
+  if (decode) rc = launch_advance_lengths(pos_or_len, B, s);
+  return finish(rc);
+}
+
+// ----------------------------------------------------------------------------- ops
+int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* w, qwen3_bf16* out, long long ldo,
+                     int rows, int n, float eps, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(x && w && out, QWEN3_EINVAL, "rmsnorm: NULL pointer");
+  Q3_CHECK(aligned16(x) && aligned16(w) && aligned16(out), QWEN3_EALIGN, "rmsnorm: misaligned pointer");
+  Q3_CHECK(n > 0 && n % 256 == 0 && n <= 2048, QWEN3_ESHAPE, "rmsnorm: n (%d) must be a multiple of 256, <= 2048", n);
+  Q3_CHECK(rows >= 0 && ldx >= n && ldo >= n && ldx % 8 == 0 && ldo % 8 == 0, QWEN3_ESHAPE,
+           "rmsnorm: bad rows or leading dimensions");
+  int rc = check_device();
+  if (rc) return rc;
+  return finish(launch_rmsnorm(x, x_f32 != 0, ldx, w, out, ldo, rows, n, eps, static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long long ldw, void* out, long long ldo,
+                  int M, int N, int K, int epilogue, const void* resid, long long ldr, int resid_f32, int out_f32,
+                  int swap, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(A && W && out, QWEN3_EINVAL, "gemm: NULL operand");
+  Q3_CHECK(aligned16(A) && aligned16(W) && aligned16(out), QWEN3_EALIGN, "gemm: misaligned operand");
+  Q3_CHECK(M > 0 && N > 0 && K > 0, QWEN3_EINVAL, "gemm: M, N, K must be positive");
+  Q3_CHECK(K % 64 == 0 && N % 32 == 0, QWEN3_ESHAPE, "gemm: K %% 64 == 0 and N %% 32 == 0 required");
+  Q3_CHECK(lda >= K && ldw >= K && lda % 8 == 0 && ldw % 8 == 0 && ldo % 8 == 0, QWEN3_EALIGN,
+           "gemm: leading dimensions must be >= K and multiples of 8");
+  Q3_CHECK(epilogue >= 0 && epilogue <= 2, QWEN3_EINVAL, "gemm: epilogue must be 0, 1 or 2");
+  if (epilogue == kEpiResid) {
+    Q3_CHECK(resid && aligned16(resid) && ldr % 8 == 0 && ldr >= N, QWEN3_EINVAL, "gemm: residual missing or misaligned");
+  }
+  if (epilogue == kEpiSwiglu) {
+    Q3_CHECK(!out_f32, QWEN3_EINVAL, "gemm: SwiGLU output is bf16");
+    Q3_CHECK(ldo >= N / 2, QWEN3_EINVAL, "gemm: ldo too small for N/2 outputs");
+  } else {
+    Q3_CHECK(ldo >= N, QWEN3_EINVAL, "gemm: ldo (%lld) < N (%d)", ldo, N);
+  }
+  int rc = check_device();
+  if (rc) return rc;
+  GemmDesc g;
+  g.swap = swap < 0 ? swap_for(M) : swap != 0;
+  g.K = K;
+  if (g.swap) { g.P = W; g.p_rows = N; g.ldp = ldw; g.Q = A; g.q_rows = M; g.ldq = lda; }
+  else        { g.P = A; g.p_rows = M; g.ldp = lda; g.Q = W; g.q_rows = N; g.ldq = ldw; }
+  g.epi = epilogue;
+  g.resid = resid;
+  g.ldr = ldr;
+  g.resid_f32 = resid_f32 != 0;
+  g.out = out;
+  g.ldo = ldo;
+  g.out_f32 = out_f32 != 0;
+  return finish(launch_gemm(g, static_cast<cudaStream_t>(stream), device_error_word()));
+}
+
+int qwen3_op_qk_norm_rope(const qwen3_config* c, qwen3_bf16* qkv, long long ldqkv, int B, int T, const int* pos_base,
+                          const qwen3_bf16* q_norm, const qwen3_bf16* k_norm, const qwen3_kv_layer* kv,
+                          const float* rope, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(qkv && pos_base && q_norm && k_norm && rope, QWEN3_EINVAL, "qk_norm_rope: NULL pointer");
+  Q3_CHECK(B > 0 && T > 0, QWEN3_EINVAL, "qk_norm_rope: B and T must be positive");
+  if ((rc = check_kv(*c, kv, T))) return rc;
+  Q3_CHECK(ldqkv % 8 == 0 && ldqkv >= (long long)(c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim, QWEN3_EALIGN,
+           "qk_norm_rope: bad ldqkv");
+  if ((rc = check_device())) return rc;
+  return finish(launch_qk_norm_rope(qkv, ldqkv, B, T, c->n_q_heads, c->n_kv_heads, pos_base, q_norm, k_norm, rope,
+                                    kv->k, kv->v, kv->s_max, c->max_pos, c->rms_eps, device_error_word(),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_attention_prefill(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B, int T,
+                               const int* start_pos, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
+                               void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(qkv && start_pos && o, QWEN3_EINVAL, "attention_prefill: NULL pointer");
+  Q3_CHECK(aligned16(qkv) && aligned16(o), QWEN3_EALIGN, "attention_prefill: misaligned pointer");
+  Q3_CHECK(B > 0 && T > 0, QWEN3_EINVAL, "attention_prefill: B and T must be positive");
+  Q3_CHECK(ldqkv % 8 == 0 && ldo % 8 == 0 && ldo >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
+           "attention_prefill: bad leading dimension");
+  if ((rc = check_kv(*c, kv, T))) return rc;
+  if ((rc = check_device())) return rc;
+  return finish(launch_attention_prefill(qkv, ldqkv, B, T, c->n_q_heads, c->n_kv_heads, start_pos, kv->k, kv->v,
+                                         kv->s_max, o, ldo, device_error_word(), static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B,
+                              const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo, void* ws,
+                              size_t ws_bytes, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(qkv && cache_len && o && ws, QWEN3_EINVAL, "attention_decode: NULL pointer");
+  Q3_CHECK(aligned16(qkv) && aligned16(o) && aligned16(ws), QWEN3_EALIGN, "attention_decode: misaligned pointer");
+  Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode: B must be positive");
+  if ((rc = check_kv(*c, kv, 1))) return rc;
+  const size_t need = decode_partial_bytes(B, c->n_q_heads, kv->s_max);
+  Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "attention_decode: workspace has %zu bytes, needs %zu", ws_bytes, need);
+  if ((rc = check_device())) return rc;
+  return finish(launch_attention_decode(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
+                                        kv->s_max, static_cast<float*>(ws), o, ldo, device_error_word(),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,
+                   void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(ids && embed && out, QWEN3_EINVAL, "embed: NULL pointer");
+  Q3_CHECK(aligned16(embed) && aligned16(out), QWEN3_EALIGN, "embed: misaligned pointer");
+  Q3_CHECK(n >= 0 && vocab > 0 && H > 0 && H % 8 == 0, QWEN3_ESHAPE, "embed: bad sizes");
+  int rc = check_device();
+  if (rc) return rc;
+  return finish(launch_embed(ids, n, embed, vocab, H, out, out_f32 != 0, device_error_word(),
+                             static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

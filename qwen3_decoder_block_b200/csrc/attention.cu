@@ -1,0 +1,522 @@
+// K3: causal grouped-query prefill attention on tcgen05 tensor cores.
+// K4: split-KV decode attention (memory bound, CUDA cores) + log-sum-exp merge.
+//
+// Both compute, for query head h at absolute position m and its KV group
+// g = h / (Hq / Hkv),  o = softmax(q k^T / sqrt(128) + M) v  with M = -inf for keys
+// after m ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", section GQA, the
+// attention formula; section prefill 与 decode: a decoded token sees every cached
+// position and itself). Keys and values are read from the KV cache, which already
+// holds this call's tokens (written by the QK-norm/RoPE kernel).
+//
+// Prefill design: one CTA per (q tile, kv group, sequence). The 128-row MMA tile
+// packs 128/G tokens x the G query heads of one KV group, so every K/V tile is
+// loaded once for the whole group. S = Q K^T goes to tensor memory (double
+// buffered), 4 softmax warps (one row per thread) read it with tcgen05.ld, apply
+// the causal mask and an online softmax in the exp2 domain with lazy rescaling
+// of O (only when the running max grows by more than 2^8), write P as bf16 into a
+// 128-byte swizzled shared tile, and O += P V accumulates in tensor memory with V
+// as an MN-major operand. Causal tiles beyond the diagonal are skipped and the
+// heaviest q tiles are scheduled first.
+#include "common.cuh"
+#include "internal.h"
+
+namespace q3 {
+
+int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld, int box_rows);
+int make_tmap_3d(CUtensorMap* map, const void* base, long long inner, long long mid, long long outer,
+                 long long mid_stride_bytes, long long outer_stride_bytes, int box_inner, int box_mid, int box_outer);
+
+namespace {
+
+constexpr int kHeadDim = 128;
+constexpr int kTileQ = 128;   // MMA rows per CTA
+constexpr int kTileK = 128;   // keys per KV tile
+constexpr uint32_t kHalf = 128 * 64 * 2;  // one [128 rows][64] bf16 swizzled half tile: 16 KB
+// smem layout (1024-aligned): Q (2 halves), 2 stages x (K 2 halves, V 2 halves), P (2 halves)
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffKV = 2 * kHalf;
+constexpr uint32_t kStageBytes = 4 * kHalf;
+constexpr uint32_t kOffP = kOffKV + 2 * kStageBytes;
+constexpr uint32_t kOffBar = kOffP + 2 * kHalf;
+constexpr uint32_t kPrefillSmem = kOffBar + 256 + 1024;
+// log2(e) / sqrt(128)
+constexpr float kScaleLog2 = 0.12751743074380304f;
+constexpr float kRescaleThreshold = 8.0f;
+
+struct PrefillParams {
+  int B, T, Hq, Hkv, G, s_max, n_qtiles;
+  const int* start_pos;
+  uint16_t* out;
+  long long ldo;
+  int* err;
+};
+
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* v_full = bars + 3;    // [2]
+  uint64_t* kv_empty = bars + 5;  // [2]
+  uint64_t* s_full = bars + 7;    // [2]
+  uint64_t* s_free = bars + 9;    // [2]
+  uint64_t* p_full = bars + 11;
+  uint64_t* p_free = bars + 12;   // PV of the previous tile complete (O stable, P reusable)
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = p.n_qtiles - 1 - (int)blockIdx.x;  // heavy tiles first
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int G = p.G, TQ = kTileQ / G;
+  const int t0 = qt * TQ;
+  const int start = p.start_pos[b];
+  const int kv_limit = start + p.T;  // keys [0, kv_limit) are in the cache
+  const int t_last = min(t0 + TQ, p.T) - 1;
+  const int n_kv = (start + t_last) / kTileK + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1); mbar_init(&v_full[i], 1); mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128);
+    }
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_O = tmem + 256;
+  const long long kv_row0 = ((long long)b * p.Hkv + g) * p.s_max;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      bool ok = true;
+      long long issued_kv = 0;
+      mbar_arrive_expect_tx(q_full, 2 * kHalf);
+      for (int h = 0; h < 2; ++h)
+        tma_load_3d(smem + kOffQ + h * kHalf, &tmQ, q_full, 64 * h, g * G, b * p.T + t0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (*s_abort || !mbar_wait(&kv_empty[st], par ^ 1, p.err)) { ok = false; break; }
+        uint8_t* base = smem + kOffKV + st * kStageBytes;
+        const int row = (int)(kv_row0 + (long long)j * kTileK);
+        mbar_arrive_expect_tx(&k_full[st], 2 * kHalf);
+        tma_load_2d(base, &tmK, &k_full[st], 0, row);
+        tma_load_2d(base + kHalf, &tmK, &k_full[st], 64, row);
+        mbar_arrive_expect_tx(&v_full[st], 2 * kHalf);
+        tma_load_2d(base + 2 * kHalf, &tmV, &v_full[st], 0, row);
+        tma_load_2d(base + 3 * kHalf, &tmV, &v_full[st], 64, row);
+        ++issued_kv;
+      }
+      // Before exit every copy must have landed (normal path: consumers saw them all).
+      mbar_wait(q_full, 0, p.err);
+      if (!ok) {
+        *s_abort = 1;
+        for (long long i = issued_kv > 2 ? issued_kv - 2 : 0; i < issued_kv; ++i) {
+          mbar_wait(&k_full[i & 1], (uint32_t)((i >> 1) & 1), p.err);
+          mbar_wait(&v_full[i & 1], (uint32_t)((i >> 1) & 1), p.err);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileK, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim, 0, 1);  // V is MN-major
+      bool ok = mbar_wait(q_full, 0, p.err);
+      const uint32_t sq = smem_u32(smem + kOffQ);
+      const uint32_t sp = smem_u32(smem + kOffP);
+      for (int j = 0; j <= n_kv && ok; ++j) {
+        if (j < n_kv) {
+          // S_j = Q K_j^T into S buffer j&1
+          const int st = j & 1;
+          const uint32_t par = (j >> 1) & 1;
+          if (*s_abort || !mbar_wait(&k_full[st], par, p.err) || !mbar_wait(&s_free[st], par ^ 1, p.err)) {
+            ok = false; break;
+          }
+          tc_fence_after();
+          const uint32_t sk = smem_u32(smem + kOffKV + st * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = sdesc_kmajor_sw128(sq + (kk >> 2) * kHalf) + 2 * (kk & 3);
+            const uint64_t bd = sdesc_kmajor_sw128(sk + (kk >> 2) * kHalf) + 2 * (kk & 3);
+            mma_bf16_ss(tmem + st * 128, a, bd, idesc_s, kk ? 1u : 0u);
+          }
+          mma_commit(&s_full[st]);
+        }
+        if (j > 0) {
+          // O += P_{j-1} V_{j-1}
+          const int jj = j - 1, st = jj & 1;
+          const uint32_t par = (jj >> 1) & 1;
+          if (*s_abort || !mbar_wait(&v_full[st], par, p.err) || !mbar_wait(p_full, jj & 1, p.err)) {
+            ok = false; break;
+          }
+          tc_fence_after();
+          const uint32_t sv = smem_u32(smem + kOffKV + st * kStageBytes + 2 * kHalf);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = sdesc_kmajor_sw128(sp + (kk >> 2) * kHalf) + 2 * (kk & 3);
+            const uint64_t bd = sdesc_mnmajor_sw128(sv + kk * 16 * 128, kHalf, 1024);
+            mma_bf16_ss(tmem_O, a, bd, idesc_o, (jj | kk) ? 1u : 0u);
+          }
+          mma_commit(p_free);
+          mma_commit(&kv_empty[st]);
+        }
+      }
+      if (!ok) {
+        *s_abort = 1;
+        mma_commit(drain);
+        mbar_wait(drain, 0, p.err);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // tile row
+    const int t = t0 + r / G;
+    const int qpos = start + t;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    uint8_t* sP = smem + kOffP;
+    for (int j = 0; j < n_kv; ++j) {
+      const int st = j & 1;
+      const uint32_t par = (j >> 1) & 1;
+      bool w_ok = !*s_abort && mbar_wait(&s_full[st], par, p.err);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + st * 128 + c * 32 + ((uint32_t)(quad * 32) << 16), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[st]);
+      const int kv0 = j * kTileK;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 128; ++i) {
+        const int kp = kv0 + i;
+        const bool vis = kp <= qpos && kp < kv_limit;
+        s[i] = vis ? s[i] * kScaleLog2 : -INFINITY;
+        mx = fmaxf(mx, s[i]);
+      }
+      float m_use = m_run, alpha = 1.f;
+      if (mx > m_run + kRescaleThreshold || m_run == -INFINITY) {
+        m_use = fmaxf(mx, m_run);
+        alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_use);
+        m_run = m_use;
+      }
+      float sum = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = (m_use == -INFINITY) ? 0.f : exp2f(s[2 * i] - m_use);
+        const float p1 = (m_use == -INFINITY) ? 0.f : exp2f(s[2 * i + 1] - m_use);
+        sum += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      // the previous PV must be complete before O is rescaled or P overwritten
+      if (j > 0) {
+        w_ok = !*s_abort && mbar_wait(p_free, (j - 1) & 1, p.err);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            const uint32_t ta = tmem_O + c * 32 + ((uint32_t)(quad * 32) << 16);
+            tmem_ld32(ta, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+            tmem_st32(ta, v);
+          }
+          tmem_wait_st();
+        }
+      }
+      // the last KV tile may extend past the written cache: zero those V rows so
+      // that 0-probability keys cannot inject NaN/Inf through P V
+      if (kv0 + kTileK > kv_limit) {
+        w_ok = !*s_abort && mbar_wait(&v_full[st], par, p.err);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        if (kv0 + r >= kv_limit) {
+          uint4* v0 = reinterpret_cast<uint4*>(smem + kOffKV + st * kStageBytes + 2 * kHalf + r * 128);
+          uint4* v1 = reinterpret_cast<uint4*>(smem + kOffKV + st * kStageBytes + 3 * kHalf + r * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) { v0[c] = make_uint4(0, 0, 0, 0); v1[c] = make_uint4(0, 0, 0, 0); }
+        }
+      }
+      // P row r -> two 128-byte-swizzled K-major half tiles
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint8_t* rowp = sP + h * kHalf + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const int pc = c ^ (r & 7);
+          *reinterpret_cast<uint4*>(rowp + pc * 16) =
+              make_uint4(pk[h * 32 + c * 4], pk[h * 32 + c * 4 + 1], pk[h * 32 + c * 4 + 2], pk[h * 32 + c * 4 + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // epilogue: O / l -> bf16
+    if (ok) {
+      bool w_ok = !*s_abort && mbar_wait(p_free, (n_kv - 1) & 1, p.err);
+      if (__all_sync(0xffffffffu, w_ok)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        const int h = g * G + (r % G);
+        uint16_t* dst = p.out + ((long long)b * p.T + t) * p.ldo + (long long)h * kHeadDim;
+        const bool store = t < p.T;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem_O + c * 32 + ((uint32_t)(quad * 32) << 16), v);
+          tmem_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * inv_l, __uint_as_float(v[8 * i + 1]) * inv_l);
+              o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l, __uint_as_float(v[8 * i + 3]) * inv_l);
+              o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l, __uint_as_float(v[8 * i + 5]) * inv_l);
+              o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l, __uint_as_float(v[8 * i + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(dst + c * 32 + i * 8) = o;
+            }
+          }
+        }
+      } else {
+        *s_abort = 1;
+      }
+    } else {
+      *s_abort = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv,
+                             const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
+                             long long ldo, int* err, cudaStream_t s) {
+  if (B <= 0 || T <= 0) return 0;
+  const int G = Hq / Hkv;
+  const int TQ = kTileQ / G;
+  CUtensorMap tmQ, tmK, tmV;
+  // Q: (dim, head, token) with the G heads of one group and TQ tokens per box
+  if (make_tmap_3d(&tmQ, qkv, kHeadDim, Hq, (long long)B * T, kHeadDim * 2, ldqkv * 2, 64, G, TQ) != 0) {
+    set_last_error("attention: cannot encode the query tensor map");
+    return -6;
+  }
+  const long long kv_rows = (long long)B * Hkv * s_max;
+  if (make_tmap_2d(&tmK, ck, kv_rows, kHeadDim, kHeadDim, kTileK) != 0 ||
+      make_tmap_2d(&tmV, cv, kv_rows, kHeadDim, kHeadDim, kTileK) != 0) {
+    set_last_error("attention: cannot encode the KV-cache tensor maps");
+    return -6;
+  }
+  PrefillParams p;
+  p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.s_max = s_max;
+  p.n_qtiles = (T + TQ - 1) / TQ;
+  p.start_pos = start_pos;
+  p.out = out;
+  p.ldo = ldo;
+  p.err = err;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+    attr = true;
+  }
+  dim3 grid(p.n_qtiles, Hkv, B);
+  attn_prefill_kernel<<<grid, 192, kPrefillSmem, s>>>(tmQ, tmK, tmV, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("attention prefill launch failed: %s", cudaGetErrorString(e));
+    return -6;
+  }
+  return 0;
+}
+
+// ============================================================================
+// K4: split-KV decode attention. CTA (split, group, sequence) handles keys
+// [split*128, split*128+128) of one sequence's KV group for all G query heads of
+// the group, so each K/V line is read once. K and V chunks arrive by two bulk
+// copies; scores use one warp per key (lanes split the 128 dims); the partial
+// (max, sum, unnormalised o) goes to the workspace and a second kernel merges
+// the splits with log-sum-exp weights.
+// ============================================================================
+constexpr int kDecChunk = 128;
+constexpr int kDecThreads = 256;
+
+__global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
+    const uint16_t* __restrict__ qkv, long long ldqkv, int Hq, int Hkv, const int* __restrict__ cache_len,
+    const uint16_t* __restrict__ ck, const uint16_t* __restrict__ cv, int s_max, int n_splits,
+    float* __restrict__ part, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint16_t* sK = reinterpret_cast<uint16_t*>(smem);
+  uint16_t* sV = sK + kDecChunk * kHeadDim;
+  float* sQ = reinterpret_cast<float*>(sV + kDecChunk * kHeadDim);  // [G][128]
+  const int G = Hq / Hkv;
+  float* sS = sQ + G * kHeadDim;                                     // [G][128]
+  float* sM = sS + G * kDecChunk;                                    // [G]
+  float* sL = sM + G;                                                // [G]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sL + G + 2);
+  bar = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(bar) + 7) & ~uintptr_t(7));
+
+  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_keys_total = cache_len[b] + 1;  // cached tokens + the new one
+  const int k0 = split * kDecChunk;
+  const int nk = min(kDecChunk, n_keys_total - k0);
+  float* my_part = part + (((long long)b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
+  const long long head_stride = (long long)n_splits * (kHeadDim + 2);
+  if (nk <= 0 || n_keys_total > s_max) {
+    if (n_keys_total > s_max && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
+    for (int i = threadIdx.x; i < G; i += blockDim.x) {
+      my_part[i * head_stride + kHeadDim] = -INFINITY;
+      my_part[i * head_stride + kHeadDim + 1] = 0.f;
+    }
+    return;
+  }
+  const long long row0 = ((long long)b * Hkv + g) * s_max + k0;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, 2u * nk * kHeadDim * 2);
+    bulk_load(sK, ck + row0 * kHeadDim, nk * kHeadDim * 2, bar);
+    bulk_load(sV, cv + row0 * kHeadDim, nk * kHeadDim * 2, bar);
+  }
+  // query heads of this group (already normed and rotated) -> fp32 smem
+  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+    const int j = i / kHeadDim, d = i % kHeadDim;
+    sQ[i] = __uint_as_float((uint32_t)qkv[(long long)b * ldqkv + (long long)(g * G + j) * kHeadDim + d] << 16) *
+            kScaleLog2;
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(bar, 0, err);
+  if (!__syncthreads_and(ok)) {
+    return;  // nothing left in flight: the wait either completed or its budget ran out
+  }
+  // scores: warp per key, lane owns dims [4*lane, 4*lane+4)
+  for (int k = warp; k < nk; k += kDecThreads / 32) {
+    const uint2 kv = *reinterpret_cast<const uint2*>(sK + k * kHeadDim + 4 * lane);
+    const float k0f = bf16_lo(kv.x), k1f = bf16_hi(kv.x), k2f = bf16_lo(kv.y), k3f = bf16_hi(kv.y);
+    for (int j = 0; j < G; ++j) {
+      const float4 q = *reinterpret_cast<const float4*>(sQ + j * kHeadDim + 4 * lane);
+      float d = q.x * k0f + q.y * k1f + q.z * k2f + q.w * k3f;
+      d = warp_sum(d);
+      if (lane == 0) sS[j * kDecChunk + k] = d;
+    }
+  }
+  __syncthreads();
+  // per-head max and sum over this chunk
+  for (int j = warp; j < G; j += kDecThreads / 32) {
+    float mx = -INFINITY;
+    for (int k = lane; k < nk; k += 32) mx = fmaxf(mx, sS[j * kDecChunk + k]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int k = lane; k < nk; k += 32) {
+      const float e = exp2f(sS[j * kDecChunk + k] - mx);
+      sS[j * kDecChunk + k] = e;
+      sum += e;
+    }
+    sum = warp_sum(sum);
+    if (lane == 0) { sM[j] = mx; sL[j] = sum; }
+  }
+  __syncthreads();
+  // o[j][d] = sum_k p[j][k] v[k][d]
+  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+    const int j = i / kHeadDim, d = i % kHeadDim;
+    const float* pj = sS + j * kDecChunk;
+    float acc = 0.f;
+    for (int k = 0; k < nk; ++k) acc += pj[k] * __uint_as_float((uint32_t)sV[k * kHeadDim + d] << 16);
+    my_part[j * head_stride + d] = acc;
+  }
+  if (threadIdx.x < G) {
+    my_part[threadIdx.x * head_stride + kHeadDim] = sM[threadIdx.x];
+    my_part[threadIdx.x * head_stride + kHeadDim + 1] = sL[threadIdx.x];
+  }
+}
+
+__global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
+                                         uint16_t* __restrict__ out, long long ldo) {
+  const int bh = blockIdx.x;  // b * Hq + h
+  const int b = bh / Hq, h = bh % Hq;
+  const float* pp = part + (long long)bh * n_splits * (kHeadDim + 2);
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pp[s * (kHeadDim + 2) + kHeadDim]);
+  const int d = threadIdx.x;
+  float L = 0.f, acc = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float* q = pp + s * (kHeadDim + 2);
+    const float m = q[kHeadDim];
+    if (m == -INFINITY) continue;
+    const float w = exp2f(m - M);
+    L += q[kHeadDim + 1] * w;
+    acc += q[d] * w;
+  }
+  out[(long long)b * ldo + (long long)h * kHeadDim + d] = to_bf16_bits(acc / L);
+}
+
+int decode_splits(int s_max) { return (s_max + kDecChunk - 1) / kDecChunk; }
+
+size_t decode_partial_bytes(int B, int Hq, int s_max) {
+  return (size_t)B * Hq * decode_splits(s_max) * (kHeadDim + 2) * sizeof(float);
+}
+
+int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
+                            const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
+                            long long ldo, int* err, cudaStream_t s) {
+  if (B <= 0) return 0;
+  const int G = Hq / Hkv;
+  const int n_splits = decode_splits(s_max);
+  const size_t smem = 128 + 2 * kDecChunk * kHeadDim * 2 + (size_t)G * kHeadDim * 4 + (size_t)G * kDecChunk * 4 +
+                      (size_t)2 * G * 4 + 64;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attn_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    attr = true;
+  }
+  dim3 grid(n_splits, Hkv, B);
+  attn_decode_split_kernel<<<grid, kDecThreads, smem, s>>>(qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max, n_splits,
+                                                            part, err);
+  attn_decode_merge_kernel<<<B * Hq, kHeadDim, 0, s>>>(part, Hq, n_splits, out, ldo);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
+    return -6;
+  }
+  return 0;
+}
+
+}  // namespace q3

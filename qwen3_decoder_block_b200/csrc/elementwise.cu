@@ -1,0 +1,228 @@
+// K1 RMSNorm, K5 per-head QK-RMSNorm + rotate-half RoPE + KV-cache write, the
+// embedding gather and the weight-interleave pack. All are HBM-bound: one warp
+// per row (or per head), 16-byte (RMSNorm) or 4-byte coalesced accesses, fp32
+// arithmetic, one bf16 rounding per output.
+//
+// Pages cited:
+//   [P-Mini] "从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构" (quarkcode.cn)
+//   [P-MoE]  "从零构建 Qwen-3 MoE" (adg.csdn.net)
+#include "common.cuh"
+#include "internal.h"
+
+namespace q3 {
+
+// ---------------------------------------------------------------------------
+// K1: out = x * rsqrt(mean(x^2) + eps) * w  ([P-Mini] section RMSNorm, the
+// x-hat formula: computed in fp32, cast back once). x is bf16 or fp32.
+// One warp per row; each lane owns 8 consecutive elements of every 256-wide
+// slice (n <= 2048, n % 256 == 0).
+// ---------------------------------------------------------------------------
+template <bool IN_F32>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
+                                                      const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
+                                                      long long ldo, int rows, int n, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int n_warps = (gridDim.x * blockDim.x) >> 5;
+  const int slices = n >> 8;
+  for (int row = warp_global; row < rows; row += n_warps) {
+    float v[8][8];
+    float ss = 0.f;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      if (s < slices) {
+        const int col = s * 256 + lane * 8;
+        if (IN_F32) {
+          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (long long)row * ldx + col);
+          float4 a = src[0], b = src[1];
+          v[s][0] = a.x; v[s][1] = a.y; v[s][2] = a.z; v[s][3] = a.w;
+          v[s][4] = b.x; v[s][5] = b.y; v[s][6] = b.z; v[s][7] = b.w;
+        } else {
+          uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (long long)row * ldx + col);
+          v[s][0] = bf16_lo(a.x); v[s][1] = bf16_hi(a.x); v[s][2] = bf16_lo(a.y); v[s][3] = bf16_hi(a.y);
+          v[s][4] = bf16_lo(a.z); v[s][5] = bf16_hi(a.z); v[s][6] = bf16_lo(a.w); v[s][7] = bf16_hi(a.w);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss += v[s][j] * v[s][j];
+      }
+    }
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)n + eps);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      if (s < slices) {
+        const int col = s * 256 + lane * 8;
+        uint4 wv = *reinterpret_cast<const uint4*>(w + col);
+        uint4 o;
+        o.x = pack_bf16x2(v[s][0] * r * bf16_lo(wv.x), v[s][1] * r * bf16_hi(wv.x));
+        o.y = pack_bf16x2(v[s][2] * r * bf16_lo(wv.y), v[s][3] * r * bf16_hi(wv.y));
+        o.z = pack_bf16x2(v[s][4] * r * bf16_lo(wv.z), v[s][5] * r * bf16_hi(wv.z));
+        o.w = pack_bf16x2(v[s][6] * r * bf16_lo(wv.w), v[s][7] * r * bf16_hi(wv.w));
+        *reinterpret_cast<uint4*>(out + (long long)row * ldo + col) = o;
+      }
+    }
+  }
+}
+
+int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
+                   int rows, int n, float eps, cudaStream_t s) {
+  if (rows <= 0) return 0;
+  const int warps_per_block = 8;
+  long long blocks = (rows + warps_per_block - 1) / warps_per_block;
+  if (blocks > (long long)num_sms() * 16) blocks = (long long)num_sms() * 16;
+  if (x_f32)
+    rmsnorm_kernel<true><<<(int)blocks, 256, 0, s>>>(x, ldx, w, out, ldo, rows, n, eps);
+  else
+    rmsnorm_kernel<false><<<(int)blocks, 256, 0, s>>>(x, ldx, w, out, ldo, rows, n, eps);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// ---------------------------------------------------------------------------
+// K5: for every token m = b*T + t at absolute position pos = pos_base[b] + t and
+// every head slot of the fused QKV row:
+//   q heads: RMSNorm over the 128 dims with q_norm weights, then RoPE, written
+//            back in place ([P-Mini] section GQA: q_norm / k_norm before RoPE);
+//   k heads: the same with k_norm, written to the cache at [b][g][pos][:];
+//   v heads: copied to the cache at [b][g][pos][:].
+// RoPE pairs dimension i with i + 64 ([P-Mini] section RoPE):
+//   (a, b) -> (a cos(pos theta_i) - b sin(pos theta_i), a sin(pos theta_i) + b cos(pos theta_i)),
+// with cos/sin read from the fp32 table [max_pos][64][2] (cos, sin).
+// One warp per (token, head slot); lane l owns dims {2l, 2l+1} and {64+2l, 65+2l}.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qk_norm_rope_kernel(uint16_t* __restrict__ qkv, long long ldqkv, int B, int T,
+                                                           int Hq, int Hkv, const int* __restrict__ pos_base,
+                                                           const uint16_t* __restrict__ qw,
+                                                           const uint16_t* __restrict__ kw,
+                                                           const float* __restrict__ rope, uint16_t* __restrict__ ck,
+                                                           uint16_t* __restrict__ cv, int s_max, int max_pos,
+                                                           float eps, int* err) {
+  const int lane = threadIdx.x & 31;
+  const long long item = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int slots = Hq + 2 * Hkv;
+  const long long total = (long long)B * T * slots;
+  if (item >= total) return;
+  const int slot = (int)(item % slots);
+  const long long m = item / slots;
+  const int b = (int)(m / T), t = (int)(m % T);
+  const int pos = pos_base[b] + t;
+  if (pos < 0 || pos >= s_max || pos >= max_pos) {
+    if (lane == 0) record_error(err, kErrCapacity);
+    return;
+  }
+  uint16_t* row = qkv + m * ldqkv + (long long)slot * 128;
+  const uint32_t x0 = *reinterpret_cast<const uint32_t*>(row + 2 * lane);
+  const uint32_t x1 = *reinterpret_cast<const uint32_t*>(row + 64 + 2 * lane);
+  if (slot >= Hq + Hkv) {  // value head: copy into the cache
+    const int g = slot - Hq - Hkv;
+    uint16_t* dst = cv + (((long long)b * Hkv + g) * s_max + pos) * 128;
+    *reinterpret_cast<uint32_t*>(dst + 2 * lane) = x0;
+    *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = x1;
+    return;
+  }
+  const bool is_q = slot < Hq;
+  const uint16_t* wn = is_q ? qw : kw;
+  float a0 = bf16_lo(x0), a1 = bf16_hi(x0), b0 = bf16_lo(x1), b1 = bf16_hi(x1);
+  const float ss = warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1);
+  const float r = rsqrtf(ss * (1.0f / 128.0f) + eps);
+  const uint32_t wa = *reinterpret_cast<const uint32_t*>(wn + 2 * lane);
+  const uint32_t wb = *reinterpret_cast<const uint32_t*>(wn + 64 + 2 * lane);
+  a0 *= r * bf16_lo(wa); a1 *= r * bf16_hi(wa);
+  b0 *= r * bf16_lo(wb); b1 *= r * bf16_hi(wb);
+  const float4 cs = *reinterpret_cast<const float4*>(rope + ((long long)pos * 64 + 2 * lane) * 2);  // (c0, s0, c1, s1)
+  const float o_a0 = a0 * cs.x - b0 * cs.y, o_b0 = a0 * cs.y + b0 * cs.x;
+  const float o_a1 = a1 * cs.z - b1 * cs.w, o_b1 = a1 * cs.w + b1 * cs.z;
+  uint16_t* dst;
+  if (is_q) {
+    dst = row;
+  } else {
+    const int g = slot - Hq;
+    dst = ck + (((long long)b * Hkv + g) * s_max + pos) * 128;
+  }
+  *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf16x2(o_a0, o_a1);
+  *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf16x2(o_b0, o_b1);
+}
+
+int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv, const int* pos_base,
+                        const uint16_t* qw, const uint16_t* kw, const float* rope, uint16_t* ck, uint16_t* cv,
+                        int s_max, int max_pos, float eps, int* err, cudaStream_t s) {
+  const long long warps = (long long)B * T * (Hq + 2 * Hkv);
+  if (warps == 0) return 0;
+  const long long blocks = (warps * 32 + 255) / 256;
+  qk_norm_rope_kernel<<<(unsigned)blocks, 256, 0, s>>>(qkv, ldqkv, B, T, Hq, Hkv, pos_base, qw, kw, rope, ck, cv,
+                                                       s_max, max_pos, eps, err);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// ---------------------------------------------------------------------------
+// Embedding gather ([P-MoE] section 5; [P-Mini] section 骨架): out[m] = E[ids[m]],
+// widened to fp32 when the residual stream is kept in fp32.
+// ---------------------------------------------------------------------------
+__global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t* __restrict__ E, int vocab, int H,
+                             void* __restrict__ out, int out_f32, int* err) {
+  const int m = blockIdx.x;
+  if (m >= n) return;
+  const int id = ids[m];
+  if (id < 0 || id >= vocab) {
+    if (threadIdx.x == 0) record_error(err, kErrInvalid);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(E + (long long)id * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    uint4 a = src[c];
+    if (out_f32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + (long long)m * H + c * 8);
+      dst[0] = make_float4(bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y));
+      dst[1] = make_float4(bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w));
+    } else {
+      reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + (long long)m * H)[c] = a;
+    }
+  }
+}
+
+int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, void* out, bool out_f32, int* err,
+                 cudaStream_t s) {
+  if (n <= 0) return 0;
+  embed_kernel<<<n, 128, 0, s>>>(ids, n, E, vocab, H, out, out_f32 ? 1 : 0, err);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// ---------------------------------------------------------------------------
+// Gate/up interleave: packed rows [32j, 32j+16) = gate rows [16j, 16j+16),
+// rows [32j+16, 32j+32) = up rows [16j, 16j+16), for n_mats matrices of I rows
+// (dense FFN: separate gate and up; MoE: fused [E, 2I, H] split by chunk(2)).
+// ---------------------------------------------------------------------------
+__global__ void pack_gate_up_kernel(const uint16_t* __restrict__ gate, const uint16_t* __restrict__ up,
+                                    long long mat_stride, int n_mats, int I, int H, uint16_t* __restrict__ out) {
+  const long long R = blockIdx.x;  // output row
+  const long long rows = (long long)n_mats * 2 * I;
+  if (R >= rows) return;
+  const int mat = (int)(R / (2 * I));
+  const int rr = (int)(R % (2 * I));
+  const int blk = rr / 32, half = (rr / 16) & 1, r = rr % 16;
+  const uint16_t* src = (half ? up : gate) + mat * mat_stride + (long long)(blk * 16 + r) * H;
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(out + R * H);
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) d4[c] = s4[c];
+}
+
+int launch_pack_gate_up(const uint16_t* gate, const uint16_t* up, long long mat_stride, int n_mats, int I, int H,
+                        uint16_t* out, cudaStream_t s) {
+  const long long rows = (long long)n_mats * 2 * I;
+  if (rows == 0) return 0;
+  pack_gate_up_kernel<<<(unsigned)rows, 128, 0, s>>>(gate, up, mat_stride, n_mats, I, H, out);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// Decode bookkeeping: every sequence's cached length grows by one token.
+__global__ void advance_lengths_kernel(int* len, int B) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) len[b] += 1;
+}
+
+int launch_advance_lengths(int* len, int B, cudaStream_t s) {
+  if (B <= 0) return 0;
+  advance_lengths_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, B);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+}  // namespace q3

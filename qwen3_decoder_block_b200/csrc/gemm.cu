@@ -1,0 +1,445 @@
+// K2: persistent tcgen05 GEMM for the block's projections (QKV, o_proj, gate/up,
+// down), the tied LM head, the MoE router and the grouped expert GEMMs.
+//
+// Every projection on the pages is an nn.Linear without bias, x @ W^T with W
+// stored [out, in] ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", section GQA;
+// section SwiGLU FFN), so both operands are K-major and the kernel computes
+// D[p][q] = sum_k P[p][k] Q[q][k].
+//
+// Design (sm_100a):
+//   * one CTA per SM, persistent over output tiles of 128 x BN;
+//   * warp 0: TMA producer (128-byte swizzled 128x64 and BNx64 tiles, mbarrier
+//     ring of STAGES); warp 1: one thread issues tcgen05.mma (M=128, N=BN, K=16)
+//     into a double-buffered fp32 accumulator in tensor memory; warps 2-5:
+//     epilogue, tcgen05.ld of the accumulator, fused epilogue, global stores;
+//   * swap mode for small M: the weight rows fill the MMA's 128-row side and the
+//     tokens become N, so decode-sized GEMMs still stream the weights;
+//   * grouped mode for MoE: per-expert row ranges of the permuted activations.
+// Every wait is bounded (1 s of %globaltimer); on expiry the kernel records
+// QWEN3_ETIMEOUT in the device error word, drains its copies and MMAs, frees
+// its tensor memory and returns.
+#include <cstdio>
+#include <mutex>
+#include <cudaTypedefs.h>
+#include "common.cuh"
+#include "internal.h"
+
+namespace q3 {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr uint32_t P_BYTES = BM * BK * 2;
+  static constexpr uint32_t Q_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t BAR_BYTES = 256;
+  static size_t smem_bytes(int n_groups) {
+    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 8 * (size_t)(n_groups + 2);
+  }
+};
+
+struct GemmParams {
+  int p_rows, q_rows, k_blocks;
+  int p_tiles, q_tiles, q_fast;
+  int epi, resid_f32, out_f32, swap;
+  void* out;
+  long long ldo;
+  const void* resid;
+  long long ldr;
+  int n_groups;
+  const int* group_offsets;
+  int* err;
+};
+
+struct Tile {
+  int p0, p_end, q0, q_end, q_load;
+};
+
+__device__ __forceinline__ int total_tiles(const GemmParams& g, const int* s_prefix) {
+  return g.n_groups > 0 ? s_prefix[g.n_groups] : g.p_tiles * g.q_tiles;
+}
+
+template <int BN>
+__device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const int* s_prefix, const int* s_off) {
+  Tile r;
+  if (g.n_groups > 0) {
+    int lo = 0, hi = g.n_groups - 1;  // largest grp with s_prefix[grp] <= t
+    while (lo < hi) {
+      int mid = (lo + hi + 1) >> 1;
+      if (s_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int grp = lo, local = t - s_prefix[grp];
+    const int pt = local / g.q_tiles, qt = local % g.q_tiles;
+    r.p0 = s_off[grp] + pt * BM;
+    r.p_end = s_off[grp + 1];
+    r.q0 = qt * BN;
+    r.q_end = g.q_rows;
+    r.q_load = grp * g.q_rows + r.q0;
+  } else {
+    int pt, qt;
+    if (g.q_fast) { pt = t / g.q_tiles; qt = t % g.q_tiles; }
+    else          { qt = t / g.p_tiles; pt = t % g.p_tiles; }
+    r.p0 = pt * BM;
+    r.p_end = g.p_rows;
+    r.q0 = qt * BN;
+    r.q_end = g.q_rows;
+    r.q_load = r.q0;
+  }
+  return r;
+}
+
+// --------------------------------------------------------------------------- epilogues
+__device__ __forceinline__ void store_row_chunk(const GemmParams& g, int p, int q, const uint32_t (&r)[32]) {
+  // non-swap: 32 accumulators of output row p, columns [q, q+32)
+  if (g.epi == kEpiSwiglu) {
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float g0 = __uint_as_float(r[2 * j]), g1 = __uint_as_float(r[2 * j + 1]);
+      float u0 = __uint_as_float(r[16 + 2 * j]), u1 = __uint_as_float(r[16 + 2 * j + 1]);
+      o[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + (q >> 1));
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    return;
+  }
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (g.epi == kEpiResid) {
+    if (g.resid_f32) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 a = src[j];
+        v[4 * j] += a.x; v[4 * j + 1] += a.y; v[4 * j + 2] += a.z; v[4 * j + 3] += a.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 a = src[j];
+        v[8 * j + 0] += bf16_lo(a.x); v[8 * j + 1] += bf16_hi(a.x);
+        v[8 * j + 2] += bf16_lo(a.y); v[8 * j + 3] += bf16_hi(a.y);
+        v[8 * j + 4] += bf16_lo(a.z); v[8 * j + 5] += bf16_hi(a.z);
+        v[8 * j + 6] += bf16_lo(a.w); v[8 * j + 7] += bf16_hi(a.w);
+      }
+    }
+  }
+  if (g.out_f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (long long)p * g.ldo + q);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) dst[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                          pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+  }
+}
+
+// swap: this thread owns feature p (one TMEM lane) and tokens [q, q+32)
+__device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int p_valid, int q, int q_end,
+                                                int lane, int feat_block, const uint32_t (&r)[32]) {
+  if (g.epi == kEpiSwiglu) {
+    // lanes 0..15 hold gate features, lanes 16..31 the matching up features
+    const int f = (feat_block >> 1) + lane;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float a = __uint_as_float(r[j]);
+      float u = __shfl_down_sync(0xffffffffu, a, 16);
+      if (lane < 16 && p_valid && q + j < q_end)
+        static_cast<uint16_t*>(g.out)[(long long)(q + j) * g.ldo + f] = to_bf16_bits(silu_f(a) * u);
+    }
+    return;
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (!p_valid || q + j >= q_end) continue;
+    float v = __uint_as_float(r[j]);
+    const long long row = q + j;
+    if (g.epi == kEpiResid) {
+      if (g.resid_f32) v += static_cast<const float*>(g.resid)[row * g.ldr + p];
+      else v += __uint_as_float((uint32_t)static_cast<const uint16_t*>(g.resid)[row * g.ldr + p] << 16);
+    }
+    if (g.out_f32) static_cast<float*>(g.out)[row * g.ldo + p] = v;
+    else static_cast<uint16_t*>(g.out)[row * g.ldo + p] = to_bf16_bits(v);
+  }
+}
+
+// --------------------------------------------------------------------------- kernel
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                   const GemmParams g) {
+  using C = GemmCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+  int* s_off = s_prefix + (g.n_groups + 1);  // only used in grouped mode (aliases past prefix)
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (threadIdx.x == 32) { tma_prefetch_desc(&tmP); tma_prefetch_desc(&tmQ); }
+  if (g.n_groups > 0) {
+    // per-group tile counts -> prefix (offsets are stored right after the prefix)
+    for (int i = threadIdx.x; i <= g.n_groups; i += blockDim.x) s_off[i] = g.group_offsets[i];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0;
+      for (int i = 0; i < g.n_groups; ++i) {
+        s_prefix[i] = acc;
+        const int m = s_off[i + 1] - s_off[i];
+        acc += ((m + BM - 1) / BM) * g.q_tiles;
+      }
+      s_prefix[g.n_groups] = acc;
+    }
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int ntiles = total_tiles(g, s_prefix);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (*s_abort || !mbar_wait(&empty[stage], phase ^ 1, g.err)) { ok = false; break; }
+          uint8_t* sp = smem + stage * C::STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          tma_load_2d(sp, &tmP, &full[stage], kb * BK, tl.p0);
+          tma_load_2d(sp + C::P_BYTES, &tmQ, &full[stage], kb * BK, tl.q_load);
+          ++issued;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        *s_abort = 1;
+        // let every copy still in flight land before the CTA exits
+        for (long long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
+          mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), g.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+        const int buf = local & 1;
+        const uint32_t use_par = (local >> 1) & 1;
+        if (*s_abort || !mbar_wait(&tempty[buf], use_par ^ 1, g.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * BN;
+        for (int kb = 0; kb < g.k_blocks; ++kb) {
+          if (*s_abort || !mbar_wait(&full[stage], phase, g.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint64_t adesc = sdesc_kmajor_sw128(sa);
+          const uint64_t bdesc = sdesc_kmajor_sw128(sa + C::P_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);
+      }
+      if (!ok) {
+        *s_abort = 1;
+        mma_commit(drain);  // completes once every issued MMA has finished
+        mbar_wait(drain, 0, g.err);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32) are reachable from this warp
+    int local = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
+      const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
+      const int buf = local & 1;
+      const uint32_t use_par = (local >> 1) & 1;
+      bool ok = !*s_abort && mbar_wait(&tfull[buf], use_par, g.err);
+      if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; break; }  // keep the warp converged
+      tc_fence_after();
+      const int row = quad * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, r);
+        tmem_wait_ld();
+        if (!g.swap) {
+          const int p = tl.p0 + row, q = tl.q0 + c * 32;
+          if (p < tl.p_end && q < tl.q_end) store_row_chunk(g, p, q, r);
+        } else {
+          const int p = tl.p0 + row;
+          store_col_chunk(g, p, p < tl.p_end, tl.q0 + c * 32, tl.q_end, lane, tl.p0 + quad * 32, r);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[buf]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// --------------------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld
+// (elements), box = box_rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
+int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return -1;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -2;
+}
+
+// 3-D bf16 tensor map: dims (inner, mid, outer) with byte strides for mid and outer.
+int make_tmap_3d(CUtensorMap* map, const void* base, long long inner, long long mid, long long outer,
+                 long long mid_stride_bytes, long long outer_stride_bytes, int box_inner, int box_mid, int box_outer) {
+  auto enc = get_encode();
+  if (!enc) return -1;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)mid, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)mid_stride_bytes, (cuuint64_t)outer_stride_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_mid, (cuuint32_t)box_outer};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -2;
+}
+
+template <int BN>
+static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
+  using C = GemmCfg<BN>;
+  CUtensorMap tmP, tmQ;
+  if (make_tmap_2d(&tmP, d.P, d.p_rows, d.K, d.ldp, BM) != 0) {
+    set_last_error("gemm: cannot encode the tensor map of operand P");
+    return -6;
+  }
+  const long long q_total = d.n_groups > 0 ? d.q_rows_total : d.q_rows;
+  if (make_tmap_2d(&tmQ, d.Q, q_total, d.K, d.ldq, BN) != 0) {
+    set_last_error("gemm: cannot encode the tensor map of operand Q");
+    return -6;
+  }
+  GemmParams g;
+  g.p_rows = d.p_rows;
+  g.q_rows = d.q_rows;
+  g.k_blocks = d.K / BK;
+  g.p_tiles = (d.p_rows + BM - 1) / BM;
+  g.q_tiles = (d.q_rows + BN - 1) / BN;
+  // Keep the smaller operand cache-resident: sweep fastest over the tiles of the
+  // operand that is re-read, so that the larger operand streams from HBM once.
+  g.q_fast = (long long)d.q_rows <= (long long)d.p_rows ? 1 : 0;
+  g.epi = d.epi;
+  g.resid_f32 = d.resid_f32;
+  g.out_f32 = d.out_f32;
+  g.swap = d.swap;
+  g.out = d.out;
+  g.ldo = d.ldo;
+  g.resid = d.resid;
+  g.ldr = d.ldr;
+  g.n_groups = d.n_groups;
+  g.group_offsets = d.group_offsets;
+  g.err = err;
+  const size_t smem = C::smem_bytes(d.n_groups);
+  static bool attr_set[4] = {false, false, false, false};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int slot = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
+    if (!attr_set[slot]) {
+      cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+      attr_set[slot] = true;
+    }
+  }
+  int grid;
+  if (d.n_groups > 0) {
+    grid = num_sms();
+  } else {
+    const long long tiles = (long long)g.p_tiles * g.q_tiles;
+    grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  }
+  if (grid <= 0) return 0;
+  gemm_tc_kernel<BN><<<grid, 192, smem, s>>>(tmP, tmQ, g);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("gemm launch failed: %s", cudaGetErrorString(e));
+    return -6;
+  }
+  return 0;
+}
+
+int launch_gemm(const GemmDesc& d, cudaStream_t s, int* err) {
+  int bn = d.force_bn;
+  if (bn == 0) {
+    if (d.swap) bn = d.q_rows <= 64 ? 64 : (d.q_rows <= 128 ? 128 : 256);
+    else bn = 256;
+  }
+  switch (bn) {
+    case 64: return launch_bn<64>(d, s, err);
+    case 128: return launch_bn<128>(d, s, err);
+    case 256: return launch_bn<256>(d, s, err);
+    default:
+      set_last_error("gemm: unsupported tile width %d", bn);
+      return -1;
+  }
+}
+
+}  // namespace q3

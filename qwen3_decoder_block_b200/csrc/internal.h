@@ -1,0 +1,46 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace q3 {
+
+enum Epilogue : int {
+  kEpiStore = 0,   // out = acc (bf16 or f32)
+  kEpiResid = 1,   // out = resid + acc (resid bf16 or f32; out bf16 or f32); may alias
+  kEpiSwiglu = 2,  // operand rows interleaved in 16-row gate/up blocks: out = silu(g) * u, bf16
+};
+
+// D[p][q] = sum_k P[p][k] * Q[q][k]; both operands bf16, K-major (row-major [rows, K]).
+// Non-swap: P = activations [M, K], Q = weights [N, K]; out[p][q].
+// Swap:     P = weights [N, K], Q = activations [M, K]; out[q][p]  (for small M).
+// Grouped (non-swap only): P rows [off[g], off[g+1]) use Q rows g*q_rows_per_group + [0, q_rows_per_group).
+struct GemmDesc {
+  const void* P = nullptr;
+  int p_rows = 0;
+  long long ldp = 0;  // elements
+  const void* Q = nullptr;
+  int q_rows = 0;     // non-grouped: rows of Q; grouped: rows per group
+  long long ldq = 0;
+  long long q_rows_total = 0;  // rows of the Q tensor map (grouped: n_groups * q_rows)
+  int K = 0;
+  bool swap = false;
+  int epi = kEpiStore;
+  bool resid_f32 = false, out_f32 = false;
+  void* out = nullptr;
+  long long ldo = 0;
+  const void* resid = nullptr;
+  long long ldr = 0;
+  int n_groups = 0;
+  const int* group_offsets = nullptr;  // device, n_groups + 1 entries
+  int force_bn = 0;                    // 0 = automatic
+};
+
+int launch_gemm(const GemmDesc& d, cudaStream_t s, int* err);
+
+int num_sms();
+int* device_error_word();  // device pointer of the library's error word
+void set_last_error(const char* fmt, ...);
+
+}  // namespace q3

@@ -1,0 +1,175 @@
+"""Block-level GPU parity (prefill, decode, MoE, stack) against the fp64 oracle."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+import oracle.qwen3_ref as R  # noqa: E402
+from qwen3_decoder_block_b200 import synth  # noqa: E402
+from helpers import (LAYER_MAX_ABS, LAYER_REL_FROB, LOGITS_ARGMAX, LOGITS_REL_FROB, Layer, Tensor,  # noqa: E402
+                     assert_device_ok, from_gpu_bf16, kv_cache, max_abs, oracle_config, rel_frob, rope_gpu,
+                     to_gpu_bf16, workspace)
+
+
+@pytest.fixture(scope="module")
+def q3():
+    import qwen3_decoder_block_b200 as m
+    return m
+
+
+def _prefill_case(q3, cfg, B, T, starts, seed, s_extra=13):
+    s_max = max(starts) + T + s_extra
+    L = Layer(cfg, seed)
+    x = Tensor(seed, synth.TID_X, (B * T, cfg.hidden))
+    pk = Tensor(seed, 901, (B, cfg.n_kv_heads, s_max, cfg.head_dim))
+    pv = Tensor(seed, 902, (B, cfg.n_kv_heads, s_max, cfg.head_dim))
+    k, v, kv = kv_cache(cfg, B, s_max)
+    for b in range(B):
+        k[b, :, :starts[b]] = pk.gpu[b, :, :starts[b]]
+        v[b, :, :starts[b]] = pv.gpu[b, :, :starts[b]]
+    rope = rope_gpu(cfg)
+    ws = workspace(cfg, q3.OP_BLOCK_PREFILL, B, T, s_max)
+    xg = x.gpu.clone()
+    pos = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    q3.block_prefill(cfg, L.c, xg, B, T, pos, kv, rope, ws)
+    assert_device_ok()
+    oc = oracle_config(cfg)
+    refs, kref = [], []
+    for b in range(B):
+        ck = pk.f[b][:, :starts[b]].transpose(1, 0, 2)
+        cv = pv.f[b][:, :starts[b]].transpose(1, 0, 2)
+        out, kn, vn = R.block_forward(x.f[b * T:(b + 1) * T], L.oracle(), oc, starts[b] + np.arange(T), ck, cv,
+                                      np.arange(starts[b]))
+        refs.append(out)
+        kref.append((kn, vn))
+    return from_gpu_bf16(xg), np.concatenate(refs), k, v, kref
+
+
+@pytest.mark.parametrize("B,T,starts", [(1, 16, [0]), (2, 77, [0, 50]), (1, 300, [0]), (3, 5, [0, 1, 200])])
+def test_block_prefill(q3, B, T, starts):
+    cfg = q3.config_qwen3_0_6b()
+    got, ref, k, v, kref = _prefill_case(q3, cfg, B, T, starts, seed=1000)
+    assert np.isfinite(got).all()
+    assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS, (rel_frob(got, ref),
+                                                                                        max_abs(got, ref))
+    # the new keys and values landed in the cache
+    for b in range(B):
+        gk = from_gpu_bf16(k[b][:, starts[b]:starts[b] + T]).transpose(1, 0, 2)
+        assert rel_frob(gk, kref[b][0]) <= 1e-2
+
+
+def test_block_decode(q3):
+    cfg = q3.config_qwen3_0_6b()
+    lens = [0, 5, 130, 1000]
+    B = len(lens)
+    s_max = 1100
+    seed = 1002
+    L = Layer(cfg, seed)
+    x = Tensor(seed, synth.TID_X, (B, cfg.hidden))
+    pk = Tensor(seed, 903, (B, cfg.n_kv_heads, s_max, cfg.head_dim))
+    pv = Tensor(seed, 904, (B, cfg.n_kv_heads, s_max, cfg.head_dim))
+    k, v, kv = kv_cache(cfg, B, s_max)
+    for b in range(B):
+        k[b, :, :lens[b]] = pk.gpu[b, :, :lens[b]]
+        v[b, :, :lens[b]] = pv.gpu[b, :, :lens[b]]
+    rope = rope_gpu(cfg)
+    ws = workspace(cfg, q3.OP_BLOCK_DECODE, B, 1, s_max)
+    xg = x.gpu.clone()
+    cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    q3.block_decode(cfg, L.c, xg, B, cl, kv, rope, ws)
+    assert_device_ok()
+    got = from_gpu_bf16(xg)
+    oc = oracle_config(cfg)
+    for b in range(B):
+        ck = pk.f[b][:, :lens[b]].transpose(1, 0, 2)
+        cv = pv.f[b][:, :lens[b]].transpose(1, 0, 2)
+        ref, _, _ = R.block_forward(x.f[b:b + 1], L.oracle(), oc, np.array([lens[b]]), ck, cv, np.arange(lens[b]))
+        assert rel_frob(got[b], ref[0]) <= LAYER_REL_FROB and max_abs(got[b], ref[0]) <= LAYER_MAX_ABS
+    assert list(cl.cpu().numpy()) == lens  # block_decode does not advance lengths
+
+
+def _small_stack_cfg(q3, n_layers=3):
+    return q3.make_config(hidden=256, n_q_heads=4, n_kv_heads=2, intermediate=512, vocab=2048, n_layers=n_layers)
+
+
+def test_stack_prefill_then_decode(q3):
+    cfg = _small_stack_cfg(q3)
+    seed = 1003
+    B, T = 2, 40
+    s_max = T + 8
+    layers = [Layer(cfg, seed, layer=l) for l in range(cfg.n_layers)]
+    E = Tensor(seed, synth.TID_EMBED, (cfg.vocab, cfg.hidden), 0.0, synth.W_STD)
+    fn = Tensor(seed, synth.TID_FINAL_NORM, (cfg.hidden,), synth.NORM_MEAN, synth.NORM_STD)
+    ids = synth.uniform_int(seed, synth.TID_IDS, (B, T + 1), cfg.vocab)
+    caches = [kv_cache(cfg, B, s_max) for _ in range(cfg.n_layers)]
+    rope = rope_gpu(cfg)
+    ws = workspace(cfg, q3.OP_STACK_PREFILL, B, T, s_max)
+    logits = torch.empty((B * T, cfg.vocab), dtype=torch.float32, device="cuda")
+    ids_pre = torch.from_numpy(np.ascontiguousarray(ids[:, :T]).reshape(-1)).cuda()
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
+                     [c[2] for c in caches], rope, logits, False, ws)
+    assert_device_ok()
+    oc = oracle_config(cfg)
+    olayers = [l.oracle() for l in layers]
+    got = logits.cpu().double().numpy()
+    for b in range(B):
+        ref, kvs = R.stack_forward(ids[b, :T], E.f, olayers, fn.f, oc)
+        g = got[b * T:(b + 1) * T]
+        assert rel_frob(g, ref) <= LOGITS_REL_FROB
+        assert np.mean(np.argmax(g, 1) == np.argmax(ref, 1)) >= LOGITS_ARGMAX
+    # one decode step for every sequence, lengths advance on the device
+    wsd = workspace(cfg, q3.OP_STACK_DECODE, B, 1, s_max)
+    lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    ld = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    ids_dec = torch.from_numpy(np.ascontiguousarray(ids[:, T])).cuda()
+    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_dec, B, 1, q3.MODE_DECODE, lens,
+                     [c[2] for c in caches], rope, ld, False, wsd)
+    assert_device_ok()
+    assert list(lens.cpu().numpy()) == [T + 1] * B
+    gd = ld.cpu().double().numpy()
+    for b in range(B):
+        ref, _ = R.stack_forward(ids[b, :T + 1], E.f, olayers, fn.f, oc, logit_rows=[T])
+        assert rel_frob(gd[b], ref[0]) <= LOGITS_REL_FROB
+    # last_only prefill equals the last rows of the full prefill
+    ws2 = workspace(cfg, q3.OP_STACK_PREFILL, B, T, s_max)
+    caches2 = [kv_cache(cfg, B, s_max) for _ in range(cfg.n_layers)]
+    ll = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
+                     [c[2] for c in caches2], rope, ll, True, ws2)
+    assert_device_ok()
+    np.testing.assert_array_equal(ll.cpu().numpy(), logits.view(B, T, -1)[:, -1].cpu().numpy())
+
+
+def test_moe_block_small(q3):
+    cfg = q3.make_config(hidden=512, n_q_heads=8, n_kv_heads=2, n_experts=32, top_k=4, moe_intermediate=128)
+    seed = 1004
+    B, T = 1, 100
+    s_max = T
+    L = Layer(cfg, seed, moe=True, dense=False)
+    x = Tensor(seed, synth.TID_X, (B * T, cfg.hidden))
+    k, v, kv = kv_cache(cfg, B, s_max)
+    rope = rope_gpu(cfg)
+    ws = workspace(cfg, q3.OP_MOE_BLOCK, B, T, s_max)
+    xg = x.gpu.clone()
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    kk = cfg.top_k
+    idx = torch.empty((B * T, kk), dtype=torch.int32, device="cuda")
+    w = torch.empty((B * T, kk), dtype=torch.float32, device="cuda")
+    off = torch.empty(cfg.n_experts + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(B * T * kk, dtype=torch.int32, device="cuda")
+    q3.moe_block(cfg, L.c, xg, B, T, pos, kv, rope, ws, idx, w, off, perm)
+    assert_device_ok()
+    oc = oracle_config(cfg)
+    ref, _, _, (ridx, rw, rp, margin) = R.moe_block_forward(x.f, L.oracle(), oc, np.arange(T))
+    got = from_gpu_bf16(xg)
+    assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS
+    gi = idx.cpu().numpy()
+    sure = margin > 1e-3
+    np.testing.assert_array_equal(gi[sure], ridx[sure])
+    np.testing.assert_allclose(w.cpu().numpy()[sure], rw[sure], rtol=1e-3, atol=1e-4)
+    if sure.all():
+        offs, ptok, _ = R.moe_permutation(ridx, cfg.n_experts)
+        np.testing.assert_array_equal(off.cpu().numpy(), offs)
+        np.testing.assert_array_equal(perm.cpu().numpy(), ptok)
