@@ -1,0 +1,462 @@
+"""Benchmark of libqwen3blk on the Qwen3-0.6B workloads (one process per GPU).
+
+Headline (one JSON line on rank 0):
+  value  = 28-layer Qwen3-0.6B stack prefill, B=4 x T=2048 (8192 tokens, all-position fp32
+           logits through the tied LM head), tokens/s summed over all ranks (replicas).
+  decode = 28-layer decode, B=64 sequences holding 4096 cached tokens, 128 successive steps
+           (positions 4096..4223), tokens/s (rank 0's GPU).
+Synthetic seeded inputs (random weights of the Qwen3-0.6B shapes, random token ids).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-decode]
+
+--impl reference times the fp64 CPU oracle (the only reference this workload has) on a
+bounded sample of the same prefill workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Qwen3-0.6B prefill & decode tokens/s on 1 B200; % of BF16/HBM roofline"
+PREFILL_B, PREFILL_T = 4, 2048
+DECODE_B, DECODE_CTX, DECODE_STEPS = 64, 4096, 128
+SEED_PREFILL, SEED_DECODE = 1001, 1002
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- model set-up
+def build_model(q3, cfg, seed, torch):
+    """Random Qwen3-0.6B weights drawn on the device straight into the packed layouts
+    (identical values to drawing the pages' layouts and calling the pack helpers)."""
+    from qwen3_decoder_block_b200 import synth
+    H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+
+    def fill(t, tid, mean, std, n0=1, n1=1, n2=None, s0=0, s1=0, offset=0):
+        n2 = t.numel() if n2 is None else n2
+        synth.normal_bf16_device(t.data_ptr() + 2 * offset, n0, n1, n2, s0, s1, seed, tid, mean, std)
+
+    layers, keep = [], []
+    for l in range(cfg.n_layers):
+        tid = lambda w: synth.layer_tid(l, w)
+        in_norm = torch.empty(H, **bf); fill(in_norm, tid(synth.L_IN_NORM), synth.NORM_MEAN, synth.NORM_STD)
+        post_norm = torch.empty(H, **bf); fill(post_norm, tid(synth.L_POST_NORM), synth.NORM_MEAN, synth.NORM_STD)
+        qn = torch.empty(D, **bf); fill(qn, tid(synth.L_Q_NORM), synth.NORM_MEAN, synth.NORM_STD)
+        kn = torch.empty(D, **bf); fill(kn, tid(synth.L_K_NORM), synth.NORM_MEAN, synth.NORM_STD)
+        wqkv = torch.empty(((hq + 2 * hkv) * D, H), **bf)
+        fill(wqkv, tid(synth.L_WQ), 0.0, synth.W_STD, n2=hq * D * H)
+        fill(wqkv, tid(synth.L_WK), 0.0, synth.W_STD, n2=hkv * D * H, offset=hq * D * H)
+        fill(wqkv, tid(synth.L_WV), 0.0, synth.W_STD, n2=hkv * D * H, offset=(hq + hkv) * D * H)
+        wo = torch.empty((H, hq * D), **bf); fill(wo, tid(synth.L_WO), 0.0, synth.W_STD)
+        wgu = torch.empty((2 * I, H), **bf)
+        fill(wgu, tid(synth.L_WGATE), 0.0, synth.W_STD, n0=I // 16, n1=16, n2=H, s0=32 * H, s1=H)
+        fill(wgu, tid(synth.L_WUP), 0.0, synth.W_STD, n0=I // 16, n1=16, n2=H, s0=32 * H, s1=H, offset=16 * H)
+        wd = torch.empty((H, I), **bf); fill(wd, tid(synth.L_WDOWN), 0.0, synth.W_STD)
+        keep += [in_norm, post_norm, qn, kn, wqkv, wo, wgu, wd]
+        layers.append(q3.layer_weights(in_norm=in_norm, w_qkv=wqkv, q_norm=qn, k_norm=kn, w_o=wo,
+                                       post_norm=post_norm, w_gate_up=wgu, w_down=wd))
+    embed = torch.empty((cfg.vocab, H), **bf); fill(embed, synth.TID_EMBED, 0.0, synth.W_STD)
+    fnorm = torch.empty(H, **bf); fill(fnorm, synth.TID_FINAL_NORM, synth.NORM_MEAN, synth.NORM_STD)
+    keep += [embed, fnorm]
+    return layers, embed, fnorm, keep
+
+
+def gemm_flops_per_token(cfg):
+    H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+    per_layer = 2 * (H * (hq + 2 * hkv) * D + hq * D * H + H * 2 * I + I * H)
+    return cfg.n_layers * per_layer, 2 * H * cfg.vocab
+
+
+def attention_prefill_flops(cfg, B, T):
+    pairs = B * T * (T + 1) // 2
+    return cfg.n_layers * 4 * cfg.head_dim * cfg.n_q_heads * pairs
+
+
+def summarize_profile(records, steps):
+    by = {}
+    for name, ms in records:
+        n, t = by.get(name, (0, 0.0))
+        by[name] = (n + 1, t + ms)
+    total = sum(t for _, t in by.values())
+    return {k: {"launches_per_step": n / steps, "ms_per_step": t / steps, "share": t / total if total else 0.0}
+            for k, (n, t) in sorted(by.items(), key=lambda kv: -kv[1][1])}, total / steps
+
+
+# --------------------------------------------------------------------------- workloads
+def run_prefill(q3, torch, args, rank, world, dist, peaks):
+    cfg = q3.config_qwen3_0_6b()
+    B, T = PREFILL_B, PREFILL_T
+    M = B * T
+    from qwen3_decoder_block_b200 import synth
+    layers, embed, fnorm, keep = build_model(q3, cfg, SEED_PREFILL, torch)
+    s_max = T
+    caches = []
+    for _ in range(cfg.n_layers):
+        k = torch.empty((B, cfg.n_kv_heads, s_max, cfg.head_dim), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        caches.append((k, v))
+    kvs = [q3.kv_layer(k, v, s_max) for k, v in caches]
+    rope = torch.empty(q3.rope_table_bytes(cfg) // 4, dtype=torch.float32, device="cuda")
+    q3.rope_table(cfg, rope)
+    ids = torch.empty(M, dtype=torch.int32, device="cuda")
+    synth.uniform_int_device(ids.data_ptr(), M, SEED_PREFILL, synth.TID_IDS, cfg.vocab)
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ws = torch.empty(q3.workspace_size(cfg, q3.OP_STACK_PREFILL, B, T, s_max), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((M, cfg.vocab), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        q3.stack_forward(cfg, embed, layers, fnorm, ids, B, T, q3.MODE_PREFILL, pos, kvs, rope, logits, False, ws,
+                         stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert q3.check_device_error() == 0
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    if rank == 0:
+        clocks.start()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    q3.profile_begin(args.steps * 400 + 16)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    records = q3.profile_end(stream)
+    ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    clk = clocks.stop() if rank == 0 else None
+    assert q3.check_device_error() == 0
+
+    # end to end through the public call with host buffers: ids H2D, logits of each
+    # sequence's last position D2H, inside the timed region
+    ids_host = ids.cpu().pin_memory()
+    out_host = torch.empty((B, cfg.vocab), dtype=torch.float32).pin_memory()
+    last_rows = logits.view(B, T, cfg.vocab)[:, T - 1]
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        ids.copy_(ids_host, non_blocking=True)
+        step()
+        out_host.copy_(last_rows, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    kernels, prof_ms = summarize_profile(records, args.steps)
+    g_tok, lm_tok = gemm_flops_per_token(cfg)
+    gemm_flops = M * (g_tok + lm_tok)
+    gemm_names = ("gemm_qkv", "gemm_o", "gemm_gate_up", "gemm_down", "lm_head")
+    gemm_ms = sum(kernels[n]["ms_per_step"] for n in gemm_names if n in kernels)
+    gemm_launches = sum(kernels[n]["launches_per_step"] for n in gemm_names if n in kernels)
+    attn_flops = attention_prefill_flops(cfg, B, T)
+    attn = kernels.get("attn_prefill", {"ms_per_step": float("nan"), "launches_per_step": 0})
+    peak = peaks["bf16_tflops_sustained"]
+    achieved = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    attn_tf = attn_flops / (attn["ms_per_step"] * 1e-3) / 1e12
+    per_step_ms = ms / args.steps
+    n_launch = len(records) / args.steps
+    return {
+        "value": world * M * args.steps / (ms * 1e-3),
+        "ms_per_step": per_step_ms,
+        "e2e": {"value": world * M * args.steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": M * 4, "d2h_bytes_per_step": B * cfg.vocab * 4},
+        "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (all projections + LM head)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} bf16 sustained", "traffic": None,
+                     "flops_per_launch": gemm_flops / gemm_launches,
+                     "avg_launch_ms": gemm_ms / gemm_launches},
+        "attention": {"achieved_tflops": attn_tf, "frac": attn_tf / peak, "ms_per_step": attn["ms_per_step"],
+                      "flops_per_step": attn_flops},
+        "kernels": {k: {kk: round(vv, 5) for kk, vv in v.items()} for k, v in kernels.items()},
+        "gpu_launches": int(round(n_launch * args.steps)),
+        "profiled_ms_per_step": prof_ms,
+        "clocks": clk,
+    }
+
+
+def run_decode(q3, torch, args, peaks):
+    cfg = q3.config_qwen3_0_6b()
+    B, L0, S = DECODE_B, DECODE_CTX, DECODE_STEPS
+    from qwen3_decoder_block_b200 import synth
+    layers, embed, fnorm, keep = build_model(q3, cfg, SEED_DECODE, torch)
+    s_max = L0 + S
+    caches = []
+    for l in range(cfg.n_layers):
+        k = torch.empty((B, cfg.n_kv_heads, s_max, cfg.head_dim), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        for t, which in ((k, synth.L_CACHE_K), (v, synth.L_CACHE_V)):
+            synth.normal_bf16_device(t.data_ptr(), B * cfg.n_kv_heads, L0, cfg.head_dim, s_max * cfg.head_dim,
+                                     cfg.head_dim, SEED_DECODE, synth.layer_tid(l, which), 0.0, 1.0)
+        caches.append((k, v))
+    kvs = [q3.kv_layer(k, v, s_max) for k, v in caches]
+    rope = torch.empty(q3.rope_table_bytes(cfg) // 4, dtype=torch.float32, device="cuda")
+    q3.rope_table(cfg, rope)
+    all_ids = torch.empty((S, B), dtype=torch.int32, device="cuda")
+    synth.uniform_int_device(all_ids.data_ptr(), S * B, SEED_DECODE, synth.TID_IDS_STEP, cfg.vocab)
+    ids = torch.empty(B, dtype=torch.int32, device="cuda")
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    ws = torch.empty(q3.workspace_size(cfg, q3.OP_STACK_DECODE, B, 1, s_max), dtype=torch.uint8, device="cuda")
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def step():
+        q3.stack_forward(cfg, embed, layers, fnorm, ids, B, 1, q3.MODE_DECODE, lens, kvs, rope, logits, False, ws,
+                         stream)
+
+    with torch.cuda.stream(stream):
+        ids.copy_(all_ids[0])
+        step()  # eager step: one-time set-up outside capture
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="thread_local"):
+            step()
+        for s in range(max(args.warmup, 3)):
+            ids.copy_(all_ids[s % S])
+            graph.replay()
+        lens.fill_(L0)  # undo the warm-up steps
+    torch.cuda.synchronize()
+    assert q3.check_device_error(stream) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(S):
+            ids.copy_(all_ids[s])
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    assert q3.check_device_error(stream) == 0
+    assert int(lens[0].item()) == L0 + S
+    # per-kernel attribution: one profiled eager window (not part of the timed value)
+    lens.fill_(L0)
+    torch.cuda.synchronize()
+    q3.profile_begin(8 * 300)
+    with torch.cuda.stream(stream):
+        for s in range(8):
+            ids.copy_(all_ids[s])
+            step()
+    records = q3.profile_end(stream)
+    kernels, _ = summarize_profile(records, 8)
+    # algorithmic bytes of the decode attention: K and V of every visible position (8 prof steps)
+    kv_bytes = sum(cfg.n_layers * B * (L0 + s + 1) * cfg.n_kv_heads * cfg.head_dim * 2 * 2 for s in range(8)) / 8
+    attn_ms = kernels["attn_decode"]["ms_per_step"]
+    achieved = kv_bytes / (attn_ms * 1e-3) / 1e9
+    step_bytes = sum(cfg.n_layers * B * (L0 + s + 1) * cfg.n_kv_heads * cfg.head_dim * 4 for s in range(S)) / S
+    w_bytes = 2 * (cfg.n_layers * (cfg.hidden * (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim +
+                                   cfg.n_q_heads * cfg.head_dim * cfg.hidden + 3 * cfg.hidden * cfg.intermediate) +
+                   cfg.vocab * cfg.hidden) + B * cfg.vocab * 4
+    step_ms = ms / S
+    hbm = peaks["hbm_gbs"]
+    del graph
+    return {
+        "value": B * S / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+        "workload": f"Qwen3-0.6B 28-layer decode, B{B}, {L0} cached tokens, {S} steps (positions {L0}..{L0 + S - 1}), "
+                    "CUDA-graph replay per step",
+        "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes + w_bytes,
+                          "achieved_gbs": (step_bytes + w_bytes) / (step_ms * 1e-3) / 1e9,
+                          "frac": (step_bytes + w_bytes) / (step_ms * 1e-3) / 1e9 / hbm},
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (split-KV + merge)", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} hbm copy",
+                     "traffic": None},
+        "kernels": {k: {kk: round(vv, 5) for kk, vv in v.items()} for k, v in kernels.items()},
+        "gpu_launches_per_step": len(records) / 8,
+    }
+
+
+# --------------------------------------------------------------------------- oracle timing
+def oracle_sample(T_s: int, seed: int = SEED_PREFILL):
+    """Times the fp64 oracle on one sequence of T_s tokens of the prefill workload
+    (28 layers + final norm + tied LM head on all T_s positions)."""
+    import numpy as np
+    import oracle.qwen3_ref as R
+    from qwen3_decoder_block_b200 import synth
+    cfg = R.QWEN3_0_6B
+    H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+    gen = lambda tid, shape, m=0.0, s=synth.W_STD: R.bf16_to_f64(synth.normal_bf16_fast(seed, tid, shape, m, s))
+    layers = []
+    for l in range(cfg.n_layers):
+        t = lambda w: synth.layer_tid(l, w)
+        layers.append(R.LayerWeights(
+            in_norm=gen(t(synth.L_IN_NORM), (H,), synth.NORM_MEAN, synth.NORM_STD),
+            wq=gen(t(synth.L_WQ), (hq * D, H)), wk=gen(t(synth.L_WK), (hkv * D, H)), wv=gen(t(synth.L_WV), (hkv * D, H)),
+            q_norm=gen(t(synth.L_Q_NORM), (D,), synth.NORM_MEAN, synth.NORM_STD),
+            k_norm=gen(t(synth.L_K_NORM), (D,), synth.NORM_MEAN, synth.NORM_STD),
+            wo=gen(t(synth.L_WO), (H, hq * D)),
+            post_norm=gen(t(synth.L_POST_NORM), (H,), synth.NORM_MEAN, synth.NORM_STD),
+            w_gate=gen(t(synth.L_WGATE), (I, H)), w_up=gen(t(synth.L_WUP), (I, H)), w_down=gen(t(synth.L_WDOWN), (H, I))))
+    embed = gen(synth.TID_EMBED, (cfg.vocab, H))
+    fnorm = gen(synth.TID_FINAL_NORM, (H,), synth.NORM_MEAN, synth.NORM_STD)
+    ids = synth.uniform_int(seed, synth.TID_IDS, (T_s,), cfg.vocab)
+    t0 = time.perf_counter()
+    R.stack_forward(ids, embed, layers, fnorm, cfg)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(T_s: int = 256):
+    dt = oracle_sample(T_s)
+    return {"value": T_s / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one sequence of {T_s} tokens (prefill workload's first {T_s} ids) through the 28-layer "
+                      f"stack + tied LM head in fp64 numpy, {dt:.1f} s"}
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-tokens", type=int, default=256)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    peaks = load_peaks()
+    config = {"workload": f"Qwen3-0.6B 28-layer stack prefill, B{PREFILL_B} x T{PREFILL_T} "
+                          "(positions 0..2047), final RMSNorm + tied LM head, fp32 logits for all positions",
+              "global_batch": PREFILL_B * world, "seq_len": PREFILL_T,
+              "parallelism": f"replicas x{world} (independent sequences, no collective)",
+              "l2": "inputs larger than L2 (1.2 GB of weights and 5 GB of logits per step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps = max(1, min(args.steps, 3))
+        times = [oracle_sample(args.oracle_tokens) for _ in range(max(1, min(args.warmup, 1)) + steps)][-steps:]
+        v = args.oracle_tokens / statistics.mean(times)
+        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+                "warmup": 1, "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "impl": "reference",
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"one sequence of {args.oracle_tokens} tokens per step"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+        dist = dist_mod
+    else:
+        torch.cuda.set_device(local)
+    import qwen3_decoder_block_b200 as q3
+
+    pre = run_prefill(q3, torch, args, rank, world, dist, peaks)
+    dec = None
+    if not args.no_decode and rank == 0:
+        torch.cuda.empty_cache()
+        dec = run_decode(q3, torch, args, peaks)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.oracle_tokens)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {"metric": METRIC, "value": pre["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random weights and token ids)",
+            "config": config, "e2e": pre["e2e"], "roofline": pre["roofline"], "cpu_baseline": cpu,
+            "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "attention": pre["attention"],
+            "kernels": pre["kernels"], "decode": dec}
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -142,6 +142,16 @@ int qwen3_pack_moe_gate_up(int E, int Im, int H, const qwen3_bf16* gate_up_proj,
  * (QWEN3_OK, QWEN3_ECAPACITY, QWEN3_EINVAL or QWEN3_ETIMEOUT). */
 int qwen3_check_device_error(void* stream);
 
+/* Per-launch timing of the block and stack calls. After qwen3_profile_begin(n), each
+ * kernel launch (up to n) is bracketed by two CUDA events on the call's stream;
+ * qwen3_profile_end(stream) stops recording, synchronises the stream and returns the
+ * number of records; qwen3_profile_record(i, ...) gives the i-th launch's role name
+ * (e.g. "gemm_qkv", "attn_prefill", "lm_head") and its device time in ms.
+ * The recorder is process-global: profile one thread's calls at a time. */
+int qwen3_profile_begin(int max_records);
+int qwen3_profile_end(void* stream);
+int qwen3_profile_record(int i, char* name, int name_cap, float* ms);
+
 /* -------------------------------------------------------------- block calls */
 
 /* Dense decoder block, prefill ([P-Mini] section TransformerBlock: pre-norm, GQA with

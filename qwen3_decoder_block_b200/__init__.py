@@ -63,6 +63,9 @@ _SIGS = {
                          _vp, _sz, _vp], _i),
     "qwen3_stack_forward": ([_P(Config), _vp, _P(LayerWeights), _vp, _vp, _i, _i, _i, _vp, _P(KVLayer), _vp, _vp,
                              _i, _vp, _sz, _vp], _i),
+    "qwen3_profile_begin": ([_i], _i),
+    "qwen3_profile_end": ([_vp], _i),
+    "qwen3_profile_record": ([_i, ctypes.c_char_p, _i, _P(_f)], _i),
     "qwen3_op_rmsnorm": ([_vp, _i, _ll, _vp, _vp, _ll, _i, _i, _f, _vp], _i),
     "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _vp], _i),
     "qwen3_op_qk_norm_rope": ([_P(Config), _vp, _ll, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
@@ -139,6 +142,23 @@ def rope_table(cfg: Config, rope, stream=None) -> None:
 
 def check_device_error(stream=None) -> int:
     return lib.qwen3_check_device_error(_stream(stream))
+
+
+def profile_begin(max_records: int = 4096) -> None:
+    _check(lib.qwen3_profile_begin(max_records), "profile_begin")
+
+
+def profile_end(stream=None) -> list[tuple[str, float]]:
+    n = lib.qwen3_profile_end(_stream(stream))
+    if n < 0:
+        _check(n, "profile_end")
+    out = []
+    buf = ctypes.create_string_buffer(64)
+    ms = ctypes.c_float()
+    for i in range(n):
+        _check(lib.qwen3_profile_record(i, buf, 64, ctypes.byref(ms)), "profile_record")
+        out.append((buf.value.decode(), ms.value))
+    return out
 
 
 # ------------------------------------------------------------------------- packing

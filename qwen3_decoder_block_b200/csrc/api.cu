@@ -89,6 +89,31 @@ int* device_error_word() {
   return g_err_ptr[d];
 }
 
+// ----------------------------------------------------------------------------- profiling
+// Optional per-launch timing: while enabled, every kernel launch made by the
+// block/stack calls is bracketed by two CUDA events on the caller's stream.
+struct ProfRec {
+  const char* name;
+  cudaEvent_t a, b;
+};
+static std::vector<ProfRec> g_prof;
+static size_t g_prof_used = 0;
+static bool g_prof_on = false;
+
+struct ProfScope {
+  ProfRec* r = nullptr;
+  cudaStream_t s;
+  ProfScope(const char* name, cudaStream_t st) : s(st) {
+    if (!g_prof_on || g_prof_used >= g_prof.size()) return;
+    r = &g_prof[g_prof_used++];
+    r->name = name;
+    cudaEventRecord(r->a, s);
+  }
+  ~ProfScope() {
+    if (r) cudaEventRecord(r->b, s);
+  }
+};
+
 // ----------------------------------------------------------------------------- validation
 #define Q3_CHECK(cond, code, ...)  \
   do {                             \
@@ -234,7 +259,11 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   const int H = c.hidden, D = c.head_dim;
   const long long M = (long long)B * T;
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * D;
-  int rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  int rc;
+  {
+    ProfScope ps("rmsnorm", k.s);
+    rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  }
   if (rc) return rc;
   GemmDesc g;
   g.swap = swap_for(M);
@@ -245,16 +274,26 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   g.epi = kEpiStore;
   g.out = b.qkv;
   g.ldo = nqkv;
-  if ((rc = launch_gemm(g, k.s, k.err))) return rc;
-  if ((rc = launch_qk_norm_rope(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, w.q_norm, w.k_norm, rope, kv.k,
-                                kv.v, kv.s_max, c.max_pos, c.rms_eps, k.err, k.s)))
-    return rc;
-  if (decode)
-    rc = launch_attention_decode(b.qkv, nqkv, B, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part, b.o,
-                                 (long long)c.n_q_heads * D, k.err, k.s);
-  else
-    rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
-                                  (long long)c.n_q_heads * D, k.err, k.s);
+  {
+    ProfScope ps("gemm_qkv", k.s);
+    rc = launch_gemm(g, k.s, k.err);
+  }
+  if (rc) return rc;
+  {
+    ProfScope ps("qk_norm_rope", k.s);
+    rc = launch_qk_norm_rope(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, w.q_norm, w.k_norm, rope, kv.k,
+                             kv.v, kv.s_max, c.max_pos, c.rms_eps, k.err, k.s);
+  }
+  if (rc) return rc;
+  {
+    ProfScope ps(decode ? "attn_decode" : "attn_prefill", k.s);
+    if (decode)
+      rc = launch_attention_decode(b.qkv, nqkv, B, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part,
+                                   b.o, (long long)c.n_q_heads * D, k.err, k.s);
+    else
+      rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
+                                    (long long)c.n_q_heads * D, k.err, k.s);
+  }
   if (rc) return rc;
   GemmDesc o;
   o.swap = swap_for(M);
@@ -268,6 +307,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   o.out = b.x1;
   o.out_f32 = true;
   o.ldo = H;
+  ProfScope ps("gemm_o", k.s);
   return launch_gemm(o, k.s, k.err);
 }
 
@@ -275,7 +315,11 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
 static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, I = c.intermediate;
-  int rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  int rc;
+  {
+    ProfScope ps("rmsnorm", k.s);
+    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  }
   if (rc) return rc;
   GemmDesc g;
   g.swap = swap_for(M);
@@ -285,7 +329,11 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   g.epi = kEpiSwiglu;
   g.out = b.act;
   g.ldo = I;
-  if ((rc = launch_gemm(g, k.s, k.err))) return rc;
+  {
+    ProfScope ps("gemm_gate_up", k.s);
+    rc = launch_gemm(g, k.s, k.err);
+  }
+  if (rc) return rc;
   GemmDesc d;
   d.swap = swap_for(M);
   d.K = I;
@@ -298,6 +346,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   d.out = out;
   d.out_f32 = out_f32;
   d.ldo = H;
+  ProfScope ps("gemm_down", k.s);
   return launch_gemm(d, k.s, k.err);
 }
 
@@ -305,7 +354,11 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
 static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, E = c.n_experts, kk = c.top_k, Im = c.moe_intermediate;
-  int rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  int rc;
+  {
+    ProfScope ps("rmsnorm", k.s);
+    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+  }
   if (rc) return rc;
   // router logits in fp32 (no bf16 rounding before the softmax)
   GemmDesc r;
@@ -317,11 +370,22 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   r.out = b.logits;
   r.out_f32 = true;
   r.ldo = E;
-  if ((rc = launch_gemm(r, k.s, k.err))) return rc;
-  if ((rc = launch_moe_route(b.logits, (int)M, E, kk, c.norm_topk_prob, b.idx, b.w, b.counts, k.s))) return rc;
-  if ((rc = launch_moe_permute(b.idx, (int)M, kk, E, b.counts, b.offsets, b.perm_token, b.perm_slot, b.inv_pos, b.h,
-                               H, b.a_perm, k.s)))
-    return rc;
+  {
+    ProfScope ps("gemm_router", k.s);
+    rc = launch_gemm(r, k.s, k.err);
+  }
+  if (rc) return rc;
+  {
+    ProfScope ps("moe_route", k.s);
+    rc = launch_moe_route(b.logits, (int)M, E, kk, c.norm_topk_prob, b.idx, b.w, b.counts, k.s);
+  }
+  if (rc) return rc;
+  {
+    ProfScope ps("moe_permute", k.s);
+    rc = launch_moe_permute(b.idx, (int)M, kk, E, b.counts, b.offsets, b.perm_token, b.perm_slot, b.inv_pos, b.h, H,
+                            b.a_perm, k.s);
+  }
+  if (rc) return rc;
   const long long rows = M * kk;
   GemmDesc gu;
   gu.P = b.a_perm; gu.p_rows = (int)rows; gu.ldp = H;
@@ -330,7 +394,11 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   gu.epi = kEpiSwiglu;
   gu.out = b.act_perm; gu.ldo = Im;
   gu.n_groups = E; gu.group_offsets = b.offsets;
-  if ((rc = launch_gemm(gu, k.s, k.err))) return rc;
+  {
+    ProfScope ps("moe_gemm_gate_up", k.s);
+    rc = launch_gemm(gu, k.s, k.err);
+  }
+  if (rc) return rc;
   GemmDesc dn;
   dn.P = b.act_perm; dn.p_rows = (int)rows; dn.ldp = Im;
   dn.Q = w.moe_down; dn.q_rows = H; dn.ldq = Im; dn.q_rows_total = (long long)E * H;
@@ -338,7 +406,12 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   dn.epi = kEpiStore;
   dn.out = b.y; dn.ldo = H;
   dn.n_groups = E; dn.group_offsets = b.offsets;
-  if ((rc = launch_gemm(dn, k.s, k.err))) return rc;
+  {
+    ProfScope ps("moe_gemm_down", k.s);
+    rc = launch_gemm(dn, k.s, k.err);
+  }
+  if (rc) return rc;
+  ProfScope ps("moe_combine", k.s);
   return launch_moe_combine(b.x1, b.y, b.w, b.inv_pos, (int)M, kk, H, out, out_f32, k.s);
 }
 
@@ -626,7 +699,11 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   Ctx k{*c, s, device_error_word()};
   const int H = c->hidden;
   const long long M = (long long)B * T;
-  if ((rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s))) return finish(rc);
+  {
+    ProfScope ps("embed", s);
+    rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s);
+  }
+  if (rc) return finish(rc);
   for (int l = 0; l < c->n_layers; ++l) {
     if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b))) return finish(rc);
     if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b))) return finish(rc);
@@ -635,7 +712,11 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   const int rows = last_only ? B : (int)M;
   const float* xf = last_only ? b.xs + (long long)(T - 1) * H : b.xs;
   const long long ldx = last_only ? (long long)T * H : H;
-  if ((rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s))) return finish(rc);
+  {
+    ProfScope ps("rmsnorm", s);
+    rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s);
+  }
+  if (rc) return finish(rc);
   GemmDesc g;
   g.swap = swap_for(rows);
   g.K = H;
@@ -645,9 +726,55 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   g.out = logits;
   g.out_f32 = true;
   g.ldo = c->vocab;
-  if ((rc = launch_gemm(g, s, k.err))) return finish(rc);
-  if (decode) rc = launch_advance_lengths(pos_or_len, B, s);
+  {
+    ProfScope ps("lm_head", s);
+    rc = launch_gemm(g, s, k.err);
+  }
+  if (rc) return finish(rc);
+  if (decode) {
+    ProfScope ps("advance_lengths", s);
+    rc = launch_advance_lengths(pos_or_len, B, s);
+  }
   return finish(rc);
+}
+
+
+int qwen3_profile_begin(int max_records) {
+  g_last_error.clear();
+  Q3_CHECK(max_records > 0, QWEN3_EINVAL, "profile_begin: max_records must be positive");
+  if ((int)g_prof.size() < max_records) {
+    const size_t old = g_prof.size();
+    g_prof.resize(max_records);
+    for (size_t i = old; i < g_prof.size(); ++i) {
+      if (cudaEventCreate(&g_prof[i].a) != cudaSuccess || cudaEventCreate(&g_prof[i].b) != cudaSuccess) {
+        g_prof.resize(i);
+        set_last_error("profile_begin: cudaEventCreate failed");
+        return QWEN3_ECUDA;
+      }
+    }
+  }
+  g_prof_used = 0;
+  g_prof_on = true;
+  return 0;
+}
+
+int qwen3_profile_end(void* stream) {
+  g_prof_on = false;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    set_last_error("profile_end: stream error");
+    return QWEN3_ECUDA;
+  }
+  return (int)g_prof_used;
+}
+
+int qwen3_profile_record(int i, char* name, int name_cap, float* ms) {
+  Q3_CHECK(i >= 0 && (size_t)i < g_prof_used, QWEN3_EINVAL, "profile_record: index %d out of range", i);
+  if (name && name_cap > 0) {
+    strncpy(name, g_prof[i].name, name_cap - 1);
+    name[name_cap - 1] = 0;
+  }
+  if (ms && cudaEventElapsedTime(ms, g_prof[i].a, g_prof[i].b) != cudaSuccess) return QWEN3_ECUDA;
+  return 0;
 }
 
 // ----------------------------------------------------------------------------- ops

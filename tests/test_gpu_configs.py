@@ -1,0 +1,258 @@
+"""Parity at the five workloads' full sizes, in the launch configuration the
+benchmark times. Where the oracle cannot afford the whole output it computes a
+sample one by one (a whole sequence, a few decode steps, a set of query rows).
+
+If PARITY_REPORT_DIR is set, each test writes its error figures there as JSON.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+import oracle.qwen3_ref as R  # noqa: E402
+from qwen3_decoder_block_b200 import synth  # noqa: E402
+from helpers import (LAYER_MAX_ABS, LAYER_REL_FROB, LOGITS_ARGMAX, LOGITS_REL_FROB, assert_device_ok,  # noqa: E402
+                     from_gpu_bf16, max_abs, oracle_config, rel_frob, rope_gpu, to_gpu_bf16, workspace)
+
+
+@pytest.fixture(scope="module")
+def q3():
+    import qwen3_decoder_block_b200 as m
+    return m
+
+
+def report(name, **kw):
+    d = os.environ.get("PARITY_REPORT_DIR")
+    if d:
+        os.makedirs(d, exist_ok=True)
+        with open(os.path.join(d, f"parity_{name}.json"), "w") as f:
+            json.dump({k: (float(v) if isinstance(v, (np.floating, float)) else v) for k, v in kw.items()}, f,
+                      indent=1)
+    print(name, kw)
+
+
+class HostLayer:
+    """Layer weights drawn with the host generator (pages' layouts), uploaded and packed."""
+
+    def __init__(self, q3, cfg, seed, l, moe=False):
+        H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+        g = lambda w, shape, m=0.0, s=synth.W_STD: synth.normal_bf16_fast(seed, synth.layer_tid(l, w), shape, m, s)
+        nm, ns = synth.NORM_MEAN, synth.NORM_STD
+        self.b = dict(in_norm=g(synth.L_IN_NORM, (H,), nm, ns), wq=g(synth.L_WQ, (hq * D, H)),
+                      wk=g(synth.L_WK, (hkv * D, H)), wv=g(synth.L_WV, (hkv * D, H)),
+                      q_norm=g(synth.L_Q_NORM, (D,), nm, ns), k_norm=g(synth.L_K_NORM, (D,), nm, ns),
+                      wo=g(synth.L_WO, (H, hq * D)), post_norm=g(synth.L_POST_NORM, (H,), nm, ns))
+        if moe:
+            E, Im = cfg.n_experts, cfg.moe_intermediate
+            self.b.update(router=g(synth.L_ROUTER, (E, H)), gate_up=g(synth.L_MOE_GATE_UP, (E, 2 * Im, H)),
+                          down=g(synth.L_MOE_DOWN, (E, H, Im)))
+        else:
+            self.b.update(w_gate=g(synth.L_WGATE, (I, H)), w_up=g(synth.L_WUP, (I, H)), w_down=g(synth.L_WDOWN, (H, I)))
+        gpu = {k: to_gpu_bf16(v) for k, v in self.b.items()}
+        w_qkv = torch.empty(((hq + 2 * hkv) * D, H), dtype=torch.bfloat16, device="cuda")
+        q3.pack_qkv(cfg, gpu["wq"], gpu["wk"], gpu["wv"], w_qkv)
+        kw = dict(in_norm=gpu["in_norm"], w_qkv=w_qkv, q_norm=gpu["q_norm"], k_norm=gpu["k_norm"], w_o=gpu["wo"],
+                  post_norm=gpu["post_norm"])
+        if moe:
+            E, Im = cfg.n_experts, cfg.moe_intermediate
+            mgu = torch.empty((E, 2 * Im, H), dtype=torch.bfloat16, device="cuda")
+            q3.pack_moe_gate_up(E, Im, H, gpu["gate_up"], mgu)
+            kw.update(router=gpu["router"], moe_gate_up=mgu, moe_down=gpu["down"])
+            self.keep = [mgu]
+        else:
+            wgu = torch.empty((2 * I, H), dtype=torch.bfloat16, device="cuda")
+            q3.pack_gate_up(I, H, gpu["w_gate"], gpu["w_up"], wgu)
+            kw.update(w_gate_up=wgu, w_down=gpu["w_down"])
+            self.keep = [wgu]
+        torch.cuda.synchronize()
+        self.keep += [w_qkv] + list(gpu.values())
+        self.c = q3.layer_weights(**kw)
+
+    def oracle(self):
+        f = {k: R.bf16_to_f64(v) for k, v in self.b.items()}
+        return R.LayerWeights(**f)
+
+
+def test_config0_single_layer_prefill(q3):
+    """1 layer, B1 T16, positions 0..15 (seed 1000)."""
+    cfg = q3.config_qwen3_0_6b()
+    seed, T = 1000, 16
+    L = HostLayer(q3, cfg, seed, 0)
+    x = synth.normal_bf16(seed, synth.TID_X, (T, cfg.hidden))
+    k = torch.empty((1, cfg.n_kv_heads, T, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    kv = q3.kv_layer(k, v, T)
+    xg = to_gpu_bf16(x)
+    q3.block_prefill(cfg, L.c, xg, 1, T, torch.zeros(1, dtype=torch.int32, device="cuda"), kv, rope_gpu(cfg),
+                     workspace(cfg, q3.OP_BLOCK_PREFILL, 1, T, T))
+    assert_device_ok()
+    ref, _, _ = R.block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg), np.arange(T))
+    got = from_gpu_bf16(xg)
+    report("c0", rel_frob=rel_frob(got, ref), max_abs=max_abs(got, ref))
+    assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS
+
+
+def _stack_weights(q3, cfg, seed):
+    layers = [HostLayer(q3, cfg, seed, l) for l in range(cfg.n_layers)]
+    E = synth.normal_bf16_fast(seed, synth.TID_EMBED, (cfg.vocab, cfg.hidden), 0.0, synth.W_STD)
+    fn = synth.normal_bf16_fast(seed, synth.TID_FINAL_NORM, (cfg.hidden,), synth.NORM_MEAN, synth.NORM_STD)
+    return layers, E, fn
+
+
+def test_config1_stack_prefill(q3):
+    """28 layers + final norm + tied LM head, B4 x T2048 on the GPU; the oracle recomputes
+    sequence 0 in full (2048 rows of 151936 logits)."""
+    cfg = q3.config_qwen3_0_6b()
+    seed, B, T = 1001, 4, 2048
+    layers, E, fn = _stack_weights(q3, cfg, seed)
+    ids = synth.uniform_int(seed, synth.TID_IDS, (B * T,), cfg.vocab)
+    Eg, fng = to_gpu_bf16(E), to_gpu_bf16(fn)
+    caches = [(torch.empty((B, 8, T, 128), dtype=torch.bfloat16, device="cuda"),
+               torch.empty((B, 8, T, 128), dtype=torch.bfloat16, device="cuda")) for _ in range(cfg.n_layers)]
+    kvs = [q3.kv_layer(k, v, T) for k, v in caches]
+    logits = torch.empty((B * T, cfg.vocab), dtype=torch.float32, device="cuda")
+    q3.stack_forward(cfg, Eg, [l.c for l in layers], fng, torch.from_numpy(ids).cuda(), B, T, q3.MODE_PREFILL,
+                     torch.zeros(B, dtype=torch.int32, device="cuda"), kvs, rope_gpu(cfg), logits, False,
+                     workspace(cfg, q3.OP_STACK_PREFILL, B, T, T))
+    assert_device_ok()
+    got = logits[:T].double().cpu().numpy()
+    del logits, caches
+    torch.cuda.empty_cache()
+    oc = oracle_config(cfg)
+    olayers = [l.oracle() for l in layers]
+    ref, _ = R.stack_forward(ids[:T], R.bf16_to_f64(E), olayers, R.bf16_to_f64(fn), oc)
+    err = rel_frob(got, ref)
+    agree = float(np.mean(np.argmax(got, 1) == np.argmax(ref, 1)))
+    top2 = np.sort(ref, axis=1)[:, -2:]
+    report("c1", rel_frob=err, argmax_agreement=agree, rows=T, max_abs=max_abs(got, ref),
+           median_top2_gap=float(np.median(top2[:, 1] - top2[:, 0])), logit_rms=float(np.sqrt(np.mean(ref ** 2))))
+    assert err <= LOGITS_REL_FROB
+    assert agree >= LOGITS_ARGMAX
+
+
+def test_config2_decode(q3):
+    """B64 sequences with 4096 cached tokens, successive decode steps at positions 4096..;
+    the oracle follows sequence 37 for the first 8 steps."""
+    cfg = q3.config_qwen3_0_6b()
+    seed, B, L0, steps, b_s = 1002, 64, 4096, 8, 37
+    s_max = L0 + 128
+    layers, E, fn = _stack_weights(q3, cfg, seed)
+    Eg, fng = to_gpu_bf16(E), to_gpu_bf16(fn)
+    caches = []
+    for l in range(cfg.n_layers):
+        k = torch.empty((B, 8, s_max, 128), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        for t, which in ((k, synth.L_CACHE_K), (v, synth.L_CACHE_V)):
+            synth.normal_bf16_device(t.data_ptr(), B * 8, L0, 128, s_max * 128, 128, seed,
+                                     synth.layer_tid(l, which), 0.0, 1.0)
+        caches.append((k, v))
+    kvs = [q3.kv_layer(k, v, s_max) for k, v in caches]
+    ids = synth.uniform_int(seed, synth.TID_IDS_STEP, (128, B), cfg.vocab)
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    ws = workspace(cfg, q3.OP_STACK_DECODE, B, 1, s_max)
+    rope = rope_gpu(cfg)
+    lg = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    got = []
+    for s in range(steps):
+        q3.stack_forward(cfg, Eg, [l.c for l in layers], fng, torch.from_numpy(ids[s]).cuda(), B, 1, q3.MODE_DECODE,
+                         lens, kvs, rope, lg, False, ws)
+        got.append(lg[b_s].double().cpu().numpy())
+    assert_device_ok()
+    assert int(lens[0].item()) == L0 + steps
+    del caches
+    torch.cuda.empty_cache()
+    # oracle: the same sequence's cache (host generator), then the same steps
+    oc = oracle_config(cfg)
+    olayers = [l.oracle() for l in layers]
+    base = b_s * 8 * L0 * 128
+    ocache = []
+    for l in range(cfg.n_layers):
+        kk = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_K), (8, L0, 128),
+                                                  index_base=base)).transpose(1, 0, 2)
+        vv = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_V), (8, L0, 128),
+                                                  index_base=base)).transpose(1, 0, 2)
+        ocache.append([kk, vv])
+    Ef, fnf = R.bf16_to_f64(E), R.bf16_to_f64(fn)
+    errs, agree = [], []
+    for s in range(steps):
+        caches_s = [(c[0], c[1], np.arange(L0 + s)) for c in ocache]
+        ref, new_kv = R.stack_forward(ids[s, b_s:b_s + 1], Ef, olayers, fnf, oc, positions=np.array([L0 + s]),
+                                      caches=caches_s)
+        for c, (kn, vn) in zip(ocache, new_kv):
+            c[0] = np.concatenate([c[0], kn])
+            c[1] = np.concatenate([c[1], vn])
+        errs.append(rel_frob(got[s], ref[0]))
+        agree.append(int(np.argmax(got[s]) == np.argmax(ref[0])))
+    report("c2", rel_frob_max=max(errs), rel_frob=errs, argmax=agree, steps=steps, sequence=b_s)
+    assert max(errs) <= LOGITS_REL_FROB
+    assert np.mean(agree) >= LOGITS_ARGMAX
+
+
+def test_config3_long_prefill(q3):
+    """1 layer, B1 T32768; the oracle computes K/V for all positions and finishes a
+    sample of query rows."""
+    cfg = q3.config_qwen3_0_6b()
+    seed, T = 1003, 32768
+    L = HostLayer(q3, cfg, seed, 0)
+    x = synth.normal_bf16_fast(seed, synth.TID_X, (T, cfg.hidden))
+    k = torch.empty((1, 8, T, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    kv = q3.kv_layer(k, v, T)
+    xg = to_gpu_bf16(x)
+    q3.block_prefill(cfg, L.c, xg, 1, T, torch.zeros(1, dtype=torch.int32, device="cuda"), kv, rope_gpu(cfg),
+                     workspace(cfg, q3.OP_BLOCK_PREFILL, 1, T, T))
+    assert_device_ok()
+    got = from_gpu_bf16(xg)
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128, 4095, 16383, 16384, 32766, 32767],
+                                     rng.integers(0, T, 245)]))
+    ref, _, _ = R.block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg), np.arange(T), rows=rows)
+    report("c3", rel_frob=rel_frob(got[rows], ref), max_abs=max_abs(got[rows], ref), rows=len(rows))
+    assert rel_frob(got[rows], ref) <= LAYER_REL_FROB and max_abs(got[rows], ref) <= LAYER_MAX_ABS
+
+
+def test_config4_moe_block(q3):
+    """MoE block: hidden 2048, 32/4 heads, 128 experts of width 768, top-8 renormalised,
+    B1 x T4096."""
+    cfg = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
+    seed, T = 1004, 4096
+    L = HostLayer(q3, cfg, seed, 0, moe=True)
+    x = synth.normal_bf16_fast(seed, synth.TID_X, (T, cfg.hidden))
+    k = torch.empty((1, 4, T, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    kv = q3.kv_layer(k, v, T)
+    xg = to_gpu_bf16(x)
+    kk = cfg.top_k
+    idx = torch.empty((T, kk), dtype=torch.int32, device="cuda")
+    w = torch.empty((T, kk), dtype=torch.float32, device="cuda")
+    off = torch.empty(cfg.n_experts + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * kk, dtype=torch.int32, device="cuda")
+    q3.moe_block(cfg, L.c, xg, 1, T, torch.zeros(1, dtype=torch.int32, device="cuda"), kv, rope_gpu(cfg),
+                 workspace(cfg, q3.OP_MOE_BLOCK, 1, T, T), idx, w, off, perm)
+    assert_device_ok()
+    got = from_gpu_bf16(xg)
+    ref, _, _, (ridx, rw, rp, margin) = R.moe_block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg),
+                                                            np.arange(T))
+    gi, goff, gperm = idx.cpu().numpy(), off.cpu().numpy(), perm.cpu().numpy()
+    sure = margin > 1e-3
+    idx_match = bool(np.array_equal(gi[sure], ridx[sure]))
+    # permutation: every expert whose tokens (on either side) all have a clear margin
+    offs, ptok, _ = R.moe_permutation(ridx, cfg.n_experts)
+    checked = 0
+    for e in range(cfg.n_experts):
+        toks_g = gperm[goff[e]:goff[e + 1]]
+        toks_o = ptok[offs[e]:offs[e + 1]]
+        if sure[np.union1d(toks_g, toks_o)].all():
+            np.testing.assert_array_equal(toks_g, toks_o)
+            checked += 1
+    report("c4", rel_frob=rel_frob(got, ref), max_abs=max_abs(got, ref), sure_tokens=int(sure.sum()),
+           idx_match=idx_match, experts_checked=checked, min_margin=float(margin.min()))
+    assert idx_match
+    assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS
+    if sure.all():
+        np.testing.assert_array_equal(goff, offs)
+        np.testing.assert_array_equal(gperm, ptok)

@@ -176,7 +176,12 @@ def test_attention_prefill(q3, hq, hkv, B, T, starts):
     ref = _attention_oracle(cfg, qf, kall.f, vall.f, starts, B, T).reshape(B * T, hq * D)
     got = from_gpu_bf16(o)
     assert np.isfinite(got).all()
-    assert max_abs(got, ref) <= 1e-2 and rel_frob(got, ref) <= 1e-2, (max_abs(got, ref), rel_frob(got, ref))
+    # bound: bf16 rounding of the output (<= 2^-8 |o|) plus bf16 rounding of each softmax
+    # weight in P.V (<= 2^-9 p_j |v_j|, summed: <= 2^-9 max|v|), plus fp32 slack
+    vmax = np.abs(vall.f).max()
+    tol = 2.0 ** -8 * np.abs(ref) + 2.0 ** -9 * vmax + 1e-4
+    assert np.all(np.abs(got - ref) <= tol), (max_abs(got, ref), rel_frob(got, ref))
+    assert rel_frob(got, ref) <= 1e-2
 
 
 @pytest.mark.parametrize("hq,hkv", [(16, 8), (32, 4)])
@@ -205,7 +210,8 @@ def test_attention_decode(q3, hq, hkv, lens):
         q = qkv.f[b, :hq * D].reshape(1, hq, D)
         ref = R.causal_gqa_attention(q, kall.f[b][:, :L].transpose(1, 0, 2), vall.f[b][:, :L].transpose(1, 0, 2),
                                      np.array([lens[b]]), np.arange(L)).reshape(-1)
-        assert max_abs(got[b], ref) <= 5e-3, (b, max_abs(got[b], ref))
+        # fp32 softmax and accumulation; the only rounding is the bf16 output (<= 2^-8 |o|)
+        assert np.all(np.abs(got[b] - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4), (b, max_abs(got[b], ref))
 
 
 def test_embed(q3):
