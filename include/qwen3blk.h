@@ -218,10 +218,12 @@ int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* 
  *            2: SwiGLU -- W rows interleaved as qwen3_pack_gate_up, out [M, N/2] bf16.
  *   out_f32 / resid_f32 select fp32 (else bf16). swap: 1 = weight rows on the MMA's 128-row
  *   side (small M), 0 = activations there, -1 = automatic (swap when M <= 256).
+ *   ws (may be NULL): scratch for split-K when the output has too few tiles to fill the GPU;
+ *   it holds fp32 partials, up to ws_bytes (split count = largest that fits).
  *   K % 64 == 0, N % 32 == 0, leading dimensions multiples of 8 elements. */
 int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long long ldw, void* out, long long ldo,
                   int M, int N, int K, int epilogue, const void* resid, long long ldr, int resid_f32, int out_f32,
-                  int swap, void* stream);
+                  int swap, void* ws, size_t ws_bytes, void* stream);
 
 /* Per-head QK RMSNorm + rotate-half RoPE + KV-cache write (see qwen3_block_prefill for
  * positions). qkv [B*T, (Hq+2Hkv)*D] (row stride ldqkv): q heads are normalised and rotated

@@ -67,7 +67,7 @@ _SIGS = {
     "qwen3_profile_end": ([_vp], _i),
     "qwen3_profile_record": ([_i, ctypes.c_char_p, _i, _P(_f)], _i),
     "qwen3_op_rmsnorm": ([_vp, _i, _ll, _vp, _vp, _ll, _i, _i, _f, _vp], _i),
-    "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _vp], _i),
+    "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _vp, _sz, _vp], _i),
     "qwen3_op_qk_norm_rope": ([_P(Config), _vp, _ll, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
     "qwen3_op_attention_prefill": ([_P(Config), _vp, _ll, _i, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_attention_decode": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp, _sz, _vp], _i),
@@ -225,14 +225,15 @@ def op_rmsnorm(x, w, out, rows, n, eps, ldx=None, ldo=None, stream=None) -> None
 
 
 def op_gemm(A, W, out, M, N, K, epilogue=EPI_STORE, resid=None, swap=-1, lda=None, ldw=None, ldo=None, ldr=None,
-            stream=None) -> None:
+            ws=None, stream=None) -> None:
     import torch
     out_f32 = 1 if out.dtype == torch.float32 else 0
     resid_f32 = 1 if (resid is not None and resid.dtype == torch.float32) else 0
     if ldo is None:
         ldo = N // 2 if epilogue == EPI_SWIGLU else N
     _check(lib.qwen3_op_gemm(_ptr(A), lda or K, _ptr(W), ldw or K, _ptr(out), ldo, M, N, K, epilogue, _ptr(resid),
-                             ldr or N, resid_f32, out_f32, swap, _stream(stream)), "op_gemm")
+                             ldr or N, resid_f32, out_f32, swap, _ptr(ws),
+                             0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)), "op_gemm")
 
 
 def op_qk_norm_rope(cfg, qkv, B, T, pos_base, q_norm, k_norm, kv, rope, ldqkv=None, stream=None) -> None:

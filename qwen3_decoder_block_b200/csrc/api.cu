@@ -190,6 +190,7 @@ struct Buffers {
   float* x1 = nullptr;       // [M, H] residual after attention (fp32)
   uint16_t* act = nullptr;   // [M, I] SwiGLU output
   float* part = nullptr;     // decode partials
+  float* gpart = nullptr;    // split-K partials of small-M GEMMs
   // MoE
   float* logits = nullptr;   // [M, E]
   int* idx = nullptr;        // [M, k]
@@ -219,6 +220,7 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
   b.o = cv.take<uint16_t>(M * c.n_q_heads * D);
   b.x1 = cv.take<float>(M * H);
   if (decode) b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, s_max) / sizeof(float));
+  if (M <= 256) b.gpart = cv.take<float>(kSplitKBytes / sizeof(float));
   if (op == QWEN3_OP_MOE_BLOCK) {
     const int E = c.n_experts, k = c.top_k;
     b.logits = cv.take<float>(M * E);
@@ -274,6 +276,8 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   g.epi = kEpiStore;
   g.out = b.qkv;
   g.ldo = nqkv;
+  g.partial = b.gpart;
+  g.partial_bytes = b.gpart ? kSplitKBytes : 0;
   {
     ProfScope ps("gemm_qkv", k.s);
     rc = launch_gemm(g, k.s, k.err);
@@ -307,6 +311,8 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   o.out = b.x1;
   o.out_f32 = true;
   o.ldo = H;
+  o.partial = b.gpart;
+  o.partial_bytes = b.gpart ? kSplitKBytes : 0;
   ProfScope ps("gemm_o", k.s);
   return launch_gemm(o, k.s, k.err);
 }
@@ -329,6 +335,8 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   g.epi = kEpiSwiglu;
   g.out = b.act;
   g.ldo = I;
+  g.partial = b.gpart;
+  g.partial_bytes = b.gpart ? kSplitKBytes : 0;
   {
     ProfScope ps("gemm_gate_up", k.s);
     rc = launch_gemm(g, k.s, k.err);
@@ -346,6 +354,8 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   d.out = out;
   d.out_f32 = out_f32;
   d.ldo = H;
+  d.partial = b.gpart;
+  d.partial_bytes = b.gpart ? kSplitKBytes : 0;
   ProfScope ps("gemm_down", k.s);
   return launch_gemm(d, k.s, k.err);
 }
@@ -370,6 +380,8 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   r.out = b.logits;
   r.out_f32 = true;
   r.ldo = E;
+  r.partial = b.gpart;
+  r.partial_bytes = b.gpart ? kSplitKBytes : 0;
   {
     ProfScope ps("gemm_router", k.s);
     rc = launch_gemm(r, k.s, k.err);
@@ -793,7 +805,7 @@ int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* 
 
 int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long long ldw, void* out, long long ldo,
                   int M, int N, int K, int epilogue, const void* resid, long long ldr, int resid_f32, int out_f32,
-                  int swap, void* stream) {
+                  int swap, void* ws, size_t ws_bytes, void* stream) {
   g_last_error.clear();
   Q3_CHECK(A && W && out, QWEN3_EINVAL, "gemm: NULL operand");
   Q3_CHECK(aligned16(A) && aligned16(W) && aligned16(out), QWEN3_EALIGN, "gemm: misaligned operand");
@@ -825,6 +837,10 @@ int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long 
   g.out = out;
   g.ldo = ldo;
   g.out_f32 = out_f32 != 0;
+  if (ws && aligned16(ws)) {
+    g.partial = static_cast<float*>(ws);
+    g.partial_bytes = ws_bytes;
+  }
   return finish(launch_gemm(g, static_cast<cudaStream_t>(stream), device_error_word()));
 }
 

@@ -365,106 +365,137 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
 
 // ============================================================================
 // K4: split-KV decode attention. CTA (split, group, sequence) handles keys
-// [split*128, split*128+128) of one sequence's KV group for all G query heads of
-// the group, so each K/V line is read once. K and V chunks arrive by two bulk
-// copies; scores use one warp per key (lanes split the 128 dims); the partial
-// (max, sum, unnormalised o) goes to the workspace and a second kernel merges
-// the splits with log-sum-exp weights.
+// [split*256, split*256+256) of one sequence's KV group for all G query heads of
+// the group, so each K/V line is read once. Warp w owns 32 consecutive keys:
+//   scores: lane = key; the lane reads its key's 256-byte row straight from HBM
+//           (16 x 16-byte loads in flight) and dots it with the G queries, which
+//           sit pre-scaled in shared memory (broadcast reads);
+//   softmax: per head over the warp's 32 keys (warp max / sum);
+//   P V:    lane = 4 head dims; each key's V row is one coalesced 256-byte warp read.
+// The 8 warps merge in shared memory; the split's (max, sum, unnormalised o) goes
+// to the workspace and a second kernel merges the splits with log-sum-exp weights.
 // ============================================================================
-constexpr int kDecChunk = 128;
+constexpr int kDecChunk = 256;
 constexpr int kDecThreads = 256;
+constexpr int kDecWarps = kDecThreads / 32;
 
+template <int G>
 __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
     const uint16_t* __restrict__ qkv, long long ldqkv, int Hq, int Hkv, const int* __restrict__ cache_len,
     const uint16_t* __restrict__ ck, const uint16_t* __restrict__ cv, int s_max, int n_splits,
     float* __restrict__ part, int* err) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  uint16_t* sK = reinterpret_cast<uint16_t*>(smem);
-  uint16_t* sV = sK + kDecChunk * kHeadDim;
-  float* sQ = reinterpret_cast<float*>(sV + kDecChunk * kHeadDim);  // [G][128]
-  const int G = Hq / Hkv;
-  float* sS = sQ + G * kHeadDim;                                     // [G][128]
-  float* sM = sS + G * kDecChunk;                                    // [G]
-  float* sL = sM + G;                                                // [G]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sL + G + 2);
-  bar = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(bar) + 7) & ~uintptr_t(7));
+  __shared__ __align__(16) float sQ[G][kHeadDim];
+  __shared__ float sP[kDecWarps][G][32];
+  __shared__ float sM[kDecWarps][G], sL[kDecWarps][G];
+  __shared__ __align__(16) float sO[kDecWarps][G][kHeadDim];
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_keys_total = cache_len[b] + 1;  // cached tokens + the new one
   const int k0 = split * kDecChunk;
-  const int nk = min(kDecChunk, n_keys_total - k0);
   float* my_part = part + (((long long)b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
   const long long head_stride = (long long)n_splits * (kHeadDim + 2);
-  if (nk <= 0 || n_keys_total > s_max) {
+  if (k0 >= n_keys_total || n_keys_total > s_max) {
     if (n_keys_total > s_max && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
-    for (int i = threadIdx.x; i < G; i += blockDim.x) {
-      my_part[i * head_stride + kHeadDim] = -INFINITY;
-      my_part[i * head_stride + kHeadDim + 1] = 0.f;
+    if (threadIdx.x < G) {
+      my_part[threadIdx.x * head_stride + kHeadDim] = -INFINITY;
+      my_part[threadIdx.x * head_stride + kHeadDim + 1] = 0.f;
     }
     return;
   }
-  const long long row0 = ((long long)b * Hkv + g) * s_max + k0;
-  if (threadIdx.x == 0) {
-    mbar_init(bar, 1);
-    fence_barrier_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(bar, 2u * nk * kHeadDim * 2);
-    bulk_load(sK, ck + row0 * kHeadDim, nk * kHeadDim * 2, bar);
-    bulk_load(sV, cv + row0 * kHeadDim, nk * kHeadDim * 2, bar);
-  }
-  // query heads of this group (already normed and rotated) -> fp32 smem
-  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+  for (int i = threadIdx.x; i < G * kHeadDim; i += kDecThreads) {
     const int j = i / kHeadDim, d = i % kHeadDim;
-    sQ[i] = __uint_as_float((uint32_t)qkv[(long long)b * ldqkv + (long long)(g * G + j) * kHeadDim + d] << 16) *
-            kScaleLog2;
+    sQ[j][d] = __uint_as_float((uint32_t)qkv[(long long)b * ldqkv + (long long)(g * G + j) * kHeadDim + d] << 16) *
+               kScaleLog2;
   }
   __syncthreads();
-  const bool ok = mbar_wait(bar, 0, err);
-  if (!__syncthreads_and(ok)) {
-    return;  // nothing left in flight: the wait either completed or its budget ran out
-  }
-  // scores: warp per key, lane owns dims [4*lane, 4*lane+4)
-  for (int k = warp; k < nk; k += kDecThreads / 32) {
-    const uint2 kv = *reinterpret_cast<const uint2*>(sK + k * kHeadDim + 4 * lane);
-    const float k0f = bf16_lo(kv.x), k1f = bf16_hi(kv.x), k2f = bf16_lo(kv.y), k3f = bf16_hi(kv.y);
-    for (int j = 0; j < G; ++j) {
-      const float4 q = *reinterpret_cast<const float4*>(sQ + j * kHeadDim + 4 * lane);
-      float d = q.x * k0f + q.y * k1f + q.z * k2f + q.w * k3f;
-      d = warp_sum(d);
-      if (lane == 0) sS[j * kDecChunk + k] = d;
+
+  const long long row0 = ((long long)b * Hkv + g) * s_max;
+  const int kw0 = k0 + warp * 32;  // first key of this warp
+  const int key = kw0 + lane;
+  const bool valid = key < n_keys_total;
+  // ---- scores: one key per lane
+  float s[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) s[j] = 0.f;
+  if (valid) {
+    const uint4* kr = reinterpret_cast<const uint4*>(ck + (row0 + key) * kHeadDim);
+    uint4 kv[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) kv[c] = __ldg(kr + c);
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const float k8[8] = {bf16_lo(kv[c].x), bf16_hi(kv[c].x), bf16_lo(kv[c].y), bf16_hi(kv[c].y),
+                           bf16_lo(kv[c].z), bf16_hi(kv[c].z), bf16_lo(kv[c].w), bf16_hi(kv[c].w)};
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        const float4 qa = *reinterpret_cast<const float4*>(&sQ[j][8 * c]);
+        const float4 qb = *reinterpret_cast<const float4*>(&sQ[j][8 * c + 4]);
+        s[j] += qa.x * k8[0] + qa.y * k8[1] + qa.z * k8[2] + qa.w * k8[3] + qb.x * k8[4] + qb.y * k8[5] +
+                qb.z * k8[6] + qb.w * k8[7];
+      }
     }
   }
-  __syncthreads();
-  // per-head max and sum over this chunk
-  for (int j = warp; j < G; j += kDecThreads / 32) {
-    float mx = -INFINITY;
-    for (int k = lane; k < nk; k += 32) mx = fmaxf(mx, sS[j * kDecChunk + k]);
-    mx = warp_max(mx);
-    float sum = 0.f;
-    for (int k = lane; k < nk; k += 32) {
-      const float e = exp2f(sS[j * kDecChunk + k] - mx);
-      sS[j * kDecChunk + k] = e;
-      sum += e;
+  // ---- softmax over the warp's keys
+  float m[G], l[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    const float sj = valid ? s[j] : -INFINITY;
+    m[j] = warp_max(sj);
+    const float p = valid ? exp2f(sj - m[j]) : 0.f;
+    l[j] = warp_sum(p);
+    sP[warp][j][lane] = p;
+  }
+  __syncwarp();
+  // ---- o = P V over the warp's keys, lane owns dims [4*lane, 4*lane+4)
+  float o[G][4];
+#pragma unroll
+  for (int j = 0; j < G; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  const int nk = min(32, n_keys_total - kw0);
+  const uint16_t* vbase = cv + (row0 + kw0) * kHeadDim + 4 * lane;
+#pragma unroll 4
+  for (int kk0 = 0; kk0 < 32; kk0 += 8) {
+    uint2 vv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (kk0 + u < nk) vv[u] = __ldg(reinterpret_cast<const uint2*>(vbase + (long long)(kk0 + u) * kHeadDim));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (kk0 + u < nk) {
+        const float v0 = bf16_lo(vv[u].x), v1 = bf16_hi(vv[u].x), v2 = bf16_lo(vv[u].y), v3 = bf16_hi(vv[u].y);
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float p = sP[warp][j][kk0 + u];
+          o[j][0] += p * v0; o[j][1] += p * v1; o[j][2] += p * v2; o[j][3] += p * v3;
+        }
+      }
     }
-    sum = warp_sum(sum);
-    if (lane == 0) { sM[j] = mx; sL[j] = sum; }
+  }
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    *reinterpret_cast<float4*>(&sO[warp][j][4 * lane]) = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
+    if (lane == 0) { sM[warp][j] = nk > 0 ? m[j] : -INFINITY; sL[warp][j] = nk > 0 ? l[j] : 0.f; }
   }
   __syncthreads();
-  // o[j][d] = sum_k p[j][k] v[k][d]
-  for (int i = threadIdx.x; i < G * kHeadDim; i += blockDim.x) {
+  // ---- merge the warps into this split's partial
+  for (int i = threadIdx.x; i < G * kHeadDim; i += kDecThreads) {
     const int j = i / kHeadDim, d = i % kHeadDim;
-    const float* pj = sS + j * kDecChunk;
-    float acc = 0.f;
-    for (int k = 0; k < nk; ++k) acc += pj[k] * __uint_as_float((uint32_t)sV[k * kHeadDim + d] << 16);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sM[w][j]);
+    float acc = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+      if (sM[w][j] == -INFINITY) continue;
+      const float sc = exp2f(sM[w][j] - M);
+      acc += sO[w][j][d] * sc;
+      L += sL[w][j] * sc;
+    }
     my_part[j * head_stride + d] = acc;
-  }
-  if (threadIdx.x < G) {
-    my_part[threadIdx.x * head_stride + kHeadDim] = sM[threadIdx.x];
-    my_part[threadIdx.x * head_stride + kHeadDim + 1] = sL[threadIdx.x];
+    if (d == 0) {
+      my_part[j * head_stride + kHeadDim] = M;
+      my_part[j * head_stride + kHeadDim + 1] = L;
+    }
   }
 }
 
@@ -500,16 +531,22 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
   const int n_splits = decode_splits(s_max);
-  const size_t smem = 128 + 2 * kDecChunk * kHeadDim * 2 + (size_t)G * kHeadDim * 4 + (size_t)G * kDecChunk * 4 +
-                      (size_t)2 * G * 4 + 64;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(attn_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr = true;
-  }
   dim3 grid(n_splits, Hkv, B);
-  attn_decode_split_kernel<<<grid, kDecThreads, smem, s>>>(qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max, n_splits,
-                                                            part, err);
+  switch (G) {
+#define Q3_DEC_CASE(GG)                                                                                         \
+  case GG:                                                                                                      \
+    attn_decode_split_kernel<GG><<<grid, kDecThreads, 0, s>>>(qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max,    \
+                                                              n_splits, part, err);                            \
+    break;
+    Q3_DEC_CASE(1)
+    Q3_DEC_CASE(2)
+    Q3_DEC_CASE(4)
+    Q3_DEC_CASE(8)
+#undef Q3_DEC_CASE
+    default:
+      set_last_error("attention decode: %d query heads per KV group is not supported (1, 2, 4 or 8)", G);
+      return -2;
+  }
   attn_decode_merge_kernel<<<B * Hq, kHeadDim, 0, s>>>(part, Hq, n_splits, out, ldo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -45,6 +45,8 @@ struct GemmCfg {
 struct GemmParams {
   int p_rows, q_rows, k_blocks;
   int p_tiles, q_tiles, q_fast;
+  int k_splits, kb_per_split;  // split-K: tile t covers k-blocks [ks*kb_per_split, ...)
+  float* partial;              // split-K partials [k_splits][tokens][features] (fp32)
   int epi, resid_f32, out_f32, swap;
   void* out;
   long long ldo;
@@ -56,16 +58,19 @@ struct GemmParams {
 };
 
 struct Tile {
-  int p0, p_end, q0, q_end, q_load;
+  int p0, p_end, q0, q_end, q_load, kb0, kb1, ks;
 };
 
 __device__ __forceinline__ int total_tiles(const GemmParams& g, const int* s_prefix) {
-  return g.n_groups > 0 ? s_prefix[g.n_groups] : g.p_tiles * g.q_tiles;
+  return g.n_groups > 0 ? s_prefix[g.n_groups] : g.p_tiles * g.q_tiles * g.k_splits;
 }
 
 template <int BN>
 __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const int* s_prefix, const int* s_off) {
   Tile r;
+  r.kb0 = 0;
+  r.kb1 = g.k_blocks;
+  r.ks = 0;
   if (g.n_groups > 0) {
     int lo = 0, hi = g.n_groups - 1;  // largest grp with s_prefix[grp] <= t
     while (lo < hi) {
@@ -80,6 +85,12 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const in
     r.q_end = g.q_rows;
     r.q_load = grp * g.q_rows + r.q0;
   } else {
+    if (g.k_splits > 1) {
+      r.ks = t % g.k_splits;
+      t /= g.k_splits;
+      r.kb0 = r.ks * g.kb_per_split;
+      r.kb1 = min(g.k_blocks, r.kb0 + g.kb_per_split);
+    }
     int pt, qt;
     if (g.q_fast) { pt = t / g.q_tiles; qt = t % g.q_tiles; }
     else          { qt = t / g.p_tiles; pt = t % g.p_tiles; }
@@ -231,7 +242,7 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
         const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
-        for (int kb = 0; kb < g.k_blocks; ++kb) {
+        for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
           if (*s_abort || !mbar_wait(&empty[stage], phase ^ 1, g.err)) { ok = false; break; }
           uint8_t* sp = smem + stage * C::STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -257,12 +268,13 @@ __global__ void __launch_bounds__(192, 1)
       int local = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
+        const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
         const int buf = local & 1;
         const uint32_t use_par = (local >> 1) & 1;
         if (*s_abort || !mbar_wait(&tempty[buf], use_par ^ 1, g.err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * BN;
-        for (int kb = 0; kb < g.k_blocks; ++kb) {
+        for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
           if (*s_abort || !mbar_wait(&full[stage], phase, g.err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -270,7 +282,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t bdesc = sdesc_kmajor_sw128(sa + C::P_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) ? 1u : 0u);
+            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > tl.kb0 || kk) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -300,7 +312,27 @@ __global__ void __launch_bounds__(192, 1)
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, r);
         tmem_wait_ld();
-        if (!g.swap) {
+        if (g.partial) {
+          // split-K: raw fp32 partial sums, [ks][token][feature]
+          if (!g.swap) {
+            const int p = tl.p0 + row, q = tl.q0 + c * 32;
+            if (p < tl.p_end && q < tl.q_end) {
+              float4* dst = reinterpret_cast<float4*>(g.partial + ((long long)tl.ks * g.p_rows + p) * g.q_rows + q);
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                dst[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+            }
+          } else {
+            const int p = tl.p0 + row;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int q = tl.q0 + c * 32 + j;
+              if (p < tl.p_end && q < tl.q_end)
+                g.partial[((long long)tl.ks * g.q_rows + q) * g.p_rows + p] = __uint_as_float(r[j]);
+            }
+          }
+        } else if (!g.swap) {
           const int p = tl.p0 + row, q = tl.q0 + c * 32;
           if (p < tl.p_end && q < tl.q_end) store_row_chunk(g, p, q, r);
         } else {
@@ -319,6 +351,37 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+}
+
+// --------------------------------------------------------------------------- split-K reduce
+// out[m][n] = epilogue(sum_s part[s][m][n']) over tokens m and output features n;
+// SwiGLU reads the packed gate column (n/16)*32 + n%16 and the up column 16 after it.
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N, int epi, int resid_f32,
+                                     int out_f32, const void* __restrict__ resid, long long ldr,
+                                     void* __restrict__ out, long long ldo) {
+  const int n_out = epi == kEpiSwiglu ? N / 2 : N;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)M * n_out) return;
+  const int m = (int)(idx / n_out), n = (int)(idx % n_out);
+  const long long plane = (long long)M * N;
+  if (epi == kEpiSwiglu) {
+    const int pg = (n / 16) * 32 + (n % 16);
+    float gsum = 0.f, usum = 0.f;
+    for (int s = 0; s < S; ++s) {
+      gsum += part[s * plane + (long long)m * N + pg];
+      usum += part[s * plane + (long long)m * N + pg + 16];
+    }
+    static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_bf16_bits(silu_f(gsum) * usum);
+    return;
+  }
+  float acc = 0.f;
+  for (int s = 0; s < S; ++s) acc += part[s * plane + (long long)m * N + n];
+  if (epi == kEpiResid) {
+    if (resid_f32) acc += static_cast<const float*>(resid)[(long long)m * ldr + n];
+    else acc += __uint_as_float((uint32_t)static_cast<const uint16_t*>(resid)[(long long)m * ldr + n] << 16);
+  }
+  if (out_f32) static_cast<float*>(out)[(long long)m * ldo + n] = acc;
+  else static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_bf16_bits(acc);
 }
 
 // --------------------------------------------------------------------------- host side
@@ -398,6 +461,23 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   g.n_groups = d.n_groups;
   g.group_offsets = d.group_offsets;
   g.err = err;
+  g.k_splits = 1;
+  g.kb_per_split = g.k_blocks;
+  g.partial = nullptr;
+  // Split K when the output has too few tiles to keep the SMs streaming: each split
+  // writes fp32 partials, and a reduce kernel applies the epilogue.
+  const long long out_tiles = (long long)g.p_tiles * g.q_tiles;
+  if (d.n_groups == 0 && d.partial && out_tiles * 2 <= num_sms() && g.k_blocks > 1) {
+    int S = (int)(num_sms() / out_tiles);
+    if (S > g.k_blocks) S = g.k_blocks;
+    const size_t per_split = (size_t)d.p_rows * d.q_rows * sizeof(float);
+    while (S > 1 && (size_t)S * per_split > d.partial_bytes) --S;
+    if (S > 1) {
+      g.kb_per_split = (g.k_blocks + S - 1) / S;
+      g.k_splits = (g.k_blocks + g.kb_per_split - 1) / g.kb_per_split;
+      g.partial = d.partial;
+    }
+  }
   const size_t smem = C::smem_bytes(d.n_groups);
   static bool attr_set[4] = {false, false, false, false};
   static std::mutex mu;
@@ -413,11 +493,17 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   if (d.n_groups > 0) {
     grid = num_sms();
   } else {
-    const long long tiles = (long long)g.p_tiles * g.q_tiles;
+    const long long tiles = (long long)g.p_tiles * g.q_tiles * g.k_splits;
     grid = (int)(tiles < num_sms() ? tiles : num_sms());
   }
   if (grid <= 0) return 0;
   gemm_tc_kernel<BN><<<grid, 192, smem, s>>>(tmP, tmQ, g);
+  if (g.k_splits > 1) {
+    const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
+    const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);
+    splitk_reduce_kernel<<<(unsigned)((n_out + 255) / 256), 256, 0, s>>>(
+        g.partial, g.k_splits, M, N, d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("gemm launch failed: %s", cudaGetErrorString(e));

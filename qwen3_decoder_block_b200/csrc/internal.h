@@ -35,7 +35,12 @@ struct GemmDesc {
   int n_groups = 0;
   const int* group_offsets = nullptr;  // device, n_groups + 1 entries
   int force_bn = 0;                    // 0 = automatic
+  float* partial = nullptr;            // optional split-K scratch (fp32)
+  size_t partial_bytes = 0;
 };
+
+// Scratch the block calls reserve for split-K partials of small-M GEMMs.
+constexpr size_t kSplitKBytes = (size_t)2 * 148 * 128 * 256 * sizeof(float);
 
 int launch_gemm(const GemmDesc& d, cudaStream_t s, int* err);
 

@@ -79,7 +79,8 @@ def _gemm(reps, M, N, K, epi=q3.EPI_STORE, swap=-1, out_f32=False, resid=False):
     n_out = N // 2 if epi == q3.EPI_SWIGLU else N
     out = torch.empty((M, n_out), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
     r = torch.zeros((M, N), dtype=torch.float32, device="cuda") if resid else None
-    ms = _time(lambda: q3.op_gemm(A, W, out, M, N, K, epilogue=epi, resid=r, swap=swap), reps)
+    ws = torch.empty(48 << 20, dtype=torch.uint8, device="cuda")  # split-K scratch for small M
+    ms = _time(lambda: q3.op_gemm(A, W, out, M, N, K, epilogue=epi, resid=r, swap=swap, ws=ws), reps)
     flops = 2 * M * N * K
     nbytes = 2 * (M * K + N * K) + out.numel() * out.element_size() + (r.numel() * 4 if resid else 0)
     return {"ms": ms, "tflops": flops / ms / 1e9, "gbs": nbytes / ms / 1e6, "flops": flops, "bytes": nbytes}

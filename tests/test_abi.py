@@ -86,7 +86,7 @@ def test_workspace_sizes_monotone(q3):
     M = 4 * 2048
     assert b >= M * (1024 * 2 + 4096 * 2 + 2048 * 2 + 1024 * 4 + 3072 * 2)
     d = q3.workspace_size(c, q3.OP_BLOCK_DECODE, 64, 1, 4224)
-    assert d >= 64 * 16 * 33 * 130 * 4  # split-KV partials
+    assert d >= 64 * 16 * 17 * 130 * 4  # split-KV partials (256-key chunks)
     assert q3.workspace_size(c, 99, 1, 1, 1) == 0
     assert q3.workspace_size(c, q3.OP_BLOCK_PREFILL, 0, 1, 1) == 0
 
@@ -99,9 +99,9 @@ def test_null_and_misaligned_arguments_rejected_without_launch(q3):
                                     None, 0, None)
     assert st == q3.EINVAL
     assert "NULL" in q3.lib.qwen3_last_error().decode()
-    st = q3.lib.qwen3_op_gemm(8, 1024, 16, 1024, 32, 1024, 16, 1024, 1024, 0, None, 0, 0, 0, -1, None)
+    st = q3.lib.qwen3_op_gemm(8, 1024, 16, 1024, 32, 1024, 16, 1024, 1024, 0, None, 0, 0, 0, -1, None, 0, None)
     assert st == q3.EALIGN
-    st = q3.lib.qwen3_op_gemm(16, 1024, 32, 1024, 48, 1024, 16, 1000, 1024, 0, None, 0, 0, 0, -1, None)
+    st = q3.lib.qwen3_op_gemm(16, 1024, 32, 1024, 48, 1024, 16, 1000, 1024, 0, None, 0, 0, 0, -1, None, 0, None)
     assert st == q3.ESHAPE  # N % 32
     st = q3.lib.qwen3_op_rmsnorm(16, 0, 1000, 32, 48, 1000, 4, 1000, 1e-6, None)
     assert st == q3.ESHAPE

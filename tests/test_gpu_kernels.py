@@ -75,6 +75,38 @@ def test_gemm_residual(q3, M, N, K, swap, rt, ot):
     assert np.all(np.abs(got - ref) <= tol), max_abs(got, ref)
 
 
+@pytest.mark.parametrize("M,N,K,epi", [(64, 1024, 2048, 1), (64, 6144, 1024, 2), (16, 4096, 1024, 0),
+                                       (64, 1024, 3072, 1), (200, 512, 1024, 0), (3, 4736, 1024, 0)])
+@pytest.mark.parametrize("out_f32", [0, 1])
+def test_gemm_split_k(q3, M, N, K, epi, out_f32):
+    """Small-M GEMMs split K across CTAs (fp32 partials + reduce with the epilogue)."""
+    if epi == 2 and out_f32:
+        pytest.skip("SwiGLU output is bf16")
+    A = Tensor(SEED, 37, (M, K))
+    W = Tensor(SEED, 38, (N, K), 0.0, 0.02)
+    X = Tensor(SEED, 39, (M, N))
+    n_out = N // 2 if epi == 2 else N
+    out = torch.empty((M, n_out), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
+    ws = torch.empty(64 << 20, dtype=torch.uint8, device="cuda")
+    resid = X.gpu.float() if epi == 1 else None
+    packed = W.gpu
+    if epi == 2:
+        packed = torch.empty_like(W.gpu)
+        q3.pack_gate_up(N // 2, K, W.gpu[:N // 2], W.gpu[N // 2:], packed)
+    q3.op_gemm(A.gpu, packed, out, M, N, K, epilogue=epi, resid=resid, swap=1, ws=ws)
+    assert_device_ok()
+    acc = A.f @ W.f.T
+    if epi == 2:
+        ref = R.silu(acc[:, :N // 2]) * acc[:, N // 2:]
+    elif epi == 1:
+        ref = X.f + acc
+    else:
+        ref = acc
+    got = out.cpu().double().numpy() if out_f32 else from_gpu_bf16(out)
+    tol = 1e-4 if out_f32 else bf16_tol(ref, abs_=2e-4)
+    assert np.all(np.abs(got - ref) <= tol), max_abs(got, ref)
+
+
 def test_gemm_residual_in_place(q3):
     M, N, K = 300, 1024, 1024
     A = Tensor(SEED, 34, (M, K))
