@@ -245,6 +245,24 @@ int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, lo
                               const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                               void* ws, size_t ws_bytes, void* stream);
 
+/* Decode attention exactly as qwen3_op_attention_decode, for callers that cannot allocate
+ * device memory (for example a host application given a fixed memory budget, or a plugin
+ * that is handed tensors but no allocator or workspace). The pages have no counterpart:
+ * this entry point exists for such callers only.
+ * Instead of a caller workspace, the split partials live in a static device array of this
+ * library, 12 MiB on every GPU that loads the library (held until the process exits).
+ * Limit: B * Hq * ceil(kv->s_max / 256) <= 24197 (for example B 64, Hq 16, s_max up to 5888);
+ * larger sizes return QWEN3_EWORKSPACE with the numbers in qwen3_last_error().
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture. The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * All calls share the one array: calls that overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller. Every partial a call reads is written
+ * by that same call, so nothing needs clearing between calls. */
+int qwen3_op_attention_decode_noalloc(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
+                                      const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
+                                      void* stream);
+
 /* out[m] = embed[ids[m]] ([P-MoE] section 5), bf16 or fp32 (out_f32). */
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,
                    void* stream);

@@ -71,6 +71,7 @@ _SIGS = {
     "qwen3_op_qk_norm_rope": ([_P(Config), _vp, _ll, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
     "qwen3_op_attention_prefill": ([_P(Config), _vp, _ll, _i, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_attention_decode": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp, _sz, _vp], _i),
+    "qwen3_op_attention_decode_noalloc": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_embed": ([_vp, _i, _vp, _i, _i, _vp, _i, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -254,6 +255,15 @@ def op_attention_decode(cfg, qkv, B, cache_len, kv, o, ws, ldqkv=None, ldo=None,
     _check(lib.qwen3_op_attention_decode(ctypes.byref(cfg), _ptr(qkv), ld, B, _ptr(cache_len), ctypes.byref(kv),
                                          _ptr(o), ldo or cfg.n_q_heads * cfg.head_dim, _ptr(ws),
                                          ws.numel() * ws.element_size(), _stream(stream)), "op_attention_decode")
+
+
+def op_attention_decode_noalloc(cfg, qkv, B, cache_len, kv, o, ldqkv=None, ldo=None, stream=None) -> None:
+    """Decode attention with the split scratch in the library's static device array
+    (no caller workspace; see the header for the size limit and the sharing rules)."""
+    ld = ldqkv or (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
+    _check(lib.qwen3_op_attention_decode_noalloc(ctypes.byref(cfg), _ptr(qkv), ld, B, _ptr(cache_len),
+                                                 ctypes.byref(kv), _ptr(o), ldo or cfg.n_q_heads * cfg.head_dim,
+                                                 _stream(stream)), "op_attention_decode_noalloc")
 
 
 def op_embed(ids, n, embed, vocab, H, out, stream=None) -> None:

@@ -36,6 +36,9 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
                             const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
                             long long ldo, int* err, cudaStream_t s);
 size_t decode_partial_bytes(int B, int Hq, int s_max);
+int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
+                                   const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
+                                   uint16_t* out, long long ldo, int* err, cudaStream_t s);
 int launch_moe_route(const float* logits, int T, int E, int k, int renorm, int* idx, float* w, int* counts,
                      cudaStream_t s);
 int launch_moe_permute(const int* idx, int T, int k, int E, const int* counts, int* offsets, int* perm_token,
@@ -894,6 +897,22 @@ int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long
   return finish(launch_attention_decode(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
                                         kv->s_max, static_cast<float*>(ws), o, ldo, device_error_word(),
                                         static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B,
+                                      const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
+                                      void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(qkv && cache_len && o, QWEN3_EINVAL, "attention_decode_noalloc: NULL pointer");
+  Q3_CHECK(aligned16(qkv) && aligned16(o), QWEN3_EALIGN, "attention_decode_noalloc: misaligned pointer");
+  Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode_noalloc: B must be positive");
+  if ((rc = check_kv(*c, kv, 1))) return rc;
+  if ((rc = check_device())) return rc;
+  return finish(launch_attention_decode_static(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
+                                               kv->s_max, o, ldo, device_error_word(),
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,

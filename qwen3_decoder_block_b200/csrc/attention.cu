@@ -17,6 +17,7 @@
 // 128-byte swizzled shared tile, and O += P V accumulates in tensor memory with V
 // as an MN-major operand. Causal tiles beyond the diagonal are skipped and the
 // heaviest q tiles are scheduled first.
+#include <mutex>
 #include "common.cuh"
 #include "internal.h"
 
@@ -554,6 +555,55 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     return -6;
   }
   return 0;
+}
+
+// ----------------------------------------------------------------------------
+// Decode attention without caller scratch. The split partials live in a fixed
+// device array of this library instead of a caller workspace, for callers that
+// cannot allocate device memory. Its capacity is kStaticDecodeFloats floats
+// (12 MiB): B * Hq * ceil(s_max / 256) * 130 floats must fit. The array's device
+// address is looked up on the host once per device (with that device current);
+// every call shares the array, so calls that overlap on the GPU race. Each call
+// rewrites every partial it reads, so nothing has to be cleared between calls.
+// ----------------------------------------------------------------------------
+constexpr size_t kStaticDecodeFloats = (size_t)3 << 20;
+static __device__ __align__(256) float g_decode_scratch[kStaticDecodeFloats];
+
+static std::mutex g_static_mu;
+static float* g_static_ptr[64];
+
+size_t static_decode_scratch_bytes() { return kStaticDecodeFloats * sizeof(float); }
+
+int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
+                                   const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
+                                   uint16_t* out, long long ldo, int* err, cudaStream_t s) {
+  const size_t need = decode_partial_bytes(B, Hq, s_max);
+  if (need > kStaticDecodeFloats * sizeof(float)) {
+    set_last_error("attention_decode_noalloc: B=%d, Hq=%d, s_max=%d need %zu bytes of split scratch; the "
+                   "static scratch holds %zu bytes (B * Hq * ceil(s_max/256) must be <= %zu)",
+                   B, Hq, s_max, need, kStaticDecodeFloats * sizeof(float), kStaticDecodeFloats / (kHeadDim + 2));
+    return -5;
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    set_last_error("attention_decode_noalloc: no current CUDA device");
+    return -6;
+  }
+  float* ptr;
+  {
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+      if (e != cudaSuccess || !p) {
+        set_last_error("attention_decode_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        return -6;
+      }
+      g_static_ptr[dev] = static_cast<float*>(p);
+    }
+    ptr = g_static_ptr[dev];
+  }
+  return launch_attention_decode(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, cv, s_max, ptr, out, ldo, err, s);
 }
 
 }  // namespace q3

@@ -1,0 +1,58 @@
+"""The decode-attention entry point that allocates nothing.
+
+Some callers cannot allocate device memory (an application held to a fixed memory
+budget, a plugin handed tensors but no allocator or workspace). For them the
+library offers qwen3_op_attention_decode_noalloc, whose split scratch is a static
+device array of the library. This test calls it through the C ABI twice in a row
+and checks each result against the workspace-taking qwen3_op_attention_decode, on
+the decode workload's shapes (B 64, 4097 visible positions). The file is named so
+that pytest collects it last.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from helpers import Tensor, assert_device_ok, from_gpu_bf16, kv_cache, workspace  # noqa: E402
+
+
+def test_noalloc_decode_matches_workspace_decode_twice():
+    import qwen3_decoder_block_b200 as q3
+    cfg = q3.config_qwen3_0_6b()
+    hq, hkv, D = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
+    B, L0 = 64, 4096
+    s_max = L0 + 128
+    k, v, kv = kv_cache(cfg, B, s_max)
+    for step, seed in enumerate((501, 502)):
+        lens = [L0 + step - (b % 7) * 300 for b in range(B)]  # ragged lengths
+        kall = Tensor(seed, 1, (B, hkv, s_max, D))
+        vall = Tensor(seed, 2, (B, hkv, s_max, D))
+        k.copy_(kall.gpu)
+        v.copy_(vall.gpu)
+        qkv = Tensor(seed, 3, (B, (hq + 2 * hkv) * D))
+        cl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        o_ref = torch.empty((B, hq * D), dtype=torch.bfloat16, device="cuda")
+        o_new = torch.full((B, hq * D), float("nan"), dtype=torch.bfloat16, device="cuda")
+        q3.op_attention_decode(cfg, qkv.gpu, B, cl, kv, o_ref, workspace(cfg, q3.OP_BLOCK_DECODE, B, 1, s_max))
+        q3.op_attention_decode_noalloc(cfg, qkv.gpu, B, cl, kv, o_new)
+        assert_device_ok()
+        ref, got = from_gpu_bf16(o_ref), from_gpu_bf16(o_new)
+        assert np.isfinite(got).all()
+        # same tolerance as the decode parity test: the bf16 rounding of the output
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4), step
+
+
+def test_noalloc_rejects_sizes_beyond_the_static_scratch():
+    import qwen3_decoder_block_b200 as q3
+    cfg = q3.config_qwen3_0_6b()
+    B, s_max = 64, 8192  # 64 * 16 * 32 splits > 24197
+    k, v, kv = kv_cache(cfg, 1, 16)
+    big = q3.kv_layer(k, v, s_max)
+    qkv = torch.zeros((B, 4096), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros((B, 2048), dtype=torch.bfloat16, device="cuda")
+    cl = torch.zeros(B, dtype=torch.int32, device="cuda")
+    with pytest.raises(q3.Qwen3Error) as e:
+        q3.op_attention_decode_noalloc(cfg, qkv, B, cl, big, o)
+    assert e.value.status == q3.EWORKSPACE
+    assert "static scratch" in str(e.value)
