@@ -30,22 +30,22 @@ int make_tmap_3d(CUtensorMap* map, const void* base, long long inner, long long 
 namespace {
 
 constexpr int kHeadDim = 128;
-constexpr int kTileQ = 128;   // MMA rows per CTA
+constexpr int kTileQ = 128;   // rows of one MMA tile (tokens x heads of one KV group)
 constexpr int kTileK = 128;   // keys per KV tile
 constexpr uint32_t kHalf = 128 * 64 * 2;  // one [128 rows][64] bf16 swizzled half tile: 16 KB
-// smem layout (1024-aligned): Q (2 halves), 2 stages x (K 2 halves, V 2 halves), P (2 halves)
+// shared memory (1024-aligned): Q tiles 0 and 1 (2 halves each), 2 stages x (K 2 halves, V 2 halves)
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKV = 2 * kHalf;
+constexpr uint32_t kOffKV = 4 * kHalf;
 constexpr uint32_t kStageBytes = 4 * kHalf;
-constexpr uint32_t kOffP = kOffKV + 2 * kStageBytes;
-constexpr uint32_t kOffBar = kOffP + 2 * kHalf;
+constexpr uint32_t kOffBar = kOffKV + 2 * kStageBytes;
 constexpr uint32_t kPrefillSmem = kOffBar + 256 + 1024;
+constexpr int kPrefillThreads = 320;  // TMA warp, MMA warp, 2 softmax warpgroups
 // log2(e) / sqrt(128)
 constexpr float kScaleLog2 = 0.12751743074380304f;
 constexpr float kRescaleThreshold = 8.0f;
 
 struct PrefillParams {
-  int B, T, Hq, Hkv, G, s_max, n_qtiles;
+  int B, T, Hq, Hkv, G, s_max, n_cta_q;
   const int* start_pos;
   uint16_t* out;
   long long ldo;
@@ -54,42 +54,44 @@ struct PrefillParams {
 
 }  // namespace
 
-__global__ void __launch_bounds__(192, 1)
+// Tensor memory (512 columns): tile X in {0, 1} owns columns [256X, 256X+256):
+// S_X = [256X, 256X+128) (fp32 scores; its first 64 columns are reused for the bf16
+// probabilities P_X), O_X = [256X+128, 256X+256) (fp32 output accumulator).
+__global__ void __launch_bounds__(kPrefillThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* s_free = bars + 9;    // [2]
-  uint64_t* p_full = bars + 11;
-  uint64_t* p_free = bars + 12;   // PV of the previous tile complete (O stable, P reusable)
+  uint64_t* k_full = bars + 1;    // [2] per stage
+  uint64_t* v_full = bars + 3;    // [2] per stage
+  uint64_t* kv_empty = bars + 5;  // [2] per stage
+  uint64_t* s_full = bars + 7;    // [2] per Q tile
+  uint64_t* p_full = bars + 9;    // [2] per Q tile
+  uint64_t* pv_done = bars + 11;  // [2] per Q tile
   uint64_t* drain = bars + 13;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.n_qtiles - 1 - (int)blockIdx.x;  // heavy tiles first
+  const int cq = p.n_cta_q - 1 - (int)blockIdx.x;  // heavy CTAs first
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = p.G, TQ = kTileQ / G;
-  const int t0 = qt * TQ;
+  const int t0 = cq * 2 * TQ;
   const int start = p.start_pos[b];
   const int kv_limit = start + p.T;  // keys [0, kv_limit) are in the cache
-  const int t_last = min(t0 + TQ, p.T) - 1;
-  const int n_kv = (start + t_last) / kTileK + 1;
+  // KV tiles each Q tile needs (tile 1 holds the later tokens)
+  const int nk0 = t0 < p.T ? (start + min(t0 + TQ, p.T) - 1) / kTileK + 1 : 0;
+  const int nk1 = t0 + TQ < p.T ? (start + min(t0 + 2 * TQ, p.T) - 1) / kTileK + 1 : 0;
+  const int n_kv = max(nk0, nk1);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&v_full[i], 1); mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128);
+      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(p_free, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
@@ -99,17 +101,17 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_O = tmem + 256;
   const long long kv_row0 = ((long long)b * p.Hkv + g) * p.s_max;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- TMA producer
+      // -------------------------------------------------------------- TMA producer
       bool ok = true;
-      long long issued_kv = 0;
-      mbar_arrive_expect_tx(q_full, 2 * kHalf);
-      for (int h = 0; h < 2; ++h)
-        tma_load_3d(smem + kOffQ + h * kHalf, &tmQ, q_full, 64 * h, g * G, b * p.T + t0);
+      long long issued = 0;
+      mbar_arrive_expect_tx(q_full, 4 * kHalf);
+      for (int X = 0; X < 2; ++X)
+        for (int h = 0; h < 2; ++h)
+          tma_load_3d(smem + kOffQ + (2 * X + h) * kHalf, &tmQ, q_full, 64 * h, g * G, b * p.T + t0 + X * TQ);
       for (int j = 0; j < n_kv && ok; ++j) {
         const int st = j & 1;
         const uint32_t par = (j >> 1) & 1;
@@ -122,13 +124,12 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(&v_full[st], 2 * kHalf);
         tma_load_2d(base + 2 * kHalf, &tmV, &v_full[st], 0, row);
         tma_load_2d(base + 3 * kHalf, &tmV, &v_full[st], 64, row);
-        ++issued_kv;
+        ++issued;
       }
-      // Before exit every copy must have landed (normal path: consumers saw them all).
       mbar_wait(q_full, 0, p.err);
       if (!ok) {
         *s_abort = 1;
-        for (long long i = issued_kv > 2 ? issued_kv - 2 : 0; i < issued_kv; ++i) {
+        for (long long i = issued > 2 ? issued - 2 : 0; i < issued; ++i) {
           mbar_wait(&k_full[i & 1], (uint32_t)((i >> 1) & 1), p.err);
           mbar_wait(&v_full[i & 1], (uint32_t)((i >> 1) & 1), p.err);
         }
@@ -136,48 +137,46 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
+      // -------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileK, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim, 0, 1);  // V is MN-major
       bool ok = mbar_wait(q_full, 0, p.err);
       const uint32_t sq = smem_u32(smem + kOffQ);
-      const uint32_t sp = smem_u32(smem + kOffP);
-      for (int j = 0; j <= n_kv && ok; ++j) {
-        if (j < n_kv) {
-          // S_j = Q K_j^T into S buffer j&1
-          const int st = j & 1;
-          const uint32_t par = (j >> 1) & 1;
-          if (*s_abort || !mbar_wait(&k_full[st], par, p.err) || !mbar_wait(&s_free[st], par ^ 1, p.err)) {
-            ok = false; break;
-          }
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int st = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (*s_abort || !mbar_wait(&k_full[st], par, p.err)) { ok = false; break; }
+        const uint32_t sk = smem_u32(smem + kOffKV + st * kStageBytes);
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (j >= (X ? nk1 : nk0)) continue;
+          // S_X reuses the columns of P_X of the previous tile: wait until that P.V is done
+          if (j > 0 && (*s_abort || !mbar_wait(&pv_done[X], (j - 1) & 1, p.err))) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sk = smem_u32(smem + kOffKV + st * kStageBytes);
+          const uint32_t qa = sq + 2 * X * kHalf;
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_kmajor_sw128(sq + (kk >> 2) * kHalf) + 2 * (kk & 3);
+            const uint64_t a = sdesc_kmajor_sw128(qa + (kk >> 2) * kHalf) + 2 * (kk & 3);
             const uint64_t bd = sdesc_kmajor_sw128(sk + (kk >> 2) * kHalf) + 2 * (kk & 3);
-            mma_bf16_ss(tmem + st * 128, a, bd, idesc_s, kk ? 1u : 0u);
+            mma_bf16_ss(tmem + 256 * X, a, bd, idesc_s, kk ? 1u : 0u);
           }
-          mma_commit(&s_full[st]);
+          mma_commit(&s_full[X]);
         }
-        if (j > 0) {
-          // O += P_{j-1} V_{j-1}
-          const int jj = j - 1, st = jj & 1;
-          const uint32_t par = (jj >> 1) & 1;
-          if (*s_abort || !mbar_wait(&v_full[st], par, p.err) || !mbar_wait(p_full, jj & 1, p.err)) {
-            ok = false; break;
-          }
+        if (!ok) break;
+        if (*s_abort || !mbar_wait(&v_full[st], par, p.err)) { ok = false; break; }
+        const uint32_t sv = sk + 2 * kHalf;
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (j >= (X ? nk1 : nk0)) continue;
+          if (*s_abort || !mbar_wait(&p_full[X], j & 1, p.err)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sv = smem_u32(smem + kOffKV + st * kStageBytes + 2 * kHalf);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_kmajor_sw128(sp + (kk >> 2) * kHalf) + 2 * (kk & 3);
             const uint64_t bd = sdesc_mnmajor_sw128(sv + kk * 16 * 128, kHalf, 1024);
-            mma_bf16_ss(tmem_O, a, bd, idesc_o, (jj | kk) ? 1u : 0u);
+            mma_bf16_ts(tmem + 256 * X + 128, tmem + 256 * X + kk * 8, bd, idesc_o, (j | kk) ? 1u : 0u);
           }
-          mma_commit(p_free);
-          mma_commit(&kv_empty[st]);
+          mma_commit(&pv_done[X]);
         }
+        if (!ok) break;
+        mma_commit(&kv_empty[st]);
       }
       if (!ok) {
         *s_abort = 1;
@@ -186,79 +185,106 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // tile row
-    const int t = t0 + r / G;
+    // ---------------------------------------------------------------- softmax
+    const int X = (warp - 2) >> 2;  // which Q tile this warpgroup owns
+    const int quad = warp & 3;      // tensor-memory lanes [32 quad, 32 quad + 32)
+    const int r = quad * 32 + lane;
+    const int t = t0 + X * TQ + r / G;
     const int qpos = start + t;
+    const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + 256 * X + lane_base;
+    const uint32_t tO = tS + 128;
+    const int nkx = X ? nk1 : nk0;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    uint8_t* sP = smem + kOffP;
-    for (int j = 0; j < n_kv; ++j) {
+    for (int j = 0; j < nkx; ++j) {
       const int st = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      bool w_ok = !*s_abort && mbar_wait(&s_full[st], par, p.err);
+      bool w_ok = !*s_abort && mbar_wait(&s_full[X], j & 1, p.err);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + st * 128 + c * 32 + ((uint32_t)(quad * 32) << 16), v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free[st]);
       const int kv0 = j * kTileK;
+      // only tiles touching the diagonal or the end of the cache need the mask
+      const bool need_mask = __any_sync(0xffffffffu, kv0 + kTileK - 1 > qpos || kv0 + kTileK > kv_limit);
+      // pass 1: row max, two 32-column chunks per tensor-memory round trip
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        const int kp = kv0 + i;
-        const bool vis = kp <= qpos && kp < kv_limit;
-        s[i] = vis ? s[i] * kScaleLog2 : -INFINITY;
-        mx = fmaxf(mx, s[i]);
-      }
-      float m_use = m_run, alpha = 1.f;
-      if (mx > m_run + kRescaleThreshold || m_run == -INFINITY) {
-        m_use = fmaxf(mx, m_run);
-        alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_use);
-        m_run = m_use;
-      }
-      float sum = 0.f;
-      uint32_t pk[64];
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(tS + c2 * 32, v[0]);
+        tmem_ld32(tS + c2 * 32 + 32, v[1]);
+        tmem_wait_ld_regs(v[0]);
+        tmem_wait_ld_regs(v[1]);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = (m_use == -INFINITY) ? 0.f : exp2f(s[2 * i] - m_use);
-        const float p1 = (m_use == -INFINITY) ? 0.f : exp2f(s[2 * i + 1] - m_use);
-        sum += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l_run = l_run * alpha + sum;
-      // the previous PV must be complete before O is rescaled or P overwritten
-      if (j > 0) {
-        w_ok = !*s_abort && mbar_wait(p_free, (j - 1) & 1, p.err);
-        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        for (int h = 0; h < 2; ++h) {
+          if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            const uint32_t ta = tmem_O + c * 32 + ((uint32_t)(quad * 32) << 16);
-            tmem_ld32(ta, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
-            tmem_st32(ta, v);
+            for (int i = 0; i < 32; ++i) {
+              const int kp = kv0 + (c2 + h) * 32 + i;
+              if (kp > qpos || kp >= kv_limit) v[h][i] = __float_as_uint(-INFINITY);
+            }
           }
-          tmem_wait_st();
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(v[h][i]), __uint_as_float(v[h][i + 1]));
         }
       }
-      // the last KV tile may extend past the written cache: zero those V rows so
-      // that 0-probability keys cannot inject NaN/Inf through P V
-      if (kv0 + kTileK > kv_limit) {
-        w_ok = !*s_abort && mbar_wait(&v_full[st], par, p.err);
+      const float mxs = mx * kScaleLog2;
+      float alpha = 1.f;
+      if (mxs > m_run + kRescaleThreshold || m_run == -INFINITY) {
+        alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mxs);
+        m_run = mxs;
+      }
+      // pass 2: p = 2^(s*scale - m) (packed fp32x2 FMA), row sums (packed adds), bf16 pairs
+      // written over the columns already consumed
+      const uint64_t scale2 = f2_pack(__float_as_uint(kScaleLog2), __float_as_uint(kScaleLog2));
+      const uint64_t neg2 = f2_pack(__float_as_uint(-m_run), __float_as_uint(-m_run));
+      uint64_t acc2[2] = {0ull, 0ull};
+#pragma unroll
+      for (int c2 = 0; c2 < 4; c2 += 2) {
+        uint32_t v[2][32];
+        tmem_ld32(tS + c2 * 32, v[0]);
+        tmem_ld32(tS + c2 * 32 + 32, v[1]);
+        tmem_wait_ld_regs(v[0]);
+        tmem_wait_ld_regs(v[1]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (need_mask) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int kp = kv0 + (c2 + h) * 32 + i;
+              if (kp > qpos || kp >= kv_limit) v[h][i] = __float_as_uint(-INFINITY);
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const uint64_t e = f2_fma(f2_pack(v[h][i], v[h][i + 1]), scale2, neg2);
+            const float p0 = ex2_approx(f2_lo(e));
+            const float p1 = ex2_approx(f2_hi(e));
+            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+            v[h][i >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + (c2 + h) * 16, v[h]);  // columns [16c, 16c+16) were read already
+        }
+      }
+      const uint64_t acc = f2_add(acc2[0], acc2[1]);
+      const float sum_tile = f2_lo(acc) + f2_hi(acc);
+      l_run = l_run * alpha + sum_tile;
+      // O_X is stable here: S_X of this tile was issued only after the previous P.V completed
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld_regs(v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+          tmem_st32(tO + c * 32, v);
+        }
+      }
+      // The last KV tile may extend past the written cache: zero those V rows so that
+      // 0-probability keys cannot inject NaN/Inf through P.V. One warpgroup does it:
+      // tile 0's if tile 0 takes part in this KV tile (its P.V is issued first).
+      if (kv0 + kTileK > kv_limit && (X == 0 || j >= nk0)) {
+        w_ok = !*s_abort && mbar_wait(&v_full[st], (j >> 1) & 1, p.err);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         if (kv0 + r >= kv_limit) {
           uint4* v0 = reinterpret_cast<uint4*>(smem + kOffKV + st * kStageBytes + 2 * kHalf + r * 128);
@@ -266,25 +292,15 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int c = 0; c < 8; ++c) { v0[c] = make_uint4(0, 0, 0, 0); v1[c] = make_uint4(0, 0, 0, 0); }
         }
+        fence_proxy_async_smem();
       }
-      // P row r -> two 128-byte-swizzled K-major half tiles
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint8_t* rowp = sP + h * kHalf + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const int pc = c ^ (r & 7);
-          *reinterpret_cast<uint4*>(rowp + pc * 16) =
-              make_uint4(pk[h * 32 + c * 4], pk[h * 32 + c * 4 + 1], pk[h * 32 + c * 4 + 2], pk[h * 32 + c * 4 + 3]);
-        }
-      }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[X]);
     }
     // epilogue: O / l -> bf16
-    if (ok) {
-      bool w_ok = !*s_abort && mbar_wait(p_free, (n_kv - 1) & 1, p.err);
+    if (ok && nkx > 0) {
+      bool w_ok = !*s_abort && mbar_wait(&pv_done[X], (nkx - 1) & 1, p.err);
       if (__all_sync(0xffffffffu, w_ok)) {
         tc_fence_after();
         const float inv_l = 1.f / l_run;
@@ -294,8 +310,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
-          tmem_ld32(tmem_O + c * 32 + ((uint32_t)(quad * 32) << 16), v);
-          tmem_wait_ld();
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld_regs(v);
           if (store) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -311,7 +327,7 @@ __global__ void __launch_bounds__(192, 1)
       } else {
         *s_abort = 1;
       }
-    } else {
+    } else if (!ok) {
       *s_abort = 1;
     }
   }
@@ -344,7 +360,7 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
   }
   PrefillParams p;
   p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.s_max = s_max;
-  p.n_qtiles = (T + TQ - 1) / TQ;
+  p.n_cta_q = (T + 2 * TQ - 1) / (2 * TQ);
   p.start_pos = start_pos;
   p.out = out;
   p.ldo = ldo;
@@ -354,8 +370,8 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
     cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
     attr = true;
   }
-  dim3 grid(p.n_qtiles, Hkv, B);
-  attn_prefill_kernel<<<grid, 192, kPrefillSmem, s>>>(tmQ, tmK, tmV, p);
+  dim3 grid(p.n_cta_q, Hkv, B);
+  attn_prefill_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(tmQ, tmK, tmV, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention prefill launch failed: %s", cudaGetErrorString(e));

@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, r);
-        tmem_wait_ld();
+        tmem_wait_ld_regs(r);
         if (g.partial) {
           // split-K: raw fp32 partial sums, [ks][token][feature]
           if (!g.swap) {
