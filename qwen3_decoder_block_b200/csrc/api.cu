@@ -281,12 +281,30 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   g.ldo = nqkv;
   g.partial = b.gpart;
   g.partial_bytes = b.gpart ? kSplitKBytes : 0;
+  if (!g.swap) {
+    // prefill: QK-norm, RoPE and the KV-cache write run in the GEMM's epilogue on the
+    // fp32 accumulators (no bf16 round trip of q/k/v)
+    g.epi = kEpiQKRope;
+    g.force_bn = 256;
+    g.qk.T = T;
+    g.qk.Hq = c.n_q_heads;
+    g.qk.Hkv = c.n_kv_heads;
+    g.qk.s_max = kv.s_max;
+    g.qk.max_pos = c.max_pos;
+    g.qk.pos_base = pos;
+    g.qk.q_norm = w.q_norm;
+    g.qk.k_norm = w.k_norm;
+    g.qk.rope = rope;
+    g.qk.ck = kv.k;
+    g.qk.cv = kv.v;
+    g.qk.eps = c.rms_eps;
+  }
   {
     ProfScope ps("gemm_qkv", k.s);
     rc = launch_gemm(g, k.s, k.err);
   }
   if (rc) return rc;
-  {
+  if (g.swap) {
     ProfScope ps("qk_norm_rope", k.s);
     rc = launch_qk_norm_rope(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, w.q_norm, w.k_norm, rope, kv.k,
                              kv.v, kv.s_max, c.max_pos, c.rms_eps, k.err, k.s);

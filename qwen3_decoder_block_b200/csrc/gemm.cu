@@ -55,6 +55,7 @@ struct GemmParams {
   int n_groups;
   const int* group_offsets;
   int* err;
+  QKRopeArgs qk;
 };
 
 struct Tile {
@@ -184,6 +185,97 @@ __device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int 
   }
 }
 
+// Fused QKV epilogue for one 128-column head of a non-swap tile (one token row per
+// thread): per-head RMSNorm over the 128 fp32 accumulators, weights, rotate-half RoPE
+// at the token's absolute position, one bf16 rounding; q heads are written back in
+// place (row p of out), k and v heads go to the KV cache at [b][g][pos][:]
+// ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and RoPE).
+// All 32 lanes execute the tensor-memory loads; only valid rows store.
+__device__ __forceinline__ void qk_rope_head(const GemmParams& g, uint32_t taddr, int slot, int p, bool valid) {
+  const QKRopeArgs& a = g.qk;
+  int b = 0, pos = 0;
+  if (valid) {
+    b = p / a.T;
+    pos = a.pos_base[b] + (p - b * a.T);
+    if (pos < 0 || pos >= a.s_max || pos >= a.max_pos) {
+      record_error(g.err, kErrCapacity);
+      valid = false;
+    }
+  }
+  if (slot >= a.Hq + a.Hkv) {  // value head: straight to the cache
+    uint16_t* dst = a.cv + (((long long)b * a.Hkv + (slot - a.Hq - a.Hkv)) * a.s_max + pos) * 128;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t v[32];
+      tmem_ld32(taddr + c * 32, v);
+      tmem_wait_ld_regs(v);
+      if (valid) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          d4[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                             pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+      }
+    }
+    return;
+  }
+  const bool is_q = slot < a.Hq;
+  // pass 1: sum of squares over the head's 128 values
+  float ss = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t v[32];
+    tmem_ld32(taddr + c * 32, v);
+    tmem_wait_ld_regs(v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(v[i]), __uint_as_float(v[i]), ss);
+  }
+  const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+  const uint16_t* wn = is_q ? a.q_norm : a.k_norm;
+  uint16_t* dst = is_q ? static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + (long long)slot * 128
+                       : a.ck + (((long long)b * a.Hkv + (slot - a.Hq)) * a.s_max + pos) * 128;
+  const float* rp = a.rope + (long long)pos * 128;
+  // pass 2: dims d (first half) and d + 64 (second half) form one rotation pair
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t lo[32], hi[32];
+    tmem_ld32(taddr + c * 32, lo);
+    tmem_ld32(taddr + 64 + c * 32, hi);
+    tmem_wait_ld_regs(lo);
+    tmem_wait_ld_regs(hi);
+    if (valid) {
+      uint32_t olo[16], ohi[16];
+#pragma unroll
+      for (int i8 = 0; i8 < 4; ++i8) {
+        const uint4 wa = *reinterpret_cast<const uint4*>(wn + c * 32 + i8 * 8);
+        const uint4 wb = *reinterpret_cast<const uint4*>(wn + 64 + c * 32 + i8 * 8);
+        const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w}, wb_[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          const int i = i8 * 8 + e;
+          const int d = c * 32 + i;
+          const float4 cs = *reinterpret_cast<const float4*>(rp + d * 2);  // (cos_d, sin_d, cos_d+1, sin_d+1)
+          const float a0 = __uint_as_float(lo[i]) * r * bf16_lo(wa_[e / 2]);
+          const float a1 = __uint_as_float(lo[i + 1]) * r * bf16_hi(wa_[e / 2]);
+          const float b0 = __uint_as_float(hi[i]) * r * bf16_lo(wb_[e / 2]);
+          const float b1 = __uint_as_float(hi[i + 1]) * r * bf16_hi(wb_[e / 2]);
+          olo[i / 2] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
+          ohi[i / 2] = pack_bf16x2(a0 * cs.y + b0 * cs.x, a1 * cs.w + b1 * cs.z);
+        }
+      }
+      uint4* dlo = reinterpret_cast<uint4*>(dst + c * 32);
+      uint4* dhi = reinterpret_cast<uint4*>(dst + 64 + c * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        dlo[i] = make_uint4(olo[4 * i], olo[4 * i + 1], olo[4 * i + 2], olo[4 * i + 3]);
+        dhi[i] = make_uint4(ohi[4 * i], ohi[4 * i + 1], ohi[4 * i + 2], ohi[4 * i + 3]);
+      }
+    }
+  }
+}
+
 // --------------------------------------------------------------------------- kernel
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
@@ -307,6 +399,20 @@ __global__ void __launch_bounds__(192, 1)
       if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; break; }  // keep the warp converged
       tc_fence_after();
       const int row = quad * 32 + lane;
+      if (g.epi == kEpiQKRope) {
+        // non-swap only: the tile's BN columns are BN/128 whole heads
+        const int p = tl.p0 + row;
+#pragma unroll 1
+        for (int hh = 0; hh < BN / 128; ++hh) {
+          const int col0 = tl.q0 + hh * 128;
+          if (col0 >= tl.q_end) break;
+          qk_rope_head(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + hh * 128, col0 / 128, p,
+                       p < tl.p_end);
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[buf]);
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -461,6 +567,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   g.n_groups = d.n_groups;
   g.group_offsets = d.group_offsets;
   g.err = err;
+  g.qk = d.qk;
   g.k_splits = 1;
   g.kb_per_split = g.k_blocks;
   g.partial = nullptr;

@@ -10,6 +10,19 @@ enum Epilogue : int {
   kEpiStore = 0,   // out = acc (bf16 or f32)
   kEpiResid = 1,   // out = resid + acc (resid bf16 or f32; out bf16 or f32); may alias
   kEpiSwiglu = 2,  // operand rows interleaved in 16-row gate/up blocks: out = silu(g) * u, bf16
+  kEpiQKRope = 3,  // fused QKV epilogue: per-head QK RMSNorm + RoPE (q in place), k/v to the cache
+};
+
+// Arguments of the fused QKV epilogue (non-swap GEMM over [q heads | k heads | v heads]).
+struct QKRopeArgs {
+  int T = 1, Hq = 0, Hkv = 0, s_max = 0, max_pos = 0;
+  const int* pos_base = nullptr;  // [B]: token t of sequence b is at pos_base[b] + t
+  const uint16_t* q_norm = nullptr;
+  const uint16_t* k_norm = nullptr;
+  const float* rope = nullptr;    // [max_pos][64][2] (cos, sin)
+  uint16_t* ck = nullptr;         // [B][Hkv][s_max][128]
+  uint16_t* cv = nullptr;
+  float eps = 1e-6f;
 };
 
 // D[p][q] = sum_k P[p][k] * Q[q][k]; both operands bf16, K-major (row-major [rows, K]).
@@ -35,6 +48,7 @@ struct GemmDesc {
   int n_groups = 0;
   const int* group_offsets = nullptr;  // device, n_groups + 1 entries
   int force_bn = 0;                    // 0 = automatic
+  QKRopeArgs qk;                       // kEpiQKRope only
   float* partial = nullptr;            // optional split-K scratch (fp32)
   size_t partial_bytes = 0;
 };

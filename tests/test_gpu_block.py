@@ -46,7 +46,8 @@ def _prefill_case(q3, cfg, B, T, starts, seed, s_extra=13):
     return from_gpu_bf16(xg), np.concatenate(refs), k, v, kref
 
 
-@pytest.mark.parametrize("B,T,starts", [(1, 16, [0]), (2, 77, [0, 50]), (1, 300, [0]), (3, 5, [0, 1, 200])])
+@pytest.mark.parametrize("B,T,starts", [(1, 16, [0]), (2, 77, [0, 50]), (1, 300, [0]), (3, 5, [0, 1, 200]),
+                                        (2, 200, [0, 37]), (3, 130, [0, 5, 900])])
 def test_block_prefill(q3, B, T, starts):
     cfg = q3.config_qwen3_0_6b()
     got, ref, k, v, kref = _prefill_case(q3, cfg, B, T, starts, seed=1000)
