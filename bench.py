@@ -88,36 +88,65 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- model set-up
-def build_model(q3, cfg, seed, torch):
-    """Random Qwen3-0.6B weights drawn on the device straight into the packed layouts
-    (identical values to drawing the pages' layouts and calling the pack helpers)."""
+def _filler(seed):
     from qwen3_decoder_block_b200 import synth
-    H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
-    bf = dict(dtype=torch.bfloat16, device="cuda")
 
     def fill(t, tid, mean, std, n0=1, n1=1, n2=None, s0=0, s1=0, offset=0):
         n2 = t.numel() if n2 is None else n2
         synth.normal_bf16_device(t.data_ptr() + 2 * offset, n0, n1, n2, s0, s1, seed, tid, mean, std)
+    return fill
 
-    layers, keep = [], []
-    for l in range(cfg.n_layers):
-        tid = lambda w: synth.layer_tid(l, w)
-        in_norm = torch.empty(H, **bf); fill(in_norm, tid(synth.L_IN_NORM), synth.NORM_MEAN, synth.NORM_STD)
-        post_norm = torch.empty(H, **bf); fill(post_norm, tid(synth.L_POST_NORM), synth.NORM_MEAN, synth.NORM_STD)
-        qn = torch.empty(D, **bf); fill(qn, tid(synth.L_Q_NORM), synth.NORM_MEAN, synth.NORM_STD)
-        kn = torch.empty(D, **bf); fill(kn, tid(synth.L_K_NORM), synth.NORM_MEAN, synth.NORM_STD)
-        wqkv = torch.empty(((hq + 2 * hkv) * D, H), **bf)
-        fill(wqkv, tid(synth.L_WQ), 0.0, synth.W_STD, n2=hq * D * H)
-        fill(wqkv, tid(synth.L_WK), 0.0, synth.W_STD, n2=hkv * D * H, offset=hq * D * H)
-        fill(wqkv, tid(synth.L_WV), 0.0, synth.W_STD, n2=hkv * D * H, offset=(hq + hkv) * D * H)
-        wo = torch.empty((H, hq * D), **bf); fill(wo, tid(synth.L_WO), 0.0, synth.W_STD)
+
+def build_layer(q3, cfg, seed, l, torch, moe=False):
+    """Random weights of one layer drawn on the device straight into the packed layouts
+    (identical values to drawing the pages' layouts and calling the pack helpers)."""
+    from qwen3_decoder_block_b200 import synth
+    H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    fill = _filler(seed)
+    tid = lambda w: synth.layer_tid(l, w)
+    in_norm = torch.empty(H, **bf); fill(in_norm, tid(synth.L_IN_NORM), synth.NORM_MEAN, synth.NORM_STD)
+    post_norm = torch.empty(H, **bf); fill(post_norm, tid(synth.L_POST_NORM), synth.NORM_MEAN, synth.NORM_STD)
+    qn = torch.empty(D, **bf); fill(qn, tid(synth.L_Q_NORM), synth.NORM_MEAN, synth.NORM_STD)
+    kn = torch.empty(D, **bf); fill(kn, tid(synth.L_K_NORM), synth.NORM_MEAN, synth.NORM_STD)
+    wqkv = torch.empty(((hq + 2 * hkv) * D, H), **bf)
+    fill(wqkv, tid(synth.L_WQ), 0.0, synth.W_STD, n2=hq * D * H)
+    fill(wqkv, tid(synth.L_WK), 0.0, synth.W_STD, n2=hkv * D * H, offset=hq * D * H)
+    fill(wqkv, tid(synth.L_WV), 0.0, synth.W_STD, n2=hkv * D * H, offset=(hq + hkv) * D * H)
+    wo = torch.empty((H, hq * D), **bf); fill(wo, tid(synth.L_WO), 0.0, synth.W_STD)
+    keep = [in_norm, post_norm, qn, kn, wqkv, wo]
+    kw = dict(in_norm=in_norm, w_qkv=wqkv, q_norm=qn, k_norm=kn, w_o=wo, post_norm=post_norm)
+    if moe:
+        E, Im = cfg.n_experts, cfg.moe_intermediate
+        router = torch.empty((E, H), **bf); fill(router, tid(synth.L_ROUTER), 0.0, synth.W_STD)
+        gu_pages = torch.empty((E, 2 * Im, H), **bf); fill(gu_pages, tid(synth.L_MOE_GATE_UP), 0.0, synth.W_STD)
+        gu = torch.empty_like(gu_pages)
+        q3.pack_moe_gate_up(E, Im, H, gu_pages, gu)
+        down = torch.empty((E, H, Im), **bf); fill(down, tid(synth.L_MOE_DOWN), 0.0, synth.W_STD)
+        torch.cuda.synchronize()
+        del gu_pages
+        keep += [router, gu, down]
+        kw.update(router=router, moe_gate_up=gu, moe_down=down)
+    else:
         wgu = torch.empty((2 * I, H), **bf)
         fill(wgu, tid(synth.L_WGATE), 0.0, synth.W_STD, n0=I // 16, n1=16, n2=H, s0=32 * H, s1=H)
         fill(wgu, tid(synth.L_WUP), 0.0, synth.W_STD, n0=I // 16, n1=16, n2=H, s0=32 * H, s1=H, offset=16 * H)
         wd = torch.empty((H, I), **bf); fill(wd, tid(synth.L_WDOWN), 0.0, synth.W_STD)
-        keep += [in_norm, post_norm, qn, kn, wqkv, wo, wgu, wd]
-        layers.append(q3.layer_weights(in_norm=in_norm, w_qkv=wqkv, q_norm=qn, k_norm=kn, w_o=wo,
-                                       post_norm=post_norm, w_gate_up=wgu, w_down=wd))
+        keep += [wgu, wd]
+        kw.update(w_gate_up=wgu, w_down=wd)
+    return q3.layer_weights(**kw), keep
+
+
+def build_model(q3, cfg, seed, torch):
+    from qwen3_decoder_block_b200 import synth
+    H = cfg.hidden
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    fill = _filler(seed)
+    layers, keep = [], []
+    for l in range(cfg.n_layers):
+        w, k = build_layer(q3, cfg, seed, l, torch)
+        layers.append(w)
+        keep += k
     embed = torch.empty((cfg.vocab, H), **bf); fill(embed, synth.TID_EMBED, 0.0, synth.W_STD)
     fnorm = torch.empty(H, **bf); fill(fnorm, synth.TID_FINAL_NORM, synth.NORM_MEAN, synth.NORM_STD)
     keep += [embed, fnorm]
@@ -346,6 +375,65 @@ def run_decode(q3, torch, args, peaks):
     }
 
 
+def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
+    """One decoder block prefill (dense or MoE) timed with CUDA events: returns tokens/s,
+    time per call and the algorithmic TFLOP/s of the whole block."""
+    from qwen3_decoder_block_b200 import synth
+    if moe:
+        cfg = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
+    else:
+        cfg = q3.config_qwen3_0_6b()
+    H, D, hq, hkv = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads
+    w, keep = build_layer(q3, cfg, seed, 0, torch, moe=moe)
+    x0 = torch.empty((B * T, H), dtype=torch.bfloat16, device="cuda")
+    synth.normal_bf16_device(x0.data_ptr(), 1, 1, x0.numel(), 0, 0, seed, synth.TID_X, 0.0, 1.0)
+    x = x0.clone()
+    k = torch.empty((B, hkv, T, D), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    kv = q3.kv_layer(k, v, T)
+    rope = torch.empty(q3.rope_table_bytes(cfg) // 4, dtype=torch.float32, device="cuda")
+    q3.rope_table(cfg, rope)
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    op = q3.OP_MOE_BLOCK if moe else q3.OP_BLOCK_PREFILL
+    ws = torch.empty(q3.workspace_size(cfg, op, B, T, T), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def call():
+        x.copy_(x0)
+        if moe:
+            q3.moe_block(cfg, w, x, B, T, pos, kv, rope, ws, stream=stream)
+        else:
+            q3.block_prefill(cfg, w, x, B, T, pos, kv, rope, ws, stream)
+
+    reps = reps or max(3, args.steps)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    q3.profile_begin(400)
+    call()
+    recs = q3.profile_end(stream)
+    assert q3.check_device_error() == 0
+    M = B * T
+    lin = 2 * M * (H * (hq + 2 * hkv) * D + hq * D * H)
+    attn = 4 * D * hq * B * T * (T + 1) // 2
+    if moe:
+        ffn = 2 * M * (H * cfg.n_experts + cfg.top_k * 3 * H * cfg.moe_intermediate)
+    else:
+        ffn = 2 * M * 3 * H * cfg.intermediate
+    flops = lin + attn + ffn
+    kern, _ = summarize_profile(recs, 1)
+    return {"workload": name, "tokens_per_s": M / (ms * 1e-3), "ms_per_call": ms,
+            "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_tflop": flops / 1e12,
+            "kernels_ms": {kk: round(vv["ms_per_step"], 4) for kk, vv in kern.items()}}
+
+
 # --------------------------------------------------------------------------- oracle timing
 def oracle_sample(T_s: int, seed: int = SEED_PREFILL):
     """Times the fp64 oracle on one sequence of T_s tokens of the prefill workload
@@ -400,6 +488,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--oracle-tokens", type=int, default=2048)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -446,6 +535,17 @@ def main():
     if not args.no_decode and rank == 0:
         torch.cuda.empty_cache()
         dec = run_decode(q3, torch, args, peaks)
+    others = None
+    if rank == 0 and not args.no_configs:
+        torch.cuda.empty_cache()
+        others = {
+            "c0": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T16", 1, 16, 1000,
+                                   reps=200),
+            "c3": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T32768", 1, 32768, 1003),
+            "c4": run_single_layer(q3, torch, args, "MoE block prefill (hidden 2048, 32/4 heads, 128 experts x "
+                                   "768, top-8), B1 x T4096", 1, 4096, 1004, moe=True),
+        }
+        torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.oracle_tokens)
@@ -459,7 +559,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random weights and token ids)",
             "config": config, "e2e": pre["e2e"], "roofline": pre["roofline"], "cpu_baseline": cpu,
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "attention": pre["attention"],
-            "kernels": pre["kernels"], "decode": dec}
+            "kernels": pre["kernels"], "decode": dec, "configs": others}
     print(json.dumps(line))
 
 

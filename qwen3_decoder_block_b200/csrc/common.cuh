@@ -266,7 +266,14 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float f) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// z * sigmoid(z) with the exponential and the reciprocal on the special-function unit
+// (a few ulp, far below the bf16 rounding of the outputs that use it).
+__device__ __forceinline__ float silu_f(float z) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(z * -1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return z * r;
+}
 
 // Packed fp32x2 arithmetic (two lanes of fp32 in one 64-bit register).
 __device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
