@@ -232,6 +232,15 @@ int qwen3_op_qk_norm_rope(const qwen3_config* cfg, qwen3_bf16* qkv, long long ld
                           const int* pos_base, const qwen3_bf16* q_norm, const qwen3_bf16* k_norm,
                           const qwen3_kv_layer* kv, const float* rope, void* stream);
 
+/* The prefill QKV projection with the QK-norm/RoPE/KV-write step fused into its epilogue
+ * (the form qwen3_block_prefill uses): acc = h . w_qkv^T in fp32; q heads are normalised,
+ * rotated and written to qkv [B*T, (Hq+2Hkv)*D] (bf16, same columns); k heads (normalised,
+ * rotated) and v heads go straight to kv at their positions. The k/v columns of qkv are not
+ * written. h [B*T, H] bf16; positions as qwen3_op_qk_norm_rope. */
+int qwen3_op_gemm_qkv_rope(const qwen3_config* cfg, const qwen3_bf16* h, const qwen3_bf16* w_qkv, qwen3_bf16* qkv,
+                           int B, int T, const int* pos_base, const qwen3_bf16* q_norm, const qwen3_bf16* k_norm,
+                           const qwen3_kv_layer* kv, const float* rope, void* stream);
+
 /* Causal GQA prefill attention: queries from qkv (already normed/rotated q heads), keys and
  * values from kv positions 0..start_pos[b]+t; o [B*T, Hq*D] (stride ldo), head-major columns. */
 int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B, int T,

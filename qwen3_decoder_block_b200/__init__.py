@@ -69,6 +69,7 @@ _SIGS = {
     "qwen3_op_rmsnorm": ([_vp, _i, _ll, _vp, _vp, _ll, _i, _i, _f, _vp], _i),
     "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _vp, _sz, _vp], _i),
     "qwen3_op_qk_norm_rope": ([_P(Config), _vp, _ll, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
+    "qwen3_op_gemm_qkv_rope": ([_P(Config), _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
     "qwen3_op_attention_prefill": ([_P(Config), _vp, _ll, _i, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_attention_decode": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp, _sz, _vp], _i),
     "qwen3_op_attention_decode_noalloc": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
@@ -241,6 +242,12 @@ def op_qk_norm_rope(cfg, qkv, B, T, pos_base, q_norm, k_norm, kv, rope, ldqkv=No
     ld = ldqkv or (cfg.n_q_heads + 2 * cfg.n_kv_heads) * cfg.head_dim
     _check(lib.qwen3_op_qk_norm_rope(ctypes.byref(cfg), _ptr(qkv), ld, B, T, _ptr(pos_base), _ptr(q_norm),
                                      _ptr(k_norm), ctypes.byref(kv), _ptr(rope), _stream(stream)), "op_qk_norm_rope")
+
+
+def op_gemm_qkv_rope(cfg, h, w_qkv, qkv, B, T, pos_base, q_norm, k_norm, kv, rope, stream=None) -> None:
+    _check(lib.qwen3_op_gemm_qkv_rope(ctypes.byref(cfg), _ptr(h), _ptr(w_qkv), _ptr(qkv), B, T, _ptr(pos_base),
+                                      _ptr(q_norm), _ptr(k_norm), ctypes.byref(kv), _ptr(rope), _stream(stream)),
+           "op_gemm_qkv_rope")
 
 
 def op_attention_prefill(cfg, qkv, B, T, start_pos, kv, o, ldqkv=None, ldo=None, stream=None) -> None:

@@ -882,6 +882,44 @@ int qwen3_op_qk_norm_rope(const qwen3_config* c, qwen3_bf16* qkv, long long ldqk
                                     static_cast<cudaStream_t>(stream)));
 }
 
+int qwen3_op_gemm_qkv_rope(const qwen3_config* c, const qwen3_bf16* h, const qwen3_bf16* w_qkv, qwen3_bf16* qkv,
+                           int B, int T, const int* pos_base, const qwen3_bf16* q_norm, const qwen3_bf16* k_norm,
+                           const qwen3_kv_layer* kv, const float* rope, void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(h && w_qkv && qkv && pos_base && q_norm && k_norm && rope, QWEN3_EINVAL, "gemm_qkv_rope: NULL pointer");
+  Q3_CHECK(aligned16(h) && aligned16(w_qkv) && aligned16(qkv) && aligned16(q_norm) && aligned16(k_norm) &&
+               aligned16(rope),
+           QWEN3_EALIGN, "gemm_qkv_rope: misaligned pointer");
+  Q3_CHECK(B > 0 && T > 0, QWEN3_EINVAL, "gemm_qkv_rope: B and T must be positive");
+  if ((rc = check_kv(*c, kv, T))) return rc;
+  if ((rc = check_device())) return rc;
+  const int H = c->hidden, nqkv = (c->n_q_heads + 2 * c->n_kv_heads) * c->head_dim;
+  GemmDesc g;
+  g.swap = false;
+  g.K = H;
+  g.P = h; g.p_rows = B * T; g.ldp = H;
+  g.Q = w_qkv; g.q_rows = nqkv; g.ldq = H;
+  g.epi = kEpiQKRope;
+  g.force_bn = 256;
+  g.out = qkv;
+  g.ldo = nqkv;
+  g.qk.T = T;
+  g.qk.Hq = c->n_q_heads;
+  g.qk.Hkv = c->n_kv_heads;
+  g.qk.s_max = kv->s_max;
+  g.qk.max_pos = c->max_pos;
+  g.qk.pos_base = pos_base;
+  g.qk.q_norm = q_norm;
+  g.qk.k_norm = k_norm;
+  g.qk.rope = rope;
+  g.qk.ck = kv->k;
+  g.qk.cv = kv->v;
+  g.qk.eps = c->rms_eps;
+  return finish(launch_gemm(g, static_cast<cudaStream_t>(stream), device_error_word()));
+}
+
 int qwen3_op_attention_prefill(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B, int T,
                                const int* start_pos, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                                void* stream) {

@@ -101,6 +101,25 @@ def case_lm_head(reps):
     return _gemm(reps, 8192, 151936, 1024, out_f32=True)
 
 
+def case_gemm_qkv_fused(reps, B=4, T=2048):
+    """c1 QKV projection with the fused QK-norm + RoPE + KV-write epilogue (one block prefill
+    minus the rest): M8192, N4096, K1024, measured through the block call's first GEMM."""
+    cfg = q3.config_qwen3_0_6b()
+    h = _bf16((B * T, 1024), 13)
+    w = _bf16((4096, 1024), 14, 0.02)
+    qkv = torch.empty((B * T, 4096), dtype=torch.bfloat16, device="cuda")
+    qn, kn = _bf16((128,), 15), _bf16((128,), 16)
+    k = torch.empty((B, 8, T, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    kv = q3.kv_layer(k, v, T)
+    rope = torch.empty(q3.rope_table_bytes(cfg) // 4, dtype=torch.float32, device="cuda")
+    q3.rope_table(cfg, rope)
+    pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+    ms = _time(lambda: q3.op_gemm_qkv_rope(cfg, h, w, qkv, B, T, pos, qn, kn, kv, rope), reps)
+    flops = 2 * B * T * 4096 * 1024
+    return {"ms": ms, "tflops": flops / ms / 1e9, "flops": flops}
+
+
 def case_gemm_o_decode(reps):
     """c2 o_proj: M64 (swap), N1024, K2048, fp32 residual epilogue."""
     return _gemm(reps, 64, 1024, 2048, epi=q3.EPI_RESID, out_f32=True, resid=True)

@@ -172,6 +172,37 @@ def test_qk_norm_rope(q3):
         assert bool(torch.isnan(k[b][:, :starts[b]].float()).all()) and bool(torch.isnan(k[b][:, starts[b] + T:].float()).all())
 
 
+@pytest.mark.parametrize("B,T,starts", [(1, 300, [0]), (2, 200, [17, 3000]), (3, 129, [0, 1, 40000 - 140])])
+def test_gemm_qkv_rope_fused(q3, B, T, starts):
+    """QKV GEMM whose epilogue does QK-norm + RoPE + KV write on the fp32 accumulators."""
+    cfg = q3.config_qwen3_0_6b()
+    D, hq, hkv, H = cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.hidden
+    nqkv = (hq + 2 * hkv) * D
+    s_max = max(starts) + T + 3
+    h = Tensor(SEED, 91, (B * T, H))
+    w = Tensor(SEED, 92, (nqkv, H), 0.0, 0.02)
+    qn = Tensor(SEED, 93, (D,), 1.0, 0.1)
+    kn = Tensor(SEED, 94, (D,), 1.0, 0.1)
+    k, v, kv = kv_cache(cfg, B, s_max)
+    qkv = torch.full((B * T, nqkv), float("nan"), dtype=torch.bfloat16, device="cuda")
+    pos = torch.tensor(starts, dtype=torch.int32, device="cuda")
+    q3.op_gemm_qkv_rope(cfg, h.gpu, w.gpu, qkv, B, T, pos, qn.gpu, kn.gpu, kv, rope_gpu(cfg))
+    assert_device_ok()
+    acc = h.f @ w.f.T
+    got_q = from_gpu_bf16(qkv[:, :hq * D])
+    for b in range(B):
+        rows = acc[b * T:(b + 1) * T]
+        p = starts[b] + np.arange(T)
+        q = R.rope_rotate_half(R.rms_norm(rows[:, :hq * D].reshape(T, hq, D), qn.f, 1e-6), p, 1e6)
+        kk = R.rope_rotate_half(R.rms_norm(rows[:, hq * D:(hq + hkv) * D].reshape(T, hkv, D), kn.f, 1e-6), p, 1e6)
+        vv = rows[:, (hq + hkv) * D:].reshape(T, hkv, D)
+        gq = got_q[b * T:(b + 1) * T].reshape(T, hq, D)
+        gk = from_gpu_bf16(k[b][:, starts[b]:starts[b] + T]).transpose(1, 0, 2)
+        gv = from_gpu_bf16(v[b][:, starts[b]:starts[b] + T]).transpose(1, 0, 2)
+        for got, ref in ((gq, q), (gk, kk), (gv, vv)):
+            assert np.all(np.abs(got - ref) <= bf16_tol(ref, abs_=1e-4)), max_abs(got, ref)
+
+
 def _attention_oracle(cfg, qf, kf, vf, starts, B, T):
     """qf [B*T, Hq, D]; kf, vf [B, Hkv, S, D] cache contents; returns [B*T, Hq, D]."""
     out = []
