@@ -36,9 +36,10 @@ struct GemmCfg {
   static constexpr uint32_t Q_BYTES = BN * BK * 2;
   static constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
+  static constexpr uint32_t STAGING_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x 32x32 fp32
   static constexpr uint32_t BAR_BYTES = 256;
   static size_t smem_bytes(int n_groups) {
-    return 1024 + (size_t)STAGES * STAGE_BYTES + BAR_BYTES + 8 * (size_t)(n_groups + 2);
+    return 1024 + (size_t)STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 8 * (size_t)(n_groups + 2);
   }
 };
 
@@ -48,6 +49,7 @@ struct GemmParams {
   int k_splits, kb_per_split;  // split-K: tile t covers k-blocks [ks*kb_per_split, ...)
   float* partial;              // split-K partials [k_splits][tokens][features] (fp32)
   int epi, resid_f32, out_f32, swap;
+  int tma_store;  // non-swap store/residual epilogues: stage in shared memory, TMA tile store
   void* out;
   long long ldo;
   const void* resid;
@@ -153,6 +155,48 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams& g, int p, int 
     for (int j = 0; j < 4; ++j)
       dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+  }
+}
+
+// TMA-store epilogue: this thread's row (p < 0: outside the output, values unused) of a
+// 32 x 32 chunk goes into a swizzled staging tile (128-byte swizzle for fp32 rows of
+// 128 bytes, 64-byte swizzle for bf16 rows of 64 bytes) that one TMA store writes out.
+__device__ __forceinline__ void stage_row_chunk(const GemmParams& g, int p, int q, const uint32_t (&r)[32],
+                                                uint8_t* stg, int lane) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+  if (g.epi == kEpiResid && p >= 0) {
+    if (g.resid_f32) {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 a = src[j];
+        v[4 * j] += a.x; v[4 * j + 1] += a.y; v[4 * j + 2] += a.z; v[4 * j + 3] += a.w;
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint4 a = src[j];
+        v[8 * j + 0] += bf16_lo(a.x); v[8 * j + 1] += bf16_hi(a.x);
+        v[8 * j + 2] += bf16_lo(a.y); v[8 * j + 3] += bf16_hi(a.y);
+        v[8 * j + 4] += bf16_lo(a.z); v[8 * j + 5] += bf16_hi(a.z);
+        v[8 * j + 6] += bf16_lo(a.w); v[8 * j + 7] += bf16_hi(a.w);
+      }
+    }
+  }
+  if (g.out_f32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+          make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                     pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
   }
 }
 
@@ -280,18 +324,19 @@ __device__ __forceinline__ void qk_rope_head(const GemmParams& g, uint32_t taddr
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                   const GemmParams g) {
+                   const __grid_constant__ CUtensorMap tmO, const GemmParams g) {
   using C = GemmCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + C::STAGING_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_prefix = reinterpret_cast<int*>(smem + C::STAGES * C::STAGE_BYTES + C::BAR_BYTES);
+  int* s_prefix = reinterpret_cast<int*>(staging + C::STAGING_BYTES + C::BAR_BYTES);
   int* s_off = s_prefix + (g.n_groups + 1);  // only used in grouped mode (aliases past prefix)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -391,6 +436,7 @@ __global__ void __launch_bounds__(192, 1)
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32) are reachable from this warp
     int local = 0;
+    int sbuf = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
       const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
       const int buf = local & 1;
@@ -438,6 +484,22 @@ __global__ void __launch_bounds__(192, 1)
                 g.partial[((long long)tl.ks * g.q_rows + q) * g.p_rows + p] = __uint_as_float(r[j]);
             }
           }
+        } else if (g.tma_store) {
+          const int q = tl.q0 + c * 32;
+          if (q < tl.q_end) {  // warp-uniform
+            const int p = tl.p0 + row;
+            uint8_t* stg = staging + ((warp - 2) * 2 + sbuf) * 4096;
+            if (lane == 0) bulk_wait_read<1>();  // the store that used this buffer has read it
+            __syncwarp();
+            stage_row_chunk(g, p < tl.p_end ? p : -1, q, r, stg, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmO, stg, q, tl.p0 + quad * 32);
+              bulk_commit();
+            }
+            sbuf ^= 1;
+          }
         } else if (!g.swap) {
           const int p = tl.p0 + row, q = tl.q0 + c * 32;
           if (p < tl.p_end && q < tl.q_end) store_row_chunk(g, p, q, r);
@@ -449,6 +511,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&tempty[buf]);
     }
+    if (g.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -534,6 +597,23 @@ int make_tmap_3d(CUtensorMap* map, const void* base, long long inner, long long 
   return r == CUDA_SUCCESS ? 0 : -2;
 }
 
+// Output tensor map for the TMA-store epilogue: [rows, cols] fp32 or bf16, box 32 x 32,
+// 128-byte (fp32) or 64-byte (bf16) swizzle matching stage_row_chunk.
+static int make_tmap_out(CUtensorMap* map, void* base, long long rows, long long cols, long long ld, bool f32) {
+  auto enc = get_encode();
+  if (!enc) return -1;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? 0 : -2;
+}
+
 template <int BN>
 static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   using C = GemmCfg<BN>;
@@ -585,6 +665,13 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
       g.partial = d.partial;
     }
   }
+  // TMA-store epilogue for the plain non-swap store / residual epilogues
+  CUtensorMap tmO = tmP;
+  g.tma_store = 0;
+  if (!d.swap && d.n_groups == 0 && g.k_splits == 1 && (d.epi == kEpiStore || d.epi == kEpiResid) &&
+      (reinterpret_cast<uintptr_t>(d.out) & 15) == 0 && (d.ldo * (d.out_f32 ? 4 : 2)) % 16 == 0) {
+    if (make_tmap_out(&tmO, d.out, d.p_rows, d.q_rows, d.ldo, d.out_f32) == 0) g.tma_store = 1;
+  }
   const size_t smem = C::smem_bytes(d.n_groups);
   static bool attr_set[4] = {false, false, false, false};
   static std::mutex mu;
@@ -604,7 +691,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
     grid = (int)(tiles < num_sms() ? tiles : num_sms());
   }
   if (grid <= 0) return 0;
-  gemm_tc_kernel<BN><<<grid, 192, smem, s>>>(tmP, tmQ, g);
+  gemm_tc_kernel<BN><<<grid, 192, smem, s>>>(tmP, tmQ, tmO, g);
   if (g.k_splits > 1) {
     const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
     const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);
