@@ -229,13 +229,15 @@ __device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int 
   }
 }
 
-// Fused QKV epilogue for one 128-column head of a non-swap tile (one token row per
-// thread): per-head RMSNorm over the 128 fp32 accumulators, weights, rotate-half RoPE
-// at the token's absolute position, one bf16 rounding; q heads are written back in
-// place (row p of out), k and v heads go to the KV cache at [b][g][pos][:]
-// ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and RoPE).
-// All 32 lanes execute the tensor-memory loads; only valid rows store.
-__device__ __forceinline__ void qk_rope_head(const GemmParams& g, uint32_t taddr, int slot, int p, bool valid) {
+// Fused QKV epilogue for the two 128-column heads of a non-swap 256-column tile (one
+// token row per thread): per-head RMSNorm over the 128 fp32 accumulators, weights,
+// rotate-half RoPE at the token's absolute position, one bf16 rounding; q heads are
+// written back in place (row p of out), k and v heads go to the KV cache at
+// [b][g][pos][:] ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and
+// RoPE). The row's cos/sin values are read once for both heads. All 32 lanes execute
+// the tensor-memory loads; only valid rows store.
+__device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr, int slot0, int n_heads, int p,
+                                             bool valid) {
   const QKRopeArgs& a = g.qk;
   int b = 0, pos = 0;
   if (valid) {
@@ -246,67 +248,71 @@ __device__ __forceinline__ void qk_rope_head(const GemmParams& g, uint32_t taddr
       valid = false;
     }
   }
-  if (slot >= a.Hq + a.Hkv) {  // value head: straight to the cache
-    uint16_t* dst = a.cv + (((long long)b * a.Hkv + (slot - a.Hq - a.Hkv)) * a.s_max + pos) * 128;
+  // pass 1: per-head sum of squares (value heads skip the norm)
+  float rinv[2] = {0.f, 0.f};
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    if (hh >= n_heads || slot0 + hh >= a.Hq + a.Hkv) continue;  // warp-uniform
+    float ss = 0.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t v[32];
-      tmem_ld32(taddr + c * 32, v);
+      tmem_ld32(taddr + hh * 128 + c * 32, v);
       tmem_wait_ld_regs(v);
-      if (valid) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          d4[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]), __uint_as_float(v[8 * i + 1])),
-                             pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                             pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                             pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
-      }
+      for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(v[i]), __uint_as_float(v[i]), ss);
     }
-    return;
+    rinv[hh] = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
   }
-  const bool is_q = slot < a.Hq;
-  // pass 1: sum of squares over the head's 128 values
-  float ss = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t v[32];
-    tmem_ld32(taddr + c * 32, v);
-    tmem_wait_ld_regs(v);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(v[i]), __uint_as_float(v[i]), ss);
-  }
-  const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
-  const uint16_t* wn = is_q ? a.q_norm : a.k_norm;
-  uint16_t* dst = is_q ? static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + (long long)slot * 128
-                       : a.ck + (((long long)b * a.Hkv + (slot - a.Hq)) * a.s_max + pos) * 128;
   const float* rp = a.rope + (long long)pos * 128;
   // pass 2: dims d (first half) and d + 64 (second half) form one rotation pair
-#pragma unroll
+#pragma unroll 1
   for (int c = 0; c < 2; ++c) {
-    uint32_t lo[32], hi[32];
-    tmem_ld32(taddr + c * 32, lo);
-    tmem_ld32(taddr + 64 + c * 32, hi);
-    tmem_wait_ld_regs(lo);
-    tmem_wait_ld_regs(hi);
-    if (valid) {
+    float4 cs[16];  // (cos_d, sin_d, cos_d+1, sin_d+1) for d = 32c .. 32c+31
+#pragma unroll
+    for (int i = 0; i < 16; ++i) cs[i] = valid ? *reinterpret_cast<const float4*>(rp + (c * 32 + 2 * i) * 2)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      if (hh >= n_heads) break;
+      const int slot = slot0 + hh;
+      uint32_t lo[32], hi[32];
+      tmem_ld32(taddr + hh * 128 + c * 32, lo);
+      tmem_ld32(taddr + hh * 128 + 64 + c * 32, hi);
+      tmem_wait_ld_regs(lo);
+      tmem_wait_ld_regs(hi);
+      if (!valid) continue;
       uint32_t olo[16], ohi[16];
+      uint16_t* dst;
+      if (slot >= a.Hq + a.Hkv) {  // value head: straight to the cache
+        dst = a.cv + (((long long)b * a.Hkv + (slot - a.Hq - a.Hkv)) * a.s_max + pos) * 128;
 #pragma unroll
-      for (int i8 = 0; i8 < 4; ++i8) {
-        const uint4 wa = *reinterpret_cast<const uint4*>(wn + c * 32 + i8 * 8);
-        const uint4 wb = *reinterpret_cast<const uint4*>(wn + 64 + c * 32 + i8 * 8);
-        const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w}, wb_[4] = {wb.x, wb.y, wb.z, wb.w};
+        for (int i = 0; i < 16; ++i) {
+          olo[i] = pack_bf16x2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+          ohi[i] = pack_bf16x2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
+        }
+      } else {
+        const bool is_q = slot < a.Hq;
+        const uint16_t* wn = is_q ? a.q_norm : a.k_norm;
+        dst = is_q ? static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + (long long)slot * 128
+                   : a.ck + (((long long)b * a.Hkv + (slot - a.Hq)) * a.s_max + pos) * 128;
+        const float r = hh ? rinv[1] : rinv[0];
 #pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int i = i8 * 8 + e;
-          const int d = c * 32 + i;
-          const float4 cs = *reinterpret_cast<const float4*>(rp + d * 2);  // (cos_d, sin_d, cos_d+1, sin_d+1)
-          const float a0 = __uint_as_float(lo[i]) * r * bf16_lo(wa_[e / 2]);
-          const float a1 = __uint_as_float(lo[i + 1]) * r * bf16_hi(wa_[e / 2]);
-          const float b0 = __uint_as_float(hi[i]) * r * bf16_lo(wb_[e / 2]);
-          const float b1 = __uint_as_float(hi[i + 1]) * r * bf16_hi(wb_[e / 2]);
-          olo[i / 2] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
-          ohi[i / 2] = pack_bf16x2(a0 * cs.y + b0 * cs.x, a1 * cs.w + b1 * cs.z);
+        for (int i8 = 0; i8 < 4; ++i8) {
+          const uint4 wa = *reinterpret_cast<const uint4*>(wn + c * 32 + i8 * 8);
+          const uint4 wb = *reinterpret_cast<const uint4*>(wn + 64 + c * 32 + i8 * 8);
+          const uint32_t wa_[4] = {wa.x, wa.y, wa.z, wa.w}, wb_[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int i = i8 * 8 + e;
+            const float4 t = cs[i / 2];
+            const float a0 = __uint_as_float(lo[i]) * r * bf16_lo(wa_[e / 2]);
+            const float a1 = __uint_as_float(lo[i + 1]) * r * bf16_hi(wa_[e / 2]);
+            const float b0 = __uint_as_float(hi[i]) * r * bf16_lo(wb_[e / 2]);
+            const float b1 = __uint_as_float(hi[i + 1]) * r * bf16_hi(wb_[e / 2]);
+            olo[i / 2] = pack_bf16x2(a0 * t.x - b0 * t.y, a1 * t.z - b1 * t.w);
+            ohi[i / 2] = pack_bf16x2(a0 * t.y + b0 * t.x, a1 * t.w + b1 * t.z);
+          }
         }
       }
       uint4* dlo = reinterpret_cast<uint4*>(dst + c * 32);
@@ -448,13 +454,10 @@ __global__ void __launch_bounds__(192, 1)
       if (g.epi == kEpiQKRope) {
         // non-swap only: the tile's BN columns are BN/128 whole heads
         const int p = tl.p0 + row;
-#pragma unroll 1
-        for (int hh = 0; hh < BN / 128; ++hh) {
-          const int col0 = tl.q0 + hh * 128;
-          if (col0 >= tl.q_end) break;
-          qk_rope_head(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + hh * 128, col0 / 128, p,
+        const int heads = min(BN / 128, (tl.q_end - tl.q0) / 128);
+        if (heads > 0)
+          qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
                        p < tl.p_end);
-        }
         tc_fence_before();
         mbar_arrive(&tempty[buf]);
         continue;
