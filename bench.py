@@ -489,6 +489,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true")
+    ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
+                    help="prefill or decode alone (for profiler launch lists)")
     ap.add_argument("--oracle-tokens", type=int, default=2048)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
@@ -530,13 +532,17 @@ def main():
         torch.cuda.set_device(local)
     import qwen3_decoder_block_b200 as q3
 
+    if args.workload == "decode":
+        dec = run_decode(q3, torch, args, peaks)
+        print(json.dumps({"metric": METRIC, "workload": "decode only", "decode": dec}))
+        return
     pre = run_prefill(q3, torch, args, rank, world, dist, peaks)
     dec = None
-    if not args.no_decode and rank == 0:
+    if not args.no_decode and rank == 0 and args.workload == "all":
         torch.cuda.empty_cache()
         dec = run_decode(q3, torch, args, peaks)
     others = None
-    if rank == 0 and not args.no_configs:
+    if rank == 0 and not args.no_configs and args.workload == "all":
         torch.cuda.empty_cache()
         others = {
             "c0": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T16", 1, 16, 1000,
@@ -547,7 +553,7 @@ def main():
         }
         torch.cuda.empty_cache()
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "all":
         cpu = cpu_baseline(args.oracle_tokens)
     if dist:
         dist.barrier()

@@ -120,6 +120,16 @@ def case_gemm_qkv_fused(reps, B=4, T=2048):
     return {"ms": ms, "tflops": flops / ms / 1e9, "flops": flops}
 
 
+def case_gemm_o(reps):
+    """c1 o_proj with the fp32 residual epilogue: M8192, N1024, K2048."""
+    return _gemm(reps, 8192, 1024, 2048, epi=q3.EPI_RESID, out_f32=True, resid=True)
+
+
+def case_gemm_down(reps):
+    """c1 down projection with the fp32 residual epilogue: M8192, N1024, K3072."""
+    return _gemm(reps, 8192, 1024, 3072, epi=q3.EPI_RESID, out_f32=True, resid=True)
+
+
 def case_gemm_o_decode(reps):
     """c2 o_proj: M64 (swap), N1024, K2048, fp32 residual epilogue."""
     return _gemm(reps, 64, 1024, 2048, epi=q3.EPI_RESID, out_f32=True, resid=True)
