@@ -516,6 +516,238 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
   }
 }
 
+// ============================================================================
+// K4, pipelined form (1, 2 or 4 query heads per KV group). Persistent: one CTA per
+// SM walks the (sequence, group, 256-key split) items in a fixed order. A producer
+// warp streams each split's K and V rows as two 128-key halves into a 3-stage ring
+// of shared-memory buffers with bulk copies (the DMA engine, whole lines); 16 compute
+// warps take 8 keys each. Scores: lane l holds 4 head dims of the G queries, partial
+// dot products of the warp's 8 keys x G heads are reduced across lanes with a
+// transposing butterfly (lane l ends with value l). Softmax is online across the two
+// halves; P.V puts lane l on dims [4l, 4l+4). The 16 warps merge in shared memory and
+// the split's (max, sum, unnormalised o) goes to the workspace, as in the form above.
+// ============================================================================
+constexpr int kD3Warps = 16;             // compute warps
+constexpr int kD3Threads = 32 * (kD3Warps + 1);
+constexpr int kD3Half = 128;             // keys per stage
+constexpr int kD3Stages = 3;
+constexpr uint32_t kD3StageBytes = 2u * kD3Half * kHeadDim * 2;  // K then V: 64 KB
+
+template <int G>
+struct D3Smem {
+  static constexpr uint32_t kO = kD3Stages * kD3StageBytes;           // [16][G][128] fp32
+  static constexpr uint32_t kM = kO + kD3Warps * G * kHeadDim * 4;    // [16][G]
+  static constexpr uint32_t kL = kM + kD3Warps * G * 4;               // [16][G]
+  static constexpr uint32_t kBar = (kL + kD3Warps * G * 4 + 7) & ~7u;  // full[3], empty[3]
+  static constexpr uint32_t kAbort = kBar + 2 * kD3Stages * 8;
+  static constexpr uint32_t kBytes = kAbort + 16 + 128;
+};
+
+// Butterfly that reduces NV (power of two, <= 32) per-lane values across the warp:
+// afterwards lane l holds the full sum of value (l & (NV - 1)).
+template <int NV>
+__device__ __forceinline__ float transpose_reduce(float (&a)[NV], int lane) {
+#pragma unroll
+  for (int o = NV / 2; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float keep = upper ? a[i + o] : a[i];
+      const float send = upper ? a[i] : a[i + o];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float v = a[0];
+#pragma unroll
+  for (int o = NV; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void named_bar_compute() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kD3Warps * 32) : "memory");
+}
+
+template <int G>
+__global__ void __launch_bounds__(kD3Threads, 1) attn_decode_tma_kernel(
+    const uint16_t* __restrict__ qkv, long long ldqkv, int B, int Hq, int Hkv, const int* __restrict__ cache_len,
+    const uint16_t* __restrict__ ck, const uint16_t* __restrict__ cv, int s_max, int n_splits,
+    float* __restrict__ part, int* err) {
+  using L = D3Smem<G>;
+  constexpr int NV = 8 * G;  // 8 keys x G heads per warp
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  float* sO = reinterpret_cast<float*>(smem + L::kO);
+  float* sM = reinterpret_cast<float*>(smem + L::kM);
+  float* sL = reinterpret_cast<float*>(smem + L::kL);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* empty = full + kD3Stages;
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = B * Hkv * n_splits;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kD3Stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kD3Warps); }
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kD3Warps) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      for (int it = blockIdx.x; it < n_items && !*s_abort; it += gridDim.x) {
+        const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv;
+        const int n_total = cache_len[b] + 1;
+        if (n_total > s_max) continue;  // reported by the compute warps
+        const long long row0 = (long long)bg * s_max;
+        for (int h = 0; h < 2; ++h) {
+          const int k0 = split * 2 * kD3Half + h * kD3Half;
+          const int nk = min(kD3Half, n_total - k0);
+          if (nk <= 0) continue;
+          if (!mbar_wait(&empty[st], ph ^ 1, err)) { *s_abort = 1; break; }
+          uint8_t* base = smem + st * kD3StageBytes;
+          mbar_arrive_expect_tx(&full[st], 2u * nk * kHeadDim * 2);
+          bulk_load(base, ck + (row0 + k0) * kHeadDim, nk * kHeadDim * 2, &full[st]);
+          bulk_load(base + kD3StageBytes / 2, cv + (row0 + k0) * kHeadDim, nk * kHeadDim * 2, &full[st]);
+          ++issued;
+          if (++st == kD3Stages) { st = 0; ph ^= 1; }
+        }
+      }
+      // every copy issued lands before the CTA exits (normally all were consumed already)
+      for (long long i = issued > kD3Stages ? issued - kD3Stages : 0; i < issued; ++i)
+        mbar_wait(&full[i % kD3Stages], (uint32_t)((i / kD3Stages) & 1), err);
+    }
+    return;  // the producer warp takes no part in the compute warps' named barrier
+  }
+
+  // -------------------------------------------------------------------- compute
+  int st = 0;
+  uint32_t ph = 0;
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
+    const int n_total = cache_len[b] + 1;
+    const bool over = n_total > s_max;
+    if (over && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
+    // this lane's 4 dims of the G queries, pre-scaled into the exp2 domain
+    float qv[G][4];
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      const uint2 q2 = *reinterpret_cast<const uint2*>(qkv + (long long)b * ldqkv + (long long)(g * G + j) * kHeadDim +
+                                                      4 * lane);
+      qv[j][0] = bf16_lo(q2.x) * kScaleLog2; qv[j][1] = bf16_hi(q2.x) * kScaleLog2;
+      qv[j][2] = bf16_lo(q2.y) * kScaleLog2; qv[j][3] = bf16_hi(q2.y) * kScaleLog2;
+    }
+    float m[G], l[G], o[G][4];
+#pragma unroll
+    for (int j = 0; j < G; ++j) { m[j] = -INFINITY; l[j] = 0.f; o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f; }
+    for (int h = 0; h < 2 && !over; ++h) {
+      const int k0 = split * 2 * kD3Half + h * kD3Half;
+      const int nk = min(kD3Half, n_total - k0);
+      if (nk <= 0) continue;
+      const bool ok = !*s_abort && mbar_wait(&full[st], ph, err);
+      if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; }
+      const uint16_t* sK = reinterpret_cast<const uint16_t*>(smem + st * kD3StageBytes);
+      const uint16_t* sV = sK + kD3Half * kHeadDim;
+      const int kw = warp * 8;  // this warp's first key in the half
+      if (!*s_abort) {
+        // partial dot products: value index kk*G + j
+        float a[NV];
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          float k4[4] = {0.f, 0.f, 0.f, 0.f};
+          if (kw + kk < nk) {
+            const uint2 kr = *reinterpret_cast<const uint2*>(sK + (kw + kk) * kHeadDim + 4 * lane);
+            k4[0] = bf16_lo(kr.x); k4[1] = bf16_hi(kr.x); k4[2] = bf16_lo(kr.y); k4[3] = bf16_hi(kr.y);
+          }
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+            a[kk * G + j] = qv[j][0] * k4[0] + qv[j][1] * k4[1] + qv[j][2] * k4[2] + qv[j][3] * k4[3];
+        }
+        const float s = transpose_reduce<NV>(a, lane);
+        const int vidx = lane & (NV - 1);
+        const int my_key = vidx / G, my_j = vidx % G;
+        const bool valid = kw + my_key < nk;
+        // per-head max over the first NV lanes (lanes with the same head differ in bits >= log2 G)
+        float mh = valid ? s : -INFINITY;
+#pragma unroll
+        for (int off = G; off < NV; off <<= 1) mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, off));
+        float m_new[G], alpha[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float mj = __shfl_sync(0xffffffffu, mh, j);
+          m_new[j] = fmaxf(m[j], mj);
+          alpha[j] = (m[j] == -INFINITY) ? 0.f : exp2f(m[j] - m_new[j]);
+        }
+        float my_m = m_new[0];
+#pragma unroll
+        for (int j = 1; j < G; ++j) my_m = (my_j == j) ? m_new[j] : my_m;
+        const float p = (valid && my_m != -INFINITY) ? exp2f(s - my_m) : 0.f;
+        float ps = p;
+#pragma unroll
+        for (int off = G; off < NV; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          l[j] = l[j] * alpha[j] + __shfl_sync(0xffffffffu, ps, j);
+          m[j] = m_new[j];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) o[j][c] *= alpha[j];
+        }
+        // P.V: lane owns dims [4*lane, 4*lane+4)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          float pj[G];
+#pragma unroll
+          for (int j = 0; j < G; ++j) pj[j] = __shfl_sync(0xffffffffu, p, kk * G + j);
+          if (kw + kk < nk) {
+            const uint2 vr = *reinterpret_cast<const uint2*>(sV + (kw + kk) * kHeadDim + 4 * lane);
+            const float v0 = bf16_lo(vr.x), v1 = bf16_hi(vr.x), v2 = bf16_lo(vr.y), v3 = bf16_hi(vr.y);
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              o[j][0] += pj[j] * v0; o[j][1] += pj[j] * v1; o[j][2] += pj[j] * v2; o[j][3] += pj[j] * v3;
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+      if (++st == kD3Stages) { st = 0; ph ^= 1; }
+    }
+    // merge the 16 warps into this split's partial
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      *reinterpret_cast<float4*>(&sO[(warp * G + j) * kHeadDim + 4 * lane]) = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
+      if (lane == 0) { sM[warp * G + j] = m[j]; sL[warp * G + j] = l[j]; }
+    }
+    named_bar_compute();
+    float* my_part = part + ((long long)(b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
+    const long long head_stride = (long long)n_splits * (kHeadDim + 2);
+    for (int i = threadIdx.x; i < G * kHeadDim; i += kD3Warps * 32) {
+      const int j = i / kHeadDim, d = i % kHeadDim;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kD3Warps; ++w) M = fmaxf(M, sM[w * G + j]);
+      float acc = 0.f, Lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kD3Warps; ++w) {
+        const float mw = sM[w * G + j];
+        if (mw == -INFINITY) continue;
+        const float sc = exp2f(mw - M);
+        acc += sO[(w * G + j) * kHeadDim + d] * sc;
+        Lsum += sL[w * G + j] * sc;
+      }
+      my_part[j * head_stride + d] = acc;
+      if (d == 0) {
+        my_part[j * head_stride + kHeadDim] = M;
+        my_part[j * head_stride + kHeadDim + 1] = Lsum;
+      }
+    }
+    named_bar_compute();  // the next item overwrites sO / sM / sL
+  }
+}
+
 __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
                                          uint16_t* __restrict__ out, long long ldo) {
   const int bh = blockIdx.x;  // b * Hq + h
@@ -548,6 +780,35 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
   const int n_splits = decode_splits(s_max);
+  if (G == 1 || G == 2 || G == 4) {
+    // pipelined form: persistent CTAs, bulk copies into a 3-stage shared-memory ring
+    const long long items = (long long)B * Hkv * n_splits;
+    const int grid = (int)(items < num_sms() ? items : num_sms());
+    static bool attr[3] = {false, false, false};
+#define Q3_D3_CASE(GG, SLOT)                                                                                     \
+  case GG:                                                                                                       \
+    if (!attr[SLOT]) {                                                                                           \
+      cudaFuncSetAttribute(attn_decode_tma_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,              \
+                           D3Smem<GG>::kBytes);                                                                  \
+      attr[SLOT] = true;                                                                                         \
+    }                                                                                                            \
+    attn_decode_tma_kernel<GG><<<grid, kD3Threads, D3Smem<GG>::kBytes, s>>>(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, \
+                                                                           cv, s_max, n_splits, part, err);     \
+    break;
+    switch (G) {
+      Q3_D3_CASE(1, 0)
+      Q3_D3_CASE(2, 1)
+      Q3_D3_CASE(4, 2)
+    }
+#undef Q3_D3_CASE
+    attn_decode_merge_kernel<<<B * Hq, kHeadDim, 0, s>>>(part, Hq, n_splits, out, ldo);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
+      return -6;
+    }
+    return 0;
+  }
   dim3 grid(n_splits, Hkv, B);
   switch (G) {
 #define Q3_DEC_CASE(GG)                                                                                         \
