@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -80,6 +81,14 @@ int num_sms() {
     g_sm_count[d] = n > 0 ? n : 148;
   }
   return g_sm_count[d];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("QWEN3_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
 }
 
 int* device_error_word() {

@@ -79,12 +79,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int g = blockIdx.y, b = blockIdx.z;
   const int G = p.G, TQ = kTileQ / G;
   const int t0 = cq * 2 * TQ;
-  const int start = p.start_pos[b];
-  const int kv_limit = start + p.T;  // keys [0, kv_limit) are in the cache
-  // KV tiles each Q tile needs (tile 1 holds the later tokens)
-  const int nk0 = t0 < p.T ? (start + min(t0 + TQ, p.T) - 1) / kTileK + 1 : 0;
-  const int nk1 = t0 + TQ < p.T ? (start + min(t0 + 2 * TQ, p.T) - 1) / kTileK + 1 : 0;
-  const int n_kv = max(nk0, nk1);
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -101,6 +95,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // barrier set-up and the tensor-memory allocation overlap the previous kernel;
+  // global data (positions, Q, the cache) is read only after the wait
+  pdl_wait();
+  pdl_trigger();
+  const int start = p.start_pos[b];
+  const int kv_limit = start + p.T;  // keys [0, kv_limit) are in the cache
+  // KV tiles each Q tile needs (tile 1 holds the later tokens)
+  const int nk0 = t0 < p.T ? (start + min(t0 + TQ, p.T) - 1) / kTileK + 1 : 0;
+  const int nk1 = t0 + TQ < p.T ? (start + min(t0 + 2 * TQ, p.T) - 1) / kTileK + 1 : 0;
+  const int n_kv = max(nk0, nk1);
   const long long kv_row0 = ((long long)b * p.Hkv + g) * p.s_max;
 
   if (warp == 0) {
@@ -371,7 +375,7 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
     attr = true;
   }
   dim3 grid(p.n_cta_q, Hkv, B);
-  attn_prefill_kernel<<<grid, kPrefillThreads, kPrefillSmem, s>>>(tmQ, tmK, tmV, p);
+  q3_launch(attn_prefill_kernel, grid, kPrefillThreads, kPrefillSmem, s, tmQ, tmK, tmV, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention prefill launch failed: %s", cudaGetErrorString(e));
@@ -405,6 +409,8 @@ __global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
   __shared__ float sP[kDecWarps][G][32];
   __shared__ float sM[kDecWarps][G], sL[kDecWarps][G];
   __shared__ __align__(16) float sO[kDecWarps][G][kHeadDim];
+  pdl_wait();
+  pdl_trigger();
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -591,6 +597,8 @@ __global__ void __launch_bounds__(kD3Threads, 1) attn_decode_tma_kernel(
     fence_barrier_init();
   }
   __syncthreads();
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == kD3Warps) {
     // ------------------------------------------------------------------ producer
@@ -750,6 +758,8 @@ __global__ void __launch_bounds__(kD3Threads, 1) attn_decode_tma_kernel(
 
 __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
                                          uint16_t* __restrict__ out, long long ldo) {
+  pdl_wait();
+  pdl_trigger();
   const int bh = blockIdx.x;  // b * Hq + h
   const int b = bh / Hq, h = bh % Hq;
   const float* pp = part + (long long)bh * n_splits * (kHeadDim + 2);
@@ -792,7 +802,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
                            D3Smem<GG>::kBytes);                                                                  \
       attr[SLOT] = true;                                                                                         \
     }                                                                                                            \
-    attn_decode_tma_kernel<GG><<<grid, kD3Threads, D3Smem<GG>::kBytes, s>>>(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, \
+    q3_launch(attn_decode_tma_kernel<GG>, grid, kD3Threads, D3Smem<GG>::kBytes, s, qkv, ldqkv, B, Hq, Hkv, cache_len, ck, \
                                                                            cv, s_max, n_splits, part, err);     \
     break;
     switch (G) {
@@ -801,7 +811,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
       Q3_D3_CASE(4, 2)
     }
 #undef Q3_D3_CASE
-    attn_decode_merge_kernel<<<B * Hq, kHeadDim, 0, s>>>(part, Hq, n_splits, out, ldo);
+    q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) {
       set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
@@ -813,7 +823,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   switch (G) {
 #define Q3_DEC_CASE(GG)                                                                                         \
   case GG:                                                                                                      \
-    attn_decode_split_kernel<GG><<<grid, kDecThreads, 0, s>>>(qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max,    \
+    q3_launch(attn_decode_split_kernel<GG>, grid, kDecThreads, 0, s, qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max,    \
                                                               n_splits, part, err);                            \
     break;
     Q3_DEC_CASE(1)
@@ -825,7 +835,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
       set_last_error("attention decode: %d query heads per KV group is not supported (1, 2, 4 or 8)", G);
       return -2;
   }
-  attn_decode_merge_kernel<<<B * Hq, kHeadDim, 0, s>>>(part, Hq, n_splits, out, ldo);
+  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));

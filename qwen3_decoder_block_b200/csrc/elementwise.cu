@@ -21,6 +21,8 @@ template <bool IN_F32>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
                                                       const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
                                                       long long ldo, int rows, int n, float eps) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int n_warps = (gridDim.x * blockDim.x) >> 5;
@@ -71,9 +73,9 @@ int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, 
   long long blocks = (rows + warps_per_block - 1) / warps_per_block;
   if (blocks > (long long)num_sms() * 16) blocks = (long long)num_sms() * 16;
   if (x_f32)
-    rmsnorm_kernel<true><<<(int)blocks, 256, 0, s>>>(x, ldx, w, out, ldo, rows, n, eps);
+    q3_launch(rmsnorm_kernel<true>, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps);
   else
-    rmsnorm_kernel<false><<<(int)blocks, 256, 0, s>>>(x, ldx, w, out, ldo, rows, n, eps);
+    q3_launch(rmsnorm_kernel<false>, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -96,6 +98,8 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(uint16_t* __restrict_
                                                            const float* __restrict__ rope, uint16_t* __restrict__ ck,
                                                            uint16_t* __restrict__ cv, int s_max, int max_pos,
                                                            float eps, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const long long item = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int slots = Hq + 2 * Hkv;
@@ -148,7 +152,7 @@ int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, in
   const long long warps = (long long)B * T * (Hq + 2 * Hkv);
   if (warps == 0) return 0;
   const long long blocks = (warps * 32 + 255) / 256;
-  qk_norm_rope_kernel<<<(unsigned)blocks, 256, 0, s>>>(qkv, ldqkv, B, T, Hq, Hkv, pos_base, qw, kw, rope, ck, cv,
+  q3_launch(qk_norm_rope_kernel, (unsigned)blocks, 256, 0, s, qkv, ldqkv, B, T, Hq, Hkv, pos_base, qw, kw, rope, ck, cv,
                                                        s_max, max_pos, eps, err);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
@@ -159,6 +163,8 @@ int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, in
 // ---------------------------------------------------------------------------
 __global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t* __restrict__ E, int vocab, int H,
                              void* __restrict__ out, int out_f32, int* err) {
+  pdl_wait();
+  pdl_trigger();
   const int m = blockIdx.x;
   if (m >= n) return;
   const int id = ids[m];
@@ -182,7 +188,7 @@ __global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t*
 int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, void* out, bool out_f32, int* err,
                  cudaStream_t s) {
   if (n <= 0) return 0;
-  embed_kernel<<<n, 128, 0, s>>>(ids, n, E, vocab, H, out, out_f32 ? 1 : 0, err);
+  q3_launch(embed_kernel, n, 128, 0, s, ids, n, E, vocab, H, out, out_f32 ? 1 : 0, err);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -193,6 +199,8 @@ int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, voi
 // ---------------------------------------------------------------------------
 __global__ void pack_gate_up_kernel(const uint16_t* __restrict__ gate, const uint16_t* __restrict__ up,
                                     long long mat_stride, int n_mats, int I, int H, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const long long R = blockIdx.x;  // output row
   const long long rows = (long long)n_mats * 2 * I;
   if (R >= rows) return;
@@ -209,19 +217,21 @@ int launch_pack_gate_up(const uint16_t* gate, const uint16_t* up, long long mat_
                         uint16_t* out, cudaStream_t s) {
   const long long rows = (long long)n_mats * 2 * I;
   if (rows == 0) return 0;
-  pack_gate_up_kernel<<<(unsigned)rows, 128, 0, s>>>(gate, up, mat_stride, n_mats, I, H, out);
+  q3_launch(pack_gate_up_kernel, (unsigned)rows, 128, 0, s, gate, up, mat_stride, n_mats, I, H, out);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
 // Decode bookkeeping: every sequence's cached length grows by one token.
 __global__ void advance_lengths_kernel(int* len, int B) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) len[b] += 1;
 }
 
 int launch_advance_lengths(int* len, int B, cudaStream_t s) {
   if (B <= 0) return 0;
-  advance_lengths_kernel<<<(B + 127) / 128, 128, 0, s>>>(len, B);
+  q3_launch(advance_lengths_kernel, (B + 127) / 128, 128, 0, s, len, B);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

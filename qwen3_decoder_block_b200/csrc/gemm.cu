@@ -355,6 +355,11 @@ __global__ void __launch_bounds__(192, 1)
     fence_barrier_init();
   }
   if (threadIdx.x == 32) { tma_prefetch_desc(&tmP); tma_prefetch_desc(&tmQ); }
+  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  // Everything above touches only this CTA's own resources, so it overlaps the
+  // tail of the previous kernel on the stream; global data is read after the wait.
+  pdl_wait();
+  pdl_trigger();
   if (g.n_groups > 0) {
     // per-group tile counts -> prefix (offsets are stored right after the prefix)
     for (int i = threadIdx.x; i <= g.n_groups; i += blockDim.x) s_off[i] = g.group_offsets[i];
@@ -369,7 +374,6 @@ __global__ void __launch_bounds__(192, 1)
       s_prefix[g.n_groups] = acc;
     }
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -531,6 +535,8 @@ __global__ void __launch_bounds__(192, 1)
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N, int epi, int resid_f32,
                                      int out_f32, const void* __restrict__ resid, long long ldr,
                                      void* __restrict__ out, long long ldo) {
+  pdl_wait();
+  pdl_trigger();
   const int n_out = epi == kEpiSwiglu ? N / 2 : N;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)M * n_out) return;
@@ -694,11 +700,11 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
     grid = (int)(tiles < num_sms() ? tiles : num_sms());
   }
   if (grid <= 0) return 0;
-  gemm_tc_kernel<BN><<<grid, 192, smem, s>>>(tmP, tmQ, tmO, g);
+  q3_launch(gemm_tc_kernel<BN>, grid, 192, smem, s, tmP, tmQ, tmO, g);
   if (g.k_splits > 1) {
     const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
     const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);
-    splitk_reduce_kernel<<<(unsigned)((n_out + 255) / 256), 256, 0, s>>>(
+    q3_launch(splitk_reduce_kernel, (unsigned)((n_out + 255) / 256), 256, 0, s, 
         g.partial, g.k_splits, M, N, d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo);
   }
   cudaError_t e = cudaGetLastError();

@@ -59,6 +59,27 @@ constexpr size_t kSplitKBytes = (size_t)2 * 148 * 128 * 256 * sizeof(float);
 int launch_gemm(const GemmDesc& d, cudaStream_t s, int* err);
 
 int num_sms();
+
+// Every library kernel is launched with programmatic stream serialisation (its prologue
+// may overlap the tail of the previous kernel; the kernel waits with griddepcontrol.wait
+// before reading or writing global data). QWEN3_PDL=0 in the environment turns it off.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t q3_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 int* device_error_word();  // device pointer of the library's error word
 void set_last_error(const char* fmt, ...);
 

@@ -19,6 +19,8 @@ namespace q3 {
 // ---------------------------------------------------------------------------
 __global__ void moe_route_kernel(const float* __restrict__ logits, int T, int E, int k, int renorm,
                                  int* __restrict__ idx, float* __restrict__ w, int* __restrict__ counts) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -86,6 +88,8 @@ __global__ void __launch_bounds__(kPermThreads) moe_permute_kernel(const int* __
                                                                    int* __restrict__ perm_token,
                                                                    int* __restrict__ perm_slot,
                                                                    int* __restrict__ inv_pos) {
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   __shared__ int s_warp[kPermThreads / 32];
   __shared__ int s_base;
@@ -134,6 +138,8 @@ __global__ void __launch_bounds__(kPermThreads) moe_permute_kernel(const int* __
 // A_perm[row] = h[perm_token[row]]   (H % 8 == 0)
 __global__ void moe_gather_kernel(const uint16_t* __restrict__ h, int H, const int* __restrict__ perm_token,
                                   int n_rows, uint16_t* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x;
   if (row >= n_rows) return;
   const uint4* src = reinterpret_cast<const uint4*>(h + (long long)perm_token[row] * H);
@@ -148,6 +154,8 @@ __global__ void moe_gather_kernel(const uint16_t* __restrict__ h, int H, const i
 __global__ void moe_combine_kernel(const float* __restrict__ x1, const uint16_t* __restrict__ Y,
                                    const float* __restrict__ w, const int* __restrict__ inv_pos, int k, int H,
                                    void* __restrict__ out, int out_f32) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
     const float4* xs = reinterpret_cast<const float4*>(x1 + (long long)t * H + c * 8);
@@ -178,7 +186,7 @@ int launch_moe_route(const float* logits, int T, int E, int k, int renorm, int* 
   if (T <= 0) return 0;
   if (cudaMemsetAsync(counts, 0, sizeof(int) * E, s) != cudaSuccess) return -6;
   const int warps_per_block = 8;
-  moe_route_kernel<<<(T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s>>>(logits, T, E, k,
+  q3_launch(moe_route_kernel, (T + warps_per_block - 1) / warps_per_block, 32 * warps_per_block, 0, s, logits, T, E, k,
                                                                                              renorm, idx, w, counts);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
@@ -186,15 +194,15 @@ int launch_moe_route(const float* logits, int T, int E, int k, int renorm, int* 
 int launch_moe_permute(const int* idx, int T, int k, int E, const int* counts, int* offsets, int* perm_token,
                        int* perm_slot, int* inv_pos, const uint16_t* h, int H, uint16_t* a_perm, cudaStream_t s) {
   if (T <= 0) return 0;
-  moe_permute_kernel<<<E, kPermThreads, 0, s>>>(idx, T, k, E, counts, offsets, perm_token, perm_slot, inv_pos);
-  moe_gather_kernel<<<T * k, 128, 0, s>>>(h, H, perm_token, T * k, a_perm);
+  q3_launch(moe_permute_kernel, E, kPermThreads, 0, s, idx, T, k, E, counts, offsets, perm_token, perm_slot, inv_pos);
+  q3_launch(moe_gather_kernel, T * k, 128, 0, s, h, H, perm_token, T * k, a_perm);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
 int launch_moe_combine(const float* x1, const uint16_t* Y, const float* w, const int* inv_pos, int T, int k, int H,
                        void* out, bool out_f32, cudaStream_t s) {
   if (T <= 0) return 0;
-  moe_combine_kernel<<<T, 256, 0, s>>>(x1, Y, w, inv_pos, k, H, out, out_f32 ? 1 : 0);
+  q3_launch(moe_combine_kernel, T, 256, 0, s, x1, Y, w, inv_pos, k, H, out, out_f32 ? 1 : 0);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
