@@ -955,6 +955,8 @@ int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long
   Q3_CHECK(qkv && cache_len && o && ws, QWEN3_EINVAL, "attention_decode: NULL pointer");
   Q3_CHECK(aligned16(qkv) && aligned16(o) && aligned16(ws), QWEN3_EALIGN, "attention_decode: misaligned pointer");
   Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode: B must be positive");
+  Q3_CHECK(ldqkv % 8 == 0 && ldqkv >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
+           "attention_decode: ldqkv (%lld) must be a multiple of 8 and cover the query heads", ldqkv);
   if ((rc = check_kv(*c, kv, 1))) return rc;
   const size_t need = decode_partial_bytes(B, c->n_q_heads, kv->s_max);
   Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "attention_decode: workspace has %zu bytes, needs %zu", ws_bytes, need);
@@ -973,6 +975,8 @@ int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* q
   Q3_CHECK(qkv && cache_len && o, QWEN3_EINVAL, "attention_decode_noalloc: NULL pointer");
   Q3_CHECK(aligned16(qkv) && aligned16(o), QWEN3_EALIGN, "attention_decode_noalloc: misaligned pointer");
   Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode_noalloc: B must be positive");
+  Q3_CHECK(ldqkv % 8 == 0 && ldqkv >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
+           "attention_decode_noalloc: ldqkv (%lld) must be a multiple of 8 and cover the query heads", ldqkv);
   if ((rc = check_kv(*c, kv, 1))) return rc;
   if ((rc = check_device())) return rc;
   return finish(launch_attention_decode_static(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,

@@ -1,5 +1,6 @@
 // K3: causal grouped-query prefill attention on tcgen05 tensor cores.
-// K4: split-KV decode attention (memory bound, CUDA cores) + log-sum-exp merge.
+// K4: split-KV decode attention (memory bound; both products on tcgen05) + a
+//     log-sum-exp merge of the splits.
 //
 // Both compute, for query head h at absolute position m and its KV group
 // g = h / (Hq / Hkv),  o = softmax(q k^T / sqrt(128) + M) v  with M = -inf for keys
@@ -385,374 +386,313 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
 }
 
 // ============================================================================
-// K4: split-KV decode attention. CTA (split, group, sequence) handles keys
-// [split*256, split*256+256) of one sequence's KV group for all G query heads of
-// the group, so each K/V line is read once. Warp w owns 32 consecutive keys:
-//   scores: lane = key; the lane reads its key's 256-byte row straight from HBM
-//           (16 x 16-byte loads in flight) and dots it with the G queries, which
-//           sit pre-scaled in shared memory (broadcast reads);
-//   softmax: per head over the warp's 32 keys (warp max / sum);
-//   P V:    lane = 4 head dims; each key's V row is one coalesced 256-byte warp read.
-// The 8 warps merge in shared memory; the split's (max, sum, unnormalised o) goes
-// to the workspace and a second kernel merges the splits with log-sum-exp weights.
+// K4, tensor-core form (any G in {1, 2, 4, 8, 16}). Persistent: one CTA per SM walks
+// the (sequence, group, 256-key split) items in a fixed order. Both products of a
+// 128-key tile are tcgen05 MMAs with keys or head dims on the 128-row side and the
+// G query heads of the group (padded to 16) as N:
+//   S^T[key][j]  = sum_d K[key][d] q_j[d]      A = K tile (K-major), B = Q (K-major)
+//   O^T[d][j]   += sum_key V[key][d] P[j][key]  A = V tile (MN-major), B = P (K-major)
+// so the CUDA cores only run the softmax. A TMA warp streams Q, K and V of each tile
+// into a 3-stage shared-memory ring (128-byte swizzle, whole 256-byte rows); an MMA
+// warp issues the scores of tile i+1 before P.V of tile i (S double-buffered in
+// tensor memory); 4 softmax warps own one key each (S) and one head dim each (O):
+// the tile maximum per head is a warp reduction plus a 4-warp exchange, the online
+// softmax rescales O only when the running maximum grows by more than 2^8, and P is
+// written as bf16 into a swizzled K-major tile. At the end of a split the
+// unnormalised O, the running maximum and the sum go to the workspace, and the
+// log-sum-exp merge kernel combines the splits.
 // ============================================================================
-constexpr int kDecChunk = 256;
-constexpr int kDecThreads = 256;
-constexpr int kDecWarps = kDecThreads / 32;
+constexpr int kD4Stages = 3;
+constexpr int kD4Split = 256;                      // keys per work item (two tiles)
+constexpr uint32_t kD4Half = 128 * 128;            // [128 rows][64] bf16, swizzled: 16 KB
+constexpr uint32_t kD4QHalf = 16 * 128;            // [16 rows][64] bf16, swizzled: 2 KB
+constexpr uint32_t kD4OffK = 0;
+constexpr uint32_t kD4OffV = 2 * kD4Half;
+constexpr uint32_t kD4OffQ = 4 * kD4Half;
+constexpr uint32_t kD4StageBytes = 4 * kD4Half + 2 * kD4QHalf;  // 68 KB
+constexpr uint32_t kD4OffP = kD4Stages * kD4StageBytes;         // P [16][128] as two K halves
+constexpr uint32_t kD4OffRed = kD4OffP + 2 * kD4QHalf;          // maxima [2][4][16], sums [4][16]
+constexpr uint32_t kD4OffBar = kD4OffRed + (2 * 4 * 16 + 4 * 16) * 4;
+constexpr uint32_t kD4Smem = kD4OffBar + 16 * 8 + 16 + 1024;
+constexpr int kD4Threads = 192;  // softmax warps 0-3, TMA warp 4, MMA warp 5
+constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
+
+__device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int G>
-__global__ void __launch_bounds__(kDecThreads) attn_decode_split_kernel(
-    const uint16_t* __restrict__ qkv, long long ldqkv, int Hq, int Hkv, const int* __restrict__ cache_len,
-    const uint16_t* __restrict__ ck, const uint16_t* __restrict__ cv, int s_max, int n_splits,
-    float* __restrict__ part, int* err) {
-  __shared__ __align__(16) float sQ[G][kHeadDim];
-  __shared__ float sP[kDecWarps][G][32];
-  __shared__ float sM[kDecWarps][G], sL[kDecWarps][G];
-  __shared__ __align__(16) float sO[kDecWarps][G][kHeadDim];
-  pdl_wait();
-  pdl_trigger();
-
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_keys_total = cache_len[b] + 1;  // cached tokens + the new one
-  const int k0 = split * kDecChunk;
-  float* my_part = part + (((long long)b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
-  const long long head_stride = (long long)n_splits * (kHeadDim + 2);
-  if (k0 >= n_keys_total || n_keys_total > s_max) {
-    if (n_keys_total > s_max && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
-    if (threadIdx.x < G) {
-      my_part[threadIdx.x * head_stride + kHeadDim] = -INFINITY;
-      my_part[threadIdx.x * head_stride + kHeadDim + 1] = 0.f;
-    }
-    return;
-  }
-  for (int i = threadIdx.x; i < G * kHeadDim; i += kDecThreads) {
-    const int j = i / kHeadDim, d = i % kHeadDim;
-    sQ[j][d] = __uint_as_float((uint32_t)qkv[(long long)b * ldqkv + (long long)(g * G + j) * kHeadDim + d] << 16) *
-               kScaleLog2;
-  }
-  __syncthreads();
-
-  const long long row0 = ((long long)b * Hkv + g) * s_max;
-  const int kw0 = k0 + warp * 32;  // first key of this warp
-  const int key = kw0 + lane;
-  const bool valid = key < n_keys_total;
-  // ---- scores: one key per lane
-  float s[G];
-#pragma unroll
-  for (int j = 0; j < G; ++j) s[j] = 0.f;
-  if (valid) {
-    const uint4* kr = reinterpret_cast<const uint4*>(ck + (row0 + key) * kHeadDim);
-    uint4 kv[16];
-#pragma unroll
-    for (int c = 0; c < 16; ++c) kv[c] = __ldg(kr + c);
-#pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const float k8[8] = {bf16_lo(kv[c].x), bf16_hi(kv[c].x), bf16_lo(kv[c].y), bf16_hi(kv[c].y),
-                           bf16_lo(kv[c].z), bf16_hi(kv[c].z), bf16_lo(kv[c].w), bf16_hi(kv[c].w)};
-#pragma unroll
-      for (int j = 0; j < G; ++j) {
-        const float4 qa = *reinterpret_cast<const float4*>(&sQ[j][8 * c]);
-        const float4 qb = *reinterpret_cast<const float4*>(&sQ[j][8 * c + 4]);
-        s[j] += qa.x * k8[0] + qa.y * k8[1] + qa.z * k8[2] + qa.w * k8[3] + qb.x * k8[4] + qb.y * k8[5] +
-                qb.z * k8[6] + qb.w * k8[7];
-      }
-    }
-  }
-  // ---- softmax over the warp's keys
-  float m[G], l[G];
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    const float sj = valid ? s[j] : -INFINITY;
-    m[j] = warp_max(sj);
-    const float p = valid ? exp2f(sj - m[j]) : 0.f;
-    l[j] = warp_sum(p);
-    sP[warp][j][lane] = p;
-  }
-  __syncwarp();
-  // ---- o = P V over the warp's keys, lane owns dims [4*lane, 4*lane+4)
-  float o[G][4];
-#pragma unroll
-  for (int j = 0; j < G; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  const int nk = min(32, n_keys_total - kw0);
-  const uint16_t* vbase = cv + (row0 + kw0) * kHeadDim + 4 * lane;
-#pragma unroll 4
-  for (int kk0 = 0; kk0 < 32; kk0 += 8) {
-    uint2 vv[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (kk0 + u < nk) vv[u] = __ldg(reinterpret_cast<const uint2*>(vbase + (long long)(kk0 + u) * kHeadDim));
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (kk0 + u < nk) {
-        const float v0 = bf16_lo(vv[u].x), v1 = bf16_hi(vv[u].x), v2 = bf16_lo(vv[u].y), v3 = bf16_hi(vv[u].y);
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float p = sP[warp][j][kk0 + u];
-          o[j][0] += p * v0; o[j][1] += p * v1; o[j][2] += p * v2; o[j][3] += p * v3;
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < G; ++j) {
-    *reinterpret_cast<float4*>(&sO[warp][j][4 * lane]) = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
-    if (lane == 0) { sM[warp][j] = nk > 0 ? m[j] : -INFINITY; sL[warp][j] = nk > 0 ? l[j] : 0.f; }
-  }
-  __syncthreads();
-  // ---- merge the warps into this split's partial
-  for (int i = threadIdx.x; i < G * kHeadDim; i += kDecThreads) {
-    const int j = i / kHeadDim, d = i % kHeadDim;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, sM[w][j]);
-    float acc = 0.f, L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) {
-      if (sM[w][j] == -INFINITY) continue;
-      const float sc = exp2f(sM[w][j] - M);
-      acc += sO[w][j][d] * sc;
-      L += sL[w][j] * sc;
-    }
-    my_part[j * head_stride + d] = acc;
-    if (d == 0) {
-      my_part[j * head_stride + kHeadDim] = M;
-      my_part[j * head_stride + kHeadDim + 1] = L;
-    }
-  }
-}
-
-// ============================================================================
-// K4, pipelined form (1, 2 or 4 query heads per KV group). Persistent: one CTA per
-// SM walks the (sequence, group, 256-key split) items in a fixed order. A producer
-// warp streams each split's K and V rows as two 128-key halves into a 3-stage ring
-// of shared-memory buffers with bulk copies (the DMA engine, whole lines); 16 compute
-// warps take 8 keys each. Scores: lane l holds 4 head dims of the G queries, partial
-// dot products of the warp's 8 keys x G heads are reduced across lanes with a
-// transposing butterfly (lane l ends with value l). Softmax is online across the two
-// halves; P.V puts lane l on dims [4l, 4l+4). The 16 warps merge in shared memory and
-// the split's (max, sum, unnormalised o) goes to the workspace, as in the form above.
-// ============================================================================
-constexpr int kD3Warps = 16;             // compute warps
-constexpr int kD3Threads = 32 * (kD3Warps + 1);
-constexpr int kD3Half = 128;             // keys per stage
-constexpr int kD3Stages = 3;
-constexpr uint32_t kD3StageBytes = 2u * kD3Half * kHeadDim * 2;  // K then V: 64 KB
-
-template <int G>
-struct D3Smem {
-  static constexpr uint32_t kO = kD3Stages * kD3StageBytes;           // [16][G][128] fp32
-  static constexpr uint32_t kM = kO + kD3Warps * G * kHeadDim * 4;    // [16][G]
-  static constexpr uint32_t kL = kM + kD3Warps * G * 4;               // [16][G]
-  static constexpr uint32_t kBar = (kL + kD3Warps * G * 4 + 7) & ~7u;  // full[3], empty[3]
-  static constexpr uint32_t kAbort = kBar + 2 * kD3Stages * 8;
-  static constexpr uint32_t kBytes = kAbort + 16 + 128;
-};
-
-// Butterfly that reduces NV (power of two, <= 32) per-lane values across the warp:
-// afterwards lane l holds the full sum of value (l & (NV - 1)).
-template <int NV>
-__device__ __forceinline__ float transpose_reduce(float (&a)[NV], int lane) {
-#pragma unroll
-  for (int o = NV / 2; o >= 1; o >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float keep = upper ? a[i + o] : a[i];
-      const float send = upper ? a[i] : a[i + o];
-      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  float v = a[0];
-#pragma unroll
-  for (int o = NV; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-__device__ __forceinline__ void named_bar_compute() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kD3Warps * 32) : "memory");
-}
-
-template <int G>
-__global__ void __launch_bounds__(kD3Threads, 1) attn_decode_tma_kernel(
-    const uint16_t* __restrict__ qkv, long long ldqkv, int B, int Hq, int Hkv, const int* __restrict__ cache_len,
-    const uint16_t* __restrict__ ck, const uint16_t* __restrict__ cv, int s_max, int n_splits,
-    float* __restrict__ part, int* err) {
-  using L = D3Smem<G>;
-  constexpr int NV = 8 * G;  // 8 keys x G heads per warp
+__global__ void __launch_bounds__(kD4Threads, 1)
+    attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV, int B, int Hq, int Hkv,
+                          const int* __restrict__ cache_len, int s_max, int n_splits, float* __restrict__ part,
+                          int* err) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  float* sO = reinterpret_cast<float*>(smem + L::kO);
-  float* sM = reinterpret_cast<float*>(smem + L::kM);
-  float* sL = reinterpret_cast<float*>(smem + L::kL);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  uint64_t* empty = full + kD3Stages;
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kD4OffBar);
+  uint64_t* full = bars;         // [3] stage loaded
+  uint64_t* empty = bars + 3;    // [3] stage consumed
+  uint64_t* s_full = bars + 6;   // [2] scores ready
+  uint64_t* s_empty = bars + 8;  // [2] scores read
+  uint64_t* p_full = bars + 10;  // P written (and O rescaled)
+  uint64_t* pv_done = bars + 11;
+  uint64_t* drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red_max = reinterpret_cast<float*>(smem + kD4OffRed);  // [2][4][16]
+  float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = B * Hkv * n_splits;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kD3Stages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], kD3Warps); }
+    for (int i = 0; i < kD4Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
+    mbar_init(p_full, 128);
+    mbar_init(pv_done, 1);
+    mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
+  // Rows G..15 of the Q and P operand tiles are never written: clear all of them once.
+  for (int i = threadIdx.x; i < (2 * kD4Stages + 2) * (int)(kD4QHalf / 16); i += blockDim.x) {
+    const int buf = i / (int)(kD4QHalf / 16), off = i % (int)(kD4QHalf / 16);
+    uint8_t* base = buf < 2 * kD4Stages ? smem + (buf >> 1) * kD4StageBytes + kD4OffQ + (buf & 1) * kD4QHalf
+                                        : smem + kD4OffP + (buf - 2 * kD4Stages) * kD4QHalf;
+    reinterpret_cast<uint4*>(base)[off] = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  if (threadIdx.x == 128) { tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV); }
+  if (warp == 5) { tmem_alloc(tmem_slot, kD4TmemCols); tmem_relinquish(); }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
   pdl_wait();
   pdl_trigger();
 
-  if (warp == kD3Warps) {
-    // ------------------------------------------------------------------ producer
+  if (warp == 4) {
     if (lane == 0) {
-      int st = 0;
-      uint32_t ph = 0;
-      long long issued = 0;
-      for (int it = blockIdx.x; it < n_items && !*s_abort; it += gridDim.x) {
-        const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv;
+      // ------------------------------------------------------------------ TMA producer
+      long long tc = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
         const int n_total = cache_len[b] + 1;
-        if (n_total > s_max) continue;  // reported by the compute warps
-        const long long row0 = (long long)bg * s_max;
+        if (n_total > s_max) continue;  // reported by the softmax warps
+        const int row0 = bg * s_max;
         for (int h = 0; h < 2; ++h) {
-          const int k0 = split * 2 * kD3Half + h * kD3Half;
-          const int nk = min(kD3Half, n_total - k0);
-          if (nk <= 0) continue;
-          if (!mbar_wait(&empty[st], ph ^ 1, err)) { *s_abort = 1; break; }
-          uint8_t* base = smem + st * kD3StageBytes;
-          mbar_arrive_expect_tx(&full[st], 2u * nk * kHeadDim * 2);
-          bulk_load(base, ck + (row0 + k0) * kHeadDim, nk * kHeadDim * 2, &full[st]);
-          bulk_load(base + kD3StageBytes / 2, cv + (row0 + k0) * kHeadDim, nk * kHeadDim * 2, &full[st]);
-          ++issued;
-          if (++st == kD3Stages) { st = 0; ph ^= 1; }
+          const int k0 = split * kD4Split + h * 128;
+          if (k0 >= n_total) break;
+          const int st = (int)(tc % kD4Stages);
+          if (*s_abort || !mbar_wait(&empty[st], (uint32_t)((tc / kD4Stages) & 1) ^ 1u, err)) { ok = false; break; }
+          uint8_t* base = smem + st * kD4StageBytes;
+          mbar_arrive_expect_tx(&full[st], 4 * kD4Half + 2 * G * 128);
+          tma_load_3d(base + kD4OffQ, &tmQ, &full[st], 0, g * G, b);
+          tma_load_3d(base + kD4OffQ + kD4QHalf, &tmQ, &full[st], 64, g * G, b);
+          tma_load_2d(base + kD4OffK, &tmK, &full[st], 0, row0 + k0);
+          tma_load_2d(base + kD4OffK + kD4Half, &tmK, &full[st], 64, row0 + k0);
+          tma_load_2d(base + kD4OffV, &tmV, &full[st], 0, row0 + k0);
+          tma_load_2d(base + kD4OffV + kD4Half, &tmV, &full[st], 64, row0 + k0);
+          ++tc;
         }
       }
-      // every copy issued lands before the CTA exits (normally all were consumed already)
-      for (long long i = issued > kD3Stages ? issued - kD3Stages : 0; i < issued; ++i)
-        mbar_wait(&full[i % kD3Stages], (uint32_t)((i / kD3Stages) & 1), err);
+      if (!ok) {
+        *s_abort = 1;
+        // let the copies still in flight land before the CTA exits
+        for (long long i = tc > kD4Stages ? tc - kD4Stages : 0; i < tc; ++i)
+          mbar_wait(&full[i % kD4Stages], (uint32_t)((i / kD4Stages) & 1), err);
+      }
     }
-    return;  // the producer warp takes no part in the compute warps' named barrier
-  }
-
-  // -------------------------------------------------------------------- compute
-  int st = 0;
-  uint32_t ph = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-    const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
-    const int n_total = cache_len[b] + 1;
-    const bool over = n_total > s_max;
-    if (over && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
-    // this lane's 4 dims of the G queries, pre-scaled into the exp2 domain
-    float qv[G][4];
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      const uint2 q2 = *reinterpret_cast<const uint2*>(qkv + (long long)b * ldqkv + (long long)(g * G + j) * kHeadDim +
-                                                      4 * lane);
-      qv[j][0] = bf16_lo(q2.x) * kScaleLog2; qv[j][1] = bf16_hi(q2.x) * kScaleLog2;
-      qv[j][2] = bf16_lo(q2.y) * kScaleLog2; qv[j][3] = bf16_hi(q2.y) * kScaleLog2;
-    }
-    float m[G], l[G], o[G][4];
-#pragma unroll
-    for (int j = 0; j < G; ++j) { m[j] = -INFINITY; l[j] = 0.f; o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f; }
-    for (int h = 0; h < 2 && !over; ++h) {
-      const int k0 = split * 2 * kD3Half + h * kD3Half;
-      const int nk = min(kD3Half, n_total - k0);
-      if (nk <= 0) continue;
-      const bool ok = !*s_abort && mbar_wait(&full[st], ph, err);
-      if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; }
-      const uint16_t* sK = reinterpret_cast<const uint16_t*>(smem + st * kD3StageBytes);
-      const uint16_t* sV = sK + kD3Half * kHeadDim;
-      const int kw = warp * 8;  // this warp's first key in the half
-      if (!*s_abort) {
-        // partial dot products: value index kk*G + j
-        float a[NV];
+  } else if (warp == 5) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, 0, 0);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, 1, 0);  // V^T: MN-major A
+      const uint32_t sP = smem_u32(smem + kD4OffP);
+      // O^T += V^T P^T for tile u (the first tile of a split overwrites O)
+      auto issue_pv = [&](long long u, bool first) -> bool {
+        if (*s_abort || !mbar_wait(p_full, (uint32_t)(u & 1), err)) return false;
+        tc_fence_after();
+        const uint32_t sV = smem_u32(smem + (int)(u % kD4Stages) * kD4StageBytes + kD4OffV);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          float k4[4] = {0.f, 0.f, 0.f, 0.f};
-          if (kw + kk < nk) {
-            const uint2 kr = *reinterpret_cast<const uint2*>(sK + (kw + kk) * kHeadDim + 4 * lane);
-            k4[0] = bf16_lo(kr.x); k4[1] = bf16_hi(kr.x); k4[2] = bf16_lo(kr.y); k4[3] = bf16_hi(kr.y);
+          const uint64_t a = sdesc_mnmajor_sw128(sV + kk * 16 * 128, kD4Half, 1024);
+          const uint64_t bp = sdesc_kmajor_sw128(sP + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
+          mma_bf16_ss(tmem + 32, a, bp, idesc_o, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(pv_done);
+        mma_commit(&empty[u % kD4Stages]);
+        return true;
+      };
+      long long tc = 0;
+      bool ok = true, prev_first = false;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int split = it % n_splits, b = (it / n_splits) / Hkv;
+        const int n_total = cache_len[b] + 1;
+        if (n_total > s_max) continue;
+        for (int h = 0; h < 2; ++h) {
+          const int k0 = split * kD4Split + h * 128;
+          if (k0 >= n_total) break;
+          const int st = (int)(tc % kD4Stages), sb = (int)(tc & 1);
+          if (*s_abort || !mbar_wait(&full[st], (uint32_t)((tc / kD4Stages) & 1), err)) { ok = false; break; }
+          if (tc >= 2 && (*s_abort || !mbar_wait(&s_empty[sb], (uint32_t)(((tc - 2) >> 1) & 1), err))) {
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t sK = smem_u32(smem + st * kD4StageBytes + kD4OffK);
+          const uint32_t sQ = smem_u32(smem + st * kD4StageBytes + kD4OffQ);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = sdesc_kmajor_sw128(sK + (kk >> 2) * kD4Half) + 2 * (kk & 3);
+            const uint64_t bq = sdesc_kmajor_sw128(sQ + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
+            mma_bf16_ss(tmem + 16 * sb, a, bq, idesc_s, kk ? 1u : 0u);
+          }
+          mma_commit(&s_full[sb]);
+          if (tc > 0 && !issue_pv(tc - 1, prev_first)) { ok = false; break; }
+          prev_first = (h == 0);
+          ++tc;
+        }
+      }
+      if (ok && tc > 0) ok = issue_pv(tc - 1, prev_first);
+      if (!ok) *s_abort = 1;
+      // every MMA completes before the tensor memory is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, err);
+    }
+  } else {
+    // -------------------------------------------------------------------- softmax
+    const int t = warp * 32 + lane;  // key of the tile (S) / head dim (O)
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    long long tc = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
+      const int n_total = cache_len[b] + 1;
+      const bool over = n_total > s_max;
+      if (over && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
+      float m_run[G], l_part[G];
+#pragma unroll
+      for (int j = 0; j < G; ++j) { m_run[j] = -INFINITY; l_part[j] = 0.f; }
+      int n_tiles = 0;
+      for (int h = 0; h < 2 && !over; ++h) {
+        const int k0 = split * kD4Split + h * 128;
+        if (k0 >= n_total) break;
+        const int nk = min(128, n_total - k0);
+        const int sb = (int)(tc & 1);
+        ok = ok && !*s_abort && mbar_wait(&s_full[sb], (uint32_t)((tc >> 1) & 1), err);
+        ok = __all_sync(0xffffffffu, ok);
+        uint32_t sv[16];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld16(tl + 16 * sb, sv);
+          tmem_wait_ld_regs16(sv);
+        }
+        tc_fence_before();
+        mbar_arrive(&s_empty[sb]);
+        float s[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) s[j] = (ok && t < nk) ? __uint_as_float(sv[j]) * kScaleLog2 : -INFINITY;
+        // tile maximum per head: the warp's 32 keys, then the 4 warps
+        float* rm = red_max + (tc & 1) * 64;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float wm = warp_max(s[j]);
+          if (lane == 0) rm[warp * 16 + j] = wm;
+        }
+        named_bar_softmax();
+        float alpha[G];
+        bool rescale = false;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float mt = fmaxf(fmaxf(rm[j], rm[16 + j]), fmaxf(rm[32 + j], rm[48 + j]));
+          alpha[j] = 1.f;
+          if (mt > m_run[j] + kRescaleThreshold || m_run[j] == -INFINITY) {
+            alpha[j] = (m_run[j] == -INFINITY) ? 0.f : ex2_approx(m_run[j] - mt);
+            m_run[j] = mt;
+            rescale = true;
+          }
+        }
+        float p[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          p[j] = (t < nk && m_run[j] != -INFINITY) ? ex2_approx(s[j] - m_run[j]) : 0.f;
+          l_part[j] = l_part[j] * alpha[j] + p[j];
+        }
+        // P is single-buffered and O is rescaled below: the previous P.V must be done
+        if (tc > 0) {
+          ok = ok && !*s_abort && mbar_wait(pv_done, (uint32_t)((tc - 1) & 1), err);
+          ok = __all_sync(0xffffffffu, ok);
+        }
+        if (ok) {
+          tc_fence_after();
+          if (n_tiles > 0 && rescale) {  // uniform: every thread holds the same maxima
+            uint32_t ov[16];
+            tmem_ld16(tl + 32, ov);
+            tmem_wait_ld_regs16(ov);
+#pragma unroll
+            for (int j = 0; j < G; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha[j]);
+            tmem_st16x(tl + 32, ov);
+            tmem_wait_st();
+          }
+          // P[j][t] into the K-major B tile: row j, key t, 128-byte swizzle
+          uint8_t* pb = smem + kD4OffP + (t >> 6) * kD4QHalf + (t & 7) * 2;
+          const int chunk = (t & 63) >> 3;
 #pragma unroll
           for (int j = 0; j < G; ++j)
-            a[kk * G + j] = qv[j][0] * k4[0] + qv[j][1] * k4[1] + qv[j][2] * k4[2] + qv[j][3] * k4[3];
-        }
-        const float s = transpose_reduce<NV>(a, lane);
-        const int vidx = lane & (NV - 1);
-        const int my_key = vidx / G, my_j = vidx % G;
-        const bool valid = kw + my_key < nk;
-        // per-head max over the first NV lanes (lanes with the same head differ in bits >= log2 G)
-        float mh = valid ? s : -INFINITY;
+            *reinterpret_cast<uint16_t*>(pb + j * 128 + ((chunk ^ (j & 7)) << 4)) = to_bf16_bits(p[j]);
+          // keys past the written cache: zero their V rows (0 * NaN would poison O)
+          if (t >= nk) {
+            uint4* v0 = reinterpret_cast<uint4*>(smem + (int)(tc % kD4Stages) * kD4StageBytes + kD4OffV + t * 128);
+            uint4* v1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(v0) + kD4Half);
 #pragma unroll
-        for (int off = G; off < NV; off <<= 1) mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, off));
-        float m_new[G], alpha[G];
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float mj = __shfl_sync(0xffffffffu, mh, j);
-          m_new[j] = fmaxf(m[j], mj);
-          alpha[j] = (m[j] == -INFINITY) ? 0.f : exp2f(m[j] - m_new[j]);
-        }
-        float my_m = m_new[0];
-#pragma unroll
-        for (int j = 1; j < G; ++j) my_m = (my_j == j) ? m_new[j] : my_m;
-        const float p = (valid && my_m != -INFINITY) ? exp2f(s - my_m) : 0.f;
-        float ps = p;
-#pragma unroll
-        for (int off = G; off < NV; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          l[j] = l[j] * alpha[j] + __shfl_sync(0xffffffffu, ps, j);
-          m[j] = m_new[j];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) o[j][c] *= alpha[j];
-        }
-        // P.V: lane owns dims [4*lane, 4*lane+4)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          float pj[G];
-#pragma unroll
-          for (int j = 0; j < G; ++j) pj[j] = __shfl_sync(0xffffffffu, p, kk * G + j);
-          if (kw + kk < nk) {
-            const uint2 vr = *reinterpret_cast<const uint2*>(sV + (kw + kk) * kHeadDim + 4 * lane);
-            const float v0 = bf16_lo(vr.x), v1 = bf16_hi(vr.x), v2 = bf16_lo(vr.y), v3 = bf16_hi(vr.y);
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-              o[j][0] += pj[j] * v0; o[j][1] += pj[j] * v1; o[j][2] += pj[j] * v2; o[j][3] += pj[j] * v3;
-            }
+            for (int c = 0; c < 8; ++c) { v0[c] = make_uint4(0, 0, 0, 0); v1[c] = make_uint4(0, 0, 0, 0); }
           }
+          fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        mbar_arrive(p_full);
+        ++n_tiles;
+        ++tc;
+      }
+      // this split's partial: unnormalised o, running maximum (log2 domain), sum
+      float* my_part = part + ((long long)(b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
+      const long long head_stride = (long long)n_splits * (kHeadDim + 2);
+      uint32_t ov[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) ov[j] = 0u;
+      if (n_tiles > 0) {
+        ok = ok && !*s_abort && mbar_wait(pv_done, (uint32_t)((tc - 1) & 1), err);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          tmem_ld16(tl + 32, ov);
+          tmem_wait_ld_regs16(ov);
+        }
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          const float ws = warp_sum(l_part[j]);
+          if (lane == 0) red_sum[warp * 16 + j] = ws;
+        }
+        named_bar_softmax();
+      }
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        my_part[j * head_stride + t] = __uint_as_float(ov[j]);
+        if (t == j) {
+          const float L = n_tiles > 0 ? red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j] : 0.f;
+          my_part[j * head_stride + kHeadDim] = m_run[j];
+          my_part[j * head_stride + kHeadDim + 1] = L;
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      if (++st == kD3Stages) { st = 0; ph ^= 1; }
     }
-    // merge the 16 warps into this split's partial
-#pragma unroll
-    for (int j = 0; j < G; ++j) {
-      *reinterpret_cast<float4*>(&sO[(warp * G + j) * kHeadDim + 4 * lane]) = make_float4(o[j][0], o[j][1], o[j][2], o[j][3]);
-      if (lane == 0) { sM[warp * G + j] = m[j]; sL[warp * G + j] = l[j]; }
-    }
-    named_bar_compute();
-    float* my_part = part + ((long long)(b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
-    const long long head_stride = (long long)n_splits * (kHeadDim + 2);
-    for (int i = threadIdx.x; i < G * kHeadDim; i += kD3Warps * 32) {
-      const int j = i / kHeadDim, d = i % kHeadDim;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kD3Warps; ++w) M = fmaxf(M, sM[w * G + j]);
-      float acc = 0.f, Lsum = 0.f;
-#pragma unroll
-      for (int w = 0; w < kD3Warps; ++w) {
-        const float mw = sM[w * G + j];
-        if (mw == -INFINITY) continue;
-        const float sc = exp2f(mw - M);
-        acc += sO[(w * G + j) * kHeadDim + d] * sc;
-        Lsum += sL[w * G + j] * sc;
-      }
-      my_part[j * head_stride + d] = acc;
-      if (d == 0) {
-        my_part[j * head_stride + kHeadDim] = M;
-        my_part[j * head_stride + kHeadDim + 1] = Lsum;
-      }
-    }
-    named_bar_compute();  // the next item overwrites sO / sM / sL
+    if (!ok) *s_abort = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kD4TmemCols);
   }
 }
 
@@ -778,7 +718,7 @@ __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq,
   out[(long long)b * ldo + (long long)h * kHeadDim + d] = to_bf16_bits(acc / L);
 }
 
-int decode_splits(int s_max) { return (s_max + kDecChunk - 1) / kDecChunk; }
+int decode_splits(int s_max) { return (s_max + kD4Split - 1) / kD4Split; }
 
 size_t decode_partial_bytes(int B, int Hq, int s_max) {
   return (size_t)B * Hq * decode_splits(s_max) * (kHeadDim + 2) * sizeof(float);
@@ -789,51 +729,47 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
                             long long ldo, int* err, cudaStream_t s) {
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
-  const int n_splits = decode_splits(s_max);
-  if (G == 1 || G == 2 || G == 4) {
-    // pipelined form: persistent CTAs, bulk copies into a 3-stage shared-memory ring
-    const long long items = (long long)B * Hkv * n_splits;
-    const int grid = (int)(items < num_sms() ? items : num_sms());
-    static bool attr[3] = {false, false, false};
-#define Q3_D3_CASE(GG, SLOT)                                                                                     \
-  case GG:                                                                                                       \
-    if (!attr[SLOT]) {                                                                                           \
-      cudaFuncSetAttribute(attn_decode_tma_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize,              \
-                           D3Smem<GG>::kBytes);                                                                  \
-      attr[SLOT] = true;                                                                                         \
-    }                                                                                                            \
-    q3_launch(attn_decode_tma_kernel<GG>, grid, kD3Threads, D3Smem<GG>::kBytes, s, qkv, ldqkv, B, Hq, Hkv, cache_len, ck, \
-                                                                           cv, s_max, n_splits, part, err);     \
-    break;
-    switch (G) {
-      Q3_D3_CASE(1, 0)
-      Q3_D3_CASE(2, 1)
-      Q3_D3_CASE(4, 2)
-    }
-#undef Q3_D3_CASE
-    q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) {
-      set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
-      return -6;
-    }
-    return 0;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) {
+    set_last_error("attention decode: %d query heads per KV group is not supported (1, 2, 4, 8 or 16)", G);
+    return -2;
   }
-  dim3 grid(n_splits, Hkv, B);
+  if ((long long)B * Hkv * s_max + 128 >= (1ll << 31)) {
+    set_last_error("attention decode: B * Hkv * s_max = %lld cache rows exceed the 2^31 tensor-map range",
+                   (long long)B * Hkv * s_max);
+    return -2;
+  }
+  const int n_splits = decode_splits(s_max);
+  CUtensorMap tmQ, tmK, tmV;
+  // Q: (dim, head, token), box = the G heads of one group
+  if (make_tmap_3d(&tmQ, qkv, kHeadDim, Hq, B, kHeadDim * 2, ldqkv * 2, 64, G, 1) != 0) {
+    set_last_error("attention decode: cannot encode the query tensor map");
+    return -6;
+  }
+  const long long kv_rows = (long long)B * Hkv * s_max;
+  if (make_tmap_2d(&tmK, ck, kv_rows, kHeadDim, kHeadDim, 128) != 0 ||
+      make_tmap_2d(&tmV, cv, kv_rows, kHeadDim, kHeadDim, 128) != 0) {
+    set_last_error("attention decode: cannot encode the KV-cache tensor maps");
+    return -6;
+  }
+  const long long items = (long long)B * Hkv * n_splits;
+  const int grid = (int)(items < num_sms() ? items : num_sms());
+  static bool attr[5] = {false, false, false, false, false};
   switch (G) {
-#define Q3_DEC_CASE(GG)                                                                                         \
-  case GG:                                                                                                      \
-    q3_launch(attn_decode_split_kernel<GG>, grid, kDecThreads, 0, s, qkv, ldqkv, Hq, Hkv, cache_len, ck, cv, s_max,    \
-                                                              n_splits, part, err);                            \
+#define Q3_D4_CASE(GG, SLOT)                                                                                      \
+  case GG:                                                                                                        \
+    if (!attr[SLOT]) {                                                                                            \
+      cudaFuncSetAttribute(attn_decode_tc_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, kD4Smem);      \
+      attr[SLOT] = true;                                                                                          \
+    }                                                                                                             \
+    q3_launch(attn_decode_tc_kernel<GG>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,      \
+              s_max, n_splits, part, err);                                                                        \
     break;
-    Q3_DEC_CASE(1)
-    Q3_DEC_CASE(2)
-    Q3_DEC_CASE(4)
-    Q3_DEC_CASE(8)
-#undef Q3_DEC_CASE
-    default:
-      set_last_error("attention decode: %d query heads per KV group is not supported (1, 2, 4 or 8)", G);
-      return -2;
+    Q3_D4_CASE(1, 0)
+    Q3_D4_CASE(2, 1)
+    Q3_D4_CASE(4, 2)
+    Q3_D4_CASE(8, 3)
+    Q3_D4_CASE(16, 4)
+#undef Q3_D4_CASE
   }
   q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);
   cudaError_t e = cudaGetLastError();

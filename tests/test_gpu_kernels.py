@@ -247,8 +247,8 @@ def test_attention_prefill(q3, hq, hkv, B, T, starts):
     assert rel_frob(got, ref) <= 1e-2
 
 
-@pytest.mark.parametrize("hq,hkv", [(16, 8), (32, 4)])
-@pytest.mark.parametrize("lens", [[0, 129, 598], [4095, 4096, 1, 200]])
+@pytest.mark.parametrize("hq,hkv", [(16, 8), (32, 4), (8, 8), (16, 4), (32, 2)])
+@pytest.mark.parametrize("lens", [[0, 129, 598], [4095, 4096, 1, 200], [127, 255, 256]])
 def test_attention_decode(q3, hq, hkv, lens):
     cfg = q3.make_config(n_q_heads=hq, n_kv_heads=hkv, hidden=2048 if hq == 32 else 1024)
     D = cfg.head_dim
@@ -273,8 +273,12 @@ def test_attention_decode(q3, hq, hkv, lens):
         q = qkv.f[b, :hq * D].reshape(1, hq, D)
         ref = R.causal_gqa_attention(q, kall.f[b][:, :L].transpose(1, 0, 2), vall.f[b][:, :L].transpose(1, 0, 2),
                                      np.array([lens[b]]), np.arange(L)).reshape(-1)
-        # fp32 softmax and accumulation; the only rounding is the bf16 output (<= 2^-8 |o|)
-        assert np.all(np.abs(got[b] - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-4), (b, max_abs(got[b], ref))
+        # fp32 scores, softmax and accumulation; P is rounded to bf16 for the P.V product
+        # (relative 2^-9 per weight: at most 2^-9 max|v| on the normalised output) and the
+        # output to bf16 (2^-8 |o|)
+        vmax = np.abs(vall.f[b][:, :L]).max()
+        tol = 2.0 ** -8 * np.abs(ref) + 2.0 ** -9 * vmax + 1e-4
+        assert np.all(np.abs(got[b] - ref) <= tol), (b, max_abs(got[b], ref))
 
 
 def test_embed(q3):
