@@ -17,7 +17,7 @@
 // of O (only when the running max grows by more than 2^8), write P as bf16 into a
 // 128-byte swizzled shared tile, and O += P V accumulates in tensor memory with V
 // as an MN-major operand. Causal tiles beyond the diagonal are skipped and the
-// heaviest q tiles are scheduled first.
+// heaviest q tiles of all (group, sequence) pairs are scheduled first.
 #include <mutex>
 #include "common.cuh"
 #include "internal.h"
@@ -76,8 +76,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cq = p.n_cta_q - 1 - (int)blockIdx.x;  // heavy CTAs first
-  const int g = blockIdx.y, b = blockIdx.z;
+  // Linear order, heaviest q tiles of every (group, sequence) first: the causal
+  // work of a CTA grows with cq, so the block scheduler fills the SMs longest-first.
+  const int gb = (int)(blockIdx.x % (unsigned)(p.Hkv * p.B));
+  const int cq = p.n_cta_q - 1 - (int)(blockIdx.x / (unsigned)(p.Hkv * p.B));
+  const int g = gb % p.Hkv, b = gb / p.Hkv;
   const int G = p.G, TQ = kTileQ / G;
   const int t0 = cq * 2 * TQ;
 
@@ -375,7 +378,12 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
     cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
     attr = true;
   }
-  dim3 grid(p.n_cta_q, Hkv, B);
+  const long long n_cta = (long long)p.n_cta_q * Hkv * B;
+  if (n_cta >= (1ll << 31)) {
+    set_last_error("attention prefill: %lld CTAs exceed the grid limit", n_cta);
+    return -2;
+  }
+  dim3 grid((unsigned)n_cta);
   q3_launch(attn_prefill_kernel, grid, kPrefillThreads, kPrefillSmem, s, tmQ, tmK, tmV, p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
