@@ -40,7 +40,13 @@ constexpr uint32_t kOffKV = 4 * kHalf;
 constexpr uint32_t kStageBytes = 4 * kHalf;
 constexpr uint32_t kOffBar = kOffKV + 2 * kStageBytes;
 constexpr uint32_t kPrefillSmem = kOffBar + 256 + 1024;
-constexpr int kPrefillThreads = 320;  // TMA warp, MMA warp, 2 softmax warpgroups
+constexpr int kPrefillThreads = 384;  // softmax warpgroups (warps 0-3, 4-7), TMA warp 8, MMA warp 9
+// Register split after the prologue: the softmax warpgroups hold a whole 128-column
+// score row per thread; the third warpgroup (TMA, MMA, two idle warps) needs few.
+// (2 x 200 + 88) x 128 registers must fit the launch allocation (384 x regs/thread).
+constexpr int kPrefillRegsSoftmax = 200;
+constexpr int kPrefillRegsCtl = 88;
+constexpr int kPrefillRegBudget = (2 * kPrefillRegsSoftmax + kPrefillRegsCtl) * 128;
 // log2(e) / sqrt(128)
 constexpr float kScaleLog2 = 0.12751743074380304f;
 constexpr float kRescaleThreshold = 8.0f;
@@ -94,7 +100,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     *s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (warp == 9) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -111,7 +117,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int n_kv = max(nk0, nk1);
   const long long kv_row0 = ((long long)b * p.Hkv + g) * p.s_max;
 
-  if (warp == 0) {
+  if (warp >= 8) {
+    regs_decrease<kPrefillRegsCtl>();
+  if (warp == 8) {
     if (lane == 0) {
       // -------------------------------------------------------------- TMA producer
       bool ok = true;
@@ -143,7 +151,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 9) {
     if (lane == 0) {
       // -------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileK, 0, 0);
@@ -192,9 +200,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_wait(drain, 0, p.err);
       }
     }
+  }
   } else {
+    regs_increase<kPrefillRegsSoftmax>();
     // ---------------------------------------------------------------- softmax
-    const int X = (warp - 2) >> 2;  // which Q tile this warpgroup owns
+    const int X = warp >> 2;        // which Q tile this warpgroup owns
     const int quad = warp & 3;      // tensor-memory lanes [32 quad, 32 quad + 32)
     const int r = quad * 32 + lane;
     const int t = t0 + X * TQ + r / G;
@@ -213,65 +223,52 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int kv0 = j * kTileK;
       // only tiles touching the diagonal or the end of the cache need the mask
       const bool need_mask = __any_sync(0xffffffffu, kv0 + kTileK - 1 > qpos || kv0 + kTileK > kv_limit);
-      // pass 1: row max, two 32-column chunks per tensor-memory round trip
-      float mx = -INFINITY;
+      // the whole 128-column score row of this thread in one tensor-memory round trip
+      uint32_t v[4][32];
 #pragma unroll
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        uint32_t v[2][32];
-        tmem_ld32(tS + c2 * 32, v[0]);
-        tmem_ld32(tS + c2 * 32 + 32, v[1]);
-        tmem_wait_ld_regs(v[0]);
-        tmem_wait_ld_regs(v[1]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, v[c]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (need_mask) {
+      for (int c = 0; c < 4; ++c) tmem_wait_ld_regs(v[c]);
+      if (need_mask) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kp = kv0 + (c2 + h) * 32 + i;
-              if (kp > qpos || kp >= kv_limit) v[h][i] = __float_as_uint(-INFINITY);
-            }
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int kp = kv0 + c * 32 + i;
+            if (kp > qpos || kp >= kv_limit) v[c][i] = __float_as_uint(-INFINITY);
           }
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) mx = fmax3(mx, __uint_as_float(v[h][i]), __uint_as_float(v[h][i + 1]));
-        }
       }
-      const float mxs = mx * kScaleLog2;
+      // row max: four independent 3-input max chains
+      float mc[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        mc[c] = __uint_as_float(v[c][0]);
+#pragma unroll
+        for (int i = 1; i < 31; i += 2) mc[c] = fmax3(mc[c], __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
+        mc[c] = fmaxf(mc[c], __uint_as_float(v[c][31]));
+      }
+      const float mxs = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * kScaleLog2;
       float alpha = 1.f;
       if (mxs > m_run + kRescaleThreshold || m_run == -INFINITY) {
         alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - mxs);
         m_run = mxs;
       }
-      // pass 2: p = 2^(s*scale - m) (packed fp32x2 FMA), row sums (packed adds), bf16 pairs
-      // written over the columns already consumed
+      // p = 2^(s*scale - m) (packed fp32x2 FMA), row sums (packed adds), bf16 pairs
+      // written over the first 64 columns (all scores are in registers already)
       const uint64_t scale2 = f2_pack(__float_as_uint(kScaleLog2), __float_as_uint(kScaleLog2));
       const uint64_t neg2 = f2_pack(__float_as_uint(-m_run), __float_as_uint(-m_run));
       uint64_t acc2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int c2 = 0; c2 < 4; c2 += 2) {
-        uint32_t v[2][32];
-        tmem_ld32(tS + c2 * 32, v[0]);
-        tmem_ld32(tS + c2 * 32 + 32, v[1]);
-        tmem_wait_ld_regs(v[0]);
-        tmem_wait_ld_regs(v[1]);
+      for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (need_mask) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int kp = kv0 + (c2 + h) * 32 + i;
-              if (kp > qpos || kp >= kv_limit) v[h][i] = __float_as_uint(-INFINITY);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const uint64_t e = f2_fma(f2_pack(v[h][i], v[h][i + 1]), scale2, neg2);
-            const float p0 = ex2_approx(f2_lo(e));
-            const float p1 = ex2_approx(f2_hi(e));
-            acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
-            v[h][i >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + (c2 + h) * 16, v[h]);  // columns [16c, 16c+16) were read already
+        for (int i = 0; i < 32; i += 2) {
+          const uint64_t e = f2_fma(f2_pack(v[c][i], v[c][i + 1]), scale2, neg2);
+          const float p0 = ex2_approx(f2_lo(e));
+          const float p1 = ex2_approx(f2_hi(e));
+          acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
+          v[c][i >> 1] = pack_bf16x2(p0, p1);
         }
+        tmem_st16(tS + c * 16, v[c]);
       }
       const uint64_t acc = f2_add(acc2[0], acc2[1]);
       const float sum_tile = f2_lo(acc) + f2_hi(acc);
@@ -342,7 +339,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -376,6 +373,13 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+    // the register split must fit what the block is launched with, or the increase never returns
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_prefill_kernel) != cudaSuccess ||
+        fa.numRegs * kPrefillThreads < kPrefillRegBudget) {
+      set_last_error("attention prefill: kernel built with too few registers for its warpgroup split");
+      return -6;
+    }
     attr = true;
   }
   const long long n_cta = (long long)p.n_cta_q * Hkv * B;
