@@ -40,7 +40,7 @@ constexpr uint32_t kOffKV = 4 * kHalf;
 constexpr uint32_t kStageBytes = 4 * kHalf;
 constexpr uint32_t kOffBar = kOffKV + 2 * kStageBytes;
 constexpr uint32_t kPrefillSmem = kOffBar + 256 + 1024;
-constexpr int kPrefillThreads = 384;  // softmax warpgroups (warps 0-3, 4-7), TMA warp 8, MMA warp 9
+constexpr int kPrefillThreads = 384;  // softmax warpgroups (warps 0-3, 4-7), TMA warp 8, MMA warps 9-10
 // Register split after the prologue: the softmax warpgroups hold a whole 128-column
 // score row per thread; the third warpgroup (TMA, MMA, two idle warps) needs few.
 // (2 x 200 + 88) x 128 registers must fit the launch allocation (384 x regs/thread).
@@ -62,7 +62,7 @@ struct PrefillParams {
 }  // namespace
 
 // Tensor memory (512 columns): tile X in {0, 1} owns columns [256X, 256X+256):
-// S_X = [256X, 256X+128) (fp32 scores; its first 64 columns are reused for the bf16
+// S_X = [256X, 256X+128) (fp32 scores; columns [64, 128) are reused for the bf16
 // probabilities P_X), O_X = [256X+128, 256X+256) (fp32 output accumulator).
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -77,8 +77,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* s_full = bars + 7;    // [2] per Q tile
   uint64_t* p_full = bars + 9;    // [2] per Q tile
   uint64_t* pv_done = bars + 11;  // [2] per Q tile
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* s_read = bars + 13;   // [2] per Q tile: scores loaded into registers
+  uint64_t* drain = bars + 15;    // [2] per MMA issuer
+  uint64_t* mufu_tok = bars + 17; // [2] softmax X may start its exponentials
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -93,10 +95,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1); mbar_init(&v_full[i], 1); mbar_init(&kv_empty[i], 1);
+      mbar_init(&k_full[i], 1); mbar_init(&v_full[i], 1); mbar_init(&kv_empty[i], 2);
+      mbar_init(&s_read[i], 128); mbar_init(&drain[i], 1); mbar_init(&mufu_tok[i], 128);
       mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1);
     }
-    mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -151,53 +153,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 9 || warp == 10) {
     if (lane == 0) {
-      // -------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTileK, 0, 0);
+      // ------------------------------------------------- MMA issuers, one per Q tile
+      // Each Q tile's chain S(j) -> softmax -> P.V(j) -> S(j+1) is issued by its own
+      // thread, so neither chain waits behind the other's softmax.
+      const int X = warp - 9;
+      const int nkx = X ? nk1 : nk0;
+      const int nk_other = X ? nk0 : nk1;
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, 0, 0);        // one 64-key half of S
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, kHeadDim, 0, 1);  // V is MN-major
-      bool ok = mbar_wait(q_full, 0, p.err);
-      const uint32_t sq = smem_u32(smem + kOffQ);
-      for (int j = 0; j < n_kv && ok; ++j) {
+      const uint32_t qa = smem_u32(smem + kOffQ) + 2 * X * kHalf;
+      // S_X(j) in two N = 64 halves: keys [0, 64) into columns [0, 64) of S_X, keys
+      // [64, 128) into [64, 128). P_X occupies columns [64, 128): the first half of
+      // S_X(j+1) only needs the softmax to have read S_X(j), the second half needs
+      // P.V(j) to be complete.
+      auto issue_s_half = [&](int j, int h) -> bool {
         const int st = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (*s_abort || !mbar_wait(&k_full[st], par, p.err)) { ok = false; break; }
-        const uint32_t sk = smem_u32(smem + kOffKV + st * kStageBytes);
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (j >= (X ? nk1 : nk0)) continue;
-          // S_X reuses the columns of P_X of the previous tile: wait until that P.V is done
-          if (j > 0 && (*s_abort || !mbar_wait(&pv_done[X], (j - 1) & 1, p.err))) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t qa = sq + 2 * X * kHalf;
+        if (*s_abort || !mbar_wait(&k_full[st], (j >> 1) & 1, p.err)) return false;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(smem + kOffKV + st * kStageBytes) + h * 64 * 128;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t a = sdesc_kmajor_sw128(qa + (kk >> 2) * kHalf) + 2 * (kk & 3);
-            const uint64_t bd = sdesc_kmajor_sw128(sk + (kk >> 2) * kHalf) + 2 * (kk & 3);
-            mma_bf16_ss(tmem + 256 * X, a, bd, idesc_s, kk ? 1u : 0u);
-          }
-          mma_commit(&s_full[X]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t a = sdesc_kmajor_sw128(qa + (kk >> 2) * kHalf) + 2 * (kk & 3);
+          const uint64_t bd = sdesc_kmajor_sw128(sk + (kk >> 2) * kHalf) + 2 * (kk & 3);
+          mma_bf16_ss(tmem + 256 * X + 64 * h, a, bd, idesc_s, kk ? 1u : 0u);
         }
-        if (!ok) break;
-        if (*s_abort || !mbar_wait(&v_full[st], par, p.err)) { ok = false; break; }
-        const uint32_t sv = sk + 2 * kHalf;
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (j >= (X ? nk1 : nk0)) continue;
-          if (*s_abort || !mbar_wait(&p_full[X], j & 1, p.err)) { ok = false; break; }
-          tc_fence_after();
+        if (h == 1) mma_commit(&s_full[X]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j & 1;
+        if (*s_abort || !mbar_wait(&v_full[st], (j >> 1) & 1, p.err)) return false;
+        if (*s_abort || !mbar_wait(&p_full[X], j & 1, p.err)) return false;
+        tc_fence_after();
+        const uint32_t sv = smem_u32(smem + kOffKV + st * kStageBytes + 2 * kHalf);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t bd = sdesc_mnmajor_sw128(sv + kk * 16 * 128, kHalf, 1024);
-            mma_bf16_ts(tmem + 256 * X + 128, tmem + 256 * X + kk * 8, bd, idesc_o, (j | kk) ? 1u : 0u);
-          }
-          mma_commit(&pv_done[X]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_mnmajor_sw128(sv + kk * 16 * 128, kHalf, 1024);
+          mma_bf16_ts(tmem + 256 * X + 128, tmem + 256 * X + 64 + kk * 8, bd, idesc_o, (j | kk) ? 1u : 0u);
         }
-        if (!ok) break;
+        mma_commit(&pv_done[X]);
+        // the stage takes one arrival per Q tile; this chain also stands in for the
+        // other tile when that tile does not use KV tile j
         mma_commit(&kv_empty[st]);
+        if (j >= nk_other) mma_commit(&kv_empty[st]);
+        return true;
+      };
+      bool ok = nkx > 0 ? mbar_wait(q_full, 0, p.err) : true;
+      if (ok && nkx > 0) ok = issue_s_half(0, 0) && issue_s_half(0, 1);
+      for (int j = 0; j < nkx && ok; ++j) {
+        if (j + 1 < nkx) {
+          if (*s_abort || !mbar_wait(&s_read[X], j & 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          if (!issue_s_half(j + 1, 0)) { ok = false; break; }
+        }
+        if (!issue_pv(j)) { ok = false; break; }
+        if (j + 1 < nkx) {
+          if (*s_abort || !mbar_wait(&pv_done[X], j & 1, p.err)) { ok = false; break; }
+          tc_fence_after();
+          if (!issue_s_half(j + 1, 1)) { ok = false; break; }
+        }
       }
       if (!ok) {
         *s_abort = 1;
-        mma_commit(drain);
-        mbar_wait(drain, 0, p.err);
+        mma_commit(&drain[X]);
+        mbar_wait(&drain[X], 0, p.err);
       }
     }
   }
@@ -229,6 +250,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, v[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld_regs(v[c]);
+      tc_fence_before();
+      mbar_arrive(&s_read[X]);  // columns [0, 64) of S_X may now take the next tile's scores
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -254,10 +277,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         m_run = mxs;
       }
       // p = 2^(s*scale - m) (packed fp32x2 FMA), row sums (packed adds), bf16 pairs
-      // written over the first 64 columns (all scores are in registers already)
+      // written over columns [64, 128) (all scores are in registers already)
       const uint64_t scale2 = f2_pack(__float_as_uint(kScaleLog2), __float_as_uint(kScaleLog2));
       const uint64_t neg2 = f2_pack(__float_as_uint(-m_run), __float_as_uint(-m_run));
       uint64_t acc2[2] = {0ull, 0ull};
+      // The two softmax warpgroups take turns on the exponentials (the special-function
+      // unit is the bottleneck of the softmax): tile 0 of KV tile j goes after tile 1 of
+      // KV tile j-1, tile 1 of KV tile j after tile 0 of KV tile j. Each turn overlaps
+      // the tensor core's work on the other Q tile. A turn is only awaited while the
+      // other warpgroup still has KV tiles.
+      if (X == 0 ? (j >= 1 && j - 1 < nk1) : (j < nk0)) {
+        w_ok = !*s_abort && mbar_wait(&mufu_tok[X], (uint32_t)((X == 0 ? j - 1 : j) & 1), p.err);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
 #pragma unroll
@@ -268,12 +300,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           acc2[(i >> 1) & 1] = f2_add(acc2[(i >> 1) & 1], f2_pack(__float_as_uint(p0), __float_as_uint(p1)));
           v[c][i >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tS + c * 16, v[c]);
+        tmem_st16(tS + 64 + c * 16, v[c]);
       }
+      mbar_arrive(&mufu_tok[X ^ 1]);
       const uint64_t acc = f2_add(acc2[0], acc2[1]);
       const float sum_tile = f2_lo(acc) + f2_hi(acc);
       l_run = l_run * alpha + sum_tile;
-      // O_X is stable here: S_X of this tile was issued only after the previous P.V completed
+      // O_X is stable here: the second half of S_X(j) was issued only after P.V of tile j-1 completed
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -286,9 +319,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       // The last KV tile may extend past the written cache: zero those V rows so that
-      // 0-probability keys cannot inject NaN/Inf through P.V. One warpgroup does it:
-      // tile 0's if tile 0 takes part in this KV tile (its P.V is issued first).
-      if (kv0 + kTileK > kv_limit && (X == 0 || j >= nk0)) {
+      // 0-probability keys cannot inject NaN/Inf through P.V. Both Q tiles' P.V of
+      // this KV tile are issued independently, so each warpgroup zeroes the rows
+      // before releasing its own P (the second writes zeros over zeros).
+      if (kv0 + kTileK > kv_limit) {
         w_ok = !*s_abort && mbar_wait(&v_full[st], (j >> 1) & 1, p.err);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         if (kv0 + r >= kv_limit) {
