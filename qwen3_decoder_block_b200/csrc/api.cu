@@ -91,6 +91,15 @@ bool pdl_enabled() {
   return on;
 }
 
+// Large plain GEMMs on CTA pairs; QWEN3_GEMM_PAIR=0 keeps every GEMM on single CTAs.
+bool gemm_pair_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("QWEN3_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 int* device_error_word() {
   const int d = current_device();
   std::lock_guard<std::mutex> lk(g_dev_mu);

@@ -29,11 +29,13 @@ namespace q3 {
 constexpr int BM = 128;
 constexpr int BK = 64;
 
-template <int BN>
+// PAIR: the CTA is one half of a 2-CTA pair computing a 256 x BN tile with M = 256
+// MMAs; it loads its 128 rows of A and BN/2 rows of B per stage.
+template <int BN, bool PAIR = false>
 struct GemmCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr uint32_t P_BYTES = BM * BK * 2;
-  static constexpr uint32_t Q_BYTES = BN * BK * 2;
+  static constexpr uint32_t Q_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
   static constexpr uint32_t STAGING_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x 32x32 fp32
@@ -68,7 +70,8 @@ __device__ __forceinline__ int total_tiles(const GemmParams& g, const int* s_pre
   return g.n_groups > 0 ? s_prefix[g.n_groups] : g.p_tiles * g.q_tiles * g.k_splits;
 }
 
-template <int BN>
+// BMT: output rows per tile (128, or 256 for a CTA pair)
+template <int BN, int BMT = BM>
 __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const int* s_prefix, const int* s_off) {
   Tile r;
   r.kb0 = 0;
@@ -97,7 +100,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const in
     int pt, qt;
     if (g.q_fast) { pt = t / g.q_tiles; qt = t % g.q_tiles; }
     else          { qt = t / g.p_tiles; pt = t % g.p_tiles; }
-    r.p0 = pt * BM;
+    r.p0 = pt * BMT;
     r.p_end = g.p_rows;
     r.q0 = qt * BN;
     r.q_end = g.q_rows;
@@ -327,11 +330,12 @@ __device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr
 }
 
 // --------------------------------------------------------------------------- kernel
-template <int BN>
+template <int BN, bool PAIR>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams g) {
-  using C = GemmCfg<BN>;
+  using C = GemmCfg<BN, PAIR>;
+  constexpr int BMT = PAIR ? 2 * BM : BM;  // output rows per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + C::STAGES * C::STAGE_BYTES;
@@ -346,16 +350,24 @@ __global__ void __launch_bounds__(192, 1)
   int* s_off = s_prefix + (g.n_groups + 1);  // only used in grouped mode (aliases past prefix)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // PAIR: rank 0 issues the MMAs for both CTAs; the tile loop runs over pairs
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0;
+  const int t_first = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int t_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 128); }
+    // PAIR: the 4 epilogue warps of both CTAs release an accumulator (one arrival each)
+    for (int b = 0; b < 2; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], PAIR ? 8 : 128); }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   if (threadIdx.x == 32) { tma_prefetch_desc(&tmP); tma_prefetch_desc(&tmQ); }
-  if (warp == 1) { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  if (warp == 1) {
+    if (PAIR) { tmem_alloc_pair(tmem_slot, C::TMEM_COLS); tmem_relinquish_pair(); }
+    else      { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
+  }
   // Everything above touches only this CTA's own resources, so it overlaps the
   // tail of the previous kernel on the stream; global data is read after the wait.
   pdl_wait();
@@ -376,6 +388,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int ntiles = total_tiles(g, s_prefix);
@@ -383,39 +396,54 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
+      const uint32_t full_leader = PAIR ? mapa_shared(full, 0) : 0;
       int stage = 0;
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-        const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
+      for (int t = t_first; t < ntiles && ok; t += t_step) {
+        const Tile tl = decode_tile<BN, BMT>(t, g, s_prefix, s_off);
+        // PAIR: this CTA's 128 rows of A and BN/2 rows of B; both CTAs' copies complete
+        // on the even CTA's full barrier, which expects the bytes of both
+        const int a_row = tl.p0 + (int)rank * BM;
+        const int b_row = tl.q_load + (int)rank * (BN / 2);
         for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
           if (*s_abort || !mbar_wait(&empty[stage], phase ^ 1, g.err)) { ok = false; break; }
           uint8_t* sp = smem + stage * C::STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          tma_load_2d(sp, &tmP, &full[stage], kb * BK, tl.p0);
-          tma_load_2d(sp + C::P_BYTES, &tmQ, &full[stage], kb * BK, tl.q_load);
+          if (PAIR) {
+            const uint32_t fb = full_leader + stage * 8;
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            tma_load_2d_pair(sp, &tmP, fb, kb * BK, a_row);
+            tma_load_2d_pair(sp + C::P_BYTES, &tmQ, fb, kb * BK, b_row);
+          } else {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+            tma_load_2d(sp, &tmP, &full[stage], kb * BK, a_row);
+            tma_load_2d(sp + C::P_BYTES, &tmQ, &full[stage], kb * BK, b_row);
+          }
           ++issued;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {
         *s_abort = 1;
-        // let every copy still in flight land before the CTA exits
-        for (long long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
-          mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), g.err);
+        // let every copy still in flight land before the CTA exits (PAIR: the even
+        // CTA's barrier also counts the odd CTA's copies; neither CTA leaves before
+        // the final cluster barrier)
+        if (!PAIR || rank == 0)
+          for (long long i = issued > C::STAGES ? issued - C::STAGES : 0; i < issued; ++i)
+            mbar_wait(&full[i % C::STAGES], (uint32_t)((i / C::STAGES) & 1), g.err);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && (!PAIR || rank == 0)) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      constexpr uint32_t idesc = idesc_bf16_f32(BMT, BN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++local) {
-        const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
+      for (int t = t_first; t < ntiles && ok; t += t_step, ++local) {
+        const Tile tl = decode_tile<BN, BMT>(t, g, s_prefix, s_off);
         const int buf = local & 1;
         const uint32_t use_par = (local >> 1) & 1;
         if (*s_abort || !mbar_wait(&tempty[buf], use_par ^ 1, g.err)) { ok = false; break; }
@@ -428,17 +456,23 @@ __global__ void __launch_bounds__(192, 1)
           const uint64_t adesc = sdesc_kmajor_sw128(sa);
           const uint64_t bdesc = sdesc_kmajor_sw128(sa + C::P_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > tl.kb0 || kk) ? 1u : 0u);
-          mma_commit(&empty[stage]);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            if (PAIR) mma_bf16_ss_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > tl.kb0 || kk) ? 1u : 0u);
+            else      mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > tl.kb0 || kk) ? 1u : 0u);
+          }
+          if (PAIR) mma_commit_pair_mc(&empty[stage], 3);  // frees the stage in both CTAs
+          else      mma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        mma_commit(&tfull[buf]);
+        if (PAIR) mma_commit_pair_mc(&tfull[buf], 3);
+        else      mma_commit(&tfull[buf]);
       }
       if (!ok) {
         *s_abort = 1;
-        mma_commit(drain);  // completes once every issued MMA has finished
+        // completes once every issued MMA has finished
+        if (PAIR) mma_commit_pair(drain);
+        else      mma_commit(drain);
         mbar_wait(drain, 0, g.err);
       }
     }
@@ -447,8 +481,21 @@ __global__ void __launch_bounds__(192, 1)
     const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32) are reachable from this warp
     int local = 0;
     int sbuf = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++local) {
-      const Tile tl = decode_tile<BN>(t, g, s_prefix, s_off);
+    // PAIR: this CTA's accumulator rows are rows [128 rank, 128 rank + 128) of the tile;
+    // each warp releases the accumulator on the even CTA's barrier
+    const uint32_t tempty_addr0 = PAIR ? mapa_shared(&tempty[0], 0) : 0;
+    auto release_acc = [&](int b) {
+      tc_fence_before();
+      if (PAIR) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_addr0 + b * 8);
+      } else {
+        mbar_arrive(&tempty[b]);
+      }
+    };
+    for (int t = t_first; t < ntiles; t += t_step, ++local) {
+      Tile tl = decode_tile<BN, BMT>(t, g, s_prefix, s_off);
+      if (PAIR) tl.p0 += (int)rank * BM;
       const int buf = local & 1;
       const uint32_t use_par = (local >> 1) & 1;
       bool ok = !*s_abort && mbar_wait(&tfull[buf], use_par, g.err);
@@ -462,8 +509,7 @@ __global__ void __launch_bounds__(192, 1)
         if (heads > 0)
           qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
                        p < tl.p_end);
-        tc_fence_before();
-        mbar_arrive(&tempty[buf]);
+        release_acc(buf);
         continue;
       }
 #pragma unroll 1
@@ -515,17 +561,20 @@ __global__ void __launch_bounds__(192, 1)
           store_col_chunk(g, p, p < tl.p_end, tl.q0 + c * 32, tl.q_end, lane, tl.p0 + quad * 32, r);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[buf]);
+      release_acc(buf);
     }
     if (g.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
   __syncthreads();
+  // PAIR: the even CTA's MMAs read the odd CTA's shared memory and write its tensor
+  // memory; neither leaves before both are done
+  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -631,8 +680,10 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
     set_last_error("gemm: cannot encode the tensor map of operand P");
     return -6;
   }
+  // Large plain GEMMs run on CTA pairs (M = 256 MMAs; each CTA loads half of B)
+  const bool pair = BN == 256 && !d.swap && d.n_groups == 0 && d.p_rows >= 2 * BM && gemm_pair_enabled();
   const long long q_total = d.n_groups > 0 ? d.q_rows_total : d.q_rows;
-  if (make_tmap_2d(&tmQ, d.Q, q_total, d.K, d.ldq, BN) != 0) {
+  if (make_tmap_2d(&tmQ, d.Q, q_total, d.K, d.ldq, pair ? BN / 2 : BN) != 0) {
     set_last_error("gemm: cannot encode the tensor map of operand Q");
     return -6;
   }
@@ -640,7 +691,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   g.p_rows = d.p_rows;
   g.q_rows = d.q_rows;
   g.k_blocks = d.K / BK;
-  g.p_tiles = (d.p_rows + BM - 1) / BM;
+  g.p_tiles = (d.p_rows + (pair ? 2 * BM : BM) - 1) / (pair ? 2 * BM : BM);
   g.q_tiles = (d.q_rows + BN - 1) / BN;
   // Keep the smaller operand cache-resident: sweep fastest over the tiles of the
   // operand that is re-read, so that the larger operand streams from HBM once.
@@ -663,7 +714,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   // Split K when the output has too few tiles to keep the SMs streaming: each split
   // writes fp32 partials, and a reduce kernel applies the epilogue.
   const long long out_tiles = (long long)g.p_tiles * g.q_tiles;
-  if (d.n_groups == 0 && d.partial && out_tiles * 2 <= num_sms() && g.k_blocks > 1) {
+  if (!pair && d.n_groups == 0 && d.partial && out_tiles * 2 <= num_sms() && g.k_blocks > 1) {
     int S = (int)(num_sms() / out_tiles);
     if (S > g.k_blocks) S = g.k_blocks;
     const size_t per_split = (size_t)d.p_rows * d.q_rows * sizeof(float);
@@ -681,15 +732,31 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
       (reinterpret_cast<uintptr_t>(d.out) & 15) == 0 && (d.ldo * (d.out_f32 ? 4 : 2)) % 16 == 0) {
     if (make_tmap_out(&tmO, d.out, d.p_rows, d.q_rows, d.ldo, d.out_f32) == 0) g.tma_store = 1;
   }
-  const size_t smem = C::smem_bytes(d.n_groups);
+  const size_t smem = pair ? GemmCfg<BN, true>::smem_bytes(0) : C::smem_bytes(d.n_groups);
   static bool attr_set[4] = {false, false, false, false};
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int slot = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
     if (!attr_set[slot]) {
-      cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+      cudaFuncSetAttribute(gemm_tc_kernel<BN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+      if constexpr (BN == 256)
+        cudaFuncSetAttribute(gemm_tc_kernel<BN, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
       attr_set[slot] = true;
+    }
+  }
+  if constexpr (BN == 256) {
+    if (pair) {
+      const long long tiles = (long long)g.p_tiles * g.q_tiles;
+      const int pairs = (int)(tiles < num_sms() / 2 ? tiles : num_sms() / 2);
+      if (pairs <= 0) return 0;
+      q3_launch_cluster(gemm_tc_kernel<BN, true>, 2 * pairs, 192, smem, s, 2, tmP, tmQ, tmO, g);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) {
+        set_last_error("gemm launch failed: %s", cudaGetErrorString(e));
+        return -6;
+      }
+      return 0;
     }
   }
   int grid;
@@ -700,7 +767,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
     grid = (int)(tiles < num_sms() ? tiles : num_sms());
   }
   if (grid <= 0) return 0;
-  q3_launch(gemm_tc_kernel<BN>, grid, 192, smem, s, tmP, tmQ, tmO, g);
+  q3_launch(gemm_tc_kernel<BN, false>, grid, 192, smem, s, tmP, tmQ, tmO, g);
   if (g.k_splits > 1) {
     const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
     const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);

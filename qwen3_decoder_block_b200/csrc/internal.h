@@ -64,6 +64,7 @@ int num_sms();
 // may overlap the tail of the previous kernel; the kernel waits with griddepcontrol.wait
 // before reading or writing global data). QWEN3_PDL=0 in the environment turns it off.
 bool pdl_enabled();
+bool gemm_pair_enabled();
 
 template <typename... KArgs, typename... Args>
 inline cudaError_t q3_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
@@ -80,6 +81,28 @@ inline cudaError_t q3_launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
+
+// Same, launched as clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+inline cudaError_t q3_launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                     unsigned cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 int* device_error_word();  // device pointer of the library's error word
 void set_last_error(const char* fmt, ...);
 

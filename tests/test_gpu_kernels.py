@@ -78,8 +78,10 @@ def test_gemm_residual(q3, M, N, K, swap, rt, ot):
 @pytest.mark.parametrize("M,N,K,epi", [(64, 1024, 2048, 1), (64, 6144, 1024, 2), (16, 4096, 1024, 0),
                                        (64, 1024, 3072, 1), (200, 512, 1024, 0), (3, 4736, 1024, 0)])
 @pytest.mark.parametrize("out_f32", [0, 1])
-def test_gemm_split_k(q3, M, N, K, epi, out_f32):
-    """Small-M GEMMs split K across CTAs (fp32 partials + reduce with the epilogue)."""
+@pytest.mark.parametrize("swap", [1, 0])
+def test_gemm_split_k(q3, M, N, K, epi, out_f32, swap):
+    """Small-M GEMMs split K across CTAs (fp32 partials + reduce with the epilogue),
+    with tokens on the MMA's N side (swap) or on its 128-row side."""
     if epi == 2 and out_f32:
         pytest.skip("SwiGLU output is bf16")
     A = Tensor(SEED, 37, (M, K))
@@ -93,7 +95,7 @@ def test_gemm_split_k(q3, M, N, K, epi, out_f32):
     if epi == 2:
         packed = torch.empty_like(W.gpu)
         q3.pack_gate_up(N // 2, K, W.gpu[:N // 2], W.gpu[N // 2:], packed)
-    q3.op_gemm(A.gpu, packed, out, M, N, K, epilogue=epi, resid=resid, swap=1, ws=ws)
+    q3.op_gemm(A.gpu, packed, out, M, N, K, epilogue=epi, resid=resid, swap=swap, ws=ws)
     assert_device_ok()
     acc = A.f @ W.f.T
     if epi == 2:
