@@ -31,14 +31,17 @@ constexpr int BK = 64;
 
 // PAIR: the CTA is one half of a 2-CTA pair computing a 256 x BN tile with M = 256
 // MMAs; it loads its 128 rows of A and BN/2 rows of B per stage.
-template <int BN, bool PAIR = false>
+// ROPE: the fused QK-norm + RoPE epilogue, which keeps RoPE rows 0..127 in the
+// (otherwise unused) staging area, grown to 64 KB at the cost of one stage.
+template <int BN, bool PAIR = false, bool ROPE = false>
 struct GemmCfg {
-  static constexpr int STAGES = PAIR ? (BN == 256 ? 6 : 8) : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int STAGES = PAIR ? (BN == 256 ? (ROPE ? 5 : 6) : 8) : (BN == 256 ? (ROPE ? 3 : 4) : (BN == 128 ? 6 : 8));
   static constexpr uint32_t P_BYTES = BM * BK * 2;
   static constexpr uint32_t Q_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;
   static constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   static constexpr uint32_t TMEM_COLS = 2 * BN;
-  static constexpr uint32_t STAGING_BYTES = 4 * 2 * 4096;  // 4 epilogue warps x 2 buffers x 32x32 fp32
+  // 4 epilogue warps x 2 buffers x 32x32 fp32, or the 128 x 128 fp32 RoPE rows
+  static constexpr uint32_t STAGING_BYTES = ROPE ? 128 * 128 * 4 : 4 * 2 * 4096;
   static constexpr uint32_t BAR_BYTES = 256;
   static size_t smem_bytes(int n_groups) {
     return 1024 + (size_t)STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES + 8 * (size_t)(n_groups + 2);
@@ -239,8 +242,13 @@ __device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int 
 // [b][g][pos][:] ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and
 // RoPE). The row's cos/sin values are read once for both heads. All 32 lanes execute
 // the tensor-memory loads; only valid rows store.
+// rope_lo: RoPE rows 0..127 in shared memory, row r's 16-byte chunk k stored at chunk
+// k ^ (r & 31). The angle of position pos splits as (pos & ~127) + (pos & 127): its
+// cos/sin follow from the two rows by the angle-addition formulas, so every thread
+// reads one row shared by its warp (L1) and one row from shared memory, instead of a
+// 512-byte row of its own.
 __device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr, int slot0, int n_heads, int p,
-                                             bool valid) {
+                                             bool valid, const float* rope_lo) {
   const QKRopeArgs& a = g.qk;
   int b = 0, pos = 0;
   if (valid) {
@@ -267,14 +275,25 @@ __device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr
     }
     rinv[hh] = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
   }
-  const float* rp = a.rope + (long long)pos * 128;
+  const float* rph = a.rope + (long long)(pos & ~127) * 128;
+  const int lo = pos & 127;
+  const float4* rpl = reinterpret_cast<const float4*>(rope_lo + lo * 128);
   // pass 2: dims d (first half) and d + 64 (second half) form one rotation pair
 #pragma unroll 1
   for (int c = 0; c < 2; ++c) {
     float4 cs[16];  // (cos_d, sin_d, cos_d+1, sin_d+1) for d = 32c .. 32c+31
 #pragma unroll
-    for (int i = 0; i < 16; ++i) cs[i] = valid ? *reinterpret_cast<const float4*>(rp + (c * 32 + 2 * i) * 2)
-                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < 16; ++i) {
+      const int k = c * 16 + i;
+      if (valid) {
+        const float4 h = *reinterpret_cast<const float4*>(rph + k * 4);
+        const float4 l = rpl[k ^ (lo & 31)];
+        cs[i] = make_float4(h.x * l.x - h.y * l.y, h.y * l.x + h.x * l.y, h.z * l.z - h.w * l.w,
+                            h.w * l.z + h.z * l.w);
+      } else {
+        cs[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
       if (hh >= n_heads) break;
@@ -330,11 +349,11 @@ __device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr
 }
 
 // --------------------------------------------------------------------------- kernel
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool ROPE>
 __global__ void __launch_bounds__(192, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmO, const GemmParams g) {
-  using C = GemmCfg<BN, PAIR>;
+  using C = GemmCfg<BN, PAIR, ROPE>;
   constexpr int BMT = PAIR ? 2 * BM : BM;  // output rows per tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -493,6 +512,17 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive(&tempty[b]);
       }
     };
+    const float* rope_lo = reinterpret_cast<const float*>(staging);
+    if (ROPE) {
+      // RoPE rows 0..127 into shared memory (coalesced: a warp reads 512 contiguous bytes)
+      const int et = threadIdx.x - 64;  // 0..127
+      for (int i = et; i < 128 * 32; i += 128) {
+        const int r = i >> 5, k = i & 31;
+        const float4 v = r < g.qk.max_pos ? reinterpret_cast<const float4*>(g.qk.rope)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        reinterpret_cast<float4*>(staging)[r * 32 + (k ^ (r & 31))] = v;
+      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");  // the 4 epilogue warps only
+    }
     for (int t = t_first; t < ntiles; t += t_step, ++local) {
       Tile tl = decode_tile<BN, BMT>(t, g, s_prefix, s_off);
       if (PAIR) tl.p0 += (int)rank * BM;
@@ -502,13 +532,13 @@ __global__ void __launch_bounds__(192, 1)
       if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; break; }  // keep the warp converged
       tc_fence_after();
       const int row = quad * 32 + lane;
-      if (g.epi == kEpiQKRope) {
+      if constexpr (ROPE) {
         // non-swap only: the tile's BN columns are BN/128 whole heads
         const int p = tl.p0 + row;
         const int heads = min(BN / 128, (tl.q_end - tl.q0) / 128);
         if (heads > 0)
           qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
-                       p < tl.p_end);
+                       p < tl.p_end, rope_lo);
         release_acc(buf);
         continue;
       }
@@ -672,6 +702,41 @@ static int make_tmap_out(CUtensorMap* map, void* base, long long rows, long long
   return r == CUDA_SUCCESS ? 0 : -2;
 }
 
+// One kernel instantiation: shared-memory attribute (once), launch (CTA pairs as
+// clusters of 2), launch-error check.
+template <int BN, bool PAIR, bool ROPE>
+static int launch_variant(const GemmParams& g, const CUtensorMap& tmP, const CUtensorMap& tmQ,
+                          const CUtensorMap& tmO, cudaStream_t s) {
+  using C = GemmCfg<BN, PAIR, ROPE>;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  });
+  const size_t smem = C::smem_bytes(g.n_groups);
+  if (PAIR) {
+    const long long tiles = (long long)g.p_tiles * g.q_tiles;
+    const int pairs = (int)(tiles < num_sms() / 2 ? tiles : num_sms() / 2);
+    if (pairs <= 0) return 0;
+    q3_launch_cluster(gemm_tc_kernel<BN, PAIR, ROPE>, 2 * pairs, 192, smem, s, 2, tmP, tmQ, tmO, g);
+  } else {
+    int grid;
+    if (g.n_groups > 0) {
+      grid = num_sms();
+    } else {
+      const long long tiles = (long long)g.p_tiles * g.q_tiles * g.k_splits;
+      grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    }
+    if (grid <= 0) return 0;
+    q3_launch(gemm_tc_kernel<BN, PAIR, ROPE>, grid, 192, smem, s, tmP, tmQ, tmO, g);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_last_error("gemm launch failed: %s", cudaGetErrorString(e));
+    return -6;
+  }
+  return 0;
+}
+
 template <int BN>
 static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   using C = GemmCfg<BN>;
@@ -714,7 +779,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   // Split K when the output has too few tiles to keep the SMs streaming: each split
   // writes fp32 partials, and a reduce kernel applies the epilogue.
   const long long out_tiles = (long long)g.p_tiles * g.q_tiles;
-  if (!pair && d.n_groups == 0 && d.partial && out_tiles * 2 <= num_sms() && g.k_blocks > 1) {
+  if (!pair && d.n_groups == 0 && d.epi != kEpiQKRope && d.partial && out_tiles * 2 <= num_sms() && g.k_blocks > 1) {
     int S = (int)(num_sms() / out_tiles);
     if (S > g.k_blocks) S = g.k_blocks;
     const size_t per_split = (size_t)d.p_rows * d.q_rows * sizeof(float);
@@ -732,42 +797,18 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
       (reinterpret_cast<uintptr_t>(d.out) & 15) == 0 && (d.ldo * (d.out_f32 ? 4 : 2)) % 16 == 0) {
     if (make_tmap_out(&tmO, d.out, d.p_rows, d.q_rows, d.ldo, d.out_f32) == 0) g.tma_store = 1;
   }
-  const size_t smem = pair ? GemmCfg<BN, true>::smem_bytes(0) : C::smem_bytes(d.n_groups);
-  static bool attr_set[4] = {false, false, false, false};
-  static std::mutex mu;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    const int slot = BN == 64 ? 0 : (BN == 128 ? 1 : 2);
-    if (!attr_set[slot]) {
-      cudaFuncSetAttribute(gemm_tc_kernel<BN, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-      if constexpr (BN == 256)
-        cudaFuncSetAttribute(gemm_tc_kernel<BN, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-      attr_set[slot] = true;
-    }
-  }
   if constexpr (BN == 256) {
-    if (pair) {
-      const long long tiles = (long long)g.p_tiles * g.q_tiles;
-      const int pairs = (int)(tiles < num_sms() / 2 ? tiles : num_sms() / 2);
-      if (pairs <= 0) return 0;
-      q3_launch_cluster(gemm_tc_kernel<BN, true>, 2 * pairs, 192, smem, s, 2, tmP, tmQ, tmO, g);
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) {
-        set_last_error("gemm launch failed: %s", cudaGetErrorString(e));
-        return -6;
-      }
-      return 0;
+    if (d.epi == kEpiQKRope)
+      return pair ? launch_variant<BN, true, true>(g, tmP, tmQ, tmO, s) : launch_variant<BN, false, true>(g, tmP, tmQ, tmO, s);
+    if (pair) return launch_variant<BN, true, false>(g, tmP, tmQ, tmO, s);
+  } else {
+    if (d.epi == kEpiQKRope) {
+      set_last_error("gemm: the fused QK-norm/RoPE epilogue needs 256-column tiles");
+      return -1;
     }
   }
-  int grid;
-  if (d.n_groups > 0) {
-    grid = num_sms();
-  } else {
-    const long long tiles = (long long)g.p_tiles * g.q_tiles * g.k_splits;
-    grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  }
-  if (grid <= 0) return 0;
-  q3_launch(gemm_tc_kernel<BN, false>, grid, 192, smem, s, tmP, tmQ, tmO, g);
+  int rc = launch_variant<BN, false, false>(g, tmP, tmQ, tmO, s);
+  if (rc) return rc;
   if (g.k_splits > 1) {
     const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
     const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);
