@@ -276,14 +276,17 @@ struct Ctx {
 static inline bool swap_for(long long M) { return M <= 256; }
 
 // x1 = x + o_proj(attn(norm1(x)))   ([P-Mini] section TransformerBlock, first half)
+// h_ready: b.h already holds norm1(x) (written by the previous layer's last GEMM).
+// *h2_ready is set when the o_proj GEMM also left norm2(x1) in b.h.
 static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void* x, bool x_f32, int B, int T,
-                          bool decode, const int* pos, const qwen3_kv_layer& kv, const float* rope, Buffers& b) {
+                          bool decode, const int* pos, const qwen3_kv_layer& kv, const float* rope, Buffers& b,
+                          bool h_ready, bool* h2_ready) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, D = c.head_dim;
   const long long M = (long long)B * T;
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * D;
-  int rc;
-  {
+  int rc = 0;
+  if (!h_ready) {
     ProfScope ps("rmsnorm", k.s);
     rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
   }
@@ -299,11 +302,18 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   g.ldo = nqkv;
   g.partial = b.gpart;
   g.partial_bytes = b.gpart ? kSplitKBytes : 0;
-  if (!g.swap) {
-    // prefill: QK-norm, RoPE and the KV-cache write run in the GEMM's epilogue on the
-    // fp32 accumulators (no bf16 round trip of q/k/v)
-    g.epi = kEpiQKRope;
-    g.force_bn = 256;
+  int qk_done = 0;
+  {
+    // QK-norm, RoPE and the KV-cache write run on the fp32 accumulators (no bf16 round
+    // trip of q/k/v): in the GEMM's epilogue for prefill, in the split-K completion
+    // for small token counts
+    if (!g.swap) {
+      g.epi = kEpiQKRope;
+      g.force_bn = 256;
+    } else {
+      g.qk_in_reduce = true;
+      g.fused = &qk_done;
+    }
     g.qk.T = T;
     g.qk.Hq = c.n_q_heads;
     g.qk.Hkv = c.n_kv_heads;
@@ -322,7 +332,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     rc = launch_gemm(g, k.s, k.err);
   }
   if (rc) return rc;
-  if (g.swap) {
+  if (g.swap && !qk_done) {
     ProfScope ps("qk_norm_rope", k.s);
     rc = launch_qk_norm_rope(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, w.q_norm, w.k_norm, rope, kv.k,
                              kv.v, kv.s_max, c.max_pos, c.rms_eps, k.err, k.s);
@@ -352,16 +362,28 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   o.ldo = H;
   o.partial = b.gpart;
   o.partial_bytes = b.gpart ? kSplitKBytes : 0;
+  // with split K, the completion kernel also writes norm2(x1) into b.h
+  int h2 = 0;
+  o.norm_w = w.post_norm;
+  o.norm_out = b.h;
+  o.norm_eps = c.rms_eps;
+  o.fused = &h2;
   ProfScope ps("gemm_o", k.s);
-  return launch_gemm(o, k.s, k.err);
+  rc = launch_gemm(o, k.s, k.err);
+  *h2_ready = h2 != 0;
+  return rc;
 }
 
 // out = x1 + down(silu(gate(norm2(x1))) * up(norm2(x1)))   ([P-Mini] sections SwiGLU FFN, TransformerBlock)
-static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
+// h2_ready: b.h already holds norm2(x1). With next_norm set, the down GEMM's split-K
+// completion may also write norm(out) * next_norm into next_out (*next_ready set then).
+static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b,
+                     bool h2_ready, const uint16_t* next_norm = nullptr, uint16_t* next_out = nullptr,
+                     bool* next_ready = nullptr) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, I = c.intermediate;
-  int rc;
-  {
+  int rc = 0;
+  if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
     rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
   }
@@ -395,16 +417,26 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   d.ldo = H;
   d.partial = b.gpart;
   d.partial_bytes = b.gpart ? kSplitKBytes : 0;
+  int nr = 0;
+  if (next_norm && next_out) {
+    d.norm_w = next_norm;
+    d.norm_out = next_out;
+    d.norm_eps = c.rms_eps;
+    d.fused = &nr;
+  }
   ProfScope ps("gemm_down", k.s);
-  return launch_gemm(d, k.s, k.err);
+  rc = launch_gemm(d, k.s, k.err);
+  if (next_ready) *next_ready = nr != 0;
+  return rc;
 }
 
 // out = x1 + sum_j w_j Expert_{e_j}(norm2(x1))   ([P-Mini] section MoE)
-static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b) {
+static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b,
+                   bool h2_ready) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, E = c.n_experts, kk = c.top_k, Im = c.moe_intermediate;
-  int rc;
-  {
+  int rc = 0;
+  if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
     rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
   }
@@ -672,8 +704,9 @@ int qwen3_block_prefill(const qwen3_config* c, const qwen3_layer_weights* w, qwe
   Buffers b;
   carve(*c, QWEN3_OP_BLOCK_PREFILL, B, T, kv->s_max, ws, &b);
   Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
-  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b))) return finish(rc);
-  return finish(dense_ffn(k, *w, (long long)B * T, x, false, b));
+  bool h2 = false;
+  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b, false, &h2))) return finish(rc);
+  return finish(dense_ffn(k, *w, (long long)B * T, x, false, b, h2));
 }
 
 int qwen3_block_decode(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_bf16* x, int B,
@@ -685,8 +718,9 @@ int qwen3_block_decode(const qwen3_config* c, const qwen3_layer_weights* w, qwen
   Buffers b;
   carve(*c, QWEN3_OP_BLOCK_DECODE, B, 1, kv->s_max, ws, &b);
   Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
-  if ((rc = attention_half(k, *w, x, false, B, 1, true, cache_len, *kv, rope, b))) return finish(rc);
-  return finish(dense_ffn(k, *w, B, x, false, b));
+  bool h2 = false;
+  if ((rc = attention_half(k, *w, x, false, B, 1, true, cache_len, *kv, rope, b, false, &h2))) return finish(rc);
+  return finish(dense_ffn(k, *w, B, x, false, b, h2));
 }
 
 int qwen3_moe_block(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_bf16* x, int B, int T,
@@ -700,8 +734,9 @@ int qwen3_moe_block(const qwen3_config* c, const qwen3_layer_weights* w, qwen3_b
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   Ctx k{*c, s, device_error_word()};
   const long long M = (long long)B * T;
-  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b))) return finish(rc);
-  if ((rc = moe_ffn(k, *w, M, x, false, b))) return finish(rc);
+  bool h2 = false;
+  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b, false, &h2))) return finish(rc);
+  if ((rc = moe_ffn(k, *w, M, x, false, b, h2))) return finish(rc);
   const size_t mk = (size_t)M * c->top_k;
   if (topk_idx && cudaMemcpyAsync(topk_idx, b.idx, mk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) rc = -6;
   if (topk_w && cudaMemcpyAsync(topk_w, b.w, mk * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) rc = -6;
@@ -755,15 +790,24 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
     rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s);
   }
   if (rc) return finish(rc);
+  // With split K (small token counts), each layer's down projection also leaves the
+  // next layer's norm1 (or, after the last layer, the final norm when every row is
+  // kept) in b.h / b.hf, and the o_proj leaves norm2.
+  bool h_ready = false;
+  const bool fuse_final = !last_only || T == 1;
   for (int l = 0; l < c->n_layers; ++l) {
-    if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b))) return finish(rc);
-    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b))) return finish(rc);
+    bool h2 = false;
+    if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b, h_ready, &h2)))
+      return finish(rc);
+    const bool last = l + 1 == c->n_layers;
+    const uint16_t* nn = last ? (fuse_final ? final_norm : nullptr) : layers[l + 1].in_norm;
+    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b, h2, nn, last ? b.hf : b.h, &h_ready))) return finish(rc);
   }
   // final RMSNorm and tied LM head ([P-Mini] section 骨架; [P-SGL] section 一)
   const int rows = last_only ? B : (int)M;
   const float* xf = last_only ? b.xs + (long long)(T - 1) * H : b.xs;
   const long long ldx = last_only ? (long long)T * H : H;
-  {
+  if (!h_ready) {
     ProfScope ps("rmsnorm", s);
     rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s);
   }

@@ -641,6 +641,129 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int 
   else static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_bf16_bits(acc);
 }
 
+// Split-K completion fused with the QK-norm + RoPE + KV-cache write (swap layout:
+// part[s][token][feature]). One warp per (token m, head slot); lane l owns dims
+// {2l, 2l+1} and {64+2l, 65+2l} of the slot. Token m of sequence b = m / T sits at
+// position pos_base[b] + m % T. Sums in split order, then the same arithmetic as
+// qk_norm_rope_kernel on the fp32 sums (q/k/v are not rounded before the norm).
+__global__ void __launch_bounds__(256) splitk_qkrope_kernel(const float* __restrict__ part, int S, int M, int N,
+                                                            uint16_t* __restrict__ qkv, long long ldqkv,
+                                                            const QKRopeArgs a, int* err) {
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int slots = a.Hq + 2 * a.Hkv;
+  const long long item = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (item >= (long long)M * slots) return;
+  const int slot = (int)(item % slots);
+  const int m = (int)(item / slots);
+  const int b = m / a.T, t = m % a.T;
+  const int pos = a.pos_base[b] + t;
+  if (pos < 0 || pos >= a.s_max || pos >= a.max_pos) {
+    if (lane == 0) record_error(err, kErrCapacity);
+    return;
+  }
+  const long long plane = (long long)M * N;
+  const float* src = part + (long long)m * N + slot * 128;
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+  int s = 0;
+  for (; s + 4 <= S; s += 4) {  // four splits' loads in flight, added in split order
+    float2 x0[4], x1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x0[u] = *reinterpret_cast<const float2*>(src + (s + u) * plane + 2 * lane);
+      x1[u] = *reinterpret_cast<const float2*>(src + (s + u) * plane + 64 + 2 * lane);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) { a0 += x0[u].x; a1 += x0[u].y; b0 += x1[u].x; b1 += x1[u].y; }
+  }
+  for (; s < S; ++s) {
+    const float2 x0 = *reinterpret_cast<const float2*>(src + s * plane + 2 * lane);
+    const float2 x1 = *reinterpret_cast<const float2*>(src + s * plane + 64 + 2 * lane);
+    a0 += x0.x; a1 += x0.y; b0 += x1.x; b1 += x1.y;
+  }
+  if (slot >= a.Hq + a.Hkv) {  // value head: to the cache
+    uint16_t* dst = a.cv + (((long long)b * a.Hkv + (slot - a.Hq - a.Hkv)) * a.s_max + pos) * 128;
+    *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf16x2(a0, a1);
+    *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf16x2(b0, b1);
+    return;
+  }
+  const bool is_q = slot < a.Hq;
+  const uint16_t* wn = is_q ? a.q_norm : a.k_norm;
+  const float ss = warp_sum(a0 * a0 + a1 * a1 + b0 * b0 + b1 * b1);
+  const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+  const uint32_t wa = *reinterpret_cast<const uint32_t*>(wn + 2 * lane);
+  const uint32_t wb = *reinterpret_cast<const uint32_t*>(wn + 64 + 2 * lane);
+  a0 *= r * bf16_lo(wa); a1 *= r * bf16_hi(wa);
+  b0 *= r * bf16_lo(wb); b1 *= r * bf16_hi(wb);
+  const float4 cs = *reinterpret_cast<const float4*>(a.rope + ((long long)pos * 64 + 2 * lane) * 2);
+  const float o_a0 = a0 * cs.x - b0 * cs.y, o_b0 = a0 * cs.y + b0 * cs.x;
+  const float o_a1 = a1 * cs.z - b1 * cs.w, o_b1 = a1 * cs.w + b1 * cs.z;
+  uint16_t* dst = is_q ? qkv + (long long)m * ldqkv + (long long)slot * 128
+                       : a.ck + (((long long)b * a.Hkv + (slot - a.Hq)) * a.s_max + pos) * 128;
+  *reinterpret_cast<uint32_t*>(dst + 2 * lane) = pack_bf16x2(o_a0, o_a1);
+  *reinterpret_cast<uint32_t*>(dst + 64 + 2 * lane) = pack_bf16x2(o_b0, o_b1);
+}
+
+// Split-K completion of a residual GEMM fused with the RMSNorm that follows it: one
+// CTA of 1024 threads per token row m, PER = N / 1024 features per thread; out[m] =
+// resid[m] + sum_s part[s][m] (summed in split order), then norm_out[m] =
+// out[m] * rsqrt(mean(out[m]^2) + eps) * w on the fp32 values.
+template <int PER>
+__global__ void __launch_bounds__(1024) splitk_resid_norm_kernel(const float* __restrict__ part, int S, int M, int N,
+                                                                 int resid_f32, int out_f32,
+                                                                 const void* __restrict__ resid, long long ldr,
+                                                                 void* __restrict__ out, long long ldo,
+                                                                 const uint16_t* __restrict__ w,
+                                                                 uint16_t* __restrict__ norm_out, float eps) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_red[32];
+  const int m = blockIdx.x;
+  const long long plane = (long long)M * N;
+  const float* src = part + (long long)m * N + threadIdx.x;
+  float v[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) v[i] = 0.f;
+  int s = 0;
+  for (; s + 4 <= S; s += 4) {  // four splits' loads in flight, added in split order
+    float x[4][PER];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int i = 0; i < PER; ++i) x[u][i] = src[(s + u) * plane + i * 1024];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int i = 0; i < PER; ++i) v[i] += x[u][i];
+  }
+  for (; s < S; ++s)
+#pragma unroll
+    for (int i = 0; i < PER; ++i) v[i] += src[s * plane + i * 1024];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int n = i * 1024 + threadIdx.x;
+    v[i] += resid_f32 ? static_cast<const float*>(resid)[(long long)m * ldr + n]
+                      : __uint_as_float((uint32_t)static_cast<const uint16_t*>(resid)[(long long)m * ldr + n] << 16);
+    if (out_f32) static_cast<float*>(out)[(long long)m * ldo + n] = v[i];
+    else static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_bf16_bits(v[i]);
+    ss += v[i] * v[i];
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) tot += s_red[i];
+  const float r = rsqrtf(tot / (float)N + eps);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int n = i * 1024 + threadIdx.x;
+    norm_out[(long long)m * ldo + n] = to_bf16_bits(v[i] * r * bf16_lo((uint32_t)w[n]));
+  }
+}
+
 // --------------------------------------------------------------------------- host side
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -812,8 +935,25 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   if (g.k_splits > 1) {
     const int M = d.swap ? d.q_rows : d.p_rows, N = d.swap ? d.p_rows : d.q_rows;
     const long long n_out = (long long)M * (d.epi == kEpiSwiglu ? N / 2 : N);
-    q3_launch(splitk_reduce_kernel, (unsigned)((n_out + 255) / 256), 256, 0, s, 
-        g.partial, g.k_splits, M, N, d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo);
+    if (d.qk_in_reduce && d.swap && d.epi == kEpiStore) {
+      const long long warps = (long long)M * (d.qk.Hq + 2 * d.qk.Hkv);
+      q3_launch(splitk_qkrope_kernel, (unsigned)((warps * 32 + 255) / 256), 256, 0, s, g.partial, g.k_splits, M, N,
+                static_cast<uint16_t*>(d.out), d.ldo, d.qk, err);
+      if (d.fused) *d.fused = 1;
+    } else if (d.norm_out && d.norm_w && d.epi == kEpiResid && (N == 1024 || N == 2048)) {
+      if (N == 1024)
+        q3_launch(splitk_resid_norm_kernel<1>, (unsigned)M, 1024, 0, s, g.partial, g.k_splits, M, N,
+                  d.resid_f32 ? 1 : 0, d.out_f32 ? 1 : 0, d.resid, d.ldr, d.out, d.ldo, d.norm_w, d.norm_out,
+                  d.norm_eps);
+      else
+        q3_launch(splitk_resid_norm_kernel<2>, (unsigned)M, 1024, 0, s, g.partial, g.k_splits, M, N,
+                  d.resid_f32 ? 1 : 0, d.out_f32 ? 1 : 0, d.resid, d.ldr, d.out, d.ldo, d.norm_w, d.norm_out,
+                  d.norm_eps);
+      if (d.fused) *d.fused = 1;
+    } else {
+      q3_launch(splitk_reduce_kernel, (unsigned)((n_out + 255) / 256), 256, 0, s, g.partial, g.k_splits, M, N,
+                d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo);
+    }
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -51,6 +51,17 @@ struct GemmDesc {
   QKRopeArgs qk;                       // kEpiQKRope only
   float* partial = nullptr;            // optional split-K scratch (fp32)
   size_t partial_bytes = 0;
+  // When K is split, the kernel that sums the partials can also finish the next step:
+  //  qk_in_reduce (store epilogue of the fused QKV projection): per-head QK-norm, RoPE
+  //    and the KV-cache write, with the qk arguments (q written back to out);
+  //  norm_out (residual epilogue): norm_out = RMSNorm(out) * norm_w for every token row
+  //    (row stride ldo).
+  // *fused is set to 1 when that happened, else left as it is.
+  bool qk_in_reduce = false;
+  const uint16_t* norm_w = nullptr;
+  uint16_t* norm_out = nullptr;
+  float norm_eps = 1e-6f;
+  int* fused = nullptr;
 };
 
 // Scratch the block calls reserve for split-K partials of small-M GEMMs.
