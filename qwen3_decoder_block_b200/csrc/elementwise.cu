@@ -17,51 +17,51 @@ namespace q3 {
 // One warp per row; each lane owns 8 consecutive elements of every 256-wide
 // slice (n <= 2048, n % 256 == 0).
 // ---------------------------------------------------------------------------
+// Two passes over the row: the sum of squares, then a second read (an L1 hit) to scale
+// and store, so that a thread holds no row values and 64 warps per SM keep rows in
+// flight.
 template <bool IN_F32>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
-                                                      const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
-                                                      long long ldo, int rows, int n, float eps) {
+__device__ __forceinline__ void rms_load8(const void* x, long long off, float (&v)[8]) {
+  if (IN_F32) {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + off);
+    const float4 a = src[0], b = src[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + off);
+    v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
+    v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+  }
+}
+
+template <bool IN_F32>
+__global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
+                                                         const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
+                                                         long long ldo, int rows, int n, float eps) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int n_warps = (gridDim.x * blockDim.x) >> 5;
-  const int slices = n >> 8;
   for (int row = warp_global; row < rows; row += n_warps) {
-    float v[8][8];
     float ss = 0.f;
+    for (int col = lane * 8; col < n; col += 256) {
+      float v[8];
+      rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      if (s < slices) {
-        const int col = s * 256 + lane * 8;
-        if (IN_F32) {
-          const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (long long)row * ldx + col);
-          float4 a = src[0], b = src[1];
-          v[s][0] = a.x; v[s][1] = a.y; v[s][2] = a.z; v[s][3] = a.w;
-          v[s][4] = b.x; v[s][5] = b.y; v[s][6] = b.z; v[s][7] = b.w;
-        } else {
-          uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (long long)row * ldx + col);
-          v[s][0] = bf16_lo(a.x); v[s][1] = bf16_hi(a.x); v[s][2] = bf16_lo(a.y); v[s][3] = bf16_hi(a.y);
-          v[s][4] = bf16_lo(a.z); v[s][5] = bf16_hi(a.z); v[s][6] = bf16_lo(a.w); v[s][7] = bf16_hi(a.w);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) ss += v[s][j] * v[s][j];
-      }
+      for (int j = 0; j < 8; ++j) ss += v[j] * v[j];
     }
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)n + eps);
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      if (s < slices) {
-        const int col = s * 256 + lane * 8;
-        uint4 wv = *reinterpret_cast<const uint4*>(w + col);
-        uint4 o;
-        o.x = pack_bf16x2(v[s][0] * r * bf16_lo(wv.x), v[s][1] * r * bf16_hi(wv.x));
-        o.y = pack_bf16x2(v[s][2] * r * bf16_lo(wv.y), v[s][3] * r * bf16_hi(wv.y));
-        o.z = pack_bf16x2(v[s][4] * r * bf16_lo(wv.z), v[s][5] * r * bf16_hi(wv.z));
-        o.w = pack_bf16x2(v[s][6] * r * bf16_lo(wv.w), v[s][7] * r * bf16_hi(wv.w));
-        *reinterpret_cast<uint4*>(out + (long long)row * ldo + col) = o;
-      }
+    for (int col = lane * 8; col < n; col += 256) {
+      float v[8];
+      rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
+      const uint4 wv = *reinterpret_cast<const uint4*>(w + col);
+      uint4 o;
+      o.x = pack_bf16x2(v[0] * r * bf16_lo(wv.x), v[1] * r * bf16_hi(wv.x));
+      o.y = pack_bf16x2(v[2] * r * bf16_lo(wv.y), v[3] * r * bf16_hi(wv.y));
+      o.z = pack_bf16x2(v[4] * r * bf16_lo(wv.z), v[5] * r * bf16_hi(wv.z));
+      o.w = pack_bf16x2(v[6] * r * bf16_lo(wv.w), v[7] * r * bf16_hi(wv.w));
+      *reinterpret_cast<uint4*>(out + (long long)row * ldo + col) = o;
     }
   }
 }
