@@ -23,6 +23,10 @@
  *   - Conditions only visible on the device (a position beyond the cache, a
  *     token id outside the vocabulary, an expired bounded wait) are recorded in
  *     a device error word; qwen3_check_device_error() reads and clears it.
+ *   - Kernels are launched with programmatic dependent launch (each kernel's set-up
+ *     overlaps the end of the previous one on the stream) and large prefill GEMMs run
+ *     on pairs of CTAs (clusters of 2). The environment variables QWEN3_PDL=0 and
+ *     QWEN3_GEMM_PAIR=0, read once per process, turn either off.
  */
 #ifndef QWEN3BLK_H
 #define QWEN3BLK_H
@@ -248,8 +252,13 @@ int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, l
                                void* stream);
 
 /* Decode attention for one query per sequence at position cache_len[b] over kv positions
- * 0..cache_len[b]; split over 128-key chunks, partials in ws
- * (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max) suffices). */
+ * 0..cache_len[b] ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and
+ * prefill 与 decode). qkv: [B][ldqkv] bf16 with the Hq query heads (post-norm, post-RoPE)
+ * at its start; ldqkv a multiple of 8 and >= Hq*128. The keys are split into 256-key
+ * chunks whose (max, sum, unnormalised output) partials go to ws and are merged with
+ * log-sum-exp weights (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max)
+ * suffices). Hq / Hkv must be 1, 2, 4, 8 or 16. A position past the cache
+ * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY. */
 int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                               const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                               void* ws, size_t ws_bytes, void* stream);
