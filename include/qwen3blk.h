@@ -99,7 +99,8 @@ typedef enum {
   QWEN3_OP_BLOCK_DECODE = 2,
   QWEN3_OP_MOE_BLOCK = 3,
   QWEN3_OP_STACK_PREFILL = 4,
-  QWEN3_OP_STACK_DECODE = 5
+  QWEN3_OP_STACK_DECODE = 5,
+  QWEN3_OP_GENERATE = 6  /* qwen3_generate_greedy: T = prompt length */
 } qwen3_op;
 
 typedef enum { QWEN3_MODE_PREFILL = 0, QWEN3_MODE_DECODE = 1 } qwen3_mode;
@@ -209,6 +210,24 @@ int qwen3_stack_forward(const qwen3_config* cfg, const qwen3_bf16* embed, const 
                         const qwen3_kv_layer* kv, const float* rope, float* logits, int last_only, void* ws,
                         size_t ws_bytes, void* stream);
 
+/* Greedy generation: the prompt runs as one prefill of the stack, then one decode step
+ * per further token ([P-Mini] section prefill 与 decode; [P-MoE] last-position logits),
+ * every token chosen as the argmax of the fp32 logits (ties: lower id).
+ *   prompt_ids  [B*T] int32 (device), sequence b at rows b*T..b*T+T-1, positions 0..T-1
+ *   n_new       new tokens per sequence (>= 1): token 0 from the prompt's last logits,
+ *               token s (s >= 1) from a decode step at position T+s-1 fed token s-1
+ *   kv          host array of n_layers cache descriptors, s_max >= T + n_new - 1;
+ *               positions 0..T+n_new-2 are written
+ *   out_ids     [B, n_new] int32 (device)
+ *   ws          qwen3_workspace_size(cfg, QWEN3_OP_GENERATE, B, T, s_max) bytes; it also holds
+ *               the [B, V] fp32 logits of the current step and the cache lengths.
+ * Everything is enqueued on `stream` (one stack prefill, n_new - 1 stack decode steps and
+ * an argmax after each); the caller may capture the whole call in a CUDA graph. */
+int qwen3_generate_greedy(const qwen3_config* cfg, const qwen3_bf16* embed, const qwen3_layer_weights* layers,
+                          const qwen3_bf16* final_norm, const int* prompt_ids, int B, int T, int n_new,
+                          const qwen3_kv_layer* kv, const float* rope, int* out_ids, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* ------------------------------------------------ single kernels (ops) */
 
 /* out[r] = x[r] * rsqrt(mean(x[r]^2) + eps) * w  ([P-Mini] section RMSNorm formula).
@@ -280,6 +299,10 @@ int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, lo
 int qwen3_op_attention_decode_noalloc(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                                       const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                                       void* stream);
+
+/* out[r * ld_out] = argmax_j x[r * ldx + j], j < V (fp32 logits; ties: lower index; NaN
+ * never chosen). V % 4 == 0, x and ldx 16-byte aligned in bytes. */
+int qwen3_op_argmax(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, void* stream);
 
 /* out[m] = embed[ids[m]] ([P-MoE] section 5), bf16 or fp32 (out_f32). */
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,

@@ -20,7 +20,7 @@ if not os.path.exists(LIB_PATH):
 lib = ctypes.CDLL(LIB_PATH)
 
 OK, EINVAL, ESHAPE, EALIGN, ECAPACITY, EWORKSPACE, ECUDA, ETIMEOUT, EDEVICE = 0, -1, -2, -3, -4, -5, -6, -7, -8
-OP_BLOCK_PREFILL, OP_BLOCK_DECODE, OP_MOE_BLOCK, OP_STACK_PREFILL, OP_STACK_DECODE = 1, 2, 3, 4, 5
+OP_BLOCK_PREFILL, OP_BLOCK_DECODE, OP_MOE_BLOCK, OP_STACK_PREFILL, OP_STACK_DECODE, OP_GENERATE = 1, 2, 3, 4, 5, 6
 MODE_PREFILL, MODE_DECODE = 0, 1
 EPI_STORE, EPI_RESID, EPI_SWIGLU = 0, 1, 2
 
@@ -63,6 +63,8 @@ _SIGS = {
                          _vp, _sz, _vp], _i),
     "qwen3_stack_forward": ([_P(Config), _vp, _P(LayerWeights), _vp, _vp, _i, _i, _i, _vp, _P(KVLayer), _vp, _vp,
                              _i, _vp, _sz, _vp], _i),
+    "qwen3_generate_greedy": ([_P(Config), _vp, _P(LayerWeights), _vp, _vp, _i, _i, _i, _P(KVLayer), _vp, _vp, _vp,
+                               _sz, _vp], _i),
     "qwen3_profile_begin": ([_i], _i),
     "qwen3_profile_end": ([_vp], _i),
     "qwen3_profile_record": ([_i, ctypes.c_char_p, _i, _P(_f)], _i),
@@ -74,6 +76,7 @@ _SIGS = {
     "qwen3_op_attention_decode": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp, _sz, _vp], _i),
     "qwen3_op_attention_decode_noalloc": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_embed": ([_vp, _i, _vp, _i, _i, _vp, _i, _vp], _i),
+    "qwen3_op_argmax": ([_vp, _ll, _i, _i, _vp, _ll, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -218,7 +221,22 @@ def stack_forward(cfg, embed, layers, final_norm, ids, B, T, mode, pos_or_len, k
                                    ws.numel() * ws.element_size(), _stream(stream)), "stack_forward")
 
 
+def generate_greedy(cfg, embed, layers, final_norm, prompt_ids, B, T, n_new, kvs, rope, out_ids, ws,
+                    stream=None) -> None:
+    """Prefill the prompt, then n_new - 1 decode steps; out_ids [B, n_new] int32."""
+    n = len(layers)
+    larr = (LayerWeights * n)(*layers)
+    karr = (KVLayer * n)(*kvs)
+    _check(lib.qwen3_generate_greedy(ctypes.byref(cfg), _ptr(embed), larr, _ptr(final_norm), _ptr(prompt_ids), B, T,
+                                     n_new, karr, _ptr(rope), _ptr(out_ids), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream)), "generate_greedy")
+
+
 # ------------------------------------------------------------------------- single kernels
+def op_argmax(x, rows, V, out, ldx=None, ld_out=1, stream=None) -> None:
+    _check(lib.qwen3_op_argmax(_ptr(x), ldx or V, rows, V, _ptr(out), ld_out, _stream(stream)), "op_argmax")
+
+
 def op_rmsnorm(x, w, out, rows, n, eps, ldx=None, ldo=None, stream=None) -> None:
     import torch
     x_f32 = 1 if x.dtype == torch.float32 else 0

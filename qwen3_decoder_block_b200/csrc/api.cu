@@ -30,6 +30,9 @@ int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, voi
 int launch_pack_gate_up(const uint16_t* gate, const uint16_t* up, long long mat_stride, int n_mats, int I, int H,
                         uint16_t* out, cudaStream_t s);
 int launch_advance_lengths(int* len, int B, cudaStream_t s);
+int launch_argmax_rows(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, int* next,
+                       cudaStream_t s);
+int launch_fill_lengths(int* len, int B, int value, cudaStream_t s);
 int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv,
                              const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
                              long long ldo, int* err, cudaStream_t s);
@@ -614,8 +617,21 @@ int qwen3_rope_table(const qwen3_config* c, float* rope, void* stream) {
   return 0;
 }
 
+// Greedy generation: the stack's workspace (the larger of prefill and decode) followed
+// by the step's logits [B, V] fp32, the cache lengths [B] and the next ids [B].
+static size_t generate_stack_bytes(const qwen3_config& c, int B, int T, int s_max) {
+  const size_t a = carve(c, QWEN3_OP_STACK_PREFILL, B, T, s_max, nullptr, nullptr);
+  const size_t d = carve(c, QWEN3_OP_STACK_DECODE, B, 1, s_max, nullptr, nullptr);
+  return ((a > d ? a : d) + 255) & ~(size_t)255;
+}
+static size_t generate_extra_bytes(const qwen3_config& c, int B) {
+  return (((size_t)B * c.vocab * sizeof(float) + 255) & ~(size_t)255) + 2 * (((size_t)B * sizeof(int) + 255) & ~(size_t)255);
+}
+
 size_t qwen3_workspace_size(const qwen3_config* c, int op, int B, int T, int s_max) {
   if (!c || validate_cfg(c) != 0 || B <= 0 || s_max <= 0) return 0;
+  if (op == QWEN3_OP_GENERATE)
+    return T > 0 ? generate_stack_bytes(*c, B, T, s_max) + generate_extra_bytes(*c, B) : 0;
   if (op < QWEN3_OP_BLOCK_PREFILL || op > QWEN3_OP_STACK_DECODE) return 0;
   if (op != QWEN3_OP_BLOCK_DECODE && op != QWEN3_OP_STACK_DECODE && T <= 0) return 0;
   return carve(*c, op, B, T, s_max, nullptr, nullptr);
@@ -1035,6 +1051,58 @@ int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* q
   return finish(launch_attention_decode_static(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
                                                kv->s_max, o, ldo, device_error_word(),
                                                static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_op_argmax(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(x && out, QWEN3_EINVAL, "argmax: NULL pointer");
+  Q3_CHECK(rows > 0 && V > 0 && ld_out > 0, QWEN3_EINVAL, "argmax: rows, V and ld_out must be positive");
+  Q3_CHECK(V % 4 == 0 && aligned16(x) && ldx % 4 == 0 && ldx >= V, QWEN3_EALIGN,
+           "argmax: V and ldx must be multiples of 4 (16-byte rows), ldx >= V");
+  int rc;
+  if ((rc = check_device())) return rc;
+  return finish(launch_argmax_rows(x, ldx, rows, V, out, ld_out, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+int qwen3_generate_greedy(const qwen3_config* c, const qwen3_bf16* embed, const qwen3_layer_weights* layers,
+                          const qwen3_bf16* final_norm, const int* prompt_ids, int B, int T, int n_new,
+                          const qwen3_kv_layer* kv, const float* rope, int* out_ids, void* ws, size_t ws_bytes,
+                          void* stream) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(prompt_ids && out_ids && kv && ws && layers, QWEN3_EINVAL, "generate: NULL argument");
+  Q3_CHECK(aligned16(ws), QWEN3_EALIGN, "generate: workspace not 16-byte aligned");
+  Q3_CHECK(B > 0 && T > 0 && n_new > 0, QWEN3_EINVAL, "generate: B (%d), T (%d) and n_new (%d) must be positive", B,
+           T, n_new);
+  const long long last_pos = (long long)T + n_new - 1;  // positions 0..last_pos-1 are written
+  Q3_CHECK(last_pos - 1 < kv[0].s_max && last_pos - 1 < c->max_pos, QWEN3_ECAPACITY,
+           "generate: positions up to %lld exceed the cache capacity (%d) or max_pos (%d)", last_pos - 1, kv[0].s_max,
+           c->max_pos);
+  const size_t need = qwen3_workspace_size(c, QWEN3_OP_GENERATE, B, T, kv[0].s_max);
+  Q3_CHECK(need > 0 && ws_bytes >= need, QWEN3_EWORKSPACE, "generate: workspace has %zu bytes, needs %zu", ws_bytes,
+           need);
+  const size_t stack_bytes = generate_stack_bytes(*c, B, T, kv[0].s_max);
+  char* base = static_cast<char*>(ws);
+  float* logits = reinterpret_cast<float*>(base + stack_bytes);
+  int* lens = reinterpret_cast<int*>(base + stack_bytes + (((size_t)B * c->vocab * sizeof(float) + 255) & ~(size_t)255));
+  int* next = lens + ((((size_t)B * sizeof(int) + 255) & ~(size_t)255) / sizeof(int));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // prefill the prompt at positions 0..T-1, logits of each sequence's last position
+  if ((rc = finish(launch_fill_lengths(lens, B, 0, s)))) return rc;
+  if ((rc = qwen3_stack_forward(c, embed, layers, final_norm, prompt_ids, B, T, QWEN3_MODE_PREFILL, lens, kv, rope,
+                                logits, 1, ws, stack_bytes, stream)))
+    return rc;
+  if ((rc = finish(launch_argmax_rows(logits, c->vocab, B, c->vocab, out_ids, n_new, next, s)))) return rc;
+  if ((rc = finish(launch_fill_lengths(lens, B, T, s)))) return rc;
+  // one decode step per further token; the stack advances lens on the device
+  for (int t = 1; t < n_new; ++t) {
+    if ((rc = qwen3_stack_forward(c, embed, layers, final_norm, next, B, 1, QWEN3_MODE_DECODE, lens, kv, rope,
+                                  logits, 1, ws, stack_bytes, stream)))
+      return rc;
+    if ((rc = finish(launch_argmax_rows(logits, c->vocab, B, c->vocab, out_ids + t, n_new, next, s)))) return rc;
+  }
+  return 0;
 }
 
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,

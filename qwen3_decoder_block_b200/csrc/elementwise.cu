@@ -235,4 +235,76 @@ int launch_advance_lengths(int* len, int B, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
+// ---------------------------------------------------------------------------
+// Greedy token choice: out[r * ld_out] = next[r] = argmax_j x[r][j] over the V fp32
+// logits of row r, ties toward the lower id ([P-Mini] section prefill 与 decode: the
+// next token comes from the last position's logits). One CTA of 1024 threads per row,
+// 16-byte loads (V % 4 == 0); NaN never wins a comparison.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) argmax_rows_kernel(const float* __restrict__ x, long long ldx, int V,
+                                                           int* __restrict__ out, long long ld_out,
+                                                           int* __restrict__ next) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float s_v[32];
+  __shared__ int s_i[32];
+  const int r = blockIdx.x;
+  const float4* row = reinterpret_cast<const float4*>(x + (long long)r * ldx);
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = threadIdx.x; c < V / 4; c += blockDim.x) {  // ascending ids per thread: strict > keeps the lower id
+    const float4 v = row[c];
+    const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (e[k] > best || (e[k] == best && 4 * c + k < bi)) { best = e[k]; bi = 4 * c + k; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) { s_v[warp] = best; s_i[warp] = bi; }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    best = lane < nw ? s_v[lane] : -INFINITY;
+    bi = lane < nw ? s_i[lane] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ob > best || (ob == best && oi < bi)) { best = ob; bi = oi; }
+    }
+    if (lane == 0) {
+      const int id = bi == 0x7fffffff ? 0 : bi;  // a row of NaN picks id 0
+      out[(long long)r * ld_out] = id;
+      if (next) next[r] = id;
+    }
+  }
+}
+
+int launch_argmax_rows(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, int* next,
+                       cudaStream_t s) {
+  if (rows <= 0) return 0;
+  q3_launch(argmax_rows_kernel, rows, 1024, 0, s, x, ldx, V, out, ld_out, next);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+// len[b] = value for every sequence.
+__global__ void fill_lengths_kernel(int* len, int B, int value) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) len[b] = value;
+}
+
+int launch_fill_lengths(int* len, int B, int value, cudaStream_t s) {
+  if (B <= 0) return 0;
+  q3_launch(fill_lengths_kernel, (B + 127) / 128, 128, 0, s, len, B, value);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
 }  // namespace q3
