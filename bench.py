@@ -362,8 +362,10 @@ def run_decode(q3, torch, args, peaks):
     step_ms = ms / S
     hbm = peaks["hbm_gbs"]
     del graph
+    gen = run_generate(q3, torch, cfg, layers, embed, fnorm, kvs, rope, B, s_max, stream)
     return {
         "value": B * S / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": step_ms,
+        "generate": gen,
         "workload": f"Qwen3-0.6B 28-layer decode, B{B}, {L0} cached tokens, {S} steps (positions {L0}..{L0 + S - 1}), "
                     "CUDA-graph replay per step",
         "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes + w_bytes,
@@ -379,6 +381,33 @@ def run_decode(q3, torch, args, peaks):
         "kernels": {k: {kk: round(vv, 5) for kk, vv in v.items()} for k, v in kernels.items()},
         "gpu_launches_per_step": len(records) / 8,
     }
+
+
+def run_generate(q3, torch, cfg, layers, embed, fnorm, kvs, rope, B, s_max, stream, T=128, n_new=64):
+    """The library's greedy loop (qwen3_generate_greedy): a T-token prompt per sequence,
+    then n_new tokens (one stack prefill, n_new - 1 decode steps, an argmax after each),
+    launched eagerly on one stream and timed with CUDA events around the call."""
+    from qwen3_decoder_block_b200 import synth
+    prompt = torch.empty(B * T, dtype=torch.int32, device="cuda")
+    synth.uniform_int_device(prompt.data_ptr(), B * T, SEED_DECODE, synth.TID_IDS, cfg.vocab)
+    ws = torch.empty(q3.workspace_size(cfg, q3.OP_GENERATE, B, T, s_max), dtype=torch.uint8, device="cuda")
+    out = torch.empty((B, n_new), dtype=torch.int32, device="cuda")
+    times = []
+    with torch.cuda.stream(stream):
+        for it in range(3):
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record(stream)
+            q3.generate_greedy(cfg, embed, layers, fnorm, prompt, B, T, n_new, kvs, rope, out, ws, stream)
+            end.record(stream)
+            end.synchronize()
+            if it > 0:
+                times.append(start.elapsed_time(end))
+    if q3.check_device_error(stream) != 0:
+        raise RuntimeError("generate: device error")
+    ms = min(times)
+    return {"value": B * n_new / (ms * 1e-3), "unit": "generated tokens/s", "ms_per_call": ms,
+            "workload": f"Qwen3-0.6B greedy generation, B{B}, {T}-token prompt + {n_new} new tokens "
+                        f"(one stack prefill, {n_new - 1} decode steps, device argmax), eager launches"}
 
 
 def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
