@@ -469,6 +469,58 @@ def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
             "kernels_ms": {kk: round(vv["ms_per_step"], 4) for kk, vv in kern.items()}}
 
 
+def run_moe_decode(q3, torch, args, peaks, B=64, L0=4096, seed=1005):
+    """One decode step of the c4-shaped MoE block (hidden 2048, 32/4 heads, 128 experts x
+    768, top-8) for B sequences holding L0 cached tokens: qwen3_moe_block with T = 1 at
+    position L0. HBM-bound: the bytes are the K/V read, the attention and router weights,
+    and the weights of every expert the step routes to (counted from the routing)."""
+    from qwen3_decoder_block_b200 import synth
+    cfg = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
+    H, D, hq, hkv = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads
+    w, keep = build_layer(q3, cfg, seed, 0, torch, moe=True)
+    s_max = L0 + 8
+    k = torch.empty((B, hkv, s_max, D), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    for t, which in ((k, synth.L_CACHE_K), (v, synth.L_CACHE_V)):
+        synth.normal_bf16_device(t.data_ptr(), B * hkv, L0, D, s_max * D, D, seed, synth.layer_tid(0, which), 0.0, 1.0)
+    kv = q3.kv_layer(k, v, s_max)
+    x0 = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
+    synth.normal_bf16_device(x0.data_ptr(), 1, 1, x0.numel(), 0, 0, seed, synth.TID_X, 0.0, 1.0)
+    x = x0.clone()
+    rope = torch.empty(q3.rope_table_bytes(cfg) // 4, dtype=torch.float32, device="cuda")
+    q3.rope_table(cfg, rope)
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    ws = torch.empty(q3.workspace_size(cfg, q3.OP_MOE_BLOCK, B, 1, s_max), dtype=torch.uint8, device="cuda")
+    idx = torch.empty((B, cfg.top_k), dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def call():
+        x.copy_(x0)
+        q3.moe_block(cfg, w, x, B, 1, lens, kv, rope, ws, idx, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    reps = max(10, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    assert q3.check_device_error() == 0
+    experts_hit = int(torch.unique(idx).numel())
+    Im, E = cfg.moe_intermediate, cfg.n_experts
+    kv_bytes = B * hkv * (L0 + 1) * D * 2 * 2
+    w_bytes = 2 * (H * (hq + 2 * hkv) * D + hq * D * H + E * H + experts_hit * 3 * H * Im)
+    nbytes = kv_bytes + w_bytes
+    return {"workload": f"MoE block decode step (hidden 2048, 32/4 heads, 128 experts x 768, top-8), B{B} at "
+                        f"{L0} cached tokens", "tokens_per_s": B / (ms * 1e-3), "ms_per_call": ms,
+            "experts_hit": experts_hit, "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+
+
 # --------------------------------------------------------------------------- oracle timing
 def oracle_sample(T_s: int, seed: int = SEED_PREFILL):
     """Times the fp64 oracle on one sequence of T_s tokens of the prefill workload
@@ -585,6 +637,7 @@ def main():
             "c3": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T32768", 1, 32768, 1003),
             "c4": run_single_layer(q3, torch, args, "MoE block prefill (hidden 2048, 32/4 heads, 128 experts x "
                                    "768, top-8), B1 x T4096", 1, 4096, 1004, moe=True),
+            "moe_decode": run_moe_decode(q3, torch, args, peaks),
         }
         torch.cuda.empty_cache()
     cpu = None

@@ -137,3 +137,40 @@ def test_moe_every_expert_selected(q3):
     np.testing.assert_array_equal(np.sort(gi, axis=1), np.tile(np.arange(E), (T, 1)))
     np.testing.assert_allclose(gw.sum(axis=1), 1.0, rtol=1e-5)
     np.testing.assert_array_equal(off, np.arange(E + 1) * T)
+
+
+def test_moe_block_decode_step(q3):
+    """One decode step per sequence through the MoE block (T = 1 at position cache_len[b],
+    attending the cached positions and itself), against the oracle composed from its
+    attention half with the cache, the router and the expert FFN."""
+    cfg = q3.make_config(hidden=512, n_q_heads=8, n_kv_heads=2, n_experts=32, top_k=4, moe_intermediate=128)
+    seed, lens = 1017, [0, 5, 130, 300]
+    B, s_max = len(lens), max(lens) + 4
+    D, hkv = cfg.head_dim, cfg.n_kv_heads
+    L = Layer(cfg, seed, moe=True, dense=False)
+    x = Tensor(seed, synth.TID_X, (B, cfg.hidden))
+    pk = Tensor(seed, 905, (B, hkv, s_max, D))
+    pv = Tensor(seed, 906, (B, hkv, s_max, D))
+    k, v, kv = kv_cache(cfg, B, s_max)
+    for b in range(B):
+        k[b, :, :lens[b]] = pk.gpu[b, :, :lens[b]]
+        v[b, :, :lens[b]] = pv.gpu[b, :, :lens[b]]
+    xg = x.gpu.clone()
+    kk = cfg.top_k
+    idx = torch.empty((B, kk), dtype=torch.int32, device="cuda")
+    w = torch.empty((B, kk), dtype=torch.float32, device="cuda")
+    q3.moe_block(cfg, L.c, xg, B, 1, torch.tensor(lens, dtype=torch.int32, device="cuda"), kv, rope_gpu(cfg),
+                 workspace(cfg, q3.OP_MOE_BLOCK, B, 1, s_max), idx, w)
+    assert_device_ok()
+    got, gi = from_gpu_bf16(xg), idx.cpu().numpy()
+    oc, Lo = oracle_config(cfg), L.oracle()
+    for b in range(B):
+        x1, _, _ = R.attention_half(x.f[b:b + 1], Lo, oc, np.array([lens[b]]),
+                                    pk.f[b][:, :lens[b]].transpose(1, 0, 2), pv.f[b][:, :lens[b]].transpose(1, 0, 2),
+                                    np.arange(lens[b]))
+        h2 = R.rms_norm(x1, Lo.post_norm, oc.rms_eps)
+        ridx, rw, _, margin = R.moe_route(h2, Lo.router, oc.top_k, oc.norm_topk_prob)
+        ref = x1 + R.moe_ffn(h2, ridx, rw, Lo.gate_up, Lo.down)
+        assert rel_frob(got[b:b + 1], ref) <= LAYER_REL_FROB and max_abs(got[b:b + 1], ref) <= LAYER_MAX_ABS
+        if margin[0] > 1e-3:
+            np.testing.assert_array_equal(np.sort(gi[b]), np.sort(ridx[0]))
