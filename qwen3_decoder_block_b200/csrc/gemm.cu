@@ -539,9 +539,7 @@ __global__ void __launch_bounds__(192, 1)
         if (heads > 0)
           qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
                        p < tl.p_end, rope_lo);
-        release_acc(buf);
-        continue;
-      }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
@@ -590,6 +588,7 @@ __global__ void __launch_bounds__(192, 1)
           const int p = tl.p0 + row;
           store_col_chunk(g, p, p < tl.p_end, tl.q0 + c * 32, tl.q_end, lane, tl.p0 + quad * 32, r);
         }
+      }
       }
       release_acc(buf);
     }
