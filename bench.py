@@ -34,6 +34,22 @@ DECODE_B, DECODE_CTX, DECODE_STEPS = 64, 4096, 128
 SEED_PREFILL, SEED_DECODE = 1001, 1002
 
 
+def max_over_ranks(dist, value: float, torch, device: str = "cuda") -> float:
+    """The slowest rank's value: every rank times its own GPU, the job takes as long as
+    the slowest (a no-op for one process)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, units_per_rank_step: float, steps: int, ms: float) -> float:
+    """Units per second of the whole job: every rank processes units_per_rank_step per
+    step (replicas, weak scaling) and the job's time is the slowest rank's ms."""
+    return world * units_per_rank_step * steps / (ms * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -220,11 +236,8 @@ def run_prefill(q3, torch, args, rank, world, dist, peaks):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(dist, e0.elapsed_time(e1), torch)
     if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     clk = clocks.stop() if rank == 0 else None
     assert q3.check_device_error() == 0
@@ -250,11 +263,7 @@ def run_prefill(q3, torch, args, rank, world, dist, peaks):
         out_host.copy_(last_rows, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), torch)
 
     kernels, prof_ms = summarize_profile(records, args.steps)
     g_tok, lm_tok = gemm_flops_per_token(cfg)
@@ -270,9 +279,9 @@ def run_prefill(q3, torch, args, rank, world, dist, peaks):
     per_step_ms = ms / args.steps
     n_launch = len(records) / args.steps
     return {
-        "value": world * M * args.steps / (ms * 1e-3),
+        "value": job_throughput(world, M, args.steps, ms),
         "ms_per_step": per_step_ms,
-        "e2e": {"value": world * M * args.steps / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(world, M, args.steps, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": M * 4, "d2h_bytes_per_step": B * cfg.vocab * 4},
         "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (all projections + LM head)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,

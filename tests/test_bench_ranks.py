@@ -1,0 +1,57 @@
+"""The bench's multi-process path on CPU: two gloo ranks (replicas) agree on the slowest
+rank's time and report the whole job's throughput from it."""
+import os
+import socket
+import sys
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, local_ms, q):
+    sys.path.insert(0, ROOT)
+    import bench
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        ms = bench.max_over_ranks(dist, local_ms[rank], torch, device="cpu")
+        dist.barrier()
+        q.put((rank, ms, bench.job_throughput(world, 8192, 10, ms)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_slowest_time_and_sum_the_work():
+    world, port = 2, _free_port()
+    local_ms = [120.0, 150.0]  # rank 1 is slower
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, local_ms, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    got = sorted(q.get(timeout=5) for _ in range(world))
+    for rank, ms, value in got:
+        assert ms == 150.0
+        assert value == pytest.approx(2 * 8192 * 10 / 0.150)
+
+
+def test_single_process_is_a_no_op():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(None, 12.5, torch) == 12.5
+    assert bench.job_throughput(1, 8192, 10, 1000.0) == pytest.approx(81920.0)
