@@ -300,6 +300,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   const void* act = b.h;
   if (g.swap) { g.P = w.w_qkv; g.p_rows = nqkv; g.ldp = H; g.Q = act; g.q_rows = (int)M; g.ldq = H; }
   else        { g.P = act; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_qkv; g.q_rows = nqkv; g.ldq = H; }
+  g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
   g.epi = kEpiStore;
   g.out = b.qkv;
   g.ldo = nqkv;
@@ -356,6 +357,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   o.K = c.n_q_heads * D;
   if (o.swap) { o.P = w.w_o; o.p_rows = H; o.ldp = o.K; o.Q = b.o; o.q_rows = (int)M; o.ldq = o.K; }
   else        { o.P = b.o; o.p_rows = (int)M; o.ldp = o.K; o.Q = w.w_o; o.q_rows = H; o.ldq = o.K; }
+  o.p_early = o.swap;  // weights; a library kernel of this call runs before this GEMM
   o.epi = kEpiResid;
   o.resid = x;
   o.resid_f32 = x_f32;
@@ -396,6 +398,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   g.K = H;
   if (g.swap) { g.P = w.w_gate_up; g.p_rows = 2 * I; g.ldp = H; g.Q = b.h; g.q_rows = (int)M; g.ldq = H; }
   else        { g.P = b.h; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_gate_up; g.q_rows = 2 * I; g.ldq = H; }
+  g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
   g.epi = kEpiSwiglu;
   g.out = b.act;
   g.ldo = I;
@@ -411,6 +414,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   d.K = I;
   if (d.swap) { d.P = w.w_down; d.p_rows = H; d.ldp = I; d.Q = b.act; d.q_rows = (int)M; d.ldq = I; }
   else        { d.P = b.act; d.p_rows = (int)M; d.ldp = I; d.Q = w.w_down; d.q_rows = H; d.ldq = I; }
+  d.p_early = d.swap;  // weights; a library kernel of this call runs before this GEMM
   d.epi = kEpiResid;
   d.resid = b.x1;
   d.resid_f32 = true;
@@ -450,6 +454,7 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   r.K = H;
   if (r.swap) { r.P = w.router; r.p_rows = E; r.ldp = H; r.Q = b.h; r.q_rows = (int)M; r.ldq = H; }
   else        { r.P = b.h; r.p_rows = (int)M; r.ldp = H; r.Q = w.router; r.q_rows = E; r.ldq = H; r.force_bn = 128; }
+  r.p_early = r.swap;  // weights; a library kernel of this call runs before this GEMM
   r.epi = kEpiStore;
   r.out = b.logits;
   r.out_f32 = true;
@@ -833,6 +838,7 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   g.K = H;
   if (g.swap) { g.P = embed; g.p_rows = c->vocab; g.ldp = H; g.Q = b.hf; g.q_rows = rows; g.ldq = H; }
   else        { g.P = b.hf; g.p_rows = rows; g.ldp = H; g.Q = embed; g.q_rows = c->vocab; g.ldq = H; }
+  g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
   g.epi = kEpiStore;
   g.out = logits;
   g.out_f32 = true;

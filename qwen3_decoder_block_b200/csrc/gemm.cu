@@ -55,6 +55,7 @@ struct GemmParams {
   float* partial;              // split-K partials [k_splits][tokens][features] (fp32)
   int epi, resid_f32, out_f32, swap;
   int tma_store;  // non-swap store/residual epilogues: stage in shared memory, TMA tile store
+  int p_early;    // P is final before this grid launches: its first tile's loads precede the grid-dependency wait
   void* out;
   long long ldo;
   const void* resid;
@@ -387,8 +388,23 @@ __global__ void __launch_bounds__(192, 1)
     if (PAIR) { tmem_alloc_pair(tmem_slot, C::TMEM_COLS); tmem_relinquish_pair(); }
     else      { tmem_alloc(tmem_slot, C::TMEM_COLS); tmem_relinquish(); }
   }
-  // Everything above touches only this CTA's own resources, so it overlaps the
-  // tail of the previous kernel on the stream; global data is read after the wait.
+  // P loads of the first tile issued before the wait (producer thread only): when P is
+  // a weight matrix that no kernel of this call writes, its stream from HBM overlaps
+  // the previous kernel, and only the Q (activation) halves of these stages wait.
+  int p_pre = 0;
+  if constexpr (!PAIR) {
+    if (g.p_early && g.n_groups == 0 && threadIdx.x == 0 && t_first < g.p_tiles * g.q_tiles * g.k_splits) {
+      const Tile tl = decode_tile<BN, BMT>(t_first, g, nullptr, nullptr);
+      p_pre = min(C::STAGES, tl.kb1 - tl.kb0);
+      for (int i = 0; i < p_pre; ++i) {
+        mbar_arrive_expect_tx(&full[i], C::STAGE_BYTES);
+        tma_load_2d(smem + i * C::STAGE_BYTES, &tmP, &full[i], (tl.kb0 + i) * BK, tl.p0);
+      }
+    }
+  }
+  // Everything above touches only this CTA's own resources (and, with p_early,
+  // memory no kernel of this call writes), so it overlaps the tail of the previous
+  // kernel on the stream; all other global data is read after the wait.
   pdl_wait();
   pdl_trigger();
   if (g.n_groups > 0) {
@@ -427,8 +443,16 @@ __global__ void __launch_bounds__(192, 1)
         const int a_row = tl.p0 + (int)rank * BM;
         const int b_row = tl.q_load + (int)rank * (BN / 2);
         for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
-          if (*s_abort || !mbar_wait(&empty[stage], phase ^ 1, g.err)) { ok = false; break; }
           uint8_t* sp = smem + stage * C::STAGE_BYTES;
+          if (issued < p_pre) {
+            // P already on its way to this (fresh) stage, whose barrier expects both
+            // halves: always add Q, so that every armed stage completes
+            tma_load_2d(sp + C::P_BYTES, &tmQ, &full[stage], kb * BK, b_row);
+            ++issued;
+            if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+            continue;
+          }
+          if (*s_abort || !mbar_wait(&empty[stage], phase ^ 1, g.err)) { ok = false; break; }
           if (PAIR) {
             const uint32_t fb = full_leader + stage * 8;
             if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
@@ -725,14 +749,14 @@ __global__ void __launch_bounds__(1024) splitk_resid_norm_kernel(const float* __
 #pragma unroll
   for (int i = 0; i < PER; ++i) v[i] = 0.f;
   int s = 0;
-  for (; s + 4 <= S; s += 4) {  // four splits' loads in flight, added in split order
-    float x[4][PER];
+  for (; s + 8 <= S; s += 8) {  // eight splits' loads in flight, added in split order
+    float x[8][PER];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
       for (int i = 0; i < PER; ++i) x[u][i] = src[(s + u) * plane + i * 1024];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
+    for (int u = 0; u < 8; ++u)
 #pragma unroll
       for (int i = 0; i < PER; ++i) v[i] += x[u][i];
   }
@@ -898,6 +922,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   g.k_splits = 1;
   g.kb_per_split = g.k_blocks;
   g.partial = nullptr;
+  g.p_early = d.p_early && !pair && d.n_groups == 0 ? 1 : 0;
   // Split K when the output has too few tiles to keep the SMs streaming: each split
   // writes fp32 partials, and a reduce kernel applies the epilogue.
   const long long out_tiles = (long long)g.p_tiles * g.q_tiles;

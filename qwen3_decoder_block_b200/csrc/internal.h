@@ -48,6 +48,11 @@ struct GemmDesc {
   int n_groups = 0;
   const int* group_offsets = nullptr;  // device, n_groups + 1 entries
   int force_bn = 0;                    // 0 = automatic
+  // P is final before the kernel launched just before this GEMM on the stream started
+  // (a weight matrix, when a library kernel of the same call precedes the GEMM; every
+  // library kernel waits for its predecessor before it lets its dependents launch):
+  // the first tile's P loads may then precede the grid-dependency wait.
+  bool p_early = false;
   QKRopeArgs qk;                       // kEpiQKRope only
   float* partial = nullptr;            // optional split-K scratch (fp32)
   size_t partial_bytes = 0;
