@@ -55,3 +55,27 @@ def test_single_process_is_a_no_op():
     import bench
     assert bench.max_over_ranks(None, 12.5, torch) == 12.5
     assert bench.job_throughput(1, 8192, 10, 1000.0) == pytest.approx(81920.0)
+
+
+def test_clock_summary_keeps_only_the_timed_window():
+    import datetime
+    sys.path.insert(0, ROOT)
+    import bench
+    t = datetime.datetime(2026, 1, 2, 3, 4, 5)
+
+    def row(dt_ms, mhz, cap="Not Active", thermal="Not Active"):
+        ts = (t + datetime.timedelta(milliseconds=dt_ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {mhz}, 1965, 900.1, 0x0, Not Active, {thermal}, Not Active, {cap}"
+
+    lines = [row(0, 1965), row(50, 1965, thermal="Active"),  # idle, before the window
+             row(120, 1800, cap="Active"), row(170, 1830, cap="Active"), row(220, 1860),
+             row(400, 1965)]  # after it
+    got = bench.ClockSampler.summarize(lines, t + datetime.timedelta(milliseconds=100),
+                                       t + datetime.timedelta(milliseconds=300))
+    assert got["samples"] == 3 and got["window"] == "timed region"
+    assert got["sm_mhz"] == 1830 and got["sm_max_mhz"] == 1965
+    assert got["reasons"] == ["sw_power_cap"]  # the thermal row lies outside the window
+    # no stamped row inside: every row, and the summary says so
+    got = bench.ClockSampler.summarize(lines, t + datetime.timedelta(seconds=5), t + datetime.timedelta(seconds=6))
+    assert got["window"] == "all samples" and got["samples"] == 6
+    assert bench.ClockSampler.summarize([], None, None)["reasons"] == ["no samples"]
