@@ -178,7 +178,9 @@ def build_layer(q3, cfg, seed, l, torch, moe=False):
         wd = torch.empty((H, I), **bf); fill(wd, tid(synth.L_WDOWN), 0.0, synth.W_STD)
         keep += [wgu, wd]
         kw.update(w_gate_up=wgu, w_down=wd)
-    return q3.layer_weights(**kw), keep
+    w = q3.layer_weights(**kw)
+    q3.check_layer_weights(cfg, w, q3.LAYER_MOE if moe else q3.LAYER_DENSE)
+    return w, keep
 
 
 def build_model(q3, cfg, seed, torch):

@@ -143,6 +143,26 @@ int qwen3_pack_gate_up(int I, int H, const qwen3_bf16* w_gate, const qwen3_bf16*
  * gives gate first, then up) into the same 16-row interleave per expert. */
 int qwen3_pack_moe_gate_up(int E, int Im, int H, const qwen3_bf16* gate_up_proj, qwen3_bf16* out, void* stream);
 
+/* Block kinds for qwen3_check_layer_weights. */
+typedef enum { QWEN3_LAYER_DENSE = 0, QWEN3_LAYER_MOE = 1 } qwen3_layer_kind;
+
+/* Two-way check of one layer's weight pointers for a block kind, on the host (reads no
+ * device memory; a set-up call). It restates for raw pointers the two-way check the
+ * pages run when they load weights ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构",
+ * section 加载官方权重：名字映射与双重校验: every expected tensor present with its
+ * shape, every model parameter covered):
+ *   - every member the kind reads is non-NULL (QWEN3_EINVAL) and 16-byte aligned
+ *     (QWEN3_EALIGN);
+ *   - every member the kind does not read is NULL (QWEN3_ESHAPE), so that a layer built
+ *     for the other kind, or a config of the wrong kind, is reported;
+ *   - with each member's size from cfg, no two members overlap (QWEN3_EINVAL), which is
+ *     what an offset into one weight arena computed with a wrong dimension produces;
+ *     the same pointer for two members of equal size (a shared read-only buffer) is
+ *     allowed.
+ * qwen3_last_error() names the member(s). The block calls check only the first
+ * point, so a struct that also carries the other kind's members stays usable there. */
+int qwen3_check_layer_weights(const qwen3_config* cfg, const qwen3_layer_weights* w, int kind);
+
 /* Synchronises `stream`, then returns and clears the device error word
  * (QWEN3_OK, QWEN3_ECAPACITY, QWEN3_EINVAL or QWEN3_ETIMEOUT). */
 int qwen3_check_device_error(void* stream);

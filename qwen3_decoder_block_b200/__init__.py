@@ -57,6 +57,7 @@ _SIGS = {
     "qwen3_pack_gate_up": ([_i, _i, _vp, _vp, _vp, _vp], _i),
     "qwen3_pack_moe_gate_up": ([_i, _i, _i, _vp, _vp, _vp], _i),
     "qwen3_check_device_error": ([_vp], _i),
+    "qwen3_check_layer_weights": ([_P(Config), _P(LayerWeights), _i], _i),
     "qwen3_block_prefill": ([_P(Config), _P(LayerWeights), _vp, _i, _i, _vp, _P(KVLayer), _vp, _vp, _sz, _vp], _i),
     "qwen3_block_decode": ([_P(Config), _P(LayerWeights), _vp, _i, _vp, _P(KVLayer), _vp, _vp, _sz, _vp], _i),
     "qwen3_moe_block": ([_P(Config), _P(LayerWeights), _vp, _i, _i, _vp, _P(KVLayer), _vp, _vp, _vp, _vp, _vp,
@@ -184,6 +185,14 @@ def layer_weights(**tensors) -> LayerWeights:
     for k, v in tensors.items():
         setattr(w, k, _ptr(v))
     return w
+
+
+LAYER_DENSE, LAYER_MOE = 0, 1
+
+
+def check_layer_weights(cfg: Config, w: LayerWeights, kind: int = LAYER_DENSE) -> None:
+    """Two-way check of a layer's weight pointers (host only); raises Qwen3Error."""
+    _check(lib.qwen3_check_layer_weights(ctypes.byref(cfg), ctypes.byref(w), kind), "check_layer_weights")
 
 
 def kv_layer(k, v, s_max: int) -> KVLayer:

@@ -678,6 +678,69 @@ int qwen3_pack_moe_gate_up(int E, int Im, int H, const qwen3_bf16* gate_up, qwen
                                     static_cast<cudaStream_t>(stream)));
 }
 
+// Two-way check of a layer's weight pointers (a set-up call; reads no device memory).
+// Forward: every member the block kind reads is set and 16-byte aligned. Reverse: every
+// member it does not read is NULL, so that weights built for the other kind (or a config
+// of the wrong kind) are reported instead of silently ignored. With the byte size of
+// each member taken from the config, no two members may overlap: an offset into one
+// weight arena computed with a wrong dimension shows up here. One read-only buffer may
+// serve two members of the same size (the same pointer), e.g. shared norm weights.
+int qwen3_check_layer_weights(const qwen3_config* c, const qwen3_layer_weights* w, int kind) {
+  g_last_error.clear();
+  int rc = validate_cfg(c);
+  if (rc) return rc;
+  Q3_CHECK(w, QWEN3_EINVAL, "check_layer_weights: weights pointer is NULL");
+  Q3_CHECK(kind == QWEN3_LAYER_DENSE || kind == QWEN3_LAYER_MOE, QWEN3_EINVAL,
+           "check_layer_weights: kind %d is neither QWEN3_LAYER_DENSE nor QWEN3_LAYER_MOE", kind);
+  const bool moe = kind == QWEN3_LAYER_MOE;
+  const char* kname = moe ? "MoE" : "dense";
+  if (moe)
+    Q3_CHECK(c->n_experts > 0 && c->moe_intermediate > 0, QWEN3_ESHAPE,
+             "check_layer_weights: a MoE layer needs n_experts > 0 and moe_intermediate > 0");
+  else
+    Q3_CHECK(c->intermediate > 0, QWEN3_ESHAPE, "check_layer_weights: a dense layer needs intermediate > 0");
+  const size_t H = c->hidden, D = c->head_dim, Hq = c->n_q_heads, Hkv = c->n_kv_heads;
+  const size_t I = moe ? 0 : c->intermediate, E = moe ? c->n_experts : 0, Im = moe ? c->moe_intermediate : 0;
+  struct Member {
+    const char* name;
+    const void* p;
+    size_t bytes;
+    bool read;
+  } m[] = {
+      {"in_norm", w->in_norm, H * 2, true},
+      {"w_qkv", w->w_qkv, (Hq + 2 * Hkv) * D * H * 2, true},
+      {"q_norm", w->q_norm, D * 2, true},
+      {"k_norm", w->k_norm, D * 2, true},
+      {"w_o", w->w_o, H * Hq * D * 2, true},
+      {"post_norm", w->post_norm, H * 2, true},
+      {"w_gate_up", w->w_gate_up, 2 * I * H * 2, !moe},
+      {"w_down", w->w_down, H * I * 2, !moe},
+      {"router", w->router, E * H * 2, moe},
+      {"moe_gate_up", w->moe_gate_up, E * 2 * Im * H * 2, moe},
+      {"moe_down", w->moe_down, E * H * Im * 2, moe},
+  };
+  const int n = (int)(sizeof(m) / sizeof(m[0]));
+  for (int i = 0; i < n; ++i) {
+    if (m[i].read) {
+      Q3_CHECK(m[i].p, QWEN3_EINVAL, "weights.%s is NULL but a %s layer reads it", m[i].name, kname);
+      Q3_CHECK(aligned16(m[i].p), QWEN3_EALIGN, "weights.%s is not 16-byte aligned", m[i].name);
+    } else {
+      Q3_CHECK(!m[i].p, QWEN3_ESHAPE, "weights.%s is set but a %s layer does not read it (wrong kind or config)",
+               m[i].name, kname);
+    }
+  }
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j) {
+      if (!m[i].p || !m[j].p) continue;
+      if (m[i].p == m[j].p && m[i].bytes == m[j].bytes) continue;
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(m[i].p), b0 = reinterpret_cast<uintptr_t>(m[j].p);
+      Q3_CHECK(a0 + m[i].bytes <= b0 || b0 + m[j].bytes <= a0, QWEN3_EINVAL,
+               "weights.%s (%zu bytes at %p) overlaps weights.%s (%zu bytes at %p)", m[i].name, m[i].bytes, m[i].p,
+               m[j].name, m[j].bytes, m[j].p);
+    }
+  return 0;
+}
+
 int qwen3_check_device_error(void* stream) {
   g_last_error.clear();
   cudaStream_t s = static_cast<cudaStream_t>(stream);

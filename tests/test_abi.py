@@ -123,3 +123,89 @@ def test_workspace_too_small_rejected(q3):
     st = q3.lib.qwen3_block_prefill(ctypes.byref(c), ctypes.byref(w), fake, 1, 16, fake, ctypes.byref(kv), fake,
                                     fake, 1024, None)
     assert st == q3.EWORKSPACE
+
+
+def _arena_layout(cfg, moe):
+    """Byte offsets of one layer's members laid out back to back in one arena, sizes
+    from the config (what a caller packing all weights into one buffer computes)."""
+    H, D, hq, hkv = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads
+    sizes = dict(in_norm=H, w_qkv=(hq + 2 * hkv) * D * H, q_norm=D, k_norm=D, w_o=H * hq * D, post_norm=H)
+    if moe:
+        E, Im = cfg.n_experts, cfg.moe_intermediate
+        sizes.update(router=E * H, moe_gate_up=E * 2 * Im * H, moe_down=E * H * Im)
+    else:
+        I = cfg.intermediate
+        sizes.update(w_gate_up=2 * I * H, w_down=H * I)
+    base, ptrs = 1 << 32, {}
+    for name, n in sizes.items():
+        ptrs[name] = base
+        base += (2 * n + 255) // 256 * 256
+    return ptrs, {k: 2 * v for k, v in sizes.items()}
+
+
+def _status(q3, cfg, ptrs, kind):
+    st = q3.lib.qwen3_check_layer_weights(ctypes.byref(cfg), ctypes.byref(q3.layer_weights(**ptrs)), kind)
+    return st, q3.lib.qwen3_last_error().decode()
+
+
+def test_layer_weights_two_way_check_accepts_correct_layouts(q3):
+    cfg = q3.config_qwen3_0_6b()
+    ptrs, _ = _arena_layout(cfg, moe=False)
+    assert _status(q3, cfg, ptrs, q3.LAYER_DENSE) == (0, "")
+    q3.check_layer_weights(cfg, q3.layer_weights(**ptrs))
+    # one read-only buffer for both per-head norms (same pointer, same size) is allowed
+    ptrs["k_norm"] = ptrs["q_norm"]
+    assert _status(q3, cfg, ptrs, q3.LAYER_DENSE)[0] == 0
+    moe = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
+    mptrs, _ = _arena_layout(moe, moe=True)
+    assert _status(q3, moe, mptrs, q3.LAYER_MOE)[0] == 0
+
+
+def test_layer_weights_forward_direction_every_read_member_present_and_aligned(q3):
+    cfg = q3.config_qwen3_0_6b()
+    ptrs, _ = _arena_layout(cfg, moe=False)
+    for name in ptrs:
+        bad = dict(ptrs)
+        del bad[name]
+        st, msg = _status(q3, cfg, bad, q3.LAYER_DENSE)
+        assert st == q3.EINVAL and f"weights.{name} is NULL" in msg
+    bad = dict(ptrs, w_o=ptrs["w_o"] + 8)
+    st, msg = _status(q3, cfg, bad, q3.LAYER_DENSE)
+    assert st == q3.EALIGN and "weights.w_o" in msg
+
+
+def test_layer_weights_reverse_direction_no_member_of_the_other_kind(q3):
+    cfg = q3.make_config(hidden=1024, n_q_heads=16, n_kv_heads=8, n_experts=32, top_k=4, moe_intermediate=256)
+    dense, _ = _arena_layout(cfg, moe=False)
+    moe, _ = _arena_layout(cfg, moe=True)
+    far = 1 << 40
+    st, msg = _status(q3, cfg, dict(dense, router=far), q3.LAYER_DENSE)
+    assert st == q3.ESHAPE and "weights.router is set but a dense layer" in msg
+    st, msg = _status(q3, cfg, dict(moe, w_down=far), q3.LAYER_MOE)
+    assert st == q3.ESHAPE and "weights.w_down is set but a MoE layer" in msg
+    # a dense layer checked as MoE: its FFN members are ones a MoE layer does not read,
+    # and without them the expert members are missing
+    st, msg = _status(q3, cfg, dense, q3.LAYER_MOE)
+    assert st == q3.ESHAPE and "weights.w_gate_up is set but a MoE layer" in msg
+    st, msg = _status(q3, cfg, {k: v for k, v in dense.items() if k not in ("w_gate_up", "w_down")}, q3.LAYER_MOE)
+    assert st == q3.EINVAL and "weights.router is NULL" in msg
+    st, _ = _status(q3, cfg, dense, 7)
+    assert st == q3.EINVAL
+
+
+def test_layer_weights_overlap_from_a_wrong_dimension_is_reported(q3):
+    """An arena laid out with n_kv_heads taken as 4 instead of 8: w_qkv is then larger
+    than the space left for it and runs into q_norm, the next member (the raw-pointer
+    form of the pages' shape mismatch)."""
+    cfg = q3.config_qwen3_0_6b()
+    wrong = q3.config_qwen3_0_6b()
+    wrong.n_kv_heads = 4
+    ptrs, _ = _arena_layout(wrong, moe=False)
+    st, msg = _status(q3, cfg, ptrs, q3.LAYER_DENSE)
+    assert st == q3.EINVAL and "weights.w_qkv" in msg and "overlaps weights.q_norm" in msg
+    # the same pointer for two members of different sizes is an overlap too
+    good, _ = _arena_layout(cfg, moe=False)
+    st, msg = _status(q3, cfg, dict(good, post_norm=good["w_o"]), q3.LAYER_DENSE)
+    assert st == q3.EINVAL and "overlaps" in msg
+    with pytest.raises(q3.Qwen3Error):
+        q3.check_layer_weights(cfg, q3.layer_weights(**dict(good, post_norm=good["w_o"])))
