@@ -561,10 +561,8 @@ def run_moe_decode(q3, torch, args, peaks, B=64, L0=4096, seed=1005):
 
 
 # --------------------------------------------------------------------------- oracle timing
-def oracle_sample(T_s: int, seed: int = SEED_PREFILL):
-    """Times the fp64 oracle on one sequence of T_s tokens of the prefill workload
-    (28 layers + final norm + tied LM head on all T_s positions)."""
-    import numpy as np
+def oracle_model(seed: int = SEED_PREFILL):
+    """The prefill workload's random weights in the oracle's layouts (fp64), drawn once."""
     import oracle.qwen3_ref as R
     from qwen3_decoder_block_b200 import synth
     cfg = R.QWEN3_0_6B
@@ -583,10 +581,32 @@ def oracle_sample(T_s: int, seed: int = SEED_PREFILL):
             w_gate=gen(t(synth.L_WGATE), (I, H)), w_up=gen(t(synth.L_WUP), (I, H)), w_down=gen(t(synth.L_WDOWN), (H, I))))
     embed = gen(synth.TID_EMBED, (cfg.vocab, H))
     fnorm = gen(synth.TID_FINAL_NORM, (H,), synth.NORM_MEAN, synth.NORM_STD)
+    return cfg, layers, embed, fnorm
+
+
+def oracle_sample(T_s: int, model=None, seed: int = SEED_PREFILL):
+    """Times the fp64 oracle on one sequence of T_s tokens of the prefill workload
+    (28 layers + final norm + tied LM head on all T_s positions)."""
+    import oracle.qwen3_ref as R
+    from qwen3_decoder_block_b200 import synth
+    cfg, layers, embed, fnorm = model if model is not None else oracle_model(seed)
     ids = synth.uniform_int(seed, synth.TID_IDS, (T_s,), cfg.vocab)
     t0 = time.perf_counter()
     R.stack_forward(ids, embed, layers, fnorm, cfg)
     return time.perf_counter() - t0
+
+
+# The reference arm's whole run (warm-up and timed steps) is sized to about
+# REF_BUDGET_S seconds at the oracle's measured rate on 8-16 host cores (66-87 tokens/s).
+REF_BUDGET_S = 150.0
+ORACLE_EST_TOKENS_S = 75.0
+
+
+def reference_tokens_per_step(steps: int, warmup: int) -> int:
+    """Tokens of the prefill workload per reference-arm step: the first n ids of one
+    sequence, n a multiple of 64 in [64, 2048]."""
+    n = int(REF_BUDGET_S * ORACLE_EST_TOKENS_S / max(1, steps + warmup)) // 64 * 64
+    return max(64, min(PREFILL_T, n))
 
 
 def blas_threads():
@@ -598,7 +618,7 @@ def blas_threads():
         return os.cpu_count()
 
 
-def cpu_baseline(T_s: int = 2048):
+def cpu_baseline(T_s: int = PREFILL_T):
     dt = oracle_sample(T_s)
     return {"value": T_s / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"one sequence of {T_s} tokens (prefill workload's first {T_s} ids) through the 28-layer "
@@ -617,7 +637,9 @@ def main():
     ap.add_argument("--no-configs", action="store_true")
     ap.add_argument("--workload", choices=["all", "prefill", "decode"], default="all",
                     help="prefill or decode alone (for profiler launch lists)")
-    ap.add_argument("--oracle-tokens", type=int, default=2048)
+    ap.add_argument("--oracle-tokens", type=int, default=None,
+                    help="oracle tokens per sample (default: 2048 for cpu_baseline; sized to the run "
+                         "for --impl reference)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -633,15 +655,20 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
-        steps = max(1, min(args.steps, 3))
-        times = [oracle_sample(args.oracle_tokens) for _ in range(max(1, min(args.warmup, 1)) + steps)][-steps:]
-        v = args.oracle_tokens / statistics.mean(times)
-        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-                "warmup": 1, "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+        # K timed steps after W warm-up steps, each the oracle on one bounded sample of
+        # the prefill workload (the first n token ids of one sequence)
+        n = args.oracle_tokens or reference_tokens_per_step(args.steps, args.warmup)
+        model = oracle_model()
+        times = [oracle_sample(n, model) for _ in range(args.warmup + args.steps)][args.warmup:]
+        total = sum(times)
+        v = n * args.steps / total
+        line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
                 "impl": "reference",
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                                 "sample": f"one sequence of {args.oracle_tokens} tokens per step"},
+                                 "sample": f"one sequence of {n} tokens (the prefill workload's first {n} ids) "
+                                           f"through the 28-layer stack + tied LM head in fp64 numpy, per step"},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -681,7 +708,7 @@ def main():
         torch.cuda.empty_cache()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "all":
-        cpu = cpu_baseline(args.oracle_tokens)
+        cpu = cpu_baseline(args.oracle_tokens or PREFILL_T)
     if dist:
         dist.barrier()
         dist.destroy_process_group()

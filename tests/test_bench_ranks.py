@@ -79,3 +79,43 @@ def test_clock_summary_keeps_only_the_timed_window():
     got = bench.ClockSampler.summarize(lines, t + datetime.timedelta(seconds=5), t + datetime.timedelta(seconds=6))
     assert got["window"] == "all samples" and got["samples"] == 6
     assert bench.ClockSampler.summarize([], None, None)["reasons"] == ["no samples"]
+
+
+def _run_main(monkeypatch, capsys, argv, env):
+    sys.path.insert(0, ROOT)
+    import bench
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    monkeypatch.setattr(sys, "argv", ["bench.py"] + argv)
+    bench.main()
+    return capsys.readouterr().out.strip()
+
+
+def test_reference_arm_times_exactly_k_steps_of_the_oracle(monkeypatch, capsys):
+    import json
+    out = _run_main(monkeypatch, capsys, ["--impl", "reference", "--steps", "2", "--warmup", "3",
+                                          "--oracle-tokens", "8"], {"WORLD_SIZE": "1", "RANK": "0"})
+    line = json.loads(out.splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 3
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True and line["value"] > 0
+    assert line["value"] == pytest.approx(8 / (line["ms_per_step"] * 1e-3), rel=1e-9)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and "8 tokens" in cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    out = _run_main(monkeypatch, capsys, ["--impl", "reference", "--steps", "1", "--warmup", "3",
+                                          "--oracle-tokens", "8"], {"WORLD_SIZE": "2", "RANK": "1"})
+    assert out == ""
+
+
+def test_reference_sample_fits_the_run():
+    sys.path.insert(0, ROOT)
+    import bench
+    for k, w in [(1, 3), (3, 3), (10, 3), (50, 3), (1000, 3)]:
+        n = bench.reference_tokens_per_step(k, w)
+        assert 64 <= n <= bench.PREFILL_T and n % 64 == 0
+        if n > 64:  # the whole run stays near the budget at the oracle's rate
+            assert (k + w) * n / bench.ORACLE_EST_TOKENS_S <= bench.REF_BUDGET_S * 1.01
