@@ -12,3 +12,7 @@ if TESTS not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running (full-size workloads)")
+    # test modules import the package, which refuses to load without its library:
+    # build it (nvcc, in-tree) before collection when it is missing or stale
+    import __graft_entry__
+    __graft_entry__.build()
