@@ -20,6 +20,9 @@
  *     can be captured in a CUDA graph (argument checks happen at enqueue time).
  *   - Return value: QWEN3_OK (0) or a negative qwen3_status; on error nothing
  *     has been enqueued and qwen3_last_error() names the offending argument.
+ *   - Batch and token counts (B, T, rows, n_new) must be at least 1: an empty batch
+ *     returns QWEN3_EINVAL rather than doing nothing, and qwen3_workspace_size()
+ *     returns 0 for it.
  *   - Conditions only visible on the device (a position beyond the cache, a
  *     token id outside the vocabulary, an expired bounded wait) are recorded in
  *     a device error word; qwen3_check_device_error() reads and clears it.

@@ -209,3 +209,28 @@ def test_layer_weights_overlap_from_a_wrong_dimension_is_reported(q3):
     assert st == q3.EINVAL and "overlaps" in msg
     with pytest.raises(q3.Qwen3Error):
         q3.check_layer_weights(cfg, q3.layer_weights(**dict(good, post_norm=good["w_o"])))
+
+
+def test_empty_batches_are_rejected_before_any_launch(q3):
+    """B = 0 or T = 0: QWEN3_EINVAL from the host checks (nothing reaches a device, so
+    this runs without a GPU), and no workspace."""
+    c = q3.config_qwen3_0_6b()
+    ptrs, _ = _arena_layout(c, moe=False)
+    w = q3.layer_weights(**ptrs)
+    fake = 1 << 44
+    kv = q3.KVLayer(fake, fake + (1 << 36), 64)
+    for B, T in [(0, 16), (2, 0), (-1, 4)]:
+        st = q3.lib.qwen3_block_prefill(ctypes.byref(c), ctypes.byref(w), fake, B, T, fake, ctypes.byref(kv), fake,
+                                        fake, 1 << 30, None)
+        assert st == q3.EINVAL and "must be positive" in q3.lib.qwen3_last_error().decode(), (B, T)
+        assert q3.workspace_size(c, q3.OP_BLOCK_PREFILL, B, T, 64) == 0
+    st = q3.lib.qwen3_block_decode(ctypes.byref(c), ctypes.byref(w), fake, 0, fake, ctypes.byref(kv), fake, fake,
+                                   1 << 30, None)
+    assert st == q3.EINVAL
+    kvs = (q3.KVLayer * c.n_layers)(*[q3.KVLayer(fake, fake + (1 << 36), 64)] * c.n_layers)
+    layers = (q3.LayerWeights * c.n_layers)(*[w] * c.n_layers)
+    st = q3.lib.qwen3_stack_forward(ctypes.byref(c), fake, layers, fake, fake, 0, 16, q3.MODE_PREFILL, fake, kvs,
+                                    fake, fake, 0, fake, 1 << 30, None)
+    assert st == q3.EINVAL
+    st = q3.lib.qwen3_op_argmax(fake, 151936, 0, 151936, fake, 1, None)
+    assert st == q3.EINVAL
