@@ -509,9 +509,9 @@ def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
 
 
 def run_moe_decode(q3, torch, args, peaks, B=64, L0=4096, seed=1005):
-    """One decode step of the c4-shaped MoE block (hidden 2048, 32/4 heads, 128 experts x
-    768, top-8) for B sequences holding L0 cached tokens: qwen3_moe_block with T = 1 at
-    position L0. HBM-bound: the bytes are the K/V read, the attention and router weights,
+    """One decode step of the MoE block (hidden 2048, 32/4 heads, 128 experts x 768,
+    top-8; the block of the B1 x T4096 MoE workload) for B sequences holding L0 cached
+    tokens: qwen3_moe_block with T = 1 at position L0. HBM-bound: the bytes are the K/V read, the attention and router weights,
     and the weights of every expert the step routes to (counted from the routing)."""
     from qwen3_decoder_block_b200 import synth
     cfg = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
@@ -698,12 +698,12 @@ def main():
     if rank == 0 and not args.no_configs and args.workload == "all":
         torch.cuda.empty_cache()
         others = {
-            "c0": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T16", 1, 16, 1000,
+            "layer_B1xT16": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T16", 1, 16, 1000,
                                    reps=200),
-            "c3": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T32768", 1, 32768, 1003),
-            "c4": run_single_layer(q3, torch, args, "MoE block prefill (hidden 2048, 32/4 heads, 128 experts x "
+            "layer_B1xT32768": run_single_layer(q3, torch, args, "1 Qwen3-0.6B layer prefill, B1 x T32768", 1, 32768, 1003),
+            "moe_block_B1xT4096": run_single_layer(q3, torch, args, "MoE block prefill (hidden 2048, 32/4 heads, 128 experts x "
                                    "768, top-8), B1 x T4096", 1, 4096, 1004, moe=True),
-            "moe_decode": run_moe_decode(q3, torch, args, peaks),
+            "moe_decode_B64_ctx4096": run_moe_decode(q3, torch, args, peaks),
         }
         torch.cuda.empty_cache()
     cpu = None
@@ -719,7 +719,7 @@ def main():
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded random weights and token ids)",
             "config": config, "e2e": pre["e2e"], "roofline": pre["roofline"], "cpu_baseline": cpu,
             "gpu_launches": pre["gpu_launches"], "clocks": pre["clocks"], "attention": pre["attention"],
-            "kernels": pre["kernels"], "decode": dec, "configs": others}
+            "kernels": pre["kernels"], "decode": dec, "workloads": others}
     print(json.dumps(line))
 
 

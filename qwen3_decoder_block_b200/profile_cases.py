@@ -37,7 +37,7 @@ def _time(fn, reps):
 
 
 def case_attn_prefill(reps, B=4, T=2048, hq=16, hkv=8):
-    """One c1 layer's causal attention: B4 x T2048, 16/8 heads."""
+    """One layer's causal attention of the B4 x T2048 stack prefill, 16/8 heads."""
     cfg = q3.make_config(n_q_heads=hq, n_kv_heads=hkv, hidden=1024 if hq <= 16 else 2048)
     nqkv = (hq + 2 * hkv) * 128
     qkv = _bf16((B * T, nqkv), 1)
@@ -52,12 +52,12 @@ def case_attn_prefill(reps, B=4, T=2048, hq=16, hkv=8):
 
 
 def case_attn_prefill_long(reps):
-    """c3's attention: B1 x T32768."""
+    """The B1 x T32768 layer's attention."""
     return case_attn_prefill(reps, B=1, T=32768)
 
 
 def case_attn_decode(reps, B=64, L=4096):
-    """One c2 layer's decode attention: B64, 4097 visible positions each."""
+    """One layer's decode attention of the B64 decode at 4096 cached tokens: 4097 visible positions each."""
     cfg = q3.config_qwen3_0_6b()
     s_max = L + 128
     nqkv = 32 * 128
@@ -87,22 +87,22 @@ def _gemm(reps, M, N, K, epi=q3.EPI_STORE, swap=-1, out_f32=False, resid=False):
 
 
 def case_gemm_gate_up(reps):
-    """c1 gate/up projection with the SwiGLU epilogue: M8192, N6144, K1024."""
+    """B4 x T2048 gate/up projection with the SwiGLU epilogue: M8192, N6144, K1024."""
     return _gemm(reps, 8192, 6144, 1024, epi=q3.EPI_SWIGLU)
 
 
 def case_gemm_qkv(reps):
-    """c1 QKV projection: M8192, N4096, K1024."""
+    """B4 x T2048 QKV projection: M8192, N4096, K1024."""
     return _gemm(reps, 8192, 4096, 1024)
 
 
 def case_lm_head(reps):
-    """c1 tied LM head: M8192, N151936, K1024, fp32 logits."""
+    """B4 x T2048 tied LM head: M8192, N151936, K1024, fp32 logits."""
     return _gemm(reps, 8192, 151936, 1024, out_f32=True)
 
 
 def case_gemm_qkv_fused(reps, B=4, T=2048):
-    """c1 QKV projection with the fused QK-norm + RoPE + KV-write epilogue (one block prefill
+    """B4 x T2048 QKV projection with the fused QK-norm + RoPE + KV-write epilogue (one block prefill
     minus the rest): M8192, N4096, K1024, measured through the block call's first GEMM."""
     cfg = q3.config_qwen3_0_6b()
     h = _bf16((B * T, 1024), 13)
@@ -121,27 +121,27 @@ def case_gemm_qkv_fused(reps, B=4, T=2048):
 
 
 def case_gemm_o(reps):
-    """c1 o_proj with the fp32 residual epilogue: M8192, N1024, K2048."""
+    """B4 x T2048 o_proj with the fp32 residual epilogue: M8192, N1024, K2048."""
     return _gemm(reps, 8192, 1024, 2048, epi=q3.EPI_RESID, out_f32=True, resid=True)
 
 
 def case_gemm_down(reps):
-    """c1 down projection with the fp32 residual epilogue: M8192, N1024, K3072."""
+    """B4 x T2048 down projection with the fp32 residual epilogue: M8192, N1024, K3072."""
     return _gemm(reps, 8192, 1024, 3072, epi=q3.EPI_RESID, out_f32=True, resid=True)
 
 
 def case_gemm_o_decode(reps):
-    """c2 o_proj: M64 (swap), N1024, K2048, fp32 residual epilogue."""
+    """B64 decode o_proj: M64 (swap), N1024, K2048, fp32 residual epilogue."""
     return _gemm(reps, 64, 1024, 2048, epi=q3.EPI_RESID, out_f32=True, resid=True)
 
 
 def case_gemm_gate_up_decode(reps):
-    """c2 gate/up: M64 (swap), N6144, K1024, SwiGLU epilogue."""
+    """B64 decode gate/up: M64 (swap), N6144, K1024, SwiGLU epilogue."""
     return _gemm(reps, 64, 6144, 1024, epi=q3.EPI_SWIGLU)
 
 
 def case_qk_norm_rope(reps, B=4, T=2048):
-    """c1 per-head QK-norm + RoPE + KV write: 8192 tokens x 32 head slots."""
+    """B4 x T2048 per-head QK-norm + RoPE + KV write: 8192 tokens x 32 head slots."""
     cfg = q3.config_qwen3_0_6b()
     qkv = _bf16((B * T, 4096), 9)
     qn, kn = _bf16((128,), 10), _bf16((128,), 11)
@@ -157,7 +157,7 @@ def case_qk_norm_rope(reps, B=4, T=2048):
 
 
 def case_rmsnorm(reps, rows=8192, n=1024):
-    """c1 RMSNorm of the fp32 residual stream: 8192 x 1024."""
+    """B4 x T2048 RMSNorm of the fp32 residual stream: 8192 x 1024."""
     x = torch.randn((rows, n), dtype=torch.float32, device="cuda")
     w = _bf16((n,), 12)
     out = torch.empty((rows, n), dtype=torch.bfloat16, device="cuda")

@@ -77,7 +77,7 @@ class HostLayer:
         return R.LayerWeights(**f)
 
 
-def test_config0_single_layer_prefill(q3):
+def test_layer_prefill_B1xT16(q3):
     """1 layer, B1 T16, positions 0..15 (seed 1000)."""
     cfg = q3.config_qwen3_0_6b()
     seed, T = 1000, 16
@@ -92,7 +92,7 @@ def test_config0_single_layer_prefill(q3):
     assert_device_ok()
     ref, _, _ = R.block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg), np.arange(T))
     got = from_gpu_bf16(xg)
-    report("c0", rel_frob=rel_frob(got, ref), max_abs=max_abs(got, ref))
+    report("layer_B1xT16", rel_frob=rel_frob(got, ref), max_abs=max_abs(got, ref))
     assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS
 
 
@@ -104,7 +104,7 @@ def _stack_weights(q3, cfg, seed):
 
 
 @pytest.fixture(scope="module")
-def config1_logits(q3):
+def stack_prefill_logits(q3):
     """28 layers + final norm + tied LM head, B4 x T2048 on the GPU; the oracle recomputes
     sequence 0 in full (2048 rows of 151936 logits). Computed once for the tests below."""
     cfg = q3.config_qwen3_0_6b()
@@ -129,7 +129,7 @@ def config1_logits(q3):
     err = rel_frob(got, ref)
     agree = float(np.mean(np.argmax(got, 1) == np.argmax(ref, 1)))
     top2 = np.sort(ref, axis=1)[:, -2:]
-    report("c1", rel_frob=err, argmax_agreement=agree, rows=T, max_abs=max_abs(got, ref),
+    report("stack_prefill_B4xT2048", rel_frob=err, argmax_agreement=agree, rows=T, max_abs=max_abs(got, ref),
            median_top2_gap=float(np.median(top2[:, 1] - top2[:, 0])), logit_rms=float(np.sqrt(np.mean(ref ** 2))))
     return err, agree
 
@@ -140,21 +140,22 @@ def config1_logits(q3):
 BF16_ARGMAX_FLOOR = 0.98
 
 
-def test_config1_stack_prefill(config1_logits):
-    err, agree = config1_logits
+def test_stack_prefill_B4xT2048(stack_prefill_logits):
+    err, agree = stack_prefill_logits
     assert err <= LOGITS_REL_FROB
     assert agree >= BF16_ARGMAX_FLOOR
 
 
-@pytest.mark.xfail(strict=False, reason="argmax >= 0.99 on c1 is out of reach for bf16 intermediates between "
-                                       "kernels: an exact computation that only rounds the bf16 operands the "
-                                       "pages' modules have reaches 0.98-0.99 (tests/bf16_error_budget.py)")
-def test_config1_argmax_target(config1_logits):
-    _, agree = config1_logits
+@pytest.mark.xfail(strict=False, reason="argmax >= 0.99 on the B4 x T2048 stack prefill is out of reach for "
+                                       "bf16 intermediates between kernels: an exact computation that only "
+                                       "rounds the bf16 operands the pages' modules have reaches 0.98-0.99 "
+                                       "(tests/bf16_error_budget.py)")
+def test_stack_prefill_B4xT2048_argmax_target(stack_prefill_logits):
+    _, agree = stack_prefill_logits
     assert agree >= LOGITS_ARGMAX
 
 
-def test_config2_decode(q3):
+def test_stack_decode_B64_ctx4096(q3):
     """B64 sequences with 4096 cached tokens, successive decode steps at positions 4096..;
     the oracle follows sequence 37 for the first 8 steps."""
     cfg = q3.config_qwen3_0_6b()
@@ -207,12 +208,12 @@ def test_config2_decode(q3):
             c[1] = np.concatenate([c[1], vn])
         errs.append(rel_frob(got[s], ref[0]))
         agree.append(int(np.argmax(got[s]) == np.argmax(ref[0])))
-    report("c2", rel_frob_max=max(errs), rel_frob=errs, argmax=agree, steps=steps, sequence=b_s)
+    report("stack_decode_B64_ctx4096", rel_frob_max=max(errs), rel_frob=errs, argmax=agree, steps=steps, sequence=b_s)
     assert max(errs) <= LOGITS_REL_FROB
     assert np.mean(agree) >= LOGITS_ARGMAX
 
 
-def test_config3_long_prefill(q3):
+def test_layer_prefill_B1xT32768(q3):
     """1 layer, B1 T32768; the oracle computes K/V for all positions and finishes a
     sample of query rows."""
     cfg = q3.config_qwen3_0_6b()
@@ -231,11 +232,11 @@ def test_config3_long_prefill(q3):
     rows = np.unique(np.concatenate([[0, 1, 63, 64, 127, 128, 4095, 16383, 16384, 32766, 32767],
                                      rng.integers(0, T, 245)]))
     ref, _, _ = R.block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg), np.arange(T), rows=rows)
-    report("c3", rel_frob=rel_frob(got[rows], ref), max_abs=max_abs(got[rows], ref), rows=len(rows))
+    report("layer_B1xT32768", rel_frob=rel_frob(got[rows], ref), max_abs=max_abs(got[rows], ref), rows=len(rows))
     assert rel_frob(got[rows], ref) <= LAYER_REL_FROB and max_abs(got[rows], ref) <= LAYER_MAX_ABS
 
 
-def test_config4_moe_block(q3):
+def test_moe_block_B1xT4096(q3):
     """MoE block: hidden 2048, 32/4 heads, 128 experts of width 768, top-8 renormalised,
     B1 x T4096."""
     cfg = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
@@ -281,7 +282,7 @@ def test_config4_moe_block(q3):
     ref_g = x1 + R.moe_ffn(h2, gi, w_ref, Lo.gate_up, Lo.down)
     # 5. the permutation is a function of the indices: bit-exact for the GPU's indices
     offs, ptok, _ = R.moe_permutation(gi, cfg.n_experts)
-    report("c4", rel_frob=rel_frob(got, ref_g), max_abs=max_abs(got, ref_g),
+    report("moe_block_B1xT4096", rel_frob=rel_frob(got, ref_g), max_abs=max_abs(got, ref_g),
            rel_frob_vs_oracle_routing=rel_frob(got, ref), sure_tokens=int(sure.sum()),
            sure_sets_equal=bool(sets_equal[sure].all()), all_sets_valid=bool(valid.all()),
            tokens_with_other_set=int((~sets_equal).sum()), w_max_abs=float(np.abs(gw - w_ref).max()),
