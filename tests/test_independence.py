@@ -1,0 +1,56 @@
+"""The oracle and the CUDA path stay apart, and the product path has no fallback:
+the oracle imports nothing of the package (only the standard library and numpy), no
+file of the package imports the oracle, and importing the package without its
+compiled library raises instead of falling back to anything."""
+import ast
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "qwen3_decoder_block_b200")
+
+
+def _imports(path):
+    tree = ast.parse(open(path, encoding="utf-8").read(), path)
+    for node in ast.walk(tree):
+        if isinstance(node, ast.Import):
+            for a in node.names:
+                yield a.name.split(".")[0]
+        elif isinstance(node, ast.ImportFrom):
+            if node.level == 0 and node.module:
+                yield node.module.split(".")[0]
+
+
+def test_oracle_imports_only_stdlib_and_numpy():
+    allowed = {"__future__", "dataclasses", "typing", "math", "numpy"}
+    for name in os.listdir(os.path.join(ROOT, "oracle")):
+        if name.endswith(".py"):
+            mods = set(_imports(os.path.join(ROOT, "oracle", name)))
+            assert mods <= allowed, (name, mods - allowed)
+
+
+def test_package_never_imports_the_oracle():
+    for dirpath, _, files in os.walk(PKG):
+        for name in files:
+            path = os.path.join(dirpath, name)
+            if name.endswith(".py"):
+                assert "oracle" not in set(_imports(path)), path
+            elif name.endswith((".cu", ".cuh", ".h")):
+                assert "oracle" not in open(path, encoding="utf-8").read(), path
+
+
+def test_package_import_fails_loudly_without_its_library():
+    code = (
+        "import os, sys\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "real = os.path.exists\n"
+        "os.path.exists = lambda p: False if str(p).endswith('libqwen3blk.so') else real(p)\n"
+        "try:\n"
+        "    import qwen3_decoder_block_b200\n"
+        "except ImportError as e:\n"
+        "    print('IMPORT_ERROR', e)\n"
+        "else:\n"
+        "    print('IMPORTED')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120).stdout
+    assert out.startswith("IMPORT_ERROR") and "libqwen3blk.so is missing" in out, out
