@@ -59,7 +59,7 @@ typedef enum {
 typedef struct {
   int hidden;           /* H: 1024 for Qwen3-0.6B; multiple of 256, at most 2048 */
   int n_q_heads;        /* Hq: 16 */
-  int n_kv_heads;       /* Hkv: 8; Hq % Hkv == 0 and 128 % (Hq/Hkv) == 0 */
+  int n_kv_heads;       /* Hkv: 8; Hq % Hkv == 0 and Hq/Hkv in {1, 2, 4, 8, 16} */
   int head_dim;         /* D: must be 128 */
   int intermediate;     /* I: 3072 (dense SwiGLU); multiple of 64 */
   int vocab;            /* V: 151936; multiple of 32 */

@@ -173,8 +173,11 @@ static int validate_cfg(const qwen3_config* c) {
   // [P-Hand] section GroupedQueryAttention: num_heads must be divisible by the number of KV groups
   Q3_CHECK(c->n_q_heads % c->n_kv_heads == 0, QWEN3_ESHAPE, "n_q_heads (%d) %% n_kv_heads (%d) != 0", c->n_q_heads,
            c->n_kv_heads);
+  // a 128-row attention tile packs 128 / G tokens of one KV group; the decode kernel is
+  // instantiated for G up to 16, the largest group of the Qwen3 family's GQA configs
   const int G = c->n_q_heads / c->n_kv_heads;
-  Q3_CHECK(128 % G == 0, QWEN3_ESHAPE, "query heads per KV group (%d) must divide 128", G);
+  Q3_CHECK(G == 1 || G == 2 || G == 4 || G == 8 || G == 16, QWEN3_ESHAPE,
+           "query heads per KV group (%d) must be 1, 2, 4, 8 or 16", G);
   Q3_CHECK(c->hidden > 0 && c->hidden % 256 == 0 && c->hidden <= 2048, QWEN3_ESHAPE,
            "hidden (%d) must be a multiple of 256 and at most 2048", c->hidden);
   Q3_CHECK(c->max_pos > 0, QWEN3_ESHAPE, "max_pos must be positive");

@@ -67,6 +67,18 @@ def test_validate_config_rejects(q3, field, value, status):
     assert q3.lib.qwen3_last_error().decode()
 
 
+@pytest.mark.parametrize("hq,hkv,ok", [(16, 16, True), (16, 8, True), (32, 8, True), (64, 8, True), (16, 1, True),
+                                       (32, 1, False), (128, 1, False), (24, 8, False), (40, 8, False)])
+def test_gqa_group_sizes(q3, hq, hkv, ok):
+    """Query heads per KV group: 1, 2, 4, 8 or 16 (all the attention kernels handle);
+    32 or more, and groups that do not divide a 128-row tile (3, or 5 as in 40/8), are
+    rejected before anything runs."""
+    c = q3.config_qwen3_0_6b()
+    c.n_q_heads, c.n_kv_heads = hq, hkv
+    st = q3.validate_config(c)
+    assert (st == 0) if ok else (st == q3.ESHAPE), (hq, hkv, st)
+
+
 def test_moe_config_checks(q3):
     c = q3.make_config(hidden=2048, n_q_heads=32, n_kv_heads=4, n_experts=128, top_k=8, moe_intermediate=768)
     assert q3.validate_config(c) == 0
