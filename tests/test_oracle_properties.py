@@ -109,3 +109,27 @@ def test_moe_equals_a_tokenwise_loop_over_its_own_top_k(E, k, T, renorm, seed):
         np.testing.assert_allclose(out[t], ref, rtol=1e-10, atol=1e-12)
         if k < E:
             assert margin[t] == pytest.approx(np.sort(p)[::-1][k - 1] - np.sort(p)[::-1][k], abs=1e-15)
+
+
+@PROPS
+@given(n_layers=st.integers(1, 3), T0=st.integers(1, 6), n_dec=st.integers(1, 4), hkv=st.sampled_from([1, 2]),
+       group=st.sampled_from([1, 2, 4]), seed=seeds)
+def test_stack_decode_steps_equal_the_rows_of_one_prefill(n_layers, T0, n_dec, hkv, group, seed):
+    """A prompt of T0 tokens, then n_dec decode steps each appending its keys and
+    values to every layer's cache, give the logits of rows T0..T0+n_dec-1 of a
+    single prefill over all T0 + n_dec tokens (greedy feedback replaced by fixed ids)."""
+    rng = np.random.default_rng(seed)
+    cfg = _cfg(R, n_q_heads=hkv * group, n_kv_heads=hkv)
+    E = 0.3 * rng.standard_normal((cfg.vocab, cfg.hidden))
+    layers = [_layer(R, cfg, rng) for _ in range(n_layers)]
+    fn = 1 + 0.1 * rng.standard_normal(cfg.hidden)
+    ids = rng.integers(0, cfg.vocab, T0 + n_dec)
+    full, _ = R.stack_forward(ids, E, layers, fn, cfg)
+    _, kv = R.stack_forward(ids[:T0], E, layers, fn, cfg)
+    caches = [(k, v, np.arange(T0)) for (k, v) in kv]
+    for s in range(n_dec):
+        pos = T0 + s
+        dec, new = R.stack_forward(ids[pos:pos + 1], E, layers, fn, cfg, positions=np.array([pos]), caches=caches)
+        np.testing.assert_allclose(dec[0], full[pos], rtol=1e-10, atol=1e-11)
+        caches = [(np.concatenate([ck, k]), np.concatenate([cv, v]), np.append(cp, pos))
+                  for (ck, cv, cp), (k, v) in zip(caches, new)]
