@@ -246,3 +246,45 @@ def test_empty_batches_are_rejected_before_any_launch(q3):
     assert st == q3.EINVAL
     st = q3.lib.qwen3_op_argmax(fake, 151936, 0, 151936, fake, 1, None)
     assert st == q3.EINVAL
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include <string.h>
+#include "qwen3blk.h"
+int main(void) {
+  qwen3_config c;
+  if (qwen3_config_qwen3_0_6b(&c) != QWEN3_OK || c.hidden != 1024 || c.n_layers != 28) return 1;
+  if (qwen3_validate_config(&c) != QWEN3_OK) return 2;
+  if (qwen3_workspace_size(&c, QWEN3_OP_BLOCK_PREFILL, 1, 16, 64) == 0) return 3;
+  qwen3_layer_weights w;
+  memset(&w, 0, sizeof w);
+  if (qwen3_check_layer_weights(&c, &w, QWEN3_LAYER_DENSE) != QWEN3_EINVAL) return 4;
+  if (strstr(qwen3_last_error(), "in_norm") == NULL) return 5;
+  c.head_dim = 64;
+  if (qwen3_validate_config(&c) != QWEN3_ESHAPE) return 6;
+  printf("%s\n", qwen3_status_string(QWEN3_ESHAPE));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(q3):
+    """A C11 program (no C++) includes the header, links against the library and calls
+    its host-only entry points."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.dirname(q3.LIB_PATH)
+    src, exe = os.path.join(libdir, "abi_c_test.c"), os.path.join(libdir, "abi_c_test")
+    with open(src, "w") as f:
+        f.write(C_PROGRAM)
+    cmd = [gcc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+           "-L", libdir, "-l:libqwen3blk.so", f"-Wl,-rpath,{libdir}", "-o", exe]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.strip() != ""
