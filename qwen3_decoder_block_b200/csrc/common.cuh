@@ -326,8 +326,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
 // tcgen05.wait::ld that also ties the 32 destination registers of an earlier
 // tmem_ld32 to the wait, so that no use of them can be scheduled before it.
 __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
