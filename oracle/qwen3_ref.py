@@ -28,6 +28,9 @@ tests/test_oracle_pins.py):
                            block when o_proj and down weights are zero
   moe_route / moe_ffn      the 0.7*E2 + 0.3*E4 worked example, k = E dense weighted sum,
                            sparse == token-wise dense reference, permutation order
+  moe_ffn_half /           the block-level 0.7*E2 + 0.3*E4 example and k = E dense sum on
+  moe_block_forward        norm_2(x1); a per-token loop over an independently restated
+                           post-attention norm, router, top-k and experts; given routing
   stack_forward            zero-residual stack closed form (argmax logit = own token),
                            last-only == last row, causality across 2 layers
   param_count              0.752B untied parameter count and 3.01 GB fp32 of [P-Mini]
@@ -275,14 +278,27 @@ def moe_ffn(h2: np.ndarray, idx: np.ndarray, w: np.ndarray, gate_up: np.ndarray,
     return out
 
 
+def moe_ffn_half(x1: np.ndarray, L: LayerWeights, cfg: Config, idx: Optional[np.ndarray] = None,
+                 w: Optional[np.ndarray] = None):
+    """Second half of the MoE block ([P-Mini] sections TransformerBlock and MoE):
+    h2 = norm_2(x1) with the post-attention weights, the router reads h2, and the
+    selected experts' outputs on h2, weighted, are added to the residual x1.
+    With idx and w given, that routing is used instead of the router's (the oracle
+    evaluated on another implementation's routing). Returns (out, (idx, w, probs,
+    margin)); probs and margin are None when the routing was given."""
+    h2 = rms_norm(x1, L.post_norm, cfg.rms_eps)
+    probs = margin = None
+    if idx is None:
+        idx, w, probs, margin = moe_route(h2, L.router, cfg.top_k, cfg.norm_topk_prob)
+    return x1 + moe_ffn(h2, idx, w, L.gate_up, L.down), (idx, w, probs, margin)
+
+
 def moe_block_forward(x, L, cfg, positions, rows=None):
     """Attention half then x1 + MoE(norm_2(x1)). Returns (out, k, v, route) where
     route = (idx, w, probs, margin) for the computed rows."""
     x1, k, v = attention_half(x, L, cfg, positions, rows=rows)
-    h2 = rms_norm(x1, L.post_norm, cfg.rms_eps)
-    idx, w, probs, margin = moe_route(h2, L.router, cfg.top_k, cfg.norm_topk_prob)
-    out = x1 + moe_ffn(h2, idx, w, L.gate_up, L.down)
-    return out, k, v, (idx, w, probs, margin)
+    out, route = moe_ffn_half(x1, L, cfg)
+    return out, k, v, route
 
 
 # ---------------------------------------------------------------------------

@@ -408,6 +408,88 @@ def pin_moe_permutation(R):
         assert idx[tok[i], slot[i]] == e
 
 
+def _expert_closed(gate_up_e, down_e, r):
+    """One SwiGLU expert on one row, restated: gate rows first, then up rows."""
+    im = gate_up_e.shape[0] // 2
+    g = gate_up_e[:im] @ r
+    u = gate_up_e[im:] @ r
+    return down_e @ (g / (1 + np.exp(-g)) * u)
+
+
+def _moe_block_layer(R, rng, cfg):
+    L = _layer(R, cfg, rng, moe=True)
+    # norm weights far from 1, so that post- and pre-attention norms, and x1 versus
+    # norm_2(x1), route differently
+    L.in_norm = 1 + 0.6 * rng.standard_normal(cfg.hidden)
+    L.post_norm = 1 + 0.6 * rng.standard_normal(cfg.hidden)
+    return L
+
+
+def pin_moe_block_worked_example(R):
+    """The worked example at block level: with o_proj zero the attention half is the
+    identity (x1 = x); a router built on the token's own norm_2(x) row gives the
+    probabilities (0.05, 0.56, 0.15, 0.24), so top-2 picks E2 and E4 with weights 0.7
+    and 0.3, and out = x + 0.7 E2(h2) + 0.3 E4(h2). With k = E the output is the dense
+    sum over all experts weighted by the probabilities themselves."""
+    g = json.load(open(os.path.join(GOLDEN, "moe_worked_example.json")))
+    rng = _rng(24)
+    cfg = _moe_cfg(R, E=g["n_experts"], k=g["top_k"], Im=6)
+    L = _moe_block_layer(R, rng, cfg)
+    L.wo = np.zeros_like(L.wo)
+    x = 1.5 * rng.standard_normal((1, cfg.hidden))
+    # norm_2 of x, restated: x / sqrt(mean x^2 + eps) * post_norm
+    h2 = x[0] / math.sqrt(float(np.mean(x[0] ** 2)) + cfg.rms_eps) * L.post_norm
+    probs = np.array([0.05, 0.56, 0.15, 0.24])
+    L.router = np.log(probs)[:, None] * h2[None, :] / float(h2 @ h2)   # router . h2 = log p
+    out, _, _, (idx, w, p, _) = R.moe_block_forward(x, L, cfg, np.array([3]))
+    assert [int(i) + 1 for i in idx[0]] == g["selected_experts_1_based"], idx
+    np.testing.assert_allclose(p[0], probs, rtol=1e-12)
+    ref = x[0] + g["weights"][0] * _expert_closed(L.gate_up[1], L.down[1], h2) \
+        + g["weights"][1] * _expert_closed(L.gate_up[3], L.down[3], h2)
+    np.testing.assert_allclose(out[0], ref, rtol=1e-11, atol=1e-13)
+    dense_cfg = _moe_cfg(R, E=g["n_experts"], k=g["n_experts"], Im=6)
+    out_all, _, _, _ = R.moe_block_forward(x, L, dense_cfg, np.array([3]))
+    ref_all = x[0] + sum(probs[e] * _expert_closed(L.gate_up[e], L.down[e], h2) for e in range(len(probs)))
+    np.testing.assert_allclose(out_all[0], ref_all, rtol=1e-11, atol=1e-13)
+
+
+def pin_moe_block_tokenwise(R):
+    """The MoE block against a per-token loop that restates its second half: the
+    post-attention RMSNorm of x1 (not x, not the input norm), the router's softmax on
+    that row, top-k by descending probability (lower index first), renormalised
+    weights, experts evaluated on the normed row, and the residual x1 added back. x1
+    comes from the attention half, pinned on its own. The given-routing form of
+    moe_ffn_half must reproduce the same rows from the same routing."""
+    rng = _rng(25)
+    cfg = _moe_cfg(R, E=8, k=3, Im=5)
+    L = _moe_block_layer(R, rng, cfg)
+    T = 9
+    x = rng.standard_normal((T, cfg.hidden))
+    pos = 5 + np.arange(T)
+    out, _, _, (idx, w, _, _) = R.moe_block_forward(x, L, cfg, pos)
+    x1, _, _ = R.attention_half(x, L, cfg, pos)
+    for t in range(T):
+        r = x1[t] / math.sqrt(float(np.mean(x1[t] ** 2)) + cfg.rms_eps) * L.post_norm
+        lg = L.router @ r
+        pr = np.exp(lg - lg.max()); pr /= pr.sum()
+        top = sorted(range(cfg.n_experts), key=lambda e: (-pr[e], e))[:cfg.top_k]
+        assert list(idx[t]) == top, (t, idx[t], top)
+        tot = sum(pr[e] for e in top)
+        ref = x1[t] + sum(pr[e] / tot * _expert_closed(L.gate_up[e], L.down[e], r) for e in top)
+        np.testing.assert_allclose(out[t], ref, rtol=1e-11, atol=1e-12)
+    given, _ = R.moe_ffn_half(x1, L, cfg, idx=idx, w=w)
+    np.testing.assert_allclose(given, out, rtol=1e-13, atol=1e-14)
+    # a different, valid routing is evaluated as given: every token on experts (0, 1, 2)
+    # with equal weights
+    idx2 = np.tile(np.arange(3, dtype=np.int32), (T, 1))
+    w2 = np.full((T, 3), 1.0 / 3.0)
+    given2, _ = R.moe_ffn_half(x1, L, cfg, idx=idx2, w=w2)
+    for t in (0, T - 1):
+        r = x1[t] / math.sqrt(float(np.mean(x1[t] ** 2)) + cfg.rms_eps) * L.post_norm
+        ref = x1[t] + sum(_expert_closed(L.gate_up[e], L.down[e], r) for e in range(3)) / 3.0
+        np.testing.assert_allclose(given2[t], ref, rtol=1e-11, atol=1e-12)
+
+
 # ----------------------------------------------------------------------------- stack
 def _stack_inputs(R, rng, cfg, n_layers):
     E = rng.standard_normal((cfg.vocab, cfg.hidden))

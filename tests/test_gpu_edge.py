@@ -168,9 +168,7 @@ def test_moe_block_decode_step(q3):
         x1, _, _ = R.attention_half(x.f[b:b + 1], Lo, oc, np.array([lens[b]]),
                                     pk.f[b][:, :lens[b]].transpose(1, 0, 2), pv.f[b][:, :lens[b]].transpose(1, 0, 2),
                                     np.arange(lens[b]))
-        h2 = R.rms_norm(x1, Lo.post_norm, oc.rms_eps)
-        ridx, rw, _, margin = R.moe_route(h2, Lo.router, oc.top_k, oc.norm_topk_prob)
-        ref = x1 + R.moe_ffn(h2, ridx, rw, Lo.gate_up, Lo.down)
+        ref, (ridx, rw, _, margin) = R.moe_ffn_half(x1, Lo, oc)
         assert rel_frob(got[b:b + 1], ref) <= LAYER_REL_FROB and max_abs(got[b:b + 1], ref) <= LAYER_MAX_ABS
         if margin[0] > 1e-3:
             np.testing.assert_array_equal(np.sort(gi[b]), np.sort(ridx[0]))

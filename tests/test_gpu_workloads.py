@@ -256,8 +256,9 @@ def test_moe_block_B1xT4096(q3):
                  workspace(cfg, q3.OP_MOE_BLOCK, 1, T, T), idx, w, off, perm)
     assert_device_ok()
     got = from_gpu_bf16(xg)
-    ref, _, _, (ridx, rw, rp, margin) = R.moe_block_forward(R.bf16_to_f64(x), L.oracle(), oracle_config(cfg),
-                                                            np.arange(T))
+    oc, Lo = oracle_config(cfg), L.oracle()
+    x1, _, _ = R.attention_half(R.bf16_to_f64(x), Lo, oc, np.arange(T))
+    ref, (ridx, rw, rp, margin) = R.moe_ffn_half(x1, Lo, oc)
     gi, gw, goff, gperm = idx.cpu().numpy(), w.cpu().numpy(), off.cpu().numpy(), perm.cpu().numpy()
     kk = cfg.top_k
     # 1. where the oracle's top-k margin exceeds 1e-3 the selected experts are unique: the
@@ -275,11 +276,7 @@ def test_moe_block_B1xT4096(q3):
     w_ref = np.take_along_axis(rp, gi, 1)
     w_ref /= w_ref.sum(1, keepdims=True)
     # 4. the layer output against the oracle evaluated on the GPU's (validated) routing
-    oc = oracle_config(cfg)
-    Lo = L.oracle()
-    x1, _, _ = R.attention_half(R.bf16_to_f64(x), Lo, oc, np.arange(T))
-    h2 = R.rms_norm(x1, Lo.post_norm, oc.rms_eps)
-    ref_g = x1 + R.moe_ffn(h2, gi, w_ref, Lo.gate_up, Lo.down)
+    ref_g, _ = R.moe_ffn_half(x1, Lo, oc, idx=gi, w=w_ref)
     # 5. the permutation is a function of the indices: bit-exact for the GPU's indices
     offs, ptok, _ = R.moe_permutation(gi, cfg.n_experts)
     report("moe_block_B1xT4096", rel_frob=rel_frob(got, ref_g), max_abs=max_abs(got, ref_g),

@@ -114,7 +114,37 @@ def _attn_half_no_residual(x, L, cfg, positions, cache_k=None, cache_v=None, cac
     return x1 - x[sel], k, v
 
 
-_ORIG = {n: getattr(R, n) for n in ("moe_route", "attention_half", "stack_forward", "causal_gqa_attention")}
+def _moe_half_routes_on_x1(x1, L, cfg, idx=None, w=None):
+    h2 = R.rms_norm(x1, L.post_norm, cfg.rms_eps)
+    probs = margin = None
+    if idx is None:
+        idx, w, probs, margin = R.moe_route(x1, L.router, cfg.top_k, cfg.norm_topk_prob)
+    return x1 + R.moe_ffn(h2, idx, w, L.gate_up, L.down), (idx, w, probs, margin)
+
+
+def _moe_half_input_norm(x1, L, cfg, idx=None, w=None):
+    h2 = R.rms_norm(x1, L.in_norm, cfg.rms_eps)
+    probs = margin = None
+    if idx is None:
+        idx, w, probs, margin = R.moe_route(h2, L.router, cfg.top_k, cfg.norm_topk_prob)
+    return x1 + R.moe_ffn(h2, idx, w, L.gate_up, L.down), (idx, w, probs, margin)
+
+
+def _moe_half_no_residual(x1, L, cfg, idx=None, w=None):
+    out, route = _ORIG["moe_ffn_half"](x1, L, cfg, idx, w)
+    return out - x1, route
+
+
+def _moe_half_experts_on_x1(x1, L, cfg, idx=None, w=None):
+    h2 = R.rms_norm(x1, L.post_norm, cfg.rms_eps)
+    probs = margin = None
+    if idx is None:
+        idx, w, probs, margin = R.moe_route(h2, L.router, cfg.top_k, cfg.norm_topk_prob)
+    return x1 + R.moe_ffn(x1, idx, w, L.gate_up, L.down), (idx, w, probs, margin)
+
+
+_ORIG = {n: getattr(R, n) for n in ("moe_route", "attention_half", "stack_forward", "causal_gqa_attention",
+                                    "moe_ffn_half")}
 
 
 def _wrap_no_qk(monkeypatch):
@@ -143,6 +173,10 @@ MUTATIONS = {
     "rope_before_qk_norm": ("attention_half", _attn_half_rope_before_norm),
     "final_norm_weights_ignored": ("stack_forward", _stack_no_final_norm),
     "attention_residual_dropped": ("attention_half", _attn_half_no_residual),
+    "moe_routes_on_x1": ("moe_ffn_half", _moe_half_routes_on_x1),
+    "moe_uses_input_norm": ("moe_ffn_half", _moe_half_input_norm),
+    "moe_residual_dropped": ("moe_ffn_half", _moe_half_no_residual),
+    "moe_experts_on_x1": ("moe_ffn_half", _moe_half_experts_on_x1),
 }
 
 
