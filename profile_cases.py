@@ -1,6 +1,6 @@
 """Single-kernel cases at the workloads' shapes, for timing and for ncu captures.
 
-    python -m qwen3_decoder_block_b200.profile_cases <case> [--reps N]
+    python profile_cases.py <case> [--reps N]
 
 Each case draws seeded inputs, runs the kernel once (warm-up), then N timed
 repetitions with CUDA events, and prints one JSON line with the average device
@@ -15,7 +15,7 @@ import json
 import torch
 
 import qwen3_decoder_block_b200 as q3
-from qwen3_decoder_block_b200 import synth
+import qwen3_synth as synth
 
 
 def _bf16(shape, tid, std=1.0, seed=77):

@@ -1,7 +1,6 @@
 """Builds the in-tree shared libraries with nvcc for sm_100a.
 
     lib/libqwen3blk.so    the decoder-block library (C ABI in include/qwen3blk.h)
-    lib/libqwen3synth.so  the seeded synthetic-input generator (host + device)
 
 Each translation unit is compiled to an object in parallel, then linked; a
 library is rebuilt only when a source, header or flag changed.
@@ -27,7 +26,6 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xc
 
 LIBRARIES = {
     "libqwen3blk.so": ["api.cu", "gemm.cu", "elementwise.cu", "attention.cu", "moe.cu"],
-    "libqwen3synth.so": ["synth.cu"],
 }
 HEADERS = ["common.cuh", "internal.h"]
 

@@ -103,6 +103,26 @@ bool gemm_pair_enabled() {
   return on;
 }
 
+// The dynamic shared-memory limit of a kernel is a per-device setting: raise it once
+// per (kernel, device), under the lock, and report a failure instead of launching.
+int ensure_smem_attr(const void* func, int bytes, bool* first) {
+  const int d = current_device();
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  static std::vector<std::pair<const void*, int>> done;
+  if (first) *first = false;
+  for (const auto& e : done)
+    if (e.first == func && e.second == d) return 0;
+  const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    set_last_error("cannot raise a kernel's shared memory to %d bytes on device %d: %s", bytes, d,
+                   cudaGetErrorString(e));
+    return -6;
+  }
+  done.emplace_back(func, d);
+  if (first) *first = true;
+  return 0;
+}
+
 int* device_error_word() {
   const int d = current_device();
   std::lock_guard<std::mutex> lk(g_dev_mu);
@@ -150,9 +170,12 @@ struct ProfScope {
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 static int check_device() {
-  static int ok[64] = {0};
+  static bool ok[64] = {false};
   const int d = current_device();
-  if (ok[d] == 1) return 0;
+  {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (ok[d]) return 0;
+  }
   cudaDeviceProp prop;
   if (cudaGetDeviceProperties(&prop, d) != cudaSuccess) {
     set_last_error("no CUDA device available");
@@ -162,7 +185,8 @@ static int check_device() {
     set_last_error("device %d is sm_%d%d; libqwen3blk needs an sm_100 (B200) GPU", d, prop.major, prop.minor);
     return QWEN3_EDEVICE;
   }
-  ok[d] = 1;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  ok[d] = true;
   return 0;
 }
 
@@ -1098,6 +1122,9 @@ int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long
   Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode: B must be positive");
   Q3_CHECK(ldqkv % 8 == 0 && ldqkv >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
            "attention_decode: ldqkv (%lld) must be a multiple of 8 and cover the query heads", ldqkv);
+  Q3_CHECK(ldo % 8 == 0 && ldo >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
+           "attention_decode: ldo (%lld) must be a multiple of 8 and at least n_q_heads * head_dim (%d)", ldo,
+           c->n_q_heads * c->head_dim);
   if ((rc = check_kv(*c, kv, 1))) return rc;
   const size_t need = decode_partial_bytes(B, c->n_q_heads, kv->s_max);
   Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "attention_decode: workspace has %zu bytes, needs %zu", ws_bytes, need);
@@ -1118,6 +1145,9 @@ int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* q
   Q3_CHECK(B > 0, QWEN3_EINVAL, "attention_decode_noalloc: B must be positive");
   Q3_CHECK(ldqkv % 8 == 0 && ldqkv >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
            "attention_decode_noalloc: ldqkv (%lld) must be a multiple of 8 and cover the query heads", ldqkv);
+  Q3_CHECK(ldo % 8 == 0 && ldo >= (long long)c->n_q_heads * c->head_dim, QWEN3_EALIGN,
+           "attention_decode_noalloc: ldo (%lld) must be a multiple of 8 and at least n_q_heads * head_dim (%d)",
+           ldo, c->n_q_heads * c->head_dim);
   if ((rc = check_kv(*c, kv, 1))) return rc;
   if ((rc = check_device())) return rc;
   return finish(launch_attention_decode_static(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,

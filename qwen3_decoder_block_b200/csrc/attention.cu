@@ -404,9 +404,9 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
   p.out = out;
   p.ldo = ldo;
   p.err = err;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPrefillSmem);
+  bool first = false;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(attn_prefill_kernel), kPrefillSmem, &first)) return -6;
+  if (first) {
     // the register split must fit what the block is launched with, or the increase never returns
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, attn_prefill_kernel) != cudaSuccess ||
@@ -414,7 +414,6 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
       set_last_error("attention prefill: kernel built with too few registers for its warpgroup split");
       return -6;
     }
-    attr = true;
   }
   const long long n_cta = (long long)p.n_cta_q * Hkv * B;
   if (n_cta >= (1ll << 31)) {
@@ -799,22 +798,18 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   }
   const long long items = (long long)B * Hkv * n_splits;
   const int grid = (int)(items < num_sms() ? items : num_sms());
-  static bool attr[5] = {false, false, false, false, false};
   switch (G) {
-#define Q3_D4_CASE(GG, SLOT)                                                                                      \
+#define Q3_D4_CASE(GG)                                                                                            \
   case GG:                                                                                                        \
-    if (!attr[SLOT]) {                                                                                            \
-      cudaFuncSetAttribute(attn_decode_tc_kernel<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, kD4Smem);      \
-      attr[SLOT] = true;                                                                                          \
-    }                                                                                                             \
+    if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG>), kD4Smem)) return -6;           \
     q3_launch(attn_decode_tc_kernel<GG>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,      \
               s_max, n_splits, part, err);                                                                        \
     break;
-    Q3_D4_CASE(1, 0)
-    Q3_D4_CASE(2, 1)
-    Q3_D4_CASE(4, 2)
-    Q3_D4_CASE(8, 3)
-    Q3_D4_CASE(16, 4)
+    Q3_D4_CASE(1)
+    Q3_D4_CASE(2)
+    Q3_D4_CASE(4)
+    Q3_D4_CASE(8)
+    Q3_D4_CASE(16)
 #undef Q3_D4_CASE
   }
   q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);

@@ -848,16 +848,13 @@ static int make_tmap_out(CUtensorMap* map, void* base, long long rows, long long
   return r == CUDA_SUCCESS ? 0 : -2;
 }
 
-// One kernel instantiation: shared-memory attribute (once), launch (CTA pairs as
+// One kernel instantiation: shared-memory attribute (once per device), launch (CTA pairs as
 // clusters of 2), launch-error check.
 template <int BN, bool PAIR, bool ROPE>
 static int launch_variant(const GemmParams& g, const CUtensorMap& tmP, const CUtensorMap& tmQ,
                           const CUtensorMap& tmO, cudaStream_t s) {
   using C = GemmCfg<BN, PAIR, ROPE>;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(gemm_tc_kernel<BN, PAIR, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-  });
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_tc_kernel<BN, PAIR, ROPE>), 227 * 1024)) return -6;
   const size_t smem = C::smem_bytes(g.n_groups);
   if (PAIR) {
     const long long tiles = (long long)g.p_tiles * g.q_tiles;

@@ -120,6 +120,11 @@ inline cudaError_t q3_launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 b
 }
 
 int* device_error_word();  // device pointer of the library's error word
+
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device); *first (optional) tells whether this call set it. Returns 0 or -6
+// (with the CUDA error in the last-error message).
+int ensure_smem_attr(const void* func, int bytes, bool* first = nullptr);
 void set_last_error(const char* fmt, ...);
 
 }  // namespace q3

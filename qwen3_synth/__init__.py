@@ -1,6 +1,7 @@
-"""Seeded synthetic inputs shared by the CUDA path, the oracle and the benchmark.
+"""Seeded synthetic inputs shared by the CUDA path's tests, the oracle and the benchmark.
 
-This module holds no arithmetic of the decoder block. It only defines how the
+A package of its own, apart from the library: it holds no arithmetic of the decoder
+block, imports nothing of the library or of the oracle, and neither imports it. It only defines how the
 random weights, activations, token ids and cached keys/values of the synthetic
 workloads are drawn, so that every consumer sees identical bits.
 
@@ -145,7 +146,8 @@ def native():
     if _native is None:
         path = os.path.join(os.path.dirname(__file__), "lib", "libqwen3synth.so")
         if not os.path.exists(path):
-            raise ImportError(f"{path} is missing: run __graft_entry__.build() first")
+            from . import _build
+            _build.build()
         lib = ctypes.CDLL(path)
         i64, u64, dbl, vp = ctypes.c_int64, ctypes.c_uint64, ctypes.c_double, ctypes.c_void_p
         lib.qwen3synth_normal_bf16_host.argtypes = [vp, i64, i64, i64, i64, i64, i64, u64, u64, dbl, dbl]

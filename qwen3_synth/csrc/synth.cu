@@ -1,5 +1,5 @@
 // Seeded synthetic input generator: host (OpenMP) and device (CUDA) versions of
-// the counter-based definition documented in qwen3_decoder_block_b200/synth.py.
+// the counter-based definition documented in qwen3_synth/__init__.py.
 // It holds none of the decoder block's arithmetic; it only draws inputs.
 #include <cstdint>
 #include <cmath>

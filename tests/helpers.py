@@ -5,7 +5,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from qwen3_decoder_block_b200 import synth
+import qwen3_synth as synth
 import oracle.qwen3_ref as R
 
 # Per-layer bar: relative Frobenius error <= 1e-2 and max abs error <= 3e-2.

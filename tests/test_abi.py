@@ -42,7 +42,7 @@ def test_binding_covers_every_declared_symbol(q3):
 
 
 def test_synth_library_exports(q3):
-    from qwen3_decoder_block_b200 import synth
+    import qwen3_synth as synth
     lib = synth.native()
     for n in ("qwen3synth_normal_bf16_host", "qwen3synth_normal_bf16_device", "qwen3synth_uniform_int_host",
               "qwen3synth_uniform_int_device"):
@@ -288,3 +288,19 @@ def test_header_is_plain_c_and_links(q3):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.strip() != ""
+
+
+@pytest.mark.parametrize("ldo", [0, -2048, 2040, 2052, 1 << 3])
+def test_decode_attention_rejects_bad_output_stride_before_launch(q3, ldo):
+    """The decode attention writes o[b * ldo + h * 128 + d]: an ldo below n_q_heads * 128,
+    not a multiple of 8, zero or negative is rejected on the host (QWEN3_EALIGN) by both
+    entry points, before anything could be launched."""
+    c = q3.config_qwen3_0_6b()
+    fake = 1 << 44
+    kv = q3.KVLayer(fake, fake + (1 << 36), 4224)
+    st = q3.lib.qwen3_op_attention_decode(ctypes.byref(c), fake, 4096, 64, fake, ctypes.byref(kv), fake, ldo, fake,
+                                          1 << 30, None)
+    assert st == q3.EALIGN and "ldo" in q3.lib.qwen3_last_error().decode(), st
+    st = q3.lib.qwen3_op_attention_decode_noalloc(ctypes.byref(c), fake, 4096, 64, fake, ctypes.byref(kv), fake, ldo,
+                                                  None)
+    assert st == q3.EALIGN and "ldo" in q3.lib.qwen3_last_error().decode(), st

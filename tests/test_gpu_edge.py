@@ -7,7 +7,7 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 import oracle.qwen3_ref as R  # noqa: E402
-from qwen3_decoder_block_b200 import synth  # noqa: E402
+import qwen3_synth as synth  # noqa: E402
 from helpers import (LAYER_MAX_ABS, LAYER_REL_FROB, Layer, Tensor, assert_device_ok, from_gpu_bf16,  # noqa: E402
                      kv_cache, max_abs, oracle_config, rel_frob, rope_gpu, workspace)
 

@@ -7,7 +7,7 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 import oracle.qwen3_ref as R  # noqa: E402
-from qwen3_decoder_block_b200 import synth  # noqa: E402
+import qwen3_synth as synth  # noqa: E402
 from helpers import Layer, Tensor, assert_device_ok, kv_cache, oracle_config, rope_gpu, workspace  # noqa: E402
 
 

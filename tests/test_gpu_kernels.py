@@ -298,7 +298,7 @@ def test_embed(q3):
 
 
 def test_synth_device_matches_host(q3):
-    from qwen3_decoder_block_b200 import synth
+    import qwen3_synth as synth
     n0, n1, n2, s1 = 3, 50, 128, 200 * 128
     buf = torch.zeros((n0, 200, n2), dtype=torch.bfloat16, device="cuda")
     synth.normal_bf16_device(buf.data_ptr(), n0, n1, n2, 200 * 128, 128, 11, 12, 0.0, 1.0, index_base=777)

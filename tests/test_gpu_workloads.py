@@ -14,7 +14,7 @@ torch = pytest.importorskip("torch")
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
 import oracle.qwen3_ref as R  # noqa: E402
-from qwen3_decoder_block_b200 import synth  # noqa: E402
+import qwen3_synth as synth  # noqa: E402
 from helpers import (LAYER_MAX_ABS, LAYER_REL_FROB, LOGITS_ARGMAX, LOGITS_REL_FROB, assert_device_ok,  # noqa: E402
                      from_gpu_bf16, max_abs, oracle_config, rel_frob, rope_gpu, to_gpu_bf16, workspace)
 

@@ -54,3 +54,34 @@ def test_package_import_fails_loudly_without_its_library():
         "    print('IMPORTED')\n")
     out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120).stdout
     assert out.startswith("IMPORT_ERROR") and "libqwen3blk.so is missing" in out, out
+
+
+def test_input_generator_is_a_module_of_its_own():
+    """The seeded generator serves both sides and belongs to neither: it imports neither
+    the package nor the oracle, and the package does not import it."""
+    synth_dir = os.path.join(ROOT, "qwen3_synth")
+    for dirpath, _, files in os.walk(synth_dir):
+        for name in files:
+            if name.endswith(".py"):
+                mods = set(_imports(os.path.join(dirpath, name)))
+                assert not mods & {"oracle", "qwen3_decoder_block_b200"}, (name, mods)
+    for dirpath, _, files in os.walk(PKG):
+        for name in files:
+            if name.endswith(".py"):
+                assert "qwen3_synth" not in set(_imports(os.path.join(dirpath, name))), name
+
+
+def test_oracle_process_maps_no_product_library():
+    """A process that runs the oracle on seeded inputs (what the benchmark's oracle arm
+    does) never loads libqwen3blk.so."""
+    code = (
+        "import sys\n"
+        f"sys.path.insert(0, {ROOT!r})\n"
+        "import numpy as np\n"
+        "import oracle.qwen3_ref as R\n"
+        "import qwen3_synth as synth\n"
+        "x = R.bf16_to_f64(synth.normal_bf16_fast(1, 3, (4, 8)))\n"
+        "R.rms_norm(x, np.ones(8), 1e-6)\n"
+        "print('LOADED' if 'libqwen3blk' in open('/proc/self/maps').read() else 'CLEAN')\n")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert out.stdout.strip() == "CLEAN", (out.stdout, out.stderr)

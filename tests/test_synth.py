@@ -2,7 +2,7 @@
 import numpy as np
 import pytest
 
-from qwen3_decoder_block_b200 import synth
+import qwen3_synth as synth
 
 
 @pytest.fixture(scope="module")
