@@ -42,6 +42,7 @@ extern "C" {
 #endif
 
 typedef uint16_t qwen3_bf16;
+typedef uint16_t qwen3_f16; /* IEEE binary16 bit pattern */
 
 typedef enum {
   QWEN3_OK = 0,
@@ -71,6 +72,17 @@ typedef struct {
   int norm_topk_prob;   /* 1: renormalise the top-k probabilities to sum 1 */
   float rms_eps;        /* 1e-6 */
   double rope_theta;    /* 1e6 */
+  /* Operand type of the linear layers (projections, router, experts, tied LM head):
+   *   0: bf16, the pages' model dtype ([P-Mini] section RMSNorm: the model body is bf16);
+   *   1: fp16. Every bf16 weight converts to fp16 exactly for magnitudes in
+   *      [2^-17, 65504] (qwen3_convert_to_f16; below, within 2^-25), so the weights keep
+   *      their values, while the activations fed to the projections round to 11
+   *      significant bits instead of 8 -- at the same tensor-core rate. The linear
+   *      weights (w_qkv, w_o, w_gate_up, w_down, router, moe_gate_up, moe_down) and the
+   *      embedding / LM head must then hold fp16; norm weights stay bf16. Activations
+   *      entering a projection must stay within +-65504 (larger ones become inf).
+   * The KV cache, q and the softmax probabilities stay bf16 in both modes. */
+  int gemm_f16;
 } qwen3_config;
 
 /* One layer's weights in the library's packed layouts (see the pack helpers).
@@ -132,6 +144,11 @@ int qwen3_rope_table(const qwen3_config* cfg, float* rope, void* stream);
 /* Scratch bytes needed by `op` for B sequences of T new tokens each, with KV
  * caches of capacity s_max (decode: T is ignored and taken as 1). */
 size_t qwen3_workspace_size(const qwen3_config* cfg, int op, int B, int T, int s_max);
+
+/* Converts n bf16 values to fp16 (round to nearest even; exact for magnitudes in
+ * [2^-17, 65504]), e.g. a packed weight matrix for the gemm_f16 mode. in == out converts
+ * in place. Asynchronous on `stream`. */
+int qwen3_convert_to_f16(const qwen3_bf16* in, qwen3_f16* out, size_t n, void* stream);
 
 /* Packs q/k/v_proj ([Hq*D,H], [Hkv*D,H], [Hkv*D,H]) into w_qkv (concatenated rows). */
 int qwen3_pack_qkv(const qwen3_config* cfg, const qwen3_bf16* wq, const qwen3_bf16* wk, const qwen3_bf16* wv,
@@ -254,22 +271,26 @@ int qwen3_generate_greedy(const qwen3_config* cfg, const qwen3_bf16* embed, cons
 /* ------------------------------------------------ single kernels (ops) */
 
 /* out[r] = x[r] * rsqrt(mean(x[r]^2) + eps) * w  ([P-Mini] section RMSNorm formula).
- * x bf16 or fp32 (x_f32 = 1), row stride ldx elements; out bf16 with stride ldo;
+ * x bf16 or fp32 (x_f32 = 1), row stride ldx elements; out bf16 (out_f16 = 0) or fp16
+ * (out_f16 = 1, the projections' operand type of the gemm_f16 mode) with stride ldo;
  * n % 256 == 0 and n <= 2048. */
 int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* w, qwen3_bf16* out, long long ldo,
-                     int rows, int n, float eps, void* stream);
+                     int rows, int n, float eps, int out_f16, void* stream);
 
 /* Linear layer on the tensor cores: out = epilogue(A . W^T), A [M, K] (lda), W [N, K] (ldw).
  *   epilogue 0: out = acc;  1: out = resid + acc (resid may alias out);
  *            2: SwiGLU -- W rows interleaved as qwen3_pack_gate_up, out [M, N/2] bf16.
  *   out_f32 / resid_f32 select fp32 (else bf16). swap: 1 = weight rows on the MMA's 128-row
- *   side (small M), 0 = activations there, -1 = automatic (swap when M <= 256).
+ *   side (small M), 0 = activations there, 2 = weight rows on the 128-row side with K split
+ *   over the CTAs of a thread-block cluster and summed in the same kernel (M <= 64,
+ *   N % 128 == 0; ws unused), -1 = automatic (2 when it applies, else 1 when M <= 256).
  *   ws (may be NULL): scratch for split-K when the output has too few tiles to fill the GPU;
  *   it holds fp32 partials, up to ws_bytes (split count = largest that fits).
+ *   ab_f16: A and W hold fp16 (1) or bf16 (0); the SwiGLU output takes the same type.
  *   K % 64 == 0, N % 32 == 0, leading dimensions multiples of 8 elements. */
 int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long long ldw, void* out, long long ldo,
                   int M, int N, int K, int epilogue, const void* resid, long long ldr, int resid_f32, int out_f32,
-                  int swap, void* ws, size_t ws_bytes, void* stream);
+                  int swap, int ab_f16, void* ws, size_t ws_bytes, void* stream);
 
 /* Per-head QK RMSNorm + rotate-half RoPE + KV-cache write (see qwen3_block_prefill for
  * positions). qkv [B*T, (Hq+2Hkv)*D] (row stride ldqkv): q heads are normalised and rotated
@@ -288,7 +309,8 @@ int qwen3_op_gemm_qkv_rope(const qwen3_config* cfg, const qwen3_bf16* h, const q
                            const qwen3_kv_layer* kv, const float* rope, void* stream);
 
 /* Causal GQA prefill attention: queries from qkv (already normed/rotated q heads), keys and
- * values from kv positions 0..start_pos[b]+t; o [B*T, Hq*D] (stride ldo), head-major columns. */
+ * values from kv positions 0..start_pos[b]+t; o [B*T, Hq*D] (stride ldo), head-major columns,
+ * bf16 (fp16 when cfg->gemm_f16: o is the input of the o_proj projection). */
 int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B, int T,
                                const int* start_pos, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                                void* stream);
@@ -300,7 +322,8 @@ int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, l
  * chunks whose (max, sum, unnormalised output) partials go to ws and are merged with
  * log-sum-exp weights (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max)
  * suffices). Hq / Hkv must be 1, 2, 4, 8 or 16. A position past the cache
- * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY. */
+ * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY. o is bf16, or fp16
+ * when cfg->gemm_f16 (as qwen3_op_attention_prefill); ldo a multiple of 8 and >= Hq*128. */
 int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                               const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                               void* ws, size_t ws_bytes, void* stream);
@@ -327,9 +350,11 @@ int qwen3_op_attention_decode_noalloc(const qwen3_config* cfg, const qwen3_bf16*
  * never chosen). V % 4 == 0, x and ldx 16-byte aligned in bytes. */
 int qwen3_op_argmax(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, void* stream);
 
-/* out[m] = embed[ids[m]] ([P-MoE] section 5), bf16 or fp32 (out_f32). */
+/* out[m] = embed[ids[m]] ([P-MoE] section 5). embed holds bf16, or fp16 (embed_f16 = 1, the
+ * gemm_f16 mode's tied embedding); out is fp32 (out_f32 = 1, exact widening) or a copy in
+ * embed's own type. */
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,
-                   void* stream);
+                   int embed_f16, void* stream);
 
 #ifdef __cplusplus
 }

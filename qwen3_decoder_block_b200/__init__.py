@@ -30,7 +30,7 @@ class Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("intermediate", ctypes.c_int), ("vocab", ctypes.c_int),
                 ("n_layers", ctypes.c_int), ("max_pos", ctypes.c_int), ("n_experts", ctypes.c_int),
                 ("top_k", ctypes.c_int), ("moe_intermediate", ctypes.c_int), ("norm_topk_prob", ctypes.c_int),
-                ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_double)]
+                ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_double), ("gemm_f16", ctypes.c_int)]
 
 
 class LayerWeights(ctypes.Structure):
@@ -69,14 +69,15 @@ _SIGS = {
     "qwen3_profile_begin": ([_i], _i),
     "qwen3_profile_end": ([_vp], _i),
     "qwen3_profile_record": ([_i, ctypes.c_char_p, _i, _P(_f)], _i),
-    "qwen3_op_rmsnorm": ([_vp, _i, _ll, _vp, _vp, _ll, _i, _i, _f, _vp], _i),
-    "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _vp, _sz, _vp], _i),
+    "qwen3_op_rmsnorm": ([_vp, _i, _ll, _vp, _vp, _ll, _i, _i, _f, _i, _vp], _i),
+    "qwen3_op_gemm": ([_vp, _ll, _vp, _ll, _vp, _ll, _i, _i, _i, _i, _vp, _ll, _i, _i, _i, _i, _vp, _sz, _vp], _i),
     "qwen3_op_qk_norm_rope": ([_P(Config), _vp, _ll, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
     "qwen3_op_gemm_qkv_rope": ([_P(Config), _vp, _vp, _vp, _i, _i, _vp, _vp, _vp, _P(KVLayer), _vp, _vp], _i),
     "qwen3_op_attention_prefill": ([_P(Config), _vp, _ll, _i, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
     "qwen3_op_attention_decode": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp, _sz, _vp], _i),
     "qwen3_op_attention_decode_noalloc": ([_P(Config), _vp, _ll, _i, _vp, _P(KVLayer), _vp, _ll, _vp], _i),
-    "qwen3_op_embed": ([_vp, _i, _vp, _i, _i, _vp, _i, _vp], _i),
+    "qwen3_op_embed": ([_vp, _i, _vp, _i, _i, _vp, _i, _i, _vp], _i),
+    "qwen3_convert_to_f16": ([_vp, _vp, _sz, _vp], _i),
     "qwen3_op_argmax": ([_vp, _ll, _i, _i, _vp, _ll, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
@@ -247,21 +248,27 @@ def op_argmax(x, rows, V, out, ldx=None, ld_out=1, stream=None) -> None:
 
 
 def op_rmsnorm(x, w, out, rows, n, eps, ldx=None, ldo=None, stream=None) -> None:
+    """out: a bf16 tensor, or an fp16 one (the fp16 operand mode's projection input)."""
     import torch
     x_f32 = 1 if x.dtype == torch.float32 else 0
-    _check(lib.qwen3_op_rmsnorm(_ptr(x), x_f32, ldx or n, _ptr(w), _ptr(out), ldo or n, rows, n, eps,
+    out_f16 = 1 if out.dtype == torch.float16 else 0
+    _check(lib.qwen3_op_rmsnorm(_ptr(x), x_f32, ldx or n, _ptr(w), _ptr(out), ldo or n, rows, n, eps, out_f16,
                                 _stream(stream)), "op_rmsnorm")
 
 
 def op_gemm(A, W, out, M, N, K, epilogue=EPI_STORE, resid=None, swap=-1, lda=None, ldw=None, ldo=None, ldr=None,
             ws=None, stream=None) -> None:
+    """A and W both bf16 or both fp16 (torch dtypes decide the operand type)."""
     import torch
     out_f32 = 1 if out.dtype == torch.float32 else 0
     resid_f32 = 1 if (resid is not None and resid.dtype == torch.float32) else 0
+    ab_f16 = 1 if A.dtype == torch.float16 else 0
+    if (W.dtype == torch.float16) != bool(ab_f16):
+        raise ValueError("op_gemm: A and W must share their type (bf16 or fp16)")
     if ldo is None:
         ldo = N // 2 if epilogue == EPI_SWIGLU else N
     _check(lib.qwen3_op_gemm(_ptr(A), lda or K, _ptr(W), ldw or K, _ptr(out), ldo, M, N, K, epilogue, _ptr(resid),
-                             ldr or N, resid_f32, out_f32, swap, _ptr(ws),
+                             ldr or N, resid_f32, out_f32, swap, ab_f16, _ptr(ws),
                              0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)), "op_gemm")
 
 
@@ -303,4 +310,18 @@ def op_attention_decode_noalloc(cfg, qkv, B, cache_len, kv, o, ldqkv=None, ldo=N
 def op_embed(ids, n, embed, vocab, H, out, stream=None) -> None:
     import torch
     _check(lib.qwen3_op_embed(_ptr(ids), n, _ptr(embed), vocab, H, _ptr(out), 1 if out.dtype == torch.float32 else 0,
-                              _stream(stream)), "op_embed")
+                              1 if embed.dtype == torch.float16 else 0, _stream(stream)), "op_embed")
+
+
+def convert_to_f16(src, dst=None, stream=None):
+    """bf16 -> fp16 (round to nearest even) into dst (a float16 tensor of the same size),
+    or in place when dst is None; returns the fp16 view."""
+    import torch
+    n = src.numel()
+    if dst is None:
+        _check(lib.qwen3_convert_to_f16(_ptr(src), _ptr(src), n, _stream(stream)), "convert_to_f16")
+        return src.view(torch.float16)
+    if dst.numel() != n:
+        raise ValueError("convert_to_f16: size mismatch")
+    _check(lib.qwen3_convert_to_f16(_ptr(src), _ptr(dst), n, _stream(stream)), "convert_to_f16")
+    return dst

@@ -25,7 +25,7 @@ NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xc
               "-Xcompiler", "-fopenmp", "-Xptxas", "-v"] + ARCH
 
 LIBRARIES = {
-    "libqwen3blk.so": ["api.cu", "gemm.cu", "elementwise.cu", "attention.cu", "moe.cu"],
+    "libqwen3blk.so": ["api.cu", "gemm.cu", "gemm_skinny.cu", "elementwise.cu", "attention.cu", "moe.cu"],
 }
 HEADERS = ["common.cuh", "internal.h"]
 

@@ -21,12 +21,13 @@
 namespace q3 {
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
-                   int rows, int n, float eps, cudaStream_t s);
+                   int rows, int n, float eps, cudaStream_t s, int* zero_word = nullptr, bool out_f16 = false);
 int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv, const int* pos_base,
                         const uint16_t* qw, const uint16_t* kw, const float* rope, uint16_t* ck, uint16_t* cv,
                         int s_max, int max_pos, float eps, int* err, cudaStream_t s);
 int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, void* out, bool out_f32, int* err,
-                 cudaStream_t s);
+                 cudaStream_t s, int* zero_word = nullptr, bool e_f16 = false);
+int launch_convert_to_f16(const uint16_t* in, uint16_t* out, long long n, cudaStream_t s);
 int launch_pack_gate_up(const uint16_t* gate, const uint16_t* up, long long mat_stride, int n_mats, int I, int H,
                         uint16_t* out, cudaStream_t s);
 int launch_advance_lengths(int* len, int B, cudaStream_t s);
@@ -35,14 +36,14 @@ int launch_argmax_rows(const float* x, long long ldx, int rows, int V, int* out,
 int launch_fill_lengths(int* len, int B, int value, cudaStream_t s);
 int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv,
                              const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
-                             long long ldo, int* err, cudaStream_t s);
+                             long long ldo, int* err, cudaStream_t s, bool o_f16 = false);
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
                             const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
-                            long long ldo, int* err, cudaStream_t s);
+                            long long ldo, int* err, cudaStream_t s, bool o_f16 = false, bool q_hilo = false);
 size_t decode_partial_bytes(int B, int Hq, int s_max);
 int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
                                    const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
-                                   uint16_t* out, long long ldo, int* err, cudaStream_t s);
+                                   uint16_t* out, long long ldo, int* err, cudaStream_t s, bool o_f16 = false);
 int launch_moe_route(const float* logits, int T, int E, int k, int renorm, int* idx, float* w, int* counts,
                      cudaStream_t s);
 int launch_moe_permute(const int* idx, int T, int k, int E, const int* counts, int* offsets, int* perm_token,
@@ -209,6 +210,7 @@ static int validate_cfg(const qwen3_config* c) {
   if (c->intermediate > 0)
     Q3_CHECK(c->intermediate % 64 == 0, QWEN3_ESHAPE, "intermediate (%d) must be a multiple of 64", c->intermediate);
   if (c->vocab > 0) Q3_CHECK(c->vocab % 32 == 0, QWEN3_ESHAPE, "vocab (%d) must be a multiple of 32", c->vocab);
+  Q3_CHECK(c->gemm_f16 == 0 || c->gemm_f16 == 1, QWEN3_ESHAPE, "gemm_f16 must be 0 or 1 (got %d)", c->gemm_f16);
   if (c->n_experts > 0) {
     Q3_CHECK(c->n_experts <= 256 && c->n_experts % 32 == 0, QWEN3_ESHAPE,
              "n_experts (%d) must be a multiple of 32 and at most 256", c->n_experts);
@@ -237,6 +239,7 @@ struct Carver {
 struct Buffers {
   uint16_t* h = nullptr;     // [M, H] normed activations
   uint16_t* qkv = nullptr;   // [M, Nqkv]
+  uint16_t* q2 = nullptr;    // [M, 2*Hq*D] decode: q as hi/lo bf16 rows per KV group
   uint16_t* o = nullptr;     // [M, Hq*D]
   float* x1 = nullptr;       // [M, H] residual after attention (fp32)
   uint16_t* act = nullptr;   // [M, I] SwiGLU output
@@ -257,6 +260,9 @@ struct Buffers {
   // stack
   float* xs = nullptr;       // [M, H] fp32 residual stream
   uint16_t* hf = nullptr;    // [rows, H] final-normed
+  // ticket of the decode-sized projections' fused RMSNorm: zeroed by the first kernel
+  // of every call, left at zero by every launch that uses it
+  int* ticket = nullptr;
 };
 
 static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void* ws, Buffers* out) {
@@ -270,7 +276,11 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
   b.qkv = cv.take<uint16_t>(M * nqkv);
   b.o = cv.take<uint16_t>(M * c.n_q_heads * D);
   b.x1 = cv.take<float>(M * H);
-  if (decode) b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, s_max) / sizeof(float));
+  // one new token per sequence (decode, or a prefill of T = 1) runs the split-KV decode attention
+  if (decode || T == 1) {
+    b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, s_max) / sizeof(float));
+    b.q2 = cv.take<uint16_t>(M * 2 * c.n_q_heads * D);
+  }
   if (M <= 256) b.gpart = cv.take<float>(kSplitKBytes / sizeof(float));
   if (op == QWEN3_OP_MOE_BLOCK) {
     const int E = c.n_experts, k = c.top_k;
@@ -292,6 +302,7 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
     b.xs = cv.take<float>(M * H);
     b.hf = cv.take<uint16_t>(M * H);
   }
+  b.ticket = cv.take<int>(64);
   if (out) *out = b;
   return cv.used + 256;
 }
@@ -315,12 +326,78 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   const int H = c.hidden, D = c.head_dim;
   const long long M = (long long)B * T;
   const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * D;
+  const bool f16 = c.gemm_f16 != 0;  // projections' operand type (q and the cache stay bf16)
+  // one token per sequence at position pos[b], attending 0..pos[b]: the decode attention
+  // computes exactly that, for a prefill of T = 1 as well
+  decode = decode || T == 1;
   int rc = 0;
   if (!h_ready) {
     ProfScope ps("rmsnorm", k.s);
-    rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+    rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s, b.ticket, f16);
   }
   if (rc) return rc;
+  QKRopeArgs qa;
+  qa.T = T;
+  qa.Hq = c.n_q_heads;
+  qa.Hkv = c.n_kv_heads;
+  qa.s_max = kv.s_max;
+  qa.max_pos = c.max_pos;
+  qa.pos_base = pos;
+  qa.q_norm = w.q_norm;
+  qa.k_norm = w.k_norm;
+  qa.rope = rope;
+  qa.ck = kv.k;
+  qa.cv = kv.v;
+  qa.eps = c.rms_eps;
+  const bool skinny = skinny_supported((int)M, nqkv, H, kEpiQKRope) &&
+                      skinny_supported((int)M, H, c.n_q_heads * D, kEpiResid);
+  if (skinny) {
+    // decode-sized: K split over clusters and summed in-kernel, each projection one launch
+    SkinnyDesc q;
+    q.A = b.h; q.lda = H; q.W = w.w_qkv; q.ldw = H;
+    q.M = (int)M; q.N = nqkv; q.K = H;
+    q.epi = kEpiQKRope;
+    q.out = b.qkv; q.ldo = nqkv;
+    q.w_early = true;  // weights; a library kernel of this call runs before this GEMM
+    q.qk = qa;
+    // one token per sequence: q as hi/lo halves for the decode attention (G <= 8)
+    const bool hilo = decode && c.n_q_heads / c.n_kv_heads <= 8;
+    if (hilo) {
+      q.qk.q2 = b.q2;
+      q.qk.ldq2 = 2LL * c.n_q_heads * D;
+    }
+    q.f16 = f16;
+    {
+      ProfScope ps("gemm_qkv", k.s);
+      rc = launch_gemm_skinny(q, k.s, k.err);
+    }
+    if (rc) return rc;
+    {
+      ProfScope ps(decode ? "attn_decode" : "attn_prefill", k.s);
+      if (decode)
+        rc = launch_attention_decode(hilo ? b.q2 : b.qkv, hilo ? 2LL * c.n_q_heads * D : nqkv, B, c.n_q_heads,
+                                     c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part, b.o,
+                                     (long long)c.n_q_heads * D, k.err, k.s, f16, hilo);
+      else
+        rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
+                                      (long long)c.n_q_heads * D, k.err, k.s, f16);
+    }
+    if (rc) return rc;
+    SkinnyDesc o;
+    o.A = b.o; o.lda = c.n_q_heads * D; o.W = w.w_o; o.ldw = c.n_q_heads * D;
+    o.M = (int)M; o.N = H; o.K = c.n_q_heads * D;
+    o.epi = kEpiResid;
+    o.resid = x; o.resid_f32 = x_f32; o.ldr = H;
+    o.out = b.x1; o.out_f32 = true; o.ldo = H;
+    o.w_early = true;
+    // the post-attention RMSNorm of x1 goes to b.h in the same launch
+    o.norm_w = w.post_norm; o.norm_out = b.h; o.ld_norm = H; o.norm_eps = c.rms_eps; o.ticket = b.ticket;
+    o.f16 = f16;
+    ProfScope ps("gemm_o", k.s);
+    rc = launch_gemm_skinny(o, k.s, k.err);
+    *h2_ready = rc == 0;
+    return rc;
+  }
   GemmDesc g;
   g.swap = swap_for(M);
   g.K = H;
@@ -328,6 +405,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   if (g.swap) { g.P = w.w_qkv; g.p_rows = nqkv; g.ldp = H; g.Q = act; g.q_rows = (int)M; g.ldq = H; }
   else        { g.P = act; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_qkv; g.q_rows = nqkv; g.ldq = H; }
   g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
+  g.f16 = f16;
   g.epi = kEpiStore;
   g.out = b.qkv;
   g.ldo = nqkv;
@@ -373,10 +451,10 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     ProfScope ps(decode ? "attn_decode" : "attn_prefill", k.s);
     if (decode)
       rc = launch_attention_decode(b.qkv, nqkv, B, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part,
-                                   b.o, (long long)c.n_q_heads * D, k.err, k.s);
+                                   b.o, (long long)c.n_q_heads * D, k.err, k.s, f16);
     else
       rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
-                                    (long long)c.n_q_heads * D, k.err, k.s);
+                                    (long long)c.n_q_heads * D, k.err, k.s, f16);
   }
   if (rc) return rc;
   GemmDesc o;
@@ -385,6 +463,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   if (o.swap) { o.P = w.w_o; o.p_rows = H; o.ldp = o.K; o.Q = b.o; o.q_rows = (int)M; o.ldq = o.K; }
   else        { o.P = b.o; o.p_rows = (int)M; o.ldp = o.K; o.Q = w.w_o; o.q_rows = H; o.ldq = o.K; }
   o.p_early = o.swap;  // weights; a library kernel of this call runs before this GEMM
+  o.f16 = f16;
   o.epi = kEpiResid;
   o.resid = x;
   o.resid_f32 = x_f32;
@@ -414,18 +493,49 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
                      bool* next_ready = nullptr) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, I = c.intermediate;
+  const bool f16 = c.gemm_f16 != 0;
   int rc = 0;
   if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
-    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s, nullptr, f16);
   }
   if (rc) return rc;
+  if (skinny_supported((int)M, 2 * I, H, kEpiSwiglu) && skinny_supported((int)M, H, I, kEpiResid)) {
+    SkinnyDesc g;
+    g.A = b.h; g.lda = H; g.W = w.w_gate_up; g.ldw = H;
+    g.M = (int)M; g.N = 2 * I; g.K = H;
+    g.epi = kEpiSwiglu;
+    g.out = b.act; g.ldo = I;
+    g.w_early = true;  // weights; a library kernel of this call runs before this GEMM
+    g.f16 = f16;
+    {
+      ProfScope ps("gemm_gate_up", k.s);
+      rc = launch_gemm_skinny(g, k.s, k.err);
+    }
+    if (rc) return rc;
+    SkinnyDesc d;
+    d.A = b.act; d.lda = I; d.W = w.w_down; d.ldw = I;
+    d.M = (int)M; d.N = H; d.K = I;
+    d.epi = kEpiResid;
+    d.resid = b.x1; d.resid_f32 = true; d.ldr = H;
+    d.out = out; d.out_f32 = out_f32; d.ldo = H;
+    d.w_early = true;
+    d.f16 = f16;
+    if (next_norm && next_out) {
+      d.norm_w = next_norm; d.norm_out = next_out; d.ld_norm = H; d.norm_eps = c.rms_eps; d.ticket = b.ticket;
+    }
+    ProfScope ps("gemm_down", k.s);
+    rc = launch_gemm_skinny(d, k.s, k.err);
+    if (next_ready) *next_ready = rc == 0 && next_norm && next_out;
+    return rc;
+  }
   GemmDesc g;
   g.swap = swap_for(M);
   g.K = H;
   if (g.swap) { g.P = w.w_gate_up; g.p_rows = 2 * I; g.ldp = H; g.Q = b.h; g.q_rows = (int)M; g.ldq = H; }
   else        { g.P = b.h; g.p_rows = (int)M; g.ldp = H; g.Q = w.w_gate_up; g.q_rows = 2 * I; g.ldq = H; }
   g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
+  g.f16 = f16;
   g.epi = kEpiSwiglu;
   g.out = b.act;
   g.ldo = I;
@@ -442,6 +552,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   if (d.swap) { d.P = w.w_down; d.p_rows = H; d.ldp = I; d.Q = b.act; d.q_rows = (int)M; d.ldq = I; }
   else        { d.P = b.act; d.p_rows = (int)M; d.ldp = I; d.Q = w.w_down; d.q_rows = H; d.ldq = I; }
   d.p_early = d.swap;  // weights; a library kernel of this call runs before this GEMM
+  d.f16 = f16;
   d.epi = kEpiResid;
   d.resid = b.x1;
   d.resid_f32 = true;
@@ -469,19 +580,32 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
                    bool h2_ready) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, E = c.n_experts, kk = c.top_k, Im = c.moe_intermediate;
+  const bool f16 = c.gemm_f16 != 0;
   int rc = 0;
   if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
-    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s);
+    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s, nullptr, f16);
   }
   if (rc) return rc;
   // router logits in fp32 (no bf16 rounding before the softmax)
+  if (skinny_supported((int)M, E, H, kEpiStore)) {
+    SkinnyDesc r;
+    r.A = b.h; r.lda = H; r.W = w.router; r.ldw = H;
+    r.M = (int)M; r.N = E; r.K = H;
+    r.epi = kEpiStore;
+    r.out = b.logits; r.out_f32 = true; r.ldo = E;
+    r.w_early = true;  // weights; a library kernel of this call runs before this GEMM
+    r.f16 = f16;
+    ProfScope ps("gemm_router", k.s);
+    rc = launch_gemm_skinny(r, k.s, k.err);
+  } else {
   GemmDesc r;
   r.swap = swap_for(M);
   r.K = H;
   if (r.swap) { r.P = w.router; r.p_rows = E; r.ldp = H; r.Q = b.h; r.q_rows = (int)M; r.ldq = H; }
   else        { r.P = b.h; r.p_rows = (int)M; r.ldp = H; r.Q = w.router; r.q_rows = E; r.ldq = H; r.force_bn = 128; }
   r.p_early = r.swap;  // weights; a library kernel of this call runs before this GEMM
+  r.f16 = f16;
   r.epi = kEpiStore;
   r.out = b.logits;
   r.out_f32 = true;
@@ -491,6 +615,7 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   {
     ProfScope ps("gemm_router", k.s);
     rc = launch_gemm(r, k.s, k.err);
+  }
   }
   if (rc) return rc;
   {
@@ -505,10 +630,21 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   }
   if (rc) return rc;
   const long long rows = M * kk;
+  // few routed rows per expert (decode-sized batches): each expert's weights on the MMA's
+  // 128-row side and its rows as N, so that every hit expert's weights stream once
+  const bool per_expert_swap = rows <= 32LL * E;
   GemmDesc gu;
-  gu.P = b.a_perm; gu.p_rows = (int)rows; gu.ldp = H;
-  gu.Q = w.moe_gate_up; gu.q_rows = 2 * Im; gu.ldq = H; gu.q_rows_total = (long long)E * 2 * Im;
+  if (per_expert_swap) {
+    gu.swap = true;
+    gu.P = w.moe_gate_up; gu.p_rows = 2 * Im; gu.ldp = H; gu.p_rows_total = (long long)E * 2 * Im;
+    gu.Q = b.a_perm; gu.q_rows = (int)rows; gu.ldq = H;
+    gu.force_bn = 64;
+  } else {
+    gu.P = b.a_perm; gu.p_rows = (int)rows; gu.ldp = H;
+    gu.Q = w.moe_gate_up; gu.q_rows = 2 * Im; gu.ldq = H; gu.q_rows_total = (long long)E * 2 * Im;
+  }
   gu.K = H;
+  gu.f16 = f16;
   gu.epi = kEpiSwiglu;
   gu.out = b.act_perm; gu.ldo = Im;
   gu.n_groups = E; gu.group_offsets = b.offsets;
@@ -518,9 +654,17 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
   }
   if (rc) return rc;
   GemmDesc dn;
-  dn.P = b.act_perm; dn.p_rows = (int)rows; dn.ldp = Im;
-  dn.Q = w.moe_down; dn.q_rows = H; dn.ldq = Im; dn.q_rows_total = (long long)E * H;
+  if (per_expert_swap) {
+    dn.swap = true;
+    dn.P = w.moe_down; dn.p_rows = H; dn.ldp = Im; dn.p_rows_total = (long long)E * H;
+    dn.Q = b.act_perm; dn.q_rows = (int)rows; dn.ldq = Im;
+    dn.force_bn = 64;
+  } else {
+    dn.P = b.act_perm; dn.p_rows = (int)rows; dn.ldp = Im;
+    dn.Q = w.moe_down; dn.q_rows = H; dn.ldq = Im; dn.q_rows_total = (long long)E * H;
+  }
   dn.K = Im;
+  dn.f16 = f16;
   dn.epi = kEpiStore;
   dn.out = b.y; dn.ldo = H;
   dn.n_groups = E; dn.group_offsets = b.offsets;
@@ -898,7 +1042,7 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   const long long M = (long long)B * T;
   {
     ProfScope ps("embed", s);
-    rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s);
+    rc = launch_embed(ids, (int)M, embed, c->vocab, H, b.xs, true, k.err, s, b.ticket, c->gemm_f16 != 0);
   }
   if (rc) return finish(rc);
   // With split K (small token counts), each layer's down projection also leaves the
@@ -920,7 +1064,7 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   const long long ldx = last_only ? (long long)T * H : H;
   if (!h_ready) {
     ProfScope ps("rmsnorm", s);
-    rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s);
+    rc = launch_rmsnorm(xf, true, ldx, final_norm, b.hf, H, rows, H, c->rms_eps, s, nullptr, c->gemm_f16 != 0);
   }
   if (rc) return finish(rc);
   GemmDesc g;
@@ -929,6 +1073,7 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   if (g.swap) { g.P = embed; g.p_rows = c->vocab; g.ldp = H; g.Q = b.hf; g.q_rows = rows; g.ldq = H; }
   else        { g.P = b.hf; g.p_rows = rows; g.ldp = H; g.Q = embed; g.q_rows = c->vocab; g.ldq = H; }
   g.p_early = g.swap;  // weights; a library kernel of this call runs before this GEMM
+  g.f16 = c->gemm_f16 != 0;
   g.epi = kEpiStore;
   g.out = logits;
   g.out_f32 = true;
@@ -986,7 +1131,7 @@ int qwen3_profile_record(int i, char* name, int name_cap, float* ms) {
 
 // ----------------------------------------------------------------------------- ops
 int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* w, qwen3_bf16* out, long long ldo,
-                     int rows, int n, float eps, void* stream) {
+                     int rows, int n, float eps, int out_f16, void* stream) {
   g_last_error.clear();
   Q3_CHECK(x && w && out, QWEN3_EINVAL, "rmsnorm: NULL pointer");
   Q3_CHECK(aligned16(x) && aligned16(w) && aligned16(out), QWEN3_EALIGN, "rmsnorm: misaligned pointer");
@@ -995,12 +1140,13 @@ int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* 
            "rmsnorm: bad rows or leading dimensions");
   int rc = check_device();
   if (rc) return rc;
-  return finish(launch_rmsnorm(x, x_f32 != 0, ldx, w, out, ldo, rows, n, eps, static_cast<cudaStream_t>(stream)));
+  return finish(launch_rmsnorm(x, x_f32 != 0, ldx, w, out, ldo, rows, n, eps, static_cast<cudaStream_t>(stream),
+                               nullptr, out_f16 != 0));
 }
 
 int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long long ldw, void* out, long long ldo,
                   int M, int N, int K, int epilogue, const void* resid, long long ldr, int resid_f32, int out_f32,
-                  int swap, void* ws, size_t ws_bytes, void* stream) {
+                  int swap, int ab_f16, void* ws, size_t ws_bytes, void* stream) {
   g_last_error.clear();
   Q3_CHECK(A && W && out, QWEN3_EINVAL, "gemm: NULL operand");
   Q3_CHECK(aligned16(A) && aligned16(W) && aligned16(out), QWEN3_EALIGN, "gemm: misaligned operand");
@@ -1012,14 +1158,29 @@ int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long 
   if (epilogue == kEpiResid) {
     Q3_CHECK(resid && aligned16(resid) && ldr % 8 == 0 && ldr >= N, QWEN3_EINVAL, "gemm: residual missing or misaligned");
   }
+  Q3_CHECK(ab_f16 == 0 || ab_f16 == 1, QWEN3_EINVAL, "gemm: ab_f16 must be 0 or 1");
   if (epilogue == kEpiSwiglu) {
-    Q3_CHECK(!out_f32, QWEN3_EINVAL, "gemm: SwiGLU output is bf16");
+    Q3_CHECK(!out_f32, QWEN3_EINVAL, "gemm: SwiGLU output is 16-bit (the operand type)");
     Q3_CHECK(ldo >= N / 2, QWEN3_EINVAL, "gemm: ldo too small for N/2 outputs");
   } else {
     Q3_CHECK(ldo >= N, QWEN3_EINVAL, "gemm: ldo (%lld) < N (%d)", ldo, N);
   }
+  Q3_CHECK(swap >= -1 && swap <= 2, QWEN3_EINVAL, "gemm: swap must be -1, 0, 1 or 2 (got %d)", swap);
+  if (swap == 2)
+    Q3_CHECK(skinny_supported(M, N, K, epilogue), QWEN3_ESHAPE,
+             "gemm: the cluster split-K form needs M <= 64 and N %% 128 == 0 (M %d, N %d)", M, N);
   int rc = check_device();
   if (rc) return rc;
+  if (swap == 2 || (swap < 0 && skinny_supported(M, N, K, epilogue))) {
+    SkinnyDesc d;
+    d.A = A; d.lda = lda; d.W = W; d.ldw = ldw;
+    d.M = M; d.N = N; d.K = K;
+    d.epi = epilogue;
+    d.out = out; d.ldo = ldo; d.out_f32 = out_f32 != 0;
+    d.resid = resid; d.ldr = ldr; d.resid_f32 = resid_f32 != 0;
+    d.f16 = ab_f16 != 0;
+    return finish(launch_gemm_skinny(d, static_cast<cudaStream_t>(stream), device_error_word()));
+  }
   GemmDesc g;
   g.swap = swap < 0 ? swap_for(M) : swap != 0;
   g.K = K;
@@ -1032,6 +1193,7 @@ int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long 
   g.out = out;
   g.ldo = ldo;
   g.out_f32 = out_f32 != 0;
+  g.f16 = ab_f16 != 0;
   if (ws && aligned16(ws)) {
     g.partial = static_cast<float*>(ws);
     g.partial_bytes = ws_bytes;
@@ -1077,6 +1239,7 @@ int qwen3_op_gemm_qkv_rope(const qwen3_config* c, const qwen3_bf16* h, const qwe
   g.Q = w_qkv; g.q_rows = nqkv; g.ldq = H;
   g.epi = kEpiQKRope;
   g.force_bn = 256;
+  g.f16 = c->gemm_f16 != 0;
   g.out = qkv;
   g.ldo = nqkv;
   g.qk.T = T;
@@ -1108,7 +1271,8 @@ int qwen3_op_attention_prefill(const qwen3_config* c, const qwen3_bf16* qkv, lon
   if ((rc = check_kv(*c, kv, T))) return rc;
   if ((rc = check_device())) return rc;
   return finish(launch_attention_prefill(qkv, ldqkv, B, T, c->n_q_heads, c->n_kv_heads, start_pos, kv->k, kv->v,
-                                         kv->s_max, o, ldo, device_error_word(), static_cast<cudaStream_t>(stream)));
+                                         kv->s_max, o, ldo, device_error_word(), static_cast<cudaStream_t>(stream),
+                                         c->gemm_f16 != 0));
 }
 
 int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B,
@@ -1131,7 +1295,7 @@ int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long
   if ((rc = check_device())) return rc;
   return finish(launch_attention_decode(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
                                         kv->s_max, static_cast<float*>(ws), o, ldo, device_error_word(),
-                                        static_cast<cudaStream_t>(stream)));
+                                        static_cast<cudaStream_t>(stream), c->gemm_f16 != 0));
 }
 
 int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* qkv, long long ldqkv, int B,
@@ -1152,7 +1316,7 @@ int qwen3_op_attention_decode_noalloc(const qwen3_config* c, const qwen3_bf16* q
   if ((rc = check_device())) return rc;
   return finish(launch_attention_decode_static(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,
                                                kv->s_max, o, ldo, device_error_word(),
-                                               static_cast<cudaStream_t>(stream)));
+                                               static_cast<cudaStream_t>(stream), c->gemm_f16 != 0));
 }
 
 int qwen3_op_argmax(const float* x, long long ldx, int rows, int V, int* out, long long ld_out, void* stream) {
@@ -1208,7 +1372,7 @@ int qwen3_generate_greedy(const qwen3_config* c, const qwen3_bf16* embed, const 
 }
 
 int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, int H, void* out, int out_f32,
-                   void* stream) {
+                   int embed_f16, void* stream) {
   g_last_error.clear();
   Q3_CHECK(ids && embed && out, QWEN3_EINVAL, "embed: NULL pointer");
   Q3_CHECK(aligned16(embed) && aligned16(out), QWEN3_EALIGN, "embed: misaligned pointer");
@@ -1216,7 +1380,20 @@ int qwen3_op_embed(const int* ids, int n, const qwen3_bf16* embed, int vocab, in
   int rc = check_device();
   if (rc) return rc;
   return finish(launch_embed(ids, n, embed, vocab, H, out, out_f32 != 0, device_error_word(),
-                             static_cast<cudaStream_t>(stream)));
+                             static_cast<cudaStream_t>(stream), nullptr, embed_f16 != 0));
+}
+
+int qwen3_convert_to_f16(const qwen3_bf16* in, qwen3_f16* out, size_t n, void* stream) {
+  g_last_error.clear();
+  Q3_CHECK(in && out, QWEN3_EINVAL, "convert_to_f16: NULL pointer");
+  Q3_CHECK(aligned16(in) && aligned16(out), QWEN3_EALIGN, "convert_to_f16: misaligned pointer");
+  Q3_CHECK(n > 0, QWEN3_EINVAL, "convert_to_f16: n must be positive");
+  Q3_CHECK(in == out || reinterpret_cast<uintptr_t>(in) + 2 * n <= reinterpret_cast<uintptr_t>(out) ||
+               reinterpret_cast<uintptr_t>(out) + 2 * n <= reinterpret_cast<uintptr_t>(in),
+           QWEN3_EINVAL, "convert_to_f16: in and out overlap without being the same buffer");
+  int rc = check_device();
+  if (rc) return rc;
+  return finish(launch_convert_to_f16(in, out, (long long)n, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -53,6 +53,7 @@ constexpr float kRescaleThreshold = 8.0f;
 
 struct PrefillParams {
   int B, T, Hq, Hkv, G, s_max, n_cta_q;
+  int o_f16;  // o feeds an fp16-operand projection (bf16 otherwise)
   const int* start_pos;
   uint16_t* out;
   long long ldo;
@@ -355,10 +356,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]) * inv_l, __uint_as_float(v[8 * i + 1]) * inv_l);
-              o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l, __uint_as_float(v[8 * i + 3]) * inv_l);
-              o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l, __uint_as_float(v[8 * i + 5]) * inv_l);
-              o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l, __uint_as_float(v[8 * i + 7]) * inv_l);
+              const bool f16 = p.o_f16 != 0;
+              o.x = pack_op_x2(f16, __uint_as_float(v[8 * i + 0]) * inv_l, __uint_as_float(v[8 * i + 1]) * inv_l);
+              o.y = pack_op_x2(f16, __uint_as_float(v[8 * i + 2]) * inv_l, __uint_as_float(v[8 * i + 3]) * inv_l);
+              o.z = pack_op_x2(f16, __uint_as_float(v[8 * i + 4]) * inv_l, __uint_as_float(v[8 * i + 5]) * inv_l);
+              o.w = pack_op_x2(f16, __uint_as_float(v[8 * i + 6]) * inv_l, __uint_as_float(v[8 * i + 7]) * inv_l);
               *reinterpret_cast<uint4*>(dst + c * 32 + i * 8) = o;
             }
           }
@@ -381,7 +383,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
 int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv,
                              const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
-                             long long ldo, int* err, cudaStream_t s) {
+                             long long ldo, int* err, cudaStream_t s, bool o_f16) {
   if (B <= 0 || T <= 0) return 0;
   const int G = Hq / Hkv;
   const int TQ = kTileQ / G;
@@ -400,6 +402,7 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
   PrefillParams p;
   p.B = B; p.T = T; p.Hq = Hq; p.Hkv = Hkv; p.G = G; p.s_max = s_max;
   p.n_cta_q = (T + 2 * TQ - 1) / (2 * TQ);
+  p.o_f16 = o_f16 ? 1 : 0;
   p.start_pos = start_pos;
   p.out = out;
   p.ldo = ldo;
@@ -464,7 +467,12 @@ constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
 
 __device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-template <int G>
+// HILO (G <= 8): q arrives as 2G rows per group, q_hi = bf16(q) in rows 0..G-1 and
+// q_lo = bf16(q - q_hi) in rows G..2G-1, and P is written the same way, so the N = 16
+// columns of both MMAs carry the hi and lo halves: S = K q_hi + K q_lo and
+// O = V P_hi + V P_lo, summed in fp32 -- about 16 significant bits for q and P at no
+// extra MMA instruction (the kernel is bound by the K/V stream).
+template <int G, bool HILO>
 __global__ void __launch_bounds__(kD4Threads, 1)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, int B, int Hq, int Hkv,
@@ -530,9 +538,10 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           const int st = (int)(tc % kD4Stages);
           if (*s_abort || !mbar_wait(&empty[st], (uint32_t)((tc / kD4Stages) & 1) ^ 1u, err)) { ok = false; break; }
           uint8_t* base = smem + st * kD4StageBytes;
-          mbar_arrive_expect_tx(&full[st], 4 * kD4Half + 2 * G * 128);
-          tma_load_3d(base + kD4OffQ, &tmQ, &full[st], 0, g * G, b);
-          tma_load_3d(base + kD4OffQ + kD4QHalf, &tmQ, &full[st], 64, g * G, b);
+          constexpr int QR = HILO ? 2 * G : G;  // query rows of a group in the tile
+          mbar_arrive_expect_tx(&full[st], 4 * kD4Half + 2 * QR * 128);
+          tma_load_3d(base + kD4OffQ, &tmQ, &full[st], 0, g * QR, b);
+          tma_load_3d(base + kD4OffQ + kD4QHalf, &tmQ, &full[st], 64, g * QR, b);
           tma_load_2d(base + kD4OffK, &tmK, &full[st], 0, row0 + k0);
           tma_load_2d(base + kD4OffK + kD4Half, &tmK, &full[st], 64, row0 + k0);
           tma_load_2d(base + kD4OffV, &tmV, &full[st], 0, row0 + k0);
@@ -636,7 +645,10 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         mbar_arrive(&s_empty[sb]);
         float s[G];
 #pragma unroll
-        for (int j = 0; j < G; ++j) s[j] = (ok && t < nk) ? __uint_as_float(sv[j]) * kScaleLog2 : -INFINITY;
+        for (int j = 0; j < G; ++j) {
+          const float sj = HILO ? __uint_as_float(sv[j]) + __uint_as_float(sv[G + j]) : __uint_as_float(sv[j]);
+          s[j] = (ok && t < nk) ? sj * kScaleLog2 : -INFINITY;
+        }
         // tile maximum per head: the warp's 32 keys, then the 4 warps
         float* rm = red_max + (tc & 1) * 64;
 #pragma unroll
@@ -675,7 +687,10 @@ __global__ void __launch_bounds__(kD4Threads, 1)
             tmem_ld16(tl + 32, ov);
             tmem_wait_ld_regs16(ov);
 #pragma unroll
-            for (int j = 0; j < G; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha[j]);
+            for (int j = 0; j < G; ++j) {
+              ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha[j]);
+              if (HILO) ov[G + j] = __float_as_uint(__uint_as_float(ov[G + j]) * alpha[j]);
+            }
             tmem_st16x(tl + 32, ov);
             tmem_wait_st();
           }
@@ -683,8 +698,15 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           uint8_t* pb = smem + kD4OffP + (t >> 6) * kD4QHalf + (t & 7) * 2;
           const int chunk = (t & 63) >> 3;
 #pragma unroll
-          for (int j = 0; j < G; ++j)
-            *reinterpret_cast<uint16_t*>(pb + j * 128 + ((chunk ^ (j & 7)) << 4)) = to_bf16_bits(p[j]);
+          for (int j = 0; j < G; ++j) {
+            const uint16_t hi = to_bf16_bits(p[j]);
+            *reinterpret_cast<uint16_t*>(pb + j * 128 + ((chunk ^ (j & 7)) << 4)) = hi;
+            if (HILO) {
+              const int jl = G + j;
+              *reinterpret_cast<uint16_t*>(pb + jl * 128 + ((chunk ^ (jl & 7)) << 4)) =
+                  to_bf16_bits(p[j] - __uint_as_float((uint32_t)hi << 16));
+            }
+          }
           // keys past the written cache: zero their V rows (0 * NaN would poison O)
           if (t >= nk) {
             uint4* v0 = reinterpret_cast<uint4*>(smem + (int)(tc % kD4Stages) * kD4StageBytes + kD4OffV + t * 128);
@@ -722,7 +744,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
       }
 #pragma unroll
       for (int j = 0; j < G; ++j) {
-        my_part[j * head_stride + t] = __uint_as_float(ov[j]);
+        my_part[j * head_stride + t] = HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
         if (t == j) {
           const float L = n_tiles > 0 ? red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j] : 0.f;
           my_part[j * head_stride + kHeadDim] = m_run[j];
@@ -742,7 +764,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
 }
 
 __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
-                                         uint16_t* __restrict__ out, long long ldo) {
+                                         uint16_t* __restrict__ out, long long ldo, int o_f16) {
   pdl_wait();
   pdl_trigger();
   const int bh = blockIdx.x;  // b * Hq + h
@@ -760,7 +782,7 @@ __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq,
     L += q[kHeadDim + 1] * w;
     acc += q[d] * w;
   }
-  out[(long long)b * ldo + (long long)h * kHeadDim + d] = to_bf16_bits(acc / L);
+  out[(long long)b * ldo + (long long)h * kHeadDim + d] = to_op_bits(o_f16 != 0, acc / L);
 }
 
 int decode_splits(int s_max) { return (s_max + kD4Split - 1) / kD4Split; }
@@ -769,9 +791,12 @@ size_t decode_partial_bytes(int B, int Hq, int s_max) {
   return (size_t)B * Hq * decode_splits(s_max) * (kHeadDim + 2) * sizeof(float);
 }
 
+// qkv: [B][ldqkv] with the Hq query heads at the start of each row; with q_hilo the row
+// holds 2 * Hq heads instead, for group g the G rows q_hi then the G rows q_lo
+// (G <= 8 only).
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
                             const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
-                            long long ldo, int* err, cudaStream_t s) {
+                            long long ldo, int* err, cudaStream_t s, bool o_f16, bool q_hilo) {
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) {
@@ -784,9 +809,14 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     return -2;
   }
   const int n_splits = decode_splits(s_max);
+  if (q_hilo && G > 8) {
+    set_last_error("attention decode: the hi/lo query layout needs at most 8 query heads per KV group");
+    return -2;
+  }
   CUtensorMap tmQ, tmK, tmV;
-  // Q: (dim, head, token), box = the G heads of one group
-  if (make_tmap_3d(&tmQ, qkv, kHeadDim, Hq, B, kHeadDim * 2, ldqkv * 2, 64, G, 1) != 0) {
+  // Q: (dim, head, token), box = the G heads of one group (2G rows: hi and lo)
+  const int qr = q_hilo ? 2 * G : G;
+  if (make_tmap_3d(&tmQ, qkv, kHeadDim, (long long)qr * Hkv, B, kHeadDim * 2, ldqkv * 2, 64, qr, 1) != 0) {
     set_last_error("attention decode: cannot encode the query tensor map");
     return -6;
   }
@@ -798,21 +828,26 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   }
   const long long items = (long long)B * Hkv * n_splits;
   const int grid = (int)(items < num_sms() ? items : num_sms());
-  switch (G) {
-#define Q3_D4_CASE(GG)                                                                                            \
-  case GG:                                                                                                        \
-    if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG>), kD4Smem)) return -6;           \
-    q3_launch(attn_decode_tc_kernel<GG>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,      \
+  const int variant = G * 2 + (q_hilo ? 1 : 0);
+  switch (variant) {
+#define Q3_D4_CASE(GG, HL)                                                                                        \
+  case GG * 2 + HL:                                                                                               \
+    if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG, HL>), kD4Smem)) return -6;       \
+    q3_launch(attn_decode_tc_kernel<GG, HL>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,  \
               s_max, n_splits, part, err);                                                                        \
     break;
-    Q3_D4_CASE(1)
-    Q3_D4_CASE(2)
-    Q3_D4_CASE(4)
-    Q3_D4_CASE(8)
-    Q3_D4_CASE(16)
+    Q3_D4_CASE(1, false)
+    Q3_D4_CASE(2, false)
+    Q3_D4_CASE(4, false)
+    Q3_D4_CASE(8, false)
+    Q3_D4_CASE(16, false)
+    Q3_D4_CASE(1, true)
+    Q3_D4_CASE(2, true)
+    Q3_D4_CASE(4, true)
+    Q3_D4_CASE(8, true)
 #undef Q3_D4_CASE
   }
-  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo);
+  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo, o_f16 ? 1 : 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
@@ -840,7 +875,7 @@ size_t static_decode_scratch_bytes() { return kStaticDecodeFloats * sizeof(float
 
 int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
                                    const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
-                                   uint16_t* out, long long ldo, int* err, cudaStream_t s) {
+                                   uint16_t* out, long long ldo, int* err, cudaStream_t s, bool o_f16) {
   const size_t need = decode_partial_bytes(B, Hq, s_max);
   if (need > kStaticDecodeFloats * sizeof(float)) {
     set_last_error("attention_decode_noalloc: B=%d, Hq=%d, s_max=%d need %zu bytes of split scratch; the "
@@ -867,7 +902,8 @@ int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, 
     }
     ptr = g_static_ptr[dev];
   }
-  return launch_attention_decode(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, cv, s_max, ptr, out, ldo, err, s);
+  return launch_attention_decode(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, cv, s_max, ptr, out, ldo, err, s, o_f16,
+                                 false);
 }
 
 }  // namespace q3

@@ -33,12 +33,16 @@ __device__ __forceinline__ void rms_load8(const void* x, long long off, float (&
   }
 }
 
-template <bool IN_F32>
+// zero_word (optional): an int this kernel sets to 0 (the fused-norm ticket of the
+// call's decode-sized projections; see launch_gemm_skinny).
+// OUT_F16: the output feeds an fp16-operand projection (bf16 otherwise).
+template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
                                                          const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
-                                                         long long ldo, int rows, int n, float eps) {
+                                                         long long ldo, int rows, int n, float eps, int* zero_word) {
   pdl_wait();
   pdl_trigger();
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
   const int lane = threadIdx.x & 31;
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int n_warps = (gridDim.x * blockDim.x) >> 5;
@@ -57,25 +61,24 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
       rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
       const uint4 wv = *reinterpret_cast<const uint4*>(w + col);
       uint4 o;
-      o.x = pack_bf16x2(v[0] * r * bf16_lo(wv.x), v[1] * r * bf16_hi(wv.x));
-      o.y = pack_bf16x2(v[2] * r * bf16_lo(wv.y), v[3] * r * bf16_hi(wv.y));
-      o.z = pack_bf16x2(v[4] * r * bf16_lo(wv.z), v[5] * r * bf16_hi(wv.z));
-      o.w = pack_bf16x2(v[6] * r * bf16_lo(wv.w), v[7] * r * bf16_hi(wv.w));
+      o.x = pack_op_x2(OUT_F16, v[0] * r * bf16_lo(wv.x), v[1] * r * bf16_hi(wv.x));
+      o.y = pack_op_x2(OUT_F16, v[2] * r * bf16_lo(wv.y), v[3] * r * bf16_hi(wv.y));
+      o.z = pack_op_x2(OUT_F16, v[4] * r * bf16_lo(wv.z), v[5] * r * bf16_hi(wv.z));
+      o.w = pack_op_x2(OUT_F16, v[6] * r * bf16_lo(wv.w), v[7] * r * bf16_hi(wv.w));
       *reinterpret_cast<uint4*>(out + (long long)row * ldo + col) = o;
     }
   }
 }
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
-                   int rows, int n, float eps, cudaStream_t s) {
+                   int rows, int n, float eps, cudaStream_t s, int* zero_word, bool out_f16) {
   if (rows <= 0) return 0;
   const int warps_per_block = 8;
   long long blocks = (rows + warps_per_block - 1) / warps_per_block;
   if (blocks > (long long)num_sms() * 16) blocks = (long long)num_sms() * 16;
-  if (x_f32)
-    q3_launch(rmsnorm_kernel<true>, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps);
-  else
-    q3_launch(rmsnorm_kernel<false>, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps);
+  auto k = x_f32 ? (out_f16 ? rmsnorm_kernel<true, true> : rmsnorm_kernel<true, false>)
+                 : (out_f16 ? rmsnorm_kernel<false, true> : rmsnorm_kernel<false, false>);
+  q3_launch(k, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps, zero_word);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -161,10 +164,13 @@ int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, in
 // Embedding gather ([P-MoE] section 5; [P-Mini] section 骨架): out[m] = E[ids[m]],
 // widened to fp32 when the residual stream is kept in fp32.
 // ---------------------------------------------------------------------------
+// E holds bf16, or fp16 (e_f16) in the fp16 operand mode; the fp32 output widens
+// either exactly, a 16-bit output copies E's values unchanged.
 __global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t* __restrict__ E, int vocab, int H,
-                             void* __restrict__ out, int out_f32, int* err) {
+                             void* __restrict__ out, int out_f32, int e_f16, int* err, int* zero_word) {
   pdl_wait();
   pdl_trigger();
+  if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
   const int m = blockIdx.x;
   if (m >= n) return;
   const int id = ids[m];
@@ -177,8 +183,14 @@ __global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t*
     uint4 a = src[c];
     if (out_f32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + (long long)m * H + c * 8);
-      dst[0] = make_float4(bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y));
-      dst[1] = make_float4(bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w));
+      if (e_f16) {
+        const uint16_t* h = reinterpret_cast<const uint16_t*>(&a);
+        dst[0] = make_float4(f16_bits_to_f32(h[0]), f16_bits_to_f32(h[1]), f16_bits_to_f32(h[2]), f16_bits_to_f32(h[3]));
+        dst[1] = make_float4(f16_bits_to_f32(h[4]), f16_bits_to_f32(h[5]), f16_bits_to_f32(h[6]), f16_bits_to_f32(h[7]));
+      } else {
+        dst[0] = make_float4(bf16_lo(a.x), bf16_hi(a.x), bf16_lo(a.y), bf16_hi(a.y));
+        dst[1] = make_float4(bf16_lo(a.z), bf16_hi(a.z), bf16_lo(a.w), bf16_hi(a.w));
+      }
     } else {
       reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + (long long)m * H)[c] = a;
     }
@@ -186,9 +198,9 @@ __global__ void embed_kernel(const int* __restrict__ ids, int n, const uint16_t*
 }
 
 int launch_embed(const int* ids, int n, const uint16_t* E, int vocab, int H, void* out, bool out_f32, int* err,
-                 cudaStream_t s) {
+                 cudaStream_t s, int* zero_word, bool e_f16) {
   if (n <= 0) return 0;
-  q3_launch(embed_kernel, n, 128, 0, s, ids, n, E, vocab, H, out, out_f32 ? 1 : 0, err);
+  q3_launch(embed_kernel, n, 128, 0, s, ids, n, E, vocab, H, out, out_f32 ? 1 : 0, e_f16 ? 1 : 0, err, zero_word);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 
@@ -304,6 +316,39 @@ __global__ void fill_lengths_kernel(int* len, int B, int value) {
 int launch_fill_lengths(int* len, int B, int value, cudaStream_t s) {
   if (B <= 0) return 0;
   q3_launch(fill_lengths_kernel, (B + 127) / 128, 128, 0, s, len, B, value);
+  return cudaGetLastError() == cudaSuccess ? 0 : -6;
+}
+
+
+// ---------------------------------------------------------------------------
+// bf16 -> fp16 conversion (round to nearest even), 8 elements per thread where the
+// buffers allow; in == out converts in place (each element is read before it is
+// written, by the same thread).
+// ---------------------------------------------------------------------------
+__global__ void convert_to_f16_kernel(const uint16_t* in, uint16_t* out, long long n) {
+  pdl_wait();
+  pdl_trigger();
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long n8 = n / 8;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    const uint4 a = reinterpret_cast<const uint4*>(in)[i];
+    uint4 o;
+    o.x = pack_f16x2(bf16_lo(a.x), bf16_hi(a.x));
+    o.y = pack_f16x2(bf16_lo(a.y), bf16_hi(a.y));
+    o.z = pack_f16x2(bf16_lo(a.z), bf16_hi(a.z));
+    o.w = pack_f16x2(bf16_lo(a.w), bf16_hi(a.w));
+    reinterpret_cast<uint4*>(out)[i] = o;
+  }
+  for (long long i = n8 * 8 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = to_f16_bits(__uint_as_float((uint32_t)in[i] << 16));
+}
+
+int launch_convert_to_f16(const uint16_t* in, uint16_t* out, long long n, cudaStream_t s) {
+  if (n <= 0) return 0;
+  long long blocks = (n / 8 + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > (long long)num_sms() * 8) blocks = (long long)num_sms() * 8;
+  q3_launch(convert_to_f16_kernel, (int)blocks, 256, 0, s, in, out, n);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

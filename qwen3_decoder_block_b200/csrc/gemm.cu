@@ -55,6 +55,7 @@ struct GemmParams {
   float* partial;              // split-K partials [k_splits][tokens][features] (fp32)
   int epi, resid_f32, out_f32, swap;
   int tma_store;  // non-swap store/residual epilogues: stage in shared memory, TMA tile store
+  int f16;        // operands fp16 (else bf16); the SwiGLU output is fp16 too
   int p_early;    // P is final before this grid launches: its first tile's loads precede the grid-dependency wait
   void* out;
   long long ldo;
@@ -68,6 +69,7 @@ struct GemmParams {
 
 struct Tile {
   int p0, p_end, q0, q_end, q_load, kb0, kb1, ks;
+  int p_out;  // output column of row p0 of the tile (grouped swap: p0 minus the group's first weight row)
 };
 
 __device__ __forceinline__ int total_tiles(const GemmParams& g, const int* s_prefix) {
@@ -88,9 +90,22 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const in
       if (s_prefix[mid] <= t) lo = mid; else hi = mid - 1;
     }
     const int grp = lo, local = t - s_prefix[grp];
+    if (g.swap) {
+      // weights of group grp on the 128-row side ([grp * p_rows, (grp + 1) * p_rows)), the
+      // group's activation rows [off[grp], off[grp + 1]) as N; weight tiles fastest
+      const int pt = local % g.p_tiles, qt = local / g.p_tiles;
+      r.p0 = grp * g.p_rows + pt * BM;
+      r.p_end = (grp + 1) * g.p_rows;
+      r.p_out = pt * BM;
+      r.q0 = s_off[grp] + qt * BN;
+      r.q_end = s_off[grp + 1];
+      r.q_load = r.q0;
+      return r;
+    }
     const int pt = local / g.q_tiles, qt = local % g.q_tiles;
     r.p0 = s_off[grp] + pt * BM;
     r.p_end = s_off[grp + 1];
+    r.p_out = r.p0;
     r.q0 = qt * BN;
     r.q_end = g.q_rows;
     r.q_load = grp * g.q_rows + r.q0;
@@ -106,6 +121,7 @@ __device__ __forceinline__ Tile decode_tile(int t, const GemmParams& g, const in
     else          { qt = t / g.p_tiles; pt = t % g.p_tiles; }
     r.p0 = pt * BMT;
     r.p_end = g.p_rows;
+    r.p_out = r.p0;
     r.q0 = qt * BN;
     r.q_end = g.q_rows;
     r.q_load = r.q0;
@@ -122,7 +138,7 @@ __device__ __forceinline__ void store_row_chunk(const GemmParams& g, int p, int 
     for (int j = 0; j < 8; ++j) {
       float g0 = __uint_as_float(r[2 * j]), g1 = __uint_as_float(r[2 * j + 1]);
       float u0 = __uint_as_float(r[16 + 2 * j]), u1 = __uint_as_float(r[16 + 2 * j + 1]);
-      o[j] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
+      o[j] = pack_op_x2(g.f16, silu_f(g0) * u0, silu_f(g1) * u1);
     }
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(g.out) + (long long)p * g.ldo + (q >> 1));
     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -218,7 +234,7 @@ __device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int 
       float a = __uint_as_float(r[j]);
       float u = __shfl_down_sync(0xffffffffu, a, 16);
       if (lane < 16 && p_valid && q + j < q_end)
-        static_cast<uint16_t*>(g.out)[(long long)(q + j) * g.ldo + f] = to_bf16_bits(silu_f(a) * u);
+        static_cast<uint16_t*>(g.out)[(long long)(q + j) * g.ldo + f] = to_op_bits(g.f16, silu_f(a) * u);
     }
     return;
   }
@@ -416,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int i = 0; i < g.n_groups; ++i) {
         s_prefix[i] = acc;
         const int m = s_off[i + 1] - s_off[i];
-        acc += ((m + BM - 1) / BM) * g.q_tiles;
+        acc += g.swap ? ((m + BN - 1) / BN) * g.p_tiles : ((m + BM - 1) / BM) * g.q_tiles;
       }
       s_prefix[g.n_groups] = acc;
     }
@@ -480,7 +496,7 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0 && (!PAIR || rank == 0)) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16_f32(BMT, BN);
+      const uint32_t idesc = g.f16 ? idesc_f16_f32(BMT, BN) : idesc_bf16_f32(BMT, BN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -609,8 +625,9 @@ __global__ void __launch_bounds__(192, 1)
           const int p = tl.p0 + row, q = tl.q0 + c * 32;
           if (p < tl.p_end && q < tl.q_end) store_row_chunk(g, p, q, r);
         } else {
-          const int p = tl.p0 + row;
-          store_col_chunk(g, p, p < tl.p_end, tl.q0 + c * 32, tl.q_end, lane, tl.p0 + quad * 32, r);
+          // feature p_out + row of the output; grouped: the group's weight row p0 + row
+          store_col_chunk(g, tl.p_out + row, tl.p0 + row < tl.p_end, tl.q0 + c * 32, tl.q_end, lane,
+                          tl.p_out + quad * 32, r);
         }
       }
       }
@@ -636,7 +653,7 @@ __global__ void __launch_bounds__(192, 1)
 // SwiGLU reads the packed gate column (n/16)*32 + n%16 and the up column 16 after it.
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int M, int N, int epi, int resid_f32,
                                      int out_f32, const void* __restrict__ resid, long long ldr,
-                                     void* __restrict__ out, long long ldo) {
+                                     void* __restrict__ out, long long ldo, int f16) {
   pdl_wait();
   pdl_trigger();
   const int n_out = epi == kEpiSwiglu ? N / 2 : N;
@@ -651,7 +668,7 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ part, int S, int 
       gsum += part[s * plane + (long long)m * N + pg];
       usum += part[s * plane + (long long)m * N + pg + 16];
     }
-    static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_bf16_bits(silu_f(gsum) * usum);
+    static_cast<uint16_t*>(out)[(long long)m * ldo + n] = to_op_bits(f16 != 0, silu_f(gsum) * usum);
     return;
   }
   float acc = 0.f;
@@ -738,7 +755,7 @@ __global__ void __launch_bounds__(1024) splitk_resid_norm_kernel(const float* __
                                                                  const void* __restrict__ resid, long long ldr,
                                                                  void* __restrict__ out, long long ldo,
                                                                  const uint16_t* __restrict__ w,
-                                                                 uint16_t* __restrict__ norm_out, float eps) {
+                                                                 uint16_t* __restrict__ norm_out, float eps, int f16) {
   pdl_wait();
   pdl_trigger();
   __shared__ float s_red[32];
@@ -783,7 +800,7 @@ __global__ void __launch_bounds__(1024) splitk_resid_norm_kernel(const float* __
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int n = i * 1024 + threadIdx.x;
-    norm_out[(long long)m * ldo + n] = to_bf16_bits(v[i] * r * bf16_lo((uint32_t)w[n]));
+    norm_out[(long long)m * ldo + n] = to_op_bits(f16 != 0, v[i] * r * bf16_lo((uint32_t)w[n]));
   }
 }
 
@@ -884,13 +901,15 @@ template <int BN>
 static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   using C = GemmCfg<BN>;
   CUtensorMap tmP, tmQ;
-  if (make_tmap_2d(&tmP, d.P, d.p_rows, d.K, d.ldp, BM) != 0) {
+  // grouped: the weight operand holds every group's rows (P when swapped, else Q)
+  const long long p_total = d.n_groups > 0 && d.swap ? d.p_rows_total : d.p_rows;
+  if (make_tmap_2d(&tmP, d.P, p_total, d.K, d.ldp, BM) != 0) {
     set_last_error("gemm: cannot encode the tensor map of operand P");
     return -6;
   }
   // Large plain GEMMs run on CTA pairs (M = 256 MMAs; each CTA loads half of B)
   const bool pair = BN == 256 && !d.swap && d.n_groups == 0 && d.p_rows >= 2 * BM && gemm_pair_enabled();
-  const long long q_total = d.n_groups > 0 ? d.q_rows_total : d.q_rows;
+  const long long q_total = d.n_groups > 0 && !d.swap ? d.q_rows_total : d.q_rows;
   if (make_tmap_2d(&tmQ, d.Q, q_total, d.K, d.ldq, pair ? BN / 2 : BN) != 0) {
     set_last_error("gemm: cannot encode the tensor map of operand Q");
     return -6;
@@ -916,6 +935,7 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
   g.group_offsets = d.group_offsets;
   g.err = err;
   g.qk = d.qk;
+  g.f16 = d.f16 ? 1 : 0;
   g.k_splits = 1;
   g.kb_per_split = g.k_blocks;
   g.partial = nullptr;
@@ -965,15 +985,15 @@ static int launch_bn(const GemmDesc& d, cudaStream_t s, int* err) {
       if (N == 1024)
         q3_launch(splitk_resid_norm_kernel<1>, (unsigned)M, 1024, 0, s, g.partial, g.k_splits, M, N,
                   d.resid_f32 ? 1 : 0, d.out_f32 ? 1 : 0, d.resid, d.ldr, d.out, d.ldo, d.norm_w, d.norm_out,
-                  d.norm_eps);
+                  d.norm_eps, g.f16);
       else
         q3_launch(splitk_resid_norm_kernel<2>, (unsigned)M, 1024, 0, s, g.partial, g.k_splits, M, N,
                   d.resid_f32 ? 1 : 0, d.out_f32 ? 1 : 0, d.resid, d.ldr, d.out, d.ldo, d.norm_w, d.norm_out,
-                  d.norm_eps);
+                  d.norm_eps, g.f16);
       if (d.fused) *d.fused = 1;
     } else {
       q3_launch(splitk_reduce_kernel, (unsigned)((n_out + 255) / 256), 256, 0, s, g.partial, g.k_splits, M, N,
-                d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo);
+                d.epi, d.resid_f32, d.out_f32, d.resid, d.ldr, d.out, d.ldo, g.f16);
     }
   }
   cudaError_t e = cudaGetLastError();

@@ -23,12 +23,20 @@ struct QKRopeArgs {
   uint16_t* ck = nullptr;         // [B][Hkv][s_max][128]
   uint16_t* cv = nullptr;
   float eps = 1e-6f;
+  // decode-sized QKV only (optional): the q heads go to q2 [tokens][ldq2] instead of the
+  // output, split as q_hi = bf16(q) and q_lo = bf16(q - q_hi): for KV group g the G hi
+  // rows, then the G lo rows (the decode attention's hi/lo layout)
+  uint16_t* q2 = nullptr;
+  long long ldq2 = 0;
 };
 
 // D[p][q] = sum_k P[p][k] * Q[q][k]; both operands bf16, K-major (row-major [rows, K]).
 // Non-swap: P = activations [M, K], Q = weights [N, K]; out[p][q].
 // Swap:     P = weights [N, K], Q = activations [M, K]; out[q][p]  (for small M).
-// Grouped (non-swap only): P rows [off[g], off[g+1]) use Q rows g*q_rows_per_group + [0, q_rows_per_group).
+// Grouped, non-swap: P rows [off[g], off[g+1]) use Q rows g*q_rows_per_group + [0, q_rows_per_group).
+// Grouped, swap (few activation rows per group): P = weights, group g's rows
+// [g*p_rows, (g+1)*p_rows) (p_rows_total = n_groups * p_rows); Q = activations, group g's rows
+// [off[g], off[g+1]) of q_rows; out[q][p - g*p_rows].
 struct GemmDesc {
   const void* P = nullptr;
   int p_rows = 0;
@@ -36,7 +44,8 @@ struct GemmDesc {
   const void* Q = nullptr;
   int q_rows = 0;     // non-grouped: rows of Q; grouped: rows per group
   long long ldq = 0;
-  long long q_rows_total = 0;  // rows of the Q tensor map (grouped: n_groups * q_rows)
+  long long q_rows_total = 0;  // rows of the Q tensor map (grouped non-swap: n_groups * q_rows)
+  long long p_rows_total = 0;  // rows of the P tensor map (grouped swap: n_groups * p_rows)
   int K = 0;
   bool swap = false;
   int epi = kEpiStore;
@@ -48,6 +57,9 @@ struct GemmDesc {
   int n_groups = 0;
   const int* group_offsets = nullptr;  // device, n_groups + 1 entries
   int force_bn = 0;                    // 0 = automatic
+  // operands fp16 (else bf16); the SwiGLU output and the fused RMSNorm output (norm_out),
+  // which feed the next projection, then hold fp16 as well
+  bool f16 = false;
   // P is final before the kernel launched just before this GEMM on the stream started
   // (a weight matrix, when a library kernel of the same call precedes the GEMM; every
   // library kernel waits for its predecessor before it lets its dependents launch):
@@ -68,6 +80,38 @@ struct GemmDesc {
   float norm_eps = 1e-6f;
   int* fused = nullptr;
 };
+
+// Decode-sized projection (M <= 64 tokens, N % 128 == 0, K % 64 == 0): out[t][n] =
+// epilogue(sum_k A[t][k] W[n][k]) with K split over the CTAs of a cluster and summed
+// in-kernel (gemm_skinny.cu). Epilogues: kEpiStore, kEpiResid (optionally followed by
+// norm_out = RMSNorm(out) * norm_w over all N features, computed by the cluster that
+// finishes last; `ticket` is an int that is 0 before the launch and 0 after it),
+// kEpiSwiglu (out [M][N/2]), kEpiQKRope (q heads written back to out, k/v to the cache).
+struct SkinnyDesc {
+  const void* A = nullptr;  // activations [M][K] bf16
+  long long lda = 0;
+  const void* W = nullptr;  // weights [N][K] bf16
+  long long ldw = 0;
+  int M = 0, N = 0, K = 0;
+  int epi = kEpiStore;
+  void* out = nullptr;
+  long long ldo = 0;
+  bool out_f32 = false;
+  const void* resid = nullptr;
+  long long ldr = 0;
+  bool resid_f32 = false;
+  bool w_early = false;  // W is final before the previous kernel started (see GemmDesc::p_early)
+  const uint16_t* norm_w = nullptr;
+  uint16_t* norm_out = nullptr;
+  long long ld_norm = 0;
+  float norm_eps = 1e-6f;
+  int* ticket = nullptr;
+  QKRopeArgs qk;
+  bool f16 = false;  // as GemmDesc::f16
+};
+
+bool skinny_supported(int M, int N, int K, int epi);
+int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err);
 
 // Scratch the block calls reserve for split-K partials of small-M GEMMs.
 constexpr size_t kSplitKBytes = (size_t)2 * 148 * 128 * 256 * sizeof(float);

@@ -68,6 +68,8 @@ class Layer:
     library's packed layouts (GPU)."""
 
     def __init__(self, cfg, seed, layer=0, moe=False, dense=True):
+        """With cfg.gemm_f16 set, the linear weights are converted to fp16 after packing
+        (exact for these weights' magnitudes), the layout the fp16 operand mode reads."""
         import torch
         import qwen3_decoder_block_b200 as q3
         H, D, hq, hkv, I = cfg.hidden, cfg.head_dim, cfg.n_q_heads, cfg.n_kv_heads, cfg.intermediate
@@ -106,6 +108,14 @@ class Layer:
             self.moe_gate_up = torch.empty((E, 2 * Im, H), dtype=torch.bfloat16, device="cuda")
             q3.pack_moe_gate_up(E, Im, H, self.gate_up.gpu, self.moe_gate_up)
             kw.update(router=self.router.gpu, moe_gate_up=self.moe_gate_up, moe_down=self.down.gpu)
+        if cfg.gemm_f16:
+            self.f16 = {}
+            for name in ("w_qkv", "w_o", "w_gate_up", "w_down", "router", "moe_gate_up", "moe_down"):
+                if name in kw:
+                    self.f16[name] = q3.convert_to_f16(kw[name], torch.empty(kw[name].shape, dtype=torch.float16,
+                                                                              device="cuda"))
+            kw.update(self.f16)
+            torch.cuda.synchronize()
         self.c = q3.layer_weights(**kw)
 
     def oracle(self) -> "R.LayerWeights":
@@ -132,6 +142,13 @@ def workspace(cfg, op, B, T, s_max):
     n = q3.workspace_size(cfg, op, B, T, s_max)
     assert n > 0
     return torch.empty(n, dtype=torch.uint8, device="cuda")
+
+
+def to_f16(t):
+    """An fp16 copy of a bf16 GPU tensor made by the library's conversion."""
+    import torch
+    import qwen3_decoder_block_b200 as q3
+    return q3.convert_to_f16(t, torch.empty(t.shape, dtype=torch.float16, device="cuda"))
 
 
 def kv_cache(cfg, B, s_max, fill=None):

@@ -59,7 +59,8 @@ def test_default_config_is_qwen3_0_6b(q3):
 
 @pytest.mark.parametrize("field,value,status", [
     ("head_dim", 64, -2), ("n_kv_heads", 3, -2), ("hidden", 1000, -2), ("hidden", 4096, -2),
-    ("intermediate", 3000, -2), ("vocab", 151937, -2), ("n_q_heads", 0, -2)])
+    ("intermediate", 3000, -2), ("vocab", 151937, -2), ("n_q_heads", 0, -2), ("gemm_f16", 2, -2),
+    ("gemm_f16", -1, -2)])
 def test_validate_config_rejects(q3, field, value, status):
     c = q3.config_qwen3_0_6b()
     setattr(c, field, value)
@@ -111,11 +112,11 @@ def test_null_and_misaligned_arguments_rejected_without_launch(q3):
                                     None, 0, None)
     assert st == q3.EINVAL
     assert "NULL" in q3.lib.qwen3_last_error().decode()
-    st = q3.lib.qwen3_op_gemm(8, 1024, 16, 1024, 32, 1024, 16, 1024, 1024, 0, None, 0, 0, 0, -1, None, 0, None)
+    st = q3.lib.qwen3_op_gemm(8, 1024, 16, 1024, 32, 1024, 16, 1024, 1024, 0, None, 0, 0, 0, -1, 0, None, 0, None)
     assert st == q3.EALIGN
-    st = q3.lib.qwen3_op_gemm(16, 1024, 32, 1024, 48, 1024, 16, 1000, 1024, 0, None, 0, 0, 0, -1, None, 0, None)
+    st = q3.lib.qwen3_op_gemm(16, 1024, 32, 1024, 48, 1024, 16, 1000, 1024, 0, None, 0, 0, 0, -1, 0, None, 0, None)
     assert st == q3.ESHAPE  # N % 32
-    st = q3.lib.qwen3_op_rmsnorm(16, 0, 1000, 32, 48, 1000, 4, 1000, 1e-6, None)
+    st = q3.lib.qwen3_op_rmsnorm(16, 0, 1000, 32, 48, 1000, 4, 1000, 1e-6, 0, None)
     assert st == q3.ESHAPE
 
 
@@ -304,3 +305,20 @@ def test_decode_attention_rejects_bad_output_stride_before_launch(q3, ldo):
     st = q3.lib.qwen3_op_attention_decode_noalloc(ctypes.byref(c), fake, 4096, 64, fake, ctypes.byref(kv), fake, ldo,
                                                   None)
     assert st == q3.EALIGN and "ldo" in q3.lib.qwen3_last_error().decode(), st
+
+
+def test_operand_mode_arguments_checked_before_launch(q3):
+    """The gemm_f16 mode's host-side checks: the default configuration keeps the pages'
+    bf16 operands; op_gemm takes ab_f16 0 or 1 only; the conversion refuses partly
+    overlapping buffers (in place is allowed) and runs nothing on bad arguments."""
+    c = q3.config_qwen3_0_6b()
+    assert c.gemm_f16 == 0
+    c.gemm_f16 = 1
+    assert q3.validate_config(c) == 0
+    st = q3.lib.qwen3_op_gemm(16, 1024, 32, 1024, 48, 1024, 16, 1024, 1024, 0, None, 0, 0, 0, -1, 2, None, 0, None)
+    assert st == q3.EINVAL and "ab_f16" in q3.lib.qwen3_last_error().decode()
+    base = 1 << 40
+    assert q3.lib.qwen3_convert_to_f16(base, base + 16, 1024, None) == q3.EINVAL
+    assert "overlap" in q3.lib.qwen3_last_error().decode()
+    assert q3.lib.qwen3_convert_to_f16(base, base + 8, 4, None) == q3.EALIGN
+    assert q3.lib.qwen3_convert_to_f16(None, base, 4, None) == q3.EINVAL

@@ -9,7 +9,7 @@ import oracle.qwen3_ref as R  # noqa: E402
 import qwen3_synth as synth  # noqa: E402
 from helpers import (LAYER_MAX_ABS, LAYER_REL_FROB, LOGITS_ARGMAX, LOGITS_REL_FROB, Layer, Tensor,  # noqa: E402
                      assert_device_ok, from_gpu_bf16, kv_cache, max_abs, oracle_config, rel_frob, rope_gpu,
-                     to_gpu_bf16, workspace)
+                     to_f16, to_gpu_bf16, workspace)
 
 
 @pytest.fixture(scope="module")
@@ -46,10 +46,12 @@ def _prefill_case(q3, cfg, B, T, starts, seed, s_extra=13):
     return from_gpu_bf16(xg), np.concatenate(refs), k, v, kref
 
 
-@pytest.mark.parametrize("B,T,starts", [(1, 16, [0]), (2, 77, [0, 50]), (1, 300, [0]), (3, 5, [0, 1, 200]),
-                                        (2, 200, [0, 37]), (3, 130, [0, 5, 900])])
-def test_block_prefill(q3, B, T, starts):
-    cfg = q3.config_qwen3_0_6b()
+@pytest.mark.parametrize("B,T,starts,f16", [(1, 16, [0], 0), (2, 77, [0, 50], 0), (1, 300, [0], 0),
+                                            (3, 5, [0, 1, 200], 0), (2, 200, [0, 37], 0), (3, 130, [0, 5, 900], 0),
+                                            (1, 16, [0], 1), (3, 5, [0, 1, 200], 1), (2, 200, [0, 37], 1)])
+def test_block_prefill(q3, B, T, starts, f16):
+    """f16 = 1: the fp16 operand mode (fp16 weights and projection inputs)."""
+    cfg = q3.make_config(gemm_f16=f16)
     got, ref, k, v, kref = _prefill_case(q3, cfg, B, T, starts, seed=1000)
     assert np.isfinite(got).all()
     assert rel_frob(got, ref) <= LAYER_REL_FROB and max_abs(got, ref) <= LAYER_MAX_ABS, (rel_frob(got, ref),
@@ -60,8 +62,9 @@ def test_block_prefill(q3, B, T, starts):
         assert rel_frob(gk, kref[b][0]) <= 1e-2
 
 
-def test_block_decode(q3):
-    cfg = q3.config_qwen3_0_6b()
+@pytest.mark.parametrize("f16", [0, 1])
+def test_block_decode(q3, f16):
+    cfg = q3.make_config(gemm_f16=f16)
     lens = [0, 5, 130, 1000]
     B = len(lens)
     s_max = 1100
@@ -90,18 +93,21 @@ def test_block_decode(q3):
     assert list(cl.cpu().numpy()) == lens  # block_decode does not advance lengths
 
 
-def _small_stack_cfg(q3, n_layers=3):
-    return q3.make_config(hidden=256, n_q_heads=4, n_kv_heads=2, intermediate=512, vocab=2048, n_layers=n_layers)
+def _small_stack_cfg(q3, n_layers=3, f16=0):
+    return q3.make_config(hidden=256, n_q_heads=4, n_kv_heads=2, intermediate=512, vocab=2048, n_layers=n_layers,
+                          gemm_f16=f16)
 
 
-def test_stack_prefill_then_decode(q3):
-    cfg = _small_stack_cfg(q3)
+@pytest.mark.parametrize("f16", [0, 1])
+def test_stack_prefill_then_decode(q3, f16):
+    cfg = _small_stack_cfg(q3, f16=f16)
     seed = 1003
     B, T = 2, 40
     s_max = T + 8
     layers = [Layer(cfg, seed, layer=l) for l in range(cfg.n_layers)]
     E = Tensor(seed, synth.TID_EMBED, (cfg.vocab, cfg.hidden), 0.0, synth.W_STD)
     fn = Tensor(seed, synth.TID_FINAL_NORM, (cfg.hidden,), synth.NORM_MEAN, synth.NORM_STD)
+    Eg = to_f16(E.gpu) if f16 else E.gpu  # the tied embedding holds the operand type
     ids = synth.uniform_int(seed, synth.TID_IDS, (B, T + 1), cfg.vocab)
     caches = [kv_cache(cfg, B, s_max) for _ in range(cfg.n_layers)]
     rope = rope_gpu(cfg)
@@ -109,7 +115,7 @@ def test_stack_prefill_then_decode(q3):
     logits = torch.empty((B * T, cfg.vocab), dtype=torch.float32, device="cuda")
     ids_pre = torch.from_numpy(np.ascontiguousarray(ids[:, :T]).reshape(-1)).cuda()
     pos = torch.zeros(B, dtype=torch.int32, device="cuda")
-    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
+    q3.stack_forward(cfg, Eg, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
                      [c[2] for c in caches], rope, logits, False, ws)
     assert_device_ok()
     oc = oracle_config(cfg)
@@ -133,7 +139,7 @@ def test_stack_prefill_then_decode(q3):
     lens = torch.full((B,), T, dtype=torch.int32, device="cuda")
     ld = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
     ids_dec = torch.from_numpy(np.ascontiguousarray(ids[:, T])).cuda()
-    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_dec, B, 1, q3.MODE_DECODE, lens,
+    q3.stack_forward(cfg, Eg, [l.c for l in layers], fn.gpu, ids_dec, B, 1, q3.MODE_DECODE, lens,
                      [c[2] for c in caches], rope, ld, False, wsd)
     assert_device_ok()
     assert list(lens.cpu().numpy()) == [T + 1] * B
@@ -145,14 +151,16 @@ def test_stack_prefill_then_decode(q3):
     ws2 = workspace(cfg, q3.OP_STACK_PREFILL, B, T, s_max)
     caches2 = [kv_cache(cfg, B, s_max) for _ in range(cfg.n_layers)]
     ll = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
-    q3.stack_forward(cfg, E.gpu, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
+    q3.stack_forward(cfg, Eg, [l.c for l in layers], fn.gpu, ids_pre, B, T, q3.MODE_PREFILL, pos,
                      [c[2] for c in caches2], rope, ll, True, ws2)
     assert_device_ok()
     np.testing.assert_array_equal(ll.cpu().numpy(), logits.view(B, T, -1)[:, -1].cpu().numpy())
 
 
-def test_moe_block_small(q3):
-    cfg = q3.make_config(hidden=512, n_q_heads=8, n_kv_heads=2, n_experts=32, top_k=4, moe_intermediate=128)
+@pytest.mark.parametrize("f16", [0, 1])
+def test_moe_block_small(q3, f16):
+    cfg = q3.make_config(hidden=512, n_q_heads=8, n_kv_heads=2, n_experts=32, top_k=4, moe_intermediate=128,
+                         gemm_f16=f16)
     seed = 1004
     B, T = 1, 100
     s_max = T

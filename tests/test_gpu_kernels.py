@@ -7,7 +7,7 @@ pytestmark = pytest.mark.gpu
 
 import oracle.qwen3_ref as R  # noqa: E402
 from helpers import (Tensor, assert_device_ok, from_gpu_bf16, kv_cache, max_abs, oracle_config, rel_frob,  # noqa: E402
-                     rope_gpu, workspace)
+                     rope_gpu, to_f16, workspace)
 
 SEED = 7
 
@@ -20,6 +20,16 @@ def q3():
 
 def bf16_tol(ref, rel=2.0 ** -8, abs_=1e-6):
     return rel * np.abs(ref) + abs_
+
+
+def f16_tol(ref, abs_=1e-6):
+    """One rounding to fp16 (relative 2^-11) on top of fp32 accumulation."""
+    return 2.0 ** -11 * np.abs(ref) + abs_
+
+
+def f64_of(t):
+    """float64 numpy copy of a bf16 / fp16 / fp32 GPU tensor (exact widening)."""
+    return t.detach().cpu().double().numpy()
 
 
 @pytest.mark.parametrize("n", [1024, 2048])
@@ -310,3 +320,114 @@ def test_synth_device_matches_host(q3):
     np.testing.assert_array_equal(got, host)
     assert bool((buf[:, n1:] == 0).all())
     np.testing.assert_array_equal(ids.cpu().numpy(), synth.uniform_int(11, 13, (5000,), 151936))
+
+
+def test_convert_to_f16_rounds_like_torch(q3):
+    """bf16 -> fp16 by the library equals torch's round-to-nearest-even conversion, in
+    place and out of place, on normal, subnormal, overflowing and odd-length inputs."""
+    x = Tensor(SEED, 91, (3001,)).gpu * 0.02
+    x[:8] = torch.tensor([0.0, -0.0, 1e-7, -3e-6, 6.1e-5, 70000.0, -1e9, 2.0 ** -24], dtype=torch.bfloat16)
+    ref = x.float().half()
+    out = q3.convert_to_f16(x, torch.empty(x.shape, dtype=torch.float16, device="cuda"))
+    y = x.clone()
+    inplace = q3.convert_to_f16(y)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(inplace.view(torch.int16), ref.view(torch.int16))
+    # bf16 values with |v| in [2^-17, 65504] are kept exactly
+    keep = (x.float().abs() >= 2.0 ** -17) & (x.float().abs() <= 65504)
+    assert torch.equal(out.float()[keep], x.float()[keep])
+
+
+@pytest.mark.parametrize("rows", [1, 37, 1000])
+def test_rmsnorm_f16_output(q3, rows):
+    n = 1024
+    x = Tensor(SEED, 11, (rows, n))
+    w = Tensor(SEED, 12, (n,), 1.0, 0.1)
+    out = torch.empty((rows, n), dtype=torch.float16, device="cuda")
+    q3.op_rmsnorm(x.gpu.float(), w.gpu, out, rows, n, 1e-6)
+    assert_device_ok()
+    ref = R.rms_norm(x.f, w.f, 1e-6)
+    assert np.all(np.abs(f64_of(out) - ref) <= f16_tol(ref, abs_=1e-5))
+
+
+@pytest.mark.parametrize("M,N,K,epi,swap", [(16, 4096, 1024, 0, 2), (64, 1024, 2048, 1, 2), (64, 6144, 1024, 2, 2),
+                                            (5, 1024, 3072, 1, 2), (200, 512, 192, 0, 1), (300, 6144, 1024, 2, 0),
+                                            (1000, 1024, 3072, 1, 0), (600, 2048, 1024, 0, 0)])
+def test_gemm_f16_operands(q3, M, N, K, epi, swap):
+    """fp16 A and W (the gemm_f16 mode): the MMA's operand type switches, results within
+    one rounding of the output (fp32 outputs: accumulation order only)."""
+    A = Tensor(SEED, 51, (M, K))
+    W = Tensor(SEED, 52, (N, K), 0.0, 0.02)
+    X = Tensor(SEED, 53, (M, N))
+    Wp = W.gpu
+    if epi == 2:
+        Wp = torch.empty_like(W.gpu)
+        q3.pack_gate_up(N // 2, K, W.gpu[:N // 2], W.gpu[N // 2:], Wp)
+    A16, W16 = to_f16(A.gpu), to_f16(Wp)
+    torch.cuda.synchronize()
+    a, w = f64_of(A16), f64_of(to_f16(W.gpu))
+    acc = a @ w.T
+    if epi == 2:
+        out = torch.empty((M, N // 2), dtype=torch.float16, device="cuda")
+        q3.op_gemm(A16, W16, out, M, N, K, epilogue=2, swap=swap)
+        ref = R.silu(acc[:, :N // 2]) * acc[:, N // 2:]
+        assert_device_ok()
+        assert np.all(np.abs(f64_of(out) - ref) <= f16_tol(ref, abs_=2e-4)), max_abs(f64_of(out), ref)
+        return
+    out = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    resid = X.gpu.float() if epi == 1 else None
+    q3.op_gemm(A16, W16, out, M, N, K, epilogue=epi, resid=resid, swap=swap)
+    assert_device_ok()
+    ref = acc + (X.f if epi == 1 else 0.0)
+    assert max_abs(f64_of(out), ref) <= 2e-5 * np.sqrt(K / 1024) * 8, max_abs(f64_of(out), ref)
+
+
+@pytest.mark.parametrize("M", [1, 3, 16, 37, 64])
+@pytest.mark.parametrize("N,K,epi", [(4096, 1024, 0), (1024, 2048, 1), (6144, 1024, 2), (1024, 3072, 1), (128, 64, 0),
+                                     (2048, 4096, 1)])
+def test_gemm_cluster_split_k(q3, M, N, K, epi):
+    """The decode-sized form (swap = 2): K split over the CTAs of a cluster and summed in
+    shared memory across the cluster, in split order, with the epilogue in the same
+    kernel; ragged token counts and a single K block."""
+    A = Tensor(SEED, 61, (M, K))
+    W = Tensor(SEED, 62, (N, K), 0.0, 0.02)
+    X = Tensor(SEED, 63, (M, N))
+    packed = W.gpu
+    if epi == 2:
+        packed = torch.empty_like(W.gpu)
+        q3.pack_gate_up(N // 2, K, W.gpu[:N // 2], W.gpu[N // 2:], packed)
+    acc = A.f @ W.f.T
+    if epi == 2:
+        out = torch.empty((M, N // 2), dtype=torch.bfloat16, device="cuda")
+        q3.op_gemm(A.gpu, packed, out, M, N, K, epilogue=2, swap=2)
+        assert_device_ok()
+        ref = R.silu(acc[:, :N // 2]) * acc[:, N // 2:]
+        assert np.all(np.abs(from_gpu_bf16(out) - ref) <= bf16_tol(ref, abs_=2e-4))
+        return
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out = torch.full((M, N), float("nan"), dtype=out_dtype, device="cuda")
+        resid = X.gpu if epi == 1 else None
+        q3.op_gemm(A.gpu, packed, out, M, N, K, epilogue=epi, resid=resid, swap=2)
+        assert_device_ok()
+        ref = acc + (X.f if epi == 1 else 0.0)
+        got = f64_of(out)
+        tol = 1e-4 if out_dtype == torch.float32 else bf16_tol(ref, abs_=1e-4)
+        assert np.all(np.abs(got - ref) <= tol), (out_dtype, max_abs(got, ref))
+    # deterministic: the same call twice gives the same bits
+    again = torch.empty_like(out)
+    q3.op_gemm(A.gpu, packed, again, M, N, K, epilogue=epi, resid=resid, swap=2)
+    torch.cuda.synchronize()
+    assert torch.equal(again.view(torch.int16), out.view(torch.int16))
+
+
+def test_embed_f16_table(q3):
+    V, H, n = 4096, 1024, 77
+    E = Tensor(SEED, 81, (V, H), 0.0, 0.02)
+    E16 = to_f16(E.gpu)
+    ids_np = np.random.default_rng(5).integers(0, V, n).astype(np.int32)
+    ids = torch.from_numpy(ids_np).cuda()
+    out = torch.empty((n, H), dtype=torch.float32, device="cuda")
+    q3.op_embed(ids, n, E16, V, H, out)
+    assert_device_ok()
+    np.testing.assert_array_equal(out.cpu().double().numpy(), f64_of(E16)[ids_np])
