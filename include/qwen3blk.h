@@ -283,7 +283,10 @@ int qwen3_op_rmsnorm(const void* x, int x_f32, long long ldx, const qwen3_bf16* 
  *   out_f32 / resid_f32 select fp32 (else bf16). swap: 1 = weight rows on the MMA's 128-row
  *   side (small M), 0 = activations there, 2 = weight rows on the 128-row side with K split
  *   over the CTAs of a thread-block cluster and summed in the same kernel (M <= 64,
- *   N % 128 == 0; ws unused), -1 = automatic (2 when it applies, else 1 when M <= 256).
+ *   N % 128 == 0; ws unused), 3 = as 2 with A holding 2M rows: row t = hi(a_t) and row M + t
+ *   = lo(a_t) = a_t - hi(a_t) rounded to the operand type, the product taken on hi + lo
+ *   (about twice the operand type's significant bits; the decode path's operand form),
+ *   -1 = automatic (2 when it applies, else 1 when M <= 256).
  *   ws (may be NULL): scratch for split-K when the output has too few tiles to fill the GPU;
  *   it holds fp32 partials, up to ws_bytes (split count = largest that fits).
  *   ab_f16: A and W hold fp16 (1) or bf16 (0); the SwiGLU output takes the same type.

@@ -21,7 +21,8 @@
 namespace q3 {
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
-                   int rows, int n, float eps, cudaStream_t s, int* zero_word = nullptr, bool out_f16 = false);
+                   int rows, int n, float eps, cudaStream_t s, int* zero_word = nullptr, bool out_f16 = false,
+                   long long out_lo = 0);
 int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv, const int* pos_base,
                         const uint16_t* qw, const uint16_t* kw, const float* rope, uint16_t* ck, uint16_t* cv,
                         int s_max, int max_pos, float eps, int* err, cudaStream_t s);
@@ -39,7 +40,8 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
                              long long ldo, int* err, cudaStream_t s, bool o_f16 = false);
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
                             const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
-                            long long ldo, int* err, cudaStream_t s, bool o_f16 = false, bool q_hilo = false);
+                            long long ldo, int* err, cudaStream_t s, bool o_f16 = false, bool q_hilo = false,
+                            long long o_lo = 0);
 size_t decode_partial_bytes(int B, int Hq, int s_max);
 int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
                                    const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
@@ -272,9 +274,11 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
   const long long M = (long long)B * (decode ? 1 : T);
   const int D = c.head_dim, H = c.hidden;
   const long long nqkv = (long long)(c.n_q_heads + 2 * c.n_kv_heads) * D;
-  b.h = cv.take<uint16_t>(M * H);
+  // decode-sized calls carry projection inputs as hi/lo rows: twice the rows
+  const long long Mh = M <= 64 ? 2 * M : M;
+  b.h = cv.take<uint16_t>(Mh * H);
   b.qkv = cv.take<uint16_t>(M * nqkv);
-  b.o = cv.take<uint16_t>(M * c.n_q_heads * D);
+  b.o = cv.take<uint16_t>(Mh * c.n_q_heads * D);
   b.x1 = cv.take<float>(M * H);
   // one new token per sequence (decode, or a prefill of T = 1) runs the split-KV decode attention
   if (decode || T == 1) {
@@ -296,7 +300,7 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
     b.act_perm = cv.take<uint16_t>(M * k * c.moe_intermediate);
     b.y = cv.take<uint16_t>(M * k * H);
   } else {
-    b.act = cv.take<uint16_t>(M * c.intermediate);
+    b.act = cv.take<uint16_t>(Mh * c.intermediate);
   }
   if (op == QWEN3_OP_STACK_PREFILL || op == QWEN3_OP_STACK_DECODE) {
     b.xs = cv.take<float>(M * H);
@@ -330,10 +334,16 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   // one token per sequence at position pos[b], attending 0..pos[b]: the decode attention
   // computes exactly that, for a prefill of T = 1 as well
   decode = decode || T == 1;
+  // decode-sized (at most 64 tokens): every projection is one cluster split-K launch, and
+  // its activation operand is carried as hi/lo halves (2M rows: the weight stream bounds
+  // these GEMMs, so the doubled N costs nothing measurable)
+  const bool skinny = skinny_supported((int)M, nqkv, H, kEpiQKRope) &&
+                      skinny_supported((int)M, H, c.n_q_heads * D, kEpiResid);
   int rc = 0;
   if (!h_ready) {
     ProfScope ps("rmsnorm", k.s);
-    rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s, b.ticket, f16);
+    rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s, b.ticket, f16,
+                        skinny ? M * H : 0);
   }
   if (rc) return rc;
   QKRopeArgs qa;
@@ -349,13 +359,11 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   qa.ck = kv.k;
   qa.cv = kv.v;
   qa.eps = c.rms_eps;
-  const bool skinny = skinny_supported((int)M, nqkv, H, kEpiQKRope) &&
-                      skinny_supported((int)M, H, c.n_q_heads * D, kEpiResid);
   if (skinny) {
-    // decode-sized: K split over clusters and summed in-kernel, each projection one launch
     SkinnyDesc q;
     q.A = b.h; q.lda = H; q.W = w.w_qkv; q.ldw = H;
     q.M = (int)M; q.N = nqkv; q.K = H;
+    q.a_hilo = true;  // b.h: M hi rows, then M lo rows
     q.epi = kEpiQKRope;
     q.out = b.qkv; q.ldo = nqkv;
     q.w_early = true;  // weights; a library kernel of this call runs before this GEMM
@@ -377,7 +385,8 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
       if (decode)
         rc = launch_attention_decode(hilo ? b.q2 : b.qkv, hilo ? 2LL * c.n_q_heads * D : nqkv, B, c.n_q_heads,
                                      c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part, b.o,
-                                     (long long)c.n_q_heads * D, k.err, k.s, f16, hilo);
+                                     (long long)c.n_q_heads * D, k.err, k.s, f16, hilo,
+                                     M * c.n_q_heads * D);  // o as hi/lo rows for o_proj
       else
         rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
                                       (long long)c.n_q_heads * D, k.err, k.s, f16);
@@ -386,12 +395,14 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     SkinnyDesc o;
     o.A = b.o; o.lda = c.n_q_heads * D; o.W = w.w_o; o.ldw = c.n_q_heads * D;
     o.M = (int)M; o.N = H; o.K = c.n_q_heads * D;
+    o.a_hilo = decode;  // the decode merge writes o as hi/lo rows; the prefill attention does not
     o.epi = kEpiResid;
     o.resid = x; o.resid_f32 = x_f32; o.ldr = H;
     o.out = b.x1; o.out_f32 = true; o.ldo = H;
     o.w_early = true;
-    // the post-attention RMSNorm of x1 goes to b.h in the same launch
+    // the post-attention RMSNorm of x1 goes to b.h (hi/lo rows) in the same launch
     o.norm_w = w.post_norm; o.norm_out = b.h; o.ld_norm = H; o.norm_eps = c.rms_eps; o.ticket = b.ticket;
+    o.norm_lo = M * H;
     o.f16 = f16;
     ProfScope ps("gemm_o", k.s);
     rc = launch_gemm_skinny(o, k.s, k.err);
@@ -488,24 +499,29 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
 // out = x1 + down(silu(gate(norm2(x1))) * up(norm2(x1)))   ([P-Mini] sections SwiGLU FFN, TransformerBlock)
 // h2_ready: b.h already holds norm2(x1). With next_norm set, the down GEMM's split-K
 // completion may also write norm(out) * next_norm into next_out (*next_ready set then).
+// next_hilo: next_out feeds a decode-sized projection (it then also gets the lo rows).
 static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b,
                      bool h2_ready, const uint16_t* next_norm = nullptr, uint16_t* next_out = nullptr,
-                     bool* next_ready = nullptr) {
+                     bool* next_ready = nullptr, bool next_hilo = false) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, I = c.intermediate;
   const bool f16 = c.gemm_f16 != 0;
+  const bool skinny = skinny_supported((int)M, 2 * I, H, kEpiSwiglu) && skinny_supported((int)M, H, I, kEpiResid);
   int rc = 0;
   if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
-    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s, nullptr, f16);
+    rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s, nullptr, f16,
+                        skinny ? M * H : 0);
   }
   if (rc) return rc;
-  if (skinny_supported((int)M, 2 * I, H, kEpiSwiglu) && skinny_supported((int)M, H, I, kEpiResid)) {
+  if (skinny) {
     SkinnyDesc g;
     g.A = b.h; g.lda = H; g.W = w.w_gate_up; g.ldw = H;
     g.M = (int)M; g.N = 2 * I; g.K = H;
+    g.a_hilo = true;  // b.h: hi rows then lo rows
     g.epi = kEpiSwiglu;
     g.out = b.act; g.ldo = I;
+    g.out_lo = M * I;  // act as hi/lo rows for the down projection
     g.w_early = true;  // weights; a library kernel of this call runs before this GEMM
     g.f16 = f16;
     {
@@ -516,6 +532,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
     SkinnyDesc d;
     d.A = b.act; d.lda = I; d.W = w.w_down; d.ldw = I;
     d.M = (int)M; d.N = H; d.K = I;
+    d.a_hilo = true;
     d.epi = kEpiResid;
     d.resid = b.x1; d.resid_f32 = true; d.ldr = H;
     d.out = out; d.out_f32 = out_f32; d.ldo = H;
@@ -523,6 +540,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
     d.f16 = f16;
     if (next_norm && next_out) {
       d.norm_w = next_norm; d.norm_out = next_out; d.ld_norm = H; d.norm_eps = c.rms_eps; d.ticket = b.ticket;
+      d.norm_lo = next_hilo ? M * H : 0;
     }
     ProfScope ps("gemm_down", k.s);
     rc = launch_gemm_skinny(d, k.s, k.err);
@@ -592,6 +610,7 @@ static int moe_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void
     SkinnyDesc r;
     r.A = b.h; r.lda = H; r.W = w.router; r.ldw = H;
     r.M = (int)M; r.N = E; r.K = H;
+    r.a_hilo = h2_ready;  // the decode-sized o_proj left norm2(x1) as hi/lo rows
     r.epi = kEpiStore;
     r.out = b.logits; r.out_f32 = true; r.ldo = E;
     r.w_early = true;  // weights; a library kernel of this call runs before this GEMM
@@ -1056,7 +1075,8 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
       return finish(rc);
     const bool last = l + 1 == c->n_layers;
     const uint16_t* nn = last ? (fuse_final ? final_norm : nullptr) : layers[l + 1].in_norm;
-    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b, h2, nn, last ? b.hf : b.h, &h_ready))) return finish(rc);
+    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b, h2, nn, last ? b.hf : b.h, &h_ready, !last)))
+      return finish(rc);
   }
   // final RMSNorm and tied LM head ([P-Mini] section 骨架; [P-SGL] section 一)
   const int rows = last_only ? B : (int)M;
@@ -1165,16 +1185,17 @@ int qwen3_op_gemm(const qwen3_bf16* A, long long lda, const qwen3_bf16* W, long 
   } else {
     Q3_CHECK(ldo >= N, QWEN3_EINVAL, "gemm: ldo (%lld) < N (%d)", ldo, N);
   }
-  Q3_CHECK(swap >= -1 && swap <= 2, QWEN3_EINVAL, "gemm: swap must be -1, 0, 1 or 2 (got %d)", swap);
-  if (swap == 2)
+  Q3_CHECK(swap >= -1 && swap <= 3, QWEN3_EINVAL, "gemm: swap must be -1, 0, 1, 2 or 3 (got %d)", swap);
+  if (swap >= 2)
     Q3_CHECK(skinny_supported(M, N, K, epilogue), QWEN3_ESHAPE,
              "gemm: the cluster split-K form needs M <= 64 and N %% 128 == 0 (M %d, N %d)", M, N);
   int rc = check_device();
   if (rc) return rc;
-  if (swap == 2 || (swap < 0 && skinny_supported(M, N, K, epilogue))) {
+  if (swap >= 2 || (swap < 0 && skinny_supported(M, N, K, epilogue))) {
     SkinnyDesc d;
     d.A = A; d.lda = lda; d.W = W; d.ldw = ldw;
     d.M = M; d.N = N; d.K = K;
+    d.a_hilo = swap == 3;
     d.epi = epilogue;
     d.out = out; d.ldo = ldo; d.out_f32 = out_f32 != 0;
     d.resid = resid; d.ldr = ldr; d.resid_f32 = resid_f32 != 0;

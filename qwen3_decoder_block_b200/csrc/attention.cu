@@ -763,8 +763,10 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   }
 }
 
+// o_lo > 0: also a lo copy round(o - hi) o_lo elements after each value (the hi/lo
+// operand of the decode-sized o_proj).
 __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
-                                         uint16_t* __restrict__ out, long long ldo, int o_f16) {
+                                         uint16_t* __restrict__ out, long long ldo, int o_f16, long long o_lo) {
   pdl_wait();
   pdl_trigger();
   const int bh = blockIdx.x;  // b * Hq + h
@@ -782,7 +784,11 @@ __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq,
     L += q[kHeadDim + 1] * w;
     acc += q[d] * w;
   }
-  out[(long long)b * ldo + (long long)h * kHeadDim + d] = to_op_bits(o_f16 != 0, acc / L);
+  const float o = acc / L;
+  const uint16_t hi = to_op_bits(o_f16 != 0, o);
+  uint16_t* dst = out + (long long)b * ldo + (long long)h * kHeadDim + d;
+  *dst = hi;
+  if (o_lo) dst[o_lo] = to_op_bits(o_f16 != 0, o - op_bits_to_f32(o_f16 != 0, hi));
 }
 
 int decode_splits(int s_max) { return (s_max + kD4Split - 1) / kD4Split; }
@@ -796,7 +802,7 @@ size_t decode_partial_bytes(int B, int Hq, int s_max) {
 // (G <= 8 only).
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
                             const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
-                            long long ldo, int* err, cudaStream_t s, bool o_f16, bool q_hilo) {
+                            long long ldo, int* err, cudaStream_t s, bool o_f16, bool q_hilo, long long o_lo) {
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) {
@@ -847,7 +853,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     Q3_D4_CASE(8, true)
 #undef Q3_D4_CASE
   }
-  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo, o_f16 ? 1 : 0);
+  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo, o_f16 ? 1 : 0, o_lo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
@@ -903,7 +909,7 @@ int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, 
     ptr = g_static_ptr[dev];
   }
   return launch_attention_decode(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, cv, s_max, ptr, out, ldo, err, s, o_f16,
-                                 false);
+                                 false, 0);
 }
 
 }  // namespace q3

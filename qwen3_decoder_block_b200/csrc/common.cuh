@@ -419,6 +419,9 @@ __device__ __forceinline__ uint32_t pack_op_x2(bool f16, float lo, float hi) {
   return f16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 __device__ __forceinline__ uint16_t to_op_bits(bool f16, float f) { return f16 ? to_f16_bits(f) : to_bf16_bits(f); }
+__device__ __forceinline__ float op_bits_to_f32(bool f16, uint16_t v) {
+  return f16 ? f16_bits_to_f32(v) : __uint_as_float((uint32_t)v << 16);
+}
 
 // z * sigmoid(z) with the exponential and the reciprocal on the special-function unit
 // (a few ulp, far below the bf16 rounding of the outputs that use it).

@@ -36,10 +36,13 @@ __device__ __forceinline__ void rms_load8(const void* x, long long off, float (&
 // zero_word (optional): an int this kernel sets to 0 (the fused-norm ticket of the
 // call's decode-sized projections; see launch_gemm_skinny).
 // OUT_F16: the output feeds an fp16-operand projection (bf16 otherwise).
+// out_lo > 0: a lo copy lo = round(v - hi) of every output value, out_lo elements after it
+// (the hi/lo operand of a decode-sized projection).
 template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
                                                          const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
-                                                         long long ldo, int rows, int n, float eps, int* zero_word) {
+                                                         long long ldo, int rows, int n, float eps, int* zero_word,
+                                                         long long out_lo) {
   pdl_wait();
   pdl_trigger();
   if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
@@ -60,25 +63,32 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
       float v[8];
       rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
       const uint4 wv = *reinterpret_cast<const uint4*>(w + col);
-      uint4 o;
-      o.x = pack_op_x2(OUT_F16, v[0] * r * bf16_lo(wv.x), v[1] * r * bf16_hi(wv.x));
-      o.y = pack_op_x2(OUT_F16, v[2] * r * bf16_lo(wv.y), v[3] * r * bf16_hi(wv.y));
-      o.z = pack_op_x2(OUT_F16, v[4] * r * bf16_lo(wv.z), v[5] * r * bf16_hi(wv.z));
-      o.w = pack_op_x2(OUT_F16, v[6] * r * bf16_lo(wv.w), v[7] * r * bf16_hi(wv.w));
-      *reinterpret_cast<uint4*>(out + (long long)row * ldo + col) = o;
+      const float wf[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
+                           bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a0 = v[2 * j] * r * wf[2 * j], a1 = v[2 * j + 1] * r * wf[2 * j + 1];
+        hi[j] = pack_op_x2(OUT_F16, a0, a1);
+        lo[j] = pack_op_x2(OUT_F16, a0 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] & 0xFFFFu)),
+                           a1 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] >> 16)));
+      }
+      uint16_t* dst = out + (long long)row * ldo + col;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (out_lo) *reinterpret_cast<uint4*>(dst + out_lo) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
   }
 }
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
-                   int rows, int n, float eps, cudaStream_t s, int* zero_word, bool out_f16) {
+                   int rows, int n, float eps, cudaStream_t s, int* zero_word, bool out_f16, long long out_lo) {
   if (rows <= 0) return 0;
   const int warps_per_block = 8;
   long long blocks = (rows + warps_per_block - 1) / warps_per_block;
   if (blocks > (long long)num_sms() * 16) blocks = (long long)num_sms() * 16;
   auto k = x_f32 ? (out_f16 ? rmsnorm_kernel<true, true> : rmsnorm_kernel<true, false>)
                  : (out_f16 ? rmsnorm_kernel<false, true> : rmsnorm_kernel<false, false>);
-  q3_launch(k, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps, zero_word);
+  q3_launch(k, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps, zero_word, out_lo);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

@@ -38,17 +38,21 @@ int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long c
 
 namespace {
 
-constexpr int kSkStages = 8;
 constexpr int kSkThreads = 192;
 constexpr int kSkMaxSplits = 8;
 constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 of K, bf16
 
-template <int BN>
+// HILO: the activation operand holds 2M rows, row t = hi(a_t) and row M + t = lo(a_t)
+// (a = hi + lo to about twice the type's precision); the MMA's N covers both and the
+// accumulator columns t and M + t are added before the split sum.
+template <int BN, bool HILO>
 struct SkCfg {
-  static constexpr uint32_t Q_BYTES = BN * 64 * 2;
+  static constexpr int NQ = HILO ? 2 * BN : BN;  // activation rows per tile = MMA N
+  static constexpr int STAGES = NQ >= 128 ? 6 : 8;
+  static constexpr uint32_t Q_BYTES = NQ * 64 * 2;
   static constexpr uint32_t STAGE = kSkPBytes + Q_BYTES;
-  static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
-  static constexpr size_t SMEM = 1024 + (size_t)kSkStages * STAGE + 256;  // + barriers and flags
+  static constexpr uint32_t TMEM_COLS = NQ < 32 ? 32 : NQ;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;  // + barriers and flags
 };
 
 struct SkParams {
@@ -67,6 +71,8 @@ struct SkParams {
   const uint16_t* norm_w;
   uint16_t* norm_out;
   long long ld_norm;
+  long long norm_lo;  // > 0: also write lo(norm_out) this many elements after each hi value
+  long long out_lo;   // SwiGLU: > 0: also write lo(out) this many elements after each hi value
   int N;
   float norm_eps;
   int* ticket;
@@ -77,11 +83,12 @@ struct SkParams {
 
 }  // namespace
 
-template <int BN>
+template <int BN, bool HILO>
 __global__ void __launch_bounds__(kSkThreads, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                        const SkParams g) {
-  using C = SkCfg<BN>;
+  using C = SkCfg<BN, HILO>;
+  constexpr int kSkStages = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kSkStages * C::STAGE);
@@ -152,7 +159,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      const uint32_t idesc = g.f16 ? idesc_f16_f32(128, BN) : idesc_bf16_f32(128, BN);
+      const uint32_t idesc = g.f16 ? idesc_f16_f32(128, C::NQ) : idesc_bf16_f32(128, C::NQ);
       bool ok = true;
       for (int i = 0; i < nkb; ++i) {
         const int st = i % kSkStages;
@@ -178,20 +185,30 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     tc_fence_after();
     const int f = quad * 32 + lane;
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
-    if constexpr (BN == 16) {
+    // column j < M: token j (its hi half with HILO); column M + t: token t's lo half,
+    // added after its hi value (columns are visited in increasing order)
+    const int M = g.M;
+    auto put = [&](int j, uint32_t r) {
+      const float v = ok ? __uint_as_float(r) : 0.f;
+      if (j < M) red[j * 128 + f] = v;
+      else if (HILO && j < 2 * M) red[(j - M) * 128 + f] += v;
+    };
+    if constexpr (C::NQ == 16) {
       uint32_t r[16];
       tmem_ld16(taddr, r);
       tmem_wait_ld_regs16(r);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) red[j * 128 + f] = ok ? __uint_as_float(r[j]) : 0.f;
+      for (int j = 0; j < 16; ++j) put(j, r[j]);
     } else {
+      const int used = HILO ? 2 * M : M;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < C::NQ / 32; ++c) {
+        if (c * 32 >= used) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld32(taddr + c * 32, r);
         tmem_wait_ld_regs(r);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) red[(c * 32 + j) * 128 + f] = ok ? __uint_as_float(r[j]) : 0.f;
+        for (int j = 0; j < 32; ++j) put(c * 32 + j, r[j]);
       }
     }
   }
@@ -265,10 +282,16 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       } else if (g.epi == kEpiSwiglu) {
         // 32-feature block j: lanes 0-15 hold gate features, lanes 16-31 the matching up
         uint16_t* dst = static_cast<uint16_t*>(g.out) + (long long)t * g.ldo + tile * 64;
+        const bool f16 = g.f16 != 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float u = __shfl_down_sync(0xffffffffu, v[j], 16);
-          if (lane < 16) dst[16 * j + lane] = to_op_bits(g.f16 != 0, silu_f(v[j]) * u);
+          if (lane < 16) {
+            const float a = silu_f(v[j]) * u;
+            const uint16_t hi = to_op_bits(f16, a);
+            dst[16 * j + lane] = hi;
+            if (g.out_lo) dst[g.out_lo + 16 * j + lane] = to_op_bits(f16, a - op_bits_to_f32(f16, hi));
+          }
         }
       } else {
         const long long col = (long long)tile * 128 + lane;
@@ -337,12 +360,19 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           }
           const uint4 w = *reinterpret_cast<const uint4*>(g.norm_w + col);
           const bool f16 = g.f16 != 0;
-          uint4 o;
-          o.x = pack_op_x2(f16, x[0] * r * bf16_lo(w.x), x[1] * r * bf16_hi(w.x));
-          o.y = pack_op_x2(f16, x[2] * r * bf16_lo(w.y), x[3] * r * bf16_hi(w.y));
-          o.z = pack_op_x2(f16, x[4] * r * bf16_lo(w.z), x[5] * r * bf16_hi(w.z));
-          o.w = pack_op_x2(f16, x[6] * r * bf16_lo(w.w), x[7] * r * bf16_hi(w.w));
-          *reinterpret_cast<uint4*>(g.norm_out + (long long)t * g.ld_norm + col) = o;
+          const float wv[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
+                               bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float a0 = x[2 * j] * r * wv[2 * j], a1 = x[2 * j + 1] * r * wv[2 * j + 1];
+            hi[j] = pack_op_x2(f16, a0, a1);
+            lo[j] = pack_op_x2(f16, a0 - op_bits_to_f32(f16, (uint16_t)(hi[j] & 0xFFFFu)),
+                               a1 - op_bits_to_f32(f16, (uint16_t)(hi[j] >> 16)));
+          }
+          uint16_t* dst = g.norm_out + (long long)t * g.ld_norm + col;
+          *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          if (g.norm_lo) *reinterpret_cast<uint4*>(dst + g.norm_lo) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
       }
       // every cluster has taken its ticket: reset it for the next launch
@@ -368,11 +398,11 @@ std::mutex g_sk_mu;
 std::vector<SkChoice> g_sk_fit;
 
 // Can n_clusters clusters of S CTAs all be resident at once (one wave)?
-template <int BN>
+template <int BN, bool HILO>
 bool clusters_fit(int S, int n_clusters) {
   int dev = 0;
   cudaGetDevice(&dev);
-  const void* func = reinterpret_cast<const void*>(gemm_skinny_kernel<BN>);
+  const void* func = reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>);
   {
     std::lock_guard<std::mutex> lk(g_sk_mu);
     for (const auto& c : g_sk_fit)
@@ -381,7 +411,7 @@ bool clusters_fit(int S, int n_clusters) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(S * n_clusters);
   cfg.blockDim = dim3(kSkThreads);
-  cfg.dynamicSmemBytes = SkCfg<BN>::SMEM;
+  cfg.dynamicSmemBytes = SkCfg<BN, HILO>::SMEM;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = S;
@@ -390,32 +420,33 @@ bool clusters_fit(int S, int n_clusters) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_skinny_kernel<BN>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_skinny_kernel<BN, HILO>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     n = 0;
   }
   std::lock_guard<std::mutex> lk(g_sk_mu);
-  g_sk_fit.push_back({func, dev, S, (int)SkCfg<BN>::SMEM, n});
+  g_sk_fit.push_back({func, dev, S, (int)SkCfg<BN, HILO>::SMEM, n});
   return n >= n_clusters;
 }
 
-template <int BN>
+template <int BN, bool HILO>
 int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
-  using C = SkCfg<BN>;
-  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN>), (int)C::SMEM)) return -6;
+  using C = SkCfg<BN, HILO>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)C::SMEM)) return -6;
   const int n_tiles = d.N / 128, k_blocks = d.K / 64;
   // splits: as many as fill the SMs in one wave of co-resident clusters
   int S = 1;
   for (int c = kSkMaxSplits; c >= 1; --c) {
     if ((long long)n_tiles * c > num_sms() || c > k_blocks) continue;
-    if (c > 1 && !clusters_fit<BN>(c, n_tiles)) continue;
+    if (c > 1 && !clusters_fit<BN, HILO>(c, n_tiles)) continue;
     S = c;
     break;
   }
   const int kpb = (k_blocks + S - 1) / S;
   S = (k_blocks + kpb - 1) / kpb;  // every split gets at least one K block
   CUtensorMap tmP, tmQ;
-  if (make_tmap_2d(&tmP, d.W, d.N, d.K, d.ldw, 128) != 0 || make_tmap_2d(&tmQ, d.A, d.M, d.K, d.lda, BN) != 0) {
+  if (make_tmap_2d(&tmP, d.W, d.N, d.K, d.ldw, 128) != 0 ||
+      make_tmap_2d(&tmQ, d.A, HILO ? 2LL * d.M : d.M, d.K, d.lda, C::NQ) != 0) {
     set_last_error("skinny gemm: cannot encode the operand tensor maps");
     return -6;
   }
@@ -435,14 +466,16 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   g.norm_w = d.norm_w;
   g.norm_out = d.norm_out;
   g.ld_norm = d.ld_norm;
+  g.norm_lo = d.norm_lo;
+  g.out_lo = d.out_lo;
   g.N = d.N;
   g.norm_eps = d.norm_eps;
   g.ticket = d.ticket;
   g.qk = d.qk;
   g.f16 = d.f16 ? 1 : 0;
   g.err = err;
-  q3_launch_cluster(gemm_skinny_kernel<BN>, dim3(n_tiles * S), dim3(kSkThreads), C::SMEM, s, (unsigned)S, tmP, tmQ,
-                    g);
+  q3_launch_cluster(gemm_skinny_kernel<BN, HILO>, dim3(n_tiles * S), dim3(kSkThreads), C::SMEM, s, (unsigned)S,
+                    tmP, tmQ, g);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("skinny gemm launch failed: %s", cudaGetErrorString(e));
@@ -467,9 +500,18 @@ int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err) {
     set_last_error("skinny gemm: the fused RMSNorm needs the residual epilogue, weights, a ticket and N %% 256 == 0");
     return -1;
   }
-  if (d.M <= 16) return launch_bn<16>(d, s, err);
-  if (d.M <= 32) return launch_bn<32>(d, s, err);
-  return launch_bn<64>(d, s, err);
+  if (d.epi == kEpiSwiglu ? false : d.out_lo != 0) {
+    set_last_error("skinny gemm: a lo copy of the output is only written by the SwiGLU epilogue");
+    return -1;
+  }
+  if (d.a_hilo) {
+    if (d.M <= 16) return launch_bn<16, true>(d, s, err);
+    if (d.M <= 32) return launch_bn<32, true>(d, s, err);
+    return launch_bn<64, true>(d, s, err);
+  }
+  if (d.M <= 16) return launch_bn<16, false>(d, s, err);
+  if (d.M <= 32) return launch_bn<32, false>(d, s, err);
+  return launch_bn<64, false>(d, s, err);
 }
 
 }  // namespace q3

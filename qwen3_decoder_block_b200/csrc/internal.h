@@ -108,6 +108,13 @@ struct SkinnyDesc {
   int* ticket = nullptr;
   QKRopeArgs qk;
   bool f16 = false;  // as GemmDesc::f16
+  // a_hilo: A holds 2M rows, row t = hi(a_t), row M + t = lo(a_t) = round(a_t - hi), both in
+  // the operand type; the product uses hi + lo (twice the precision of one 16-bit value)
+  bool a_hilo = false;
+  // optional lo copies for a following hi/lo consumer, written this many elements after
+  // each hi value: norm_lo for norm_out, out_lo for the SwiGLU output
+  long long norm_lo = 0;
+  long long out_lo = 0;
 };
 
 bool skinny_supported(int M, int N, int K, int epi);

@@ -431,3 +431,43 @@ def test_embed_f16_table(q3):
     q3.op_embed(ids, n, E16, V, H, out)
     assert_device_ok()
     np.testing.assert_array_equal(out.cpu().double().numpy(), f64_of(E16)[ids_np])
+
+
+@pytest.mark.parametrize("M,N,K,epi,f16", [(64, 4096, 1024, 0, 0), (16, 1024, 2048, 1, 0), (37, 6144, 1024, 2, 0),
+                                           (64, 1024, 3072, 1, 1), (5, 2048, 4096, 0, 1)])
+def test_gemm_cluster_split_k_hilo_operand(q3, M, N, K, epi, f16):
+    """swap = 3: the activation operand as hi/lo rows (hi = round(a), lo = round(a - hi) in
+    the operand type). The product must carry the lo half: against the fp32 activations
+    the error is far below one rounding of a (asserted 16x below the typical error of one
+    bf16 rounding), which a kernel that dropped the lo rows could not reach."""
+    rng = np.random.default_rng(M * 7 + K)
+    a32 = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).cuda()
+    dt = torch.float16 if f16 else torch.bfloat16
+    hi = a32.to(dt)
+    lo = (a32 - hi.float()).to(dt)
+    A2 = torch.cat([hi, lo]).contiguous()
+    W = Tensor(SEED, 72, (N, K), 0.0, 0.02)
+    Wp = W.gpu
+    if epi == 2:
+        Wp = torch.empty_like(W.gpu)
+        q3.pack_gate_up(N // 2, K, W.gpu[:N // 2], W.gpu[N // 2:], Wp)
+    Wd = to_f16(Wp) if f16 else Wp
+    a = a32.double().cpu().numpy()
+    acc = a @ W.f.T
+    # typical size of the product's error when a is rounded once to bf16 (independent
+    # relative errors of 2^-9 / sqrt(3) per element)
+    one_rounding = np.sqrt((a * a) @ (W.f.T * W.f.T)) * 2.0 ** -9 / np.sqrt(3.0)
+    if epi == 2:
+        out = torch.empty((M, N // 2), dtype=dt, device="cuda")
+        q3.op_gemm(A2, Wd, out, M, N, K, epilogue=2, swap=3)
+        assert_device_ok()
+        ref = R.silu(acc[:, :N // 2]) * acc[:, N // 2:]
+        assert np.all(np.abs(f64_of(out) - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-3)
+        return
+    X = Tensor(SEED, 73, (M, N))
+    out = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    q3.op_gemm(A2, Wd, out, M, N, K, epilogue=epi, resid=X.gpu.float() if epi == 1 else None, swap=3)
+    assert_device_ok()
+    ref = acc + (X.f if epi == 1 else 0.0)
+    err = np.abs(f64_of(out) - ref)
+    assert np.all(err <= one_rounding / 16 + 1e-6), float(np.max(err / (one_rounding + 1e-12)))

@@ -168,14 +168,21 @@ def test_stack_prefill_B4xT2048_bf16_operands(q3, stack_prefill_model):
     assert err <= LOGITS_REL_FROB
 
 
-def test_stack_decode_B64_ctx4096(q3):
-    """B64 sequences with 4096 cached tokens, successive decode steps at positions 4096..;
-    the oracle follows sequence 37 for the first 8 steps."""
-    cfg = q3.config_qwen3_0_6b()
-    seed, B, L0, steps, b_s = 1002, 64, 4096, 8, 37
+DECODE_SEQS = (0, 9, 18, 27, 37, 46, 55, 63)
+
+
+@pytest.mark.parametrize("f16", [1, 0])
+def test_stack_decode_B64_ctx4096(q3, f16):
+    """B64 sequences with 4096 cached tokens, successive decode steps at positions
+    4096..4103; the oracle follows 8 sequences spread over the batch for all 8 steps
+    (64 rows of 151936 logits), each from its own cache drawn by the host generator."""
+    cfg = q3.make_config(gemm_f16=f16)
+    seed, B, L0, steps = 1002, 64, 4096, 8
     s_max = L0 + 128
     layers, E, fn = _stack_weights(q3, cfg, seed)
     Eg, fng = to_gpu_bf16(E), to_gpu_bf16(fn)
+    if f16:
+        Eg = to_f16(Eg)
     caches = []
     for l in range(cfg.n_layers):
         k = torch.empty((B, 8, s_max, 128), dtype=torch.bfloat16, device="cuda")
@@ -191,37 +198,44 @@ def test_stack_decode_B64_ctx4096(q3):
     rope = rope_gpu(cfg)
     lg = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
     got = []
-    for s in range(steps):
-        q3.stack_forward(cfg, Eg, [l.c for l in layers], fng, torch.from_numpy(ids[s]).cuda(), B, 1, q3.MODE_DECODE,
-                         lens, kvs, rope, lg, False, ws)
-        got.append(lg[b_s].double().cpu().numpy())
+    for s_ in range(steps):
+        q3.stack_forward(cfg, Eg, [l.c for l in layers], fng, torch.from_numpy(ids[s_]).cuda(), B, 1,
+                         q3.MODE_DECODE, lens, kvs, rope, lg, False, ws)
+        got.append(lg[list(DECODE_SEQS)].double().cpu().numpy())
     assert_device_ok()
     assert int(lens[0].item()) == L0 + steps
-    del caches
+    del caches, kvs
     torch.cuda.empty_cache()
-    # oracle: the same sequence's cache (host generator), then the same steps
+    # oracle: each followed sequence's cache (host generator), then the same steps; the
+    # new keys and values of every step are appended to its cache
     oc = oracle_config(cfg)
     olayers = [l.oracle() for l in layers]
-    base = b_s * 8 * L0 * 128
-    ocache = []
-    for l in range(cfg.n_layers):
-        kk = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_K), (8, L0, 128),
-                                                  index_base=base)).transpose(1, 0, 2)
-        vv = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_V), (8, L0, 128),
-                                                  index_base=base)).transpose(1, 0, 2)
-        ocache.append([kk, vv])
     Ef, fnf = R.bf16_to_f64(E), R.bf16_to_f64(fn)
     errs, agree = [], []
-    for s in range(steps):
-        caches_s = [(c[0], c[1], np.arange(L0 + s)) for c in ocache]
-        ref, new_kv = R.stack_forward(ids[s, b_s:b_s + 1], Ef, olayers, fnf, oc, positions=np.array([L0 + s]),
-                                      caches=caches_s)
-        for c, (kn, vn) in zip(ocache, new_kv):
-            c[0] = np.concatenate([c[0], kn])
-            c[1] = np.concatenate([c[1], vn])
-        errs.append(rel_frob(got[s], ref[0]))
-        agree.append(int(np.argmax(got[s]) == np.argmax(ref[0])))
-    report("stack_decode_B64_ctx4096", rel_frob_max=max(errs), rel_frob=errs, argmax=agree, steps=steps, sequence=b_s)
+    for i, b_s in enumerate(DECODE_SEQS):
+        base = b_s * 8 * L0 * 128
+        ocache = []
+        for l in range(cfg.n_layers):
+            kk = np.empty((L0 + steps, 8, 128))
+            vv = np.empty((L0 + steps, 8, 128))
+            kk[:L0] = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_K), (8, L0, 128),
+                                                           index_base=base)).transpose(1, 0, 2)
+            vv[:L0] = R.bf16_to_f64(synth.normal_bf16_fast(seed, synth.layer_tid(l, synth.L_CACHE_V), (8, L0, 128),
+                                                           index_base=base)).transpose(1, 0, 2)
+            ocache.append((kk, vv))
+        for s_ in range(steps):
+            n = L0 + s_
+            caches_s = [(kk[:n], vv[:n], np.arange(n)) for kk, vv in ocache]
+            ref, new_kv = R.stack_forward(ids[s_, b_s:b_s + 1], Ef, olayers, fnf, oc, positions=np.array([n]),
+                                          caches=caches_s)
+            for (kk, vv), (kn, vn) in zip(ocache, new_kv):
+                kk[n] = kn[0]
+                vv[n] = vn[0]
+            g = got[s_][i]
+            errs.append(rel_frob(g, ref[0]))
+            agree.append(int(np.argmax(g) == np.argmax(ref[0])))
+    report(f"stack_decode_B64_ctx4096_f16{f16}", rel_frob_max=max(errs), rel_frob_mean=float(np.mean(errs)),
+           argmax_agreement=float(np.mean(agree)), rows=len(agree), sequences=list(DECODE_SEQS), steps=steps)
     assert max(errs) <= LOGITS_REL_FROB
     assert np.mean(agree) >= LOGITS_ARGMAX
 

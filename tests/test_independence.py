@@ -23,7 +23,8 @@ def _imports(path):
 
 
 def test_oracle_imports_only_stdlib_and_numpy():
-    allowed = {"__future__", "dataclasses", "typing", "math", "numpy"}
+    allowed = {"__future__", "dataclasses", "typing", "math", "numpy", "ctypes", "os", "hashlib", "shutil",
+               "subprocess", "sys"}
     for name in os.listdir(os.path.join(ROOT, "oracle")):
         if name.endswith(".py"):
             mods = set(_imports(os.path.join(ROOT, "oracle", name)))
@@ -38,6 +39,13 @@ def test_package_never_imports_the_oracle():
                 assert "oracle" not in set(_imports(path)), path
             elif name.endswith((".cu", ".cuh", ".h")):
                 assert "oracle" not in open(path, encoding="utf-8").read(), path
+
+
+def test_cpp_oracle_includes_nothing_of_the_library():
+    src = open(os.path.join(ROOT, "oracle", "qwen3_ref.cpp"), encoding="utf-8").read()
+    includes = [l for l in src.splitlines() if l.startswith("#include")]
+    assert all("<" in l for l in includes), includes  # standard headers only
+    assert "qwen3blk" not in src and "csrc" not in src
 
 
 def test_package_import_fails_loudly_without_its_library():
