@@ -74,7 +74,7 @@ def case_attn_decode(reps, B=64, L=4096):
 
 
 def _gemm(reps, M, N, K, epi=q3.EPI_STORE, swap=-1, out_f32=False, resid=False):
-    A = _bf16((M, K), 7)
+    A = _bf16((2 * M if swap == 3 else M, K), 7)  # swap 3: hi rows then lo rows
     W = _bf16((N, K), 8, 0.02)
     n_out = N // 2 if epi == q3.EPI_SWIGLU else N
     out = torch.empty((M, n_out), dtype=torch.float32 if out_f32 else torch.bfloat16, device="cuda")
@@ -82,7 +82,7 @@ def _gemm(reps, M, N, K, epi=q3.EPI_STORE, swap=-1, out_f32=False, resid=False):
     ws = torch.empty(48 << 20, dtype=torch.uint8, device="cuda")  # split-K scratch for small M
     ms = _time(lambda: q3.op_gemm(A, W, out, M, N, K, epilogue=epi, resid=r, swap=swap, ws=ws), reps)
     flops = 2 * M * N * K
-    nbytes = 2 * (M * K + N * K) + out.numel() * out.element_size() + (r.numel() * 4 if resid else 0)
+    nbytes = 2 * (A.numel() + N * K) + out.numel() * out.element_size() + (r.numel() * 4 if resid else 0)
     return {"ms": ms, "tflops": flops / ms / 1e9, "gbs": nbytes / ms / 1e6, "flops": flops, "bytes": nbytes}
 
 
@@ -138,6 +138,32 @@ def case_gemm_o_decode(reps):
 def case_gemm_gate_up_decode(reps):
     """B64 decode gate/up: M64 (swap), N6144, K1024, SwiGLU epilogue."""
     return _gemm(reps, 64, 6144, 1024, epi=q3.EPI_SWIGLU)
+
+
+def case_gemm_qkv_decode(reps):
+    """B64 decode QKV projection on the cluster split-K form: M64, N4096, K1024."""
+    return _gemm(reps, 64, 4096, 1024, swap=2)
+
+
+def case_gemm_down_decode(reps):
+    """B64 decode down projection on the cluster split-K form: M64, N1024, K3072, fp32 residual."""
+    return _gemm(reps, 64, 1024, 3072, epi=q3.EPI_RESID, out_f32=True, resid=True, swap=2)
+
+
+def case_gemm_down_decode_splitk(reps):
+    """As gemm_down_decode on the persistent GEMM with K split into fp32 partials in global
+    memory and a separate completion launch (the form used for 65-256 tokens)."""
+    return _gemm(reps, 64, 1024, 3072, epi=q3.EPI_RESID, out_f32=True, resid=True, swap=1)
+
+
+def case_gemm_qkv_decode_splitk(reps):
+    """As gemm_qkv_decode on the split-K partials form."""
+    return _gemm(reps, 64, 4096, 1024, swap=1)
+
+
+def case_gemm_down_decode_hilo(reps):
+    """As gemm_down_decode with the activations as hi/lo rows (the decode path's form)."""
+    return _gemm(reps, 64, 1024, 3072, epi=q3.EPI_RESID, out_f32=True, resid=True, swap=3)
 
 
 def case_qk_norm_rope(reps, B=4, T=2048):

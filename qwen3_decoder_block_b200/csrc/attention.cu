@@ -458,14 +458,43 @@ constexpr uint32_t kD4OffK = 0;
 constexpr uint32_t kD4OffV = 2 * kD4Half;
 constexpr uint32_t kD4OffQ = 4 * kD4Half;
 constexpr uint32_t kD4StageBytes = 4 * kD4Half + 2 * kD4QHalf;  // 68 KB
-constexpr uint32_t kD4OffP = kD4Stages * kD4StageBytes;         // P [16][128] as two K halves
-constexpr uint32_t kD4OffRed = kD4OffP + 2 * kD4QHalf;          // maxima [2][4][16], sums [4][16]
+constexpr uint32_t kD4OffP = kD4Stages * kD4StageBytes;         // P [2 buffers][16][128] as two K halves each
+constexpr uint32_t kD4OffRed = kD4OffP + 4 * kD4QHalf;          // maxima [2][4][16], sums [4][16]
 constexpr uint32_t kD4OffBar = kD4OffRed + (2 * 4 * 16 + 4 * 16) * 4;
 constexpr uint32_t kD4Smem = kD4OffBar + 16 * 8 + 16 + 1024;
 constexpr int kD4Threads = 192;  // softmax warps 0-3, TMA warp 4, MMA warp 5
 constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
 
 __device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// Log-sum-exp merge of one query head's split partials (unnormalised o, running max in
+// the exp2 domain, sum) for head dim d: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),
+// M = max_s m_s, splits in order. Written as bf16 or fp16, with an optional lo copy
+// o_lo elements after it (the hi/lo operand of the decode-sized o_proj).
+struct DecodeMergeOut {
+  uint16_t* out;
+  long long ldo;
+  int o_f16;
+  long long o_lo;
+};
+__device__ __forceinline__ void merge_head_dim(const float* pp, int n_splits, int d, uint16_t* dst,
+                                               const DecodeMergeOut& mo) {
+  float M = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pp[s * (kHeadDim + 2) + kHeadDim]);
+  float L = 0.f, acc = 0.f;
+  for (int s = 0; s < n_splits; ++s) {
+    const float* q = pp + s * (kHeadDim + 2);
+    const float m = q[kHeadDim];
+    if (m == -INFINITY) continue;
+    const float w = exp2f(m - M);
+    L += q[kHeadDim + 1] * w;
+    acc += q[d] * w;
+  }
+  const float o = acc / L;
+  const uint16_t hi = to_op_bits(mo.o_f16 != 0, o);
+  dst[d] = hi;
+  if (mo.o_lo) dst[mo.o_lo + d] = to_op_bits(mo.o_f16 != 0, o - op_bits_to_f32(mo.o_f16 != 0, hi));
+}
 
 // HILO (G <= 8): q arrives as 2G rows per group, q_hi = bf16(q) in rows 0..G-1 and
 // q_lo = bf16(q - q_hi) in rows G..2G-1, and P is written the same way, so the N = 16
@@ -485,9 +514,9 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   uint64_t* empty = bars + 3;    // [3] stage consumed
   uint64_t* s_full = bars + 6;   // [2] scores ready
   uint64_t* s_empty = bars + 8;  // [2] scores read
-  uint64_t* p_full = bars + 10;  // P written (and O rescaled)
-  uint64_t* pv_done = bars + 11;
-  uint64_t* drain = bars + 12;
+  uint64_t* p_full = bars + 10;  // [2] P buffer written (and O rescaled)
+  uint64_t* pv_done = bars + 12; // [2] P.V of a tile using that buffer complete
+  uint64_t* drain = bars + 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red_max = reinterpret_cast<float*>(smem + kD4OffRed);  // [2][4][16]
@@ -499,14 +528,13 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kD4Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1); }
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   // Rows G..15 of the Q and P operand tiles are never written: clear all of them once.
-  for (int i = threadIdx.x; i < (2 * kD4Stages + 2) * (int)(kD4QHalf / 16); i += blockDim.x) {
+  for (int i = threadIdx.x; i < (2 * kD4Stages + 4) * (int)(kD4QHalf / 16); i += blockDim.x) {
     const int buf = i / (int)(kD4QHalf / 16), off = i % (int)(kD4QHalf / 16);
     uint8_t* base = buf < 2 * kD4Stages ? smem + (buf >> 1) * kD4StageBytes + kD4OffQ + (buf & 1) * kD4QHalf
                                         : smem + kD4OffP + (buf - 2 * kD4Stages) * kD4QHalf;
@@ -562,18 +590,21 @@ __global__ void __launch_bounds__(kD4Threads, 1)
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, 0, 0);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, 1, 0);  // V^T: MN-major A
       const uint32_t sP = smem_u32(smem + kD4OffP);
-      // O^T += V^T P^T for tile u (the first tile of a split overwrites O)
+      // O^T += V^T P^T for tile u (the first tile of a split overwrites O); P of tile u is
+      // in buffer u & 1, whose barriers advance once every second tile
       auto issue_pv = [&](long long u, bool first) -> bool {
-        if (*s_abort || !mbar_wait(p_full, (uint32_t)(u & 1), err)) return false;
+        const int pb = (int)(u & 1);
+        if (*s_abort || !mbar_wait(&p_full[pb], (uint32_t)((u >> 1) & 1), err)) return false;
         tc_fence_after();
         const uint32_t sV = smem_u32(smem + (int)(u % kD4Stages) * kD4StageBytes + kD4OffV);
+        const uint32_t sPb = sP + pb * 2 * kD4QHalf;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t a = sdesc_mnmajor_sw128(sV + kk * 16 * 128, kD4Half, 1024);
-          const uint64_t bp = sdesc_kmajor_sw128(sP + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
+          const uint64_t bp = sdesc_kmajor_sw128(sPb + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
           mma_bf16_ss(tmem + 32, a, bp, idesc_o, (first && kk == 0) ? 0u : 1u);
         }
-        mma_commit(pv_done);
+        mma_commit(&pv_done[pb]);
         mma_commit(&empty[u % kD4Stages]);
         return true;
       };
@@ -675,9 +706,15 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           p[j] = (t < nk && m_run[j] != -INFINITY) ? ex2_approx(s[j] - m_run[j]) : 0.f;
           l_part[j] = l_part[j] * alpha[j] + p[j];
         }
-        // P is single-buffered and O is rescaled below: the previous P.V must be done
-        if (tc > 0) {
-          ok = ok && !*s_abort && mbar_wait(pv_done, (uint32_t)((tc - 1) & 1), err);
+        // P is double-buffered: buffer tc & 1 was last read by the P.V of tile tc - 2. A
+        // rescale of O (below) needs the P.V of tile tc - 1 complete as well.
+        const int pbuf = (int)(tc & 1);
+        if (tc >= 2) {
+          ok = ok && !*s_abort && mbar_wait(&pv_done[pbuf], (uint32_t)(((tc - 2) >> 1) & 1), err);
+          ok = __all_sync(0xffffffffu, ok);
+        }
+        if (n_tiles > 0 && rescale) {  // uniform: every thread holds the same maxima
+          ok = ok && !*s_abort && mbar_wait(&pv_done[pbuf ^ 1], (uint32_t)(((tc - 1) >> 1) & 1), err);
           ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {
@@ -694,8 +731,8 @@ __global__ void __launch_bounds__(kD4Threads, 1)
             tmem_st16x(tl + 32, ov);
             tmem_wait_st();
           }
-          // P[j][t] into the K-major B tile: row j, key t, 128-byte swizzle
-          uint8_t* pb = smem + kD4OffP + (t >> 6) * kD4QHalf + (t & 7) * 2;
+          // P[j][t] into the K-major B tile of buffer pbuf: row j, key t, 128-byte swizzle
+          uint8_t* pb = smem + kD4OffP + pbuf * 2 * kD4QHalf + (t >> 6) * kD4QHalf + (t & 7) * 2;
           const int chunk = (t & 63) >> 3;
 #pragma unroll
           for (int j = 0; j < G; ++j) {
@@ -717,7 +754,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           fence_proxy_async_smem();
         }
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[pbuf]);
         ++n_tiles;
         ++tc;
       }
@@ -728,7 +765,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
 #pragma unroll
       for (int j = 0; j < 16; ++j) ov[j] = 0u;
       if (n_tiles > 0) {
-        ok = ok && !*s_abort && mbar_wait(pv_done, (uint32_t)((tc - 1) & 1), err);
+        ok = ok && !*s_abort && mbar_wait(&pv_done[(tc - 1) & 1], (uint32_t)(((tc - 1) >> 1) & 1), err);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
@@ -763,32 +800,14 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   }
 }
 
-// o_lo > 0: also a lo copy round(o - hi) o_lo elements after each value (the hi/lo
-// operand of the decode-sized o_proj).
 __global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
-                                         uint16_t* __restrict__ out, long long ldo, int o_f16, long long o_lo) {
+                                         const DecodeMergeOut mo) {
   pdl_wait();
   pdl_trigger();
   const int bh = blockIdx.x;  // b * Hq + h
   const int b = bh / Hq, h = bh % Hq;
-  const float* pp = part + (long long)bh * n_splits * (kHeadDim + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pp[s * (kHeadDim + 2) + kHeadDim]);
-  const int d = threadIdx.x;
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const float* q = pp + s * (kHeadDim + 2);
-    const float m = q[kHeadDim];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    L += q[kHeadDim + 1] * w;
-    acc += q[d] * w;
-  }
-  const float o = acc / L;
-  const uint16_t hi = to_op_bits(o_f16 != 0, o);
-  uint16_t* dst = out + (long long)b * ldo + (long long)h * kHeadDim + d;
-  *dst = hi;
-  if (o_lo) dst[o_lo] = to_op_bits(o_f16 != 0, o - op_bits_to_f32(o_f16 != 0, hi));
+  merge_head_dim(part + (long long)bh * n_splits * (kHeadDim + 2), n_splits, threadIdx.x,
+                 mo.out + (long long)b * mo.ldo + (long long)h * kHeadDim, mo);
 }
 
 int decode_splits(int s_max) { return (s_max + kD4Split - 1) / kD4Split; }
@@ -834,6 +853,11 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   }
   const long long items = (long long)B * Hkv * n_splits;
   const int grid = (int)(items < num_sms() ? items : num_sms());
+  DecodeMergeOut mo;
+  mo.out = out;
+  mo.ldo = ldo;
+  mo.o_f16 = o_f16 ? 1 : 0;
+  mo.o_lo = o_lo;
   const int variant = G * 2 + (q_hilo ? 1 : 0);
   switch (variant) {
 #define Q3_D4_CASE(GG, HL)                                                                                        \
@@ -853,7 +877,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     Q3_D4_CASE(8, true)
 #undef Q3_D4_CASE
   }
-  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, out, ldo, o_f16 ? 1 : 0, o_lo);
+  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, mo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));

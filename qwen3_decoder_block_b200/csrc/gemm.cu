@@ -223,6 +223,53 @@ __device__ __forceinline__ void stage_row_chunk(const GemmParams& g, int p, int 
   }
 }
 
+// Residual values of row p (p < 0: outside the output, zeros), columns [q, q+32), as fp32.
+__device__ __forceinline__ void load_resid_chunk(const GemmParams& g, int p, int q, float (&v)[32]) {
+  if (p < 0) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    return;
+  }
+  if (g.resid_f32) {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 a = src[j];
+      v[4 * j] = a.x; v[4 * j + 1] = a.y; v[4 * j + 2] = a.z; v[4 * j + 3] = a.w;
+    }
+  } else {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.resid) + (long long)p * g.ldr + q);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 a = src[j];
+      v[8 * j + 0] = bf16_lo(a.x); v[8 * j + 1] = bf16_hi(a.x);
+      v[8 * j + 2] = bf16_lo(a.y); v[8 * j + 3] = bf16_hi(a.y);
+      v[8 * j + 4] = bf16_lo(a.z); v[8 * j + 5] = bf16_hi(a.z);
+      v[8 * j + 6] = bf16_lo(a.w); v[8 * j + 7] = bf16_hi(a.w);
+    }
+  }
+}
+
+// TMA-store staging of acc + res (see stage_row_chunk), the residual already loaded.
+__device__ __forceinline__ void stage_row_chunk_res(const GemmParams& g, const uint32_t (&r)[32],
+                                                    const float (&res)[32], uint8_t* stg, int lane) {
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]) + res[j];
+  if (g.out_f32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+          make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+          make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                     pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+  }
+}
+
 // swap: this thread owns feature p (one TMEM lane) and tokens [q, q+32)
 __device__ __forceinline__ void store_col_chunk(const GemmParams& g, int p, int p_valid, int q, int q_end,
                                                 int lane, int feat_block, const uint32_t (&r)[32]) {
@@ -579,6 +626,39 @@ __global__ void __launch_bounds__(192, 1)
         if (heads > 0)
           qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
                        p < tl.p_end, rope_lo);
+      } else if (g.tma_store && g.epi == kEpiResid) {
+        // residual epilogue, software-pipelined: the residual loads of chunk c + 1 are in
+        // flight while chunk c is read from tensor memory, added and staged
+        const int p = tl.p0 + row;
+        const int pr = p < tl.p_end ? p : -1;
+        float res[32];
+        load_resid_chunk(g, pr, tl.q0, res);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int q = tl.q0 + c * 32;
+          if (q >= tl.q_end) break;  // warp-uniform
+          const bool more = c + 1 < BN / 32 && q + 32 < tl.q_end;
+          float nxt[32];
+          if (more) load_resid_chunk(g, pr, q + 32, nxt);
+          uint32_t r[32];
+          tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, r);
+          tmem_wait_ld_regs(r);
+          uint8_t* stg = staging + ((warp - 2) * 2 + sbuf) * 4096;
+          if (lane == 0) bulk_wait_read<1>();  // the store that used this buffer has read it
+          __syncwarp();
+          stage_row_chunk_res(g, r, res, stg, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmO, stg, q, tl.p0 + quad * 32);
+            bulk_commit();
+          }
+          sbuf ^= 1;
+          if (more) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) res[j] = nxt[j];
+          }
+        }
       } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {

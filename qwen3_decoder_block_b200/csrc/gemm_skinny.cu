@@ -45,14 +45,20 @@ constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 
 // HILO: the activation operand holds 2M rows, row t = hi(a_t) and row M + t = lo(a_t)
 // (a = hi + lo to about twice the type's precision); the MMA's N covers both and the
 // accumulator columns t and M + t are added before the split sum.
+// The ring is sized so that two CTAs fit on an SM (at most ~110 KB each): a CTA keeps
+// its shared memory through the split reduction at its end, and the next projection's
+// CTAs, which prefetch their weights before the grid-dependency wait, can then start
+// beside it instead of after it.
 template <int BN, bool HILO>
 struct SkCfg {
   static constexpr int NQ = HILO ? 2 * BN : BN;  // activation rows per tile = MMA N
-  static constexpr int STAGES = NQ >= 128 ? 6 : 8;
   static constexpr uint32_t Q_BYTES = NQ * 64 * 2;
   static constexpr uint32_t STAGE = kSkPBytes + Q_BYTES;
+  static constexpr int STAGES = (int)(((110u << 10) - 1280u) / STAGE) > 8 ? 8 : (int)(((110u << 10) - 1280u) / STAGE);
   static constexpr uint32_t TMEM_COLS = NQ < 32 ? 32 : NQ;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;  // + barriers and flags
+  static_assert(STAGES >= 3, "ring too shallow");
+  static_assert((size_t)BN * 128 * 4 <= (size_t)STAGES * STAGE, "the split partial must fit over the ring");
 };
 
 struct SkParams {
@@ -84,7 +90,7 @@ struct SkParams {
 }  // namespace
 
 template <int BN, bool HILO>
-__global__ void __launch_bounds__(kSkThreads, 1)
+__global__ void __launch_bounds__(kSkThreads, 2)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                        const SkParams g) {
   using C = SkCfg<BN, HILO>;
