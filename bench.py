@@ -576,7 +576,11 @@ def run_moe_decode(q3, torch, args, peaks, B=64, L0=4096, seed=1005):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
+    q3.profile_begin(400)
+    call()
+    recs = q3.profile_end(stream)
     assert q3.check_device_error() == 0
+    kern, _ = summarize_profile(recs, 1)
     experts_hit = int(torch.unique(idx).numel())
     Im, E = cfg.moe_intermediate, cfg.n_experts
     kv_bytes = B * hkv * (L0 + 1) * D * 2 * 2
@@ -585,7 +589,8 @@ def run_moe_decode(q3, torch, args, peaks, B=64, L0=4096, seed=1005):
     return {"workload": f"MoE block decode step (hidden 2048, 32/4 heads, 128 experts x 768, top-8), B{B} at "
                         f"{L0} cached tokens", "tokens_per_s": B / (ms * 1e-3), "ms_per_call": ms,
             "experts_hit": experts_hit, "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
-            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+            "hbm_frac": nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "kernels_ms": {kk: round(vv["ms_per_step"], 4) for kk, vv in kern.items()}}
 
 
 # --------------------------------------------------------------------------- oracle timing

@@ -321,12 +321,15 @@ int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, l
 /* Decode attention for one query per sequence at position cache_len[b] over kv positions
  * 0..cache_len[b] ("从零实现 Qwen3：拆解 mini-qwen3 的 0.6B Dense 架构", sections GQA and
  * prefill 与 decode). qkv: [B][ldqkv] bf16 with the Hq query heads (post-norm, post-RoPE)
- * at its start; ldqkv a multiple of 8 and >= Hq*128. The keys are split into 256-key
- * chunks whose (max, sum, unnormalised output) partials go to ws and are merged with
- * log-sum-exp weights (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max)
- * suffices). Hq / Hkv must be 1, 2, 4, 8 or 16. A position past the cache
- * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY. o is bf16, or fp16
- * when cfg->gemm_f16 (as qwen3_op_attention_prefill); ldo a multiple of 8 and >= Hq*128. */
+ * at its start; ldqkv a multiple of 8 and >= Hq*128. The 128-key tiles of all (sequence,
+ * KV group) rows are divided evenly among the SMs; a row shared by several SMs leaves
+ * (max, sum, unnormalised output) partials in ws that the last of them merges with
+ * log-sum-exp weights. ws also holds the call's tile plan and per-row tickets
+ * (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max) suffices; the size does
+ * not depend on s_max). Hq / Hkv must be 1, 2, 4, 8 or 16. A position past the cache
+ * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY, a negative one as
+ * QWEN3_EINVAL; that sequence's output row is not written. o is bf16, or fp16 when
+ * cfg->gemm_f16 (as qwen3_op_attention_prefill); ldo a multiple of 8 and >= Hq*128. */
 int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                               const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                               void* ws, size_t ws_bytes, void* stream);
@@ -335,16 +338,19 @@ int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, lo
  * device memory (for example a host application given a fixed memory budget, or a plugin
  * that is handed tensors but no allocator or workspace). The pages have no counterpart:
  * this entry point exists for such callers only.
- * Instead of a caller workspace, the split partials live in a static device array of this
- * library, 12 MiB on every GPU that loads the library (held until the process exits).
- * Limit: B * Hq * ceil(kv->s_max / 256) <= 24197 (for example B 64, Hq 16, s_max up to 5888);
- * larger sizes return QWEN3_EWORKSPACE with the numbers in qwen3_last_error().
+ * Instead of a caller workspace, the partials, tile plan and tickets live in a static
+ * device array of this library, 12 MiB on every GPU that loads the library (held until
+ * the process exits). Limit: (B * Hkv + 256) * G * 130 * 4 bytes of partials plus
+ * (B + 4 + B * Hkv) * 4 bytes must fit (G = Hq / Hkv; B up to 1250 for 16 query heads in
+ * 8 groups, whatever s_max); larger sizes return QWEN3_EWORKSPACE with the numbers in
+ * qwen3_last_error().
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  * with that device current; make that first call before any stream capture. The call
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  * All calls share the one array: calls that overlap on the GPU (other streams, other
- * threads) race and must be serialised by the caller. Every partial a call reads is written
- * by that same call, so nothing needs clearing between calls. */
+ * threads) race and must be serialised by the caller. Each call writes its plan and clears
+ * its tickets before use, and every partial it reads is written by that same call, so
+ * nothing needs clearing between calls. */
 int qwen3_op_attention_decode_noalloc(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                                       const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,
                                       void* stream);

@@ -24,10 +24,26 @@ def _bf16(shape, tid, std=1.0, seed=77):
     return t
 
 
+GRAPH = False  # --graph: time `reps` launches captured in one CUDA graph (no host launch cost)
+
+
 def _time(fn, reps):
     fn()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if GRAPH:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps
     a.record()
     for _ in range(reps):
         fn()
@@ -199,7 +215,10 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=sorted(CASES) + ["all"])
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--graph", action="store_true", help="time the reps as one CUDA-graph replay")
     args = ap.parse_args()
+    global GRAPH
+    GRAPH = args.graph
     names = sorted(CASES) if args.case == "all" else [args.case]
     for n in names:
         r = CASES[n](args.reps)

@@ -39,10 +39,10 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
                              const int* start_pos, const uint16_t* ck, const uint16_t* cv, int s_max, uint16_t* out,
                              long long ldo, int* err, cudaStream_t s, bool o_f16 = false);
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
-                            const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
+                            const uint16_t* ck, const uint16_t* cv, int s_max, float* scratch, uint16_t* out,
                             long long ldo, int* err, cudaStream_t s, bool o_f16 = false, bool q_hilo = false,
-                            long long o_lo = 0);
-size_t decode_partial_bytes(int B, int Hq, int s_max);
+                            long long o_lo = 0, bool plan_ready = false);
+size_t decode_partial_bytes(int B, int Hq, int Hkv);
 int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
                                    const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
                                    uint16_t* out, long long ldo, int* err, cudaStream_t s, bool o_f16 = false);
@@ -245,7 +245,8 @@ struct Buffers {
   uint16_t* o = nullptr;     // [M, Hq*D]
   float* x1 = nullptr;       // [M, H] residual after attention (fp32)
   uint16_t* act = nullptr;   // [M, I] SwiGLU output
-  float* part = nullptr;     // decode partials
+  float* part = nullptr;     // decode attention scratch (partials, tile plan, merge tickets)
+  bool plan_ready = false;   // part holds this call's decode tile plan (same lengths for every layer)
   float* gpart = nullptr;    // split-K partials of small-M GEMMs
   // MoE
   float* logits = nullptr;   // [M, E]
@@ -262,9 +263,10 @@ struct Buffers {
   // stack
   float* xs = nullptr;       // [M, H] fp32 residual stream
   uint16_t* hf = nullptr;    // [rows, H] final-normed
-  // ticket of the decode-sized projections' fused RMSNorm: zeroed by the first kernel
-  // of every call, left at zero by every launch that uses it
+  // grid barrier of the decode-sized projections' fused RMSNorm: [0] zeroed by the first
+  // kernel of every call and left at zero by every launch that uses it, [1] a generation
   int* ticket = nullptr;
+  float* ssq = nullptr;      // the fused RMSNorm's per-tile sums of squares [H / 128][64]
 };
 
 static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void* ws, Buffers* out) {
@@ -280,9 +282,9 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
   b.qkv = cv.take<uint16_t>(M * nqkv);
   b.o = cv.take<uint16_t>(Mh * c.n_q_heads * D);
   b.x1 = cv.take<float>(M * H);
-  // one new token per sequence (decode, or a prefill of T = 1) runs the split-KV decode attention
+  // one new token per sequence (decode, or a prefill of T = 1) runs the decode attention
   if (decode || T == 1) {
-    b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, s_max) / sizeof(float));
+    b.part = cv.take<float>(decode_partial_bytes(B, c.n_q_heads, c.n_kv_heads) / sizeof(float));
     b.q2 = cv.take<uint16_t>(M * 2 * c.n_q_heads * D);
   }
   if (M <= 256) b.gpart = cv.take<float>(kSplitKBytes / sizeof(float));
@@ -307,6 +309,7 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
     b.hf = cv.take<uint16_t>(M * H);
   }
   b.ticket = cv.take<int>(64);
+  if (M <= 64) b.ssq = cv.take<float>((size_t)(H / 128 + 1) * 64);
   if (out) *out = b;
   return cv.used + 256;
 }
@@ -382,12 +385,14 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     if (rc) return rc;
     {
       ProfScope ps(decode ? "attn_decode" : "attn_prefill", k.s);
-      if (decode)
+      if (decode) {
         rc = launch_attention_decode(hilo ? b.q2 : b.qkv, hilo ? 2LL * c.n_q_heads * D : nqkv, B, c.n_q_heads,
                                      c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part, b.o,
                                      (long long)c.n_q_heads * D, k.err, k.s, f16, hilo,
-                                     M * c.n_q_heads * D);  // o as hi/lo rows for o_proj
-      else
+                                     M * c.n_q_heads * D,  // o as hi/lo rows for o_proj
+                                     b.plan_ready);
+        b.plan_ready = rc == 0;
+      } else
         rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
                                       (long long)c.n_q_heads * D, k.err, k.s, f16);
     }
@@ -401,7 +406,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     o.out = b.x1; o.out_f32 = true; o.ldo = H;
     o.w_early = true;
     // the post-attention RMSNorm of x1 goes to b.h (hi/lo rows) in the same launch
-    o.norm_w = w.post_norm; o.norm_out = b.h; o.ld_norm = H; o.norm_eps = c.rms_eps; o.ticket = b.ticket;
+    o.norm_w = w.post_norm; o.norm_out = b.h; o.ld_norm = H; o.norm_eps = c.rms_eps; o.ticket = b.ticket; o.ssq = b.ssq;
     o.norm_lo = M * H;
     o.f16 = f16;
     ProfScope ps("gemm_o", k.s);
@@ -462,7 +467,8 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     ProfScope ps(decode ? "attn_decode" : "attn_prefill", k.s);
     if (decode)
       rc = launch_attention_decode(b.qkv, nqkv, B, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.part,
-                                   b.o, (long long)c.n_q_heads * D, k.err, k.s, f16);
+                                   b.o, (long long)c.n_q_heads * D, k.err, k.s, f16, false, 0, b.plan_ready);
+    if (decode) b.plan_ready = rc == 0;
     else
       rc = launch_attention_prefill(b.qkv, nqkv, B, T, c.n_q_heads, c.n_kv_heads, pos, kv.k, kv.v, kv.s_max, b.o,
                                     (long long)c.n_q_heads * D, k.err, k.s, f16);
@@ -539,7 +545,7 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
     d.w_early = true;
     d.f16 = f16;
     if (next_norm && next_out) {
-      d.norm_w = next_norm; d.norm_out = next_out; d.ld_norm = H; d.norm_eps = c.rms_eps; d.ticket = b.ticket;
+      d.norm_w = next_norm; d.norm_out = next_out; d.ld_norm = H; d.norm_eps = c.rms_eps; d.ticket = b.ticket; d.ssq = b.ssq;
       d.norm_lo = next_hilo ? M * H : 0;
     }
     ProfScope ps("gemm_down", k.s);
@@ -1311,7 +1317,7 @@ int qwen3_op_attention_decode(const qwen3_config* c, const qwen3_bf16* qkv, long
            "attention_decode: ldo (%lld) must be a multiple of 8 and at least n_q_heads * head_dim (%d)", ldo,
            c->n_q_heads * c->head_dim);
   if ((rc = check_kv(*c, kv, 1))) return rc;
-  const size_t need = decode_partial_bytes(B, c->n_q_heads, kv->s_max);
+  const size_t need = decode_partial_bytes(B, c->n_q_heads, c->n_kv_heads);
   Q3_CHECK(ws_bytes >= need, QWEN3_EWORKSPACE, "attention_decode: workspace has %zu bytes, needs %zu", ws_bytes, need);
   if ((rc = check_device())) return rc;
   return finish(launch_attention_decode(qkv, ldqkv, B, c->n_q_heads, c->n_kv_heads, cache_len, kv->k, kv->v,

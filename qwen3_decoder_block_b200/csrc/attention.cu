@@ -1,6 +1,7 @@
 // K3: causal grouped-query prefill attention on tcgen05 tensor cores.
-// K4: split-KV decode attention (memory bound; both products on tcgen05) + a
-//     log-sum-exp merge of the splits.
+// K4: decode attention (memory bound; both products on tcgen05): the cache tiles of
+//     all (sequence, KV group) rows are divided evenly among persistent CTAs, and a
+//     row shared by several CTAs is merged (log-sum-exp) by the last of them.
 //
 // Both compute, for query head h at absolute position m and its KV group
 // g = h / (Hq / Hkv),  o = softmax(q k^T / sqrt(128) + M) v  with M = -inf for keys
@@ -434,10 +435,13 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
 }
 
 // ============================================================================
-// K4, tensor-core form (any G in {1, 2, 4, 8, 16}). Persistent: one CTA per SM walks
-// the (sequence, group, 256-key split) items in a fixed order. Both products of a
-// 128-key tile are tcgen05 MMAs with keys or head dims on the 128-row side and the
-// G query heads of the group (padded to 16) as N:
+// K4, tensor-core form (any G in {1, 2, 4, 8, 16}). Persistent: the 128-key tiles of
+// every (sequence b, KV group g) row, rows in order, form one list of T tiles, and CTA
+// c of n takes tiles [c T / n, (c + 1) T / n) -- the same number of tiles per CTA
+// whatever the lengths, and only a few row boundaries per CTA. A small plan kernel
+// turns the lengths into the per-sequence tile prefix the CTAs search. Both products
+// of a tile are tcgen05 MMAs with keys or head dims on the 128-row side and the G
+// query heads of the group (padded to 16) as N:
 //   S^T[key][j]  = sum_d K[key][d] q_j[d]      A = K tile (K-major), B = Q (K-major)
 //   O^T[d][j]   += sum_key V[key][d] P[j][key]  A = V tile (MN-major), B = P (K-major)
 // so the CUDA cores only run the softmax. A TMA warp streams Q, K and V of each tile
@@ -446,12 +450,14 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
 // tensor memory); 4 softmax warps own one key each (S) and one head dim each (O):
 // the tile maximum per head is a warp reduction plus a 4-warp exchange, the online
 // softmax rescales O only when the running maximum grows by more than 2^8, and P is
-// written as bf16 into a swizzled K-major tile. At the end of a split the
-// unnormalised O, the running maximum and the sum go to the workspace, and the
-// log-sum-exp merge kernel combines the splits.
+// written as bf16 into a swizzled K-major tile. A row that lies in one CTA is
+// normalised and written at once; otherwise each CTA writes its partial (unnormalised
+// O, running maximum, sum) to the scratch, takes the row's ticket, and the CTA with
+// the last ticket merges the row's partials in CTA order.
 // ============================================================================
 constexpr int kD4Stages = 3;
-constexpr int kD4Split = 256;                      // keys per work item (two tiles)
+constexpr int kD4MaxCtas = 256;                    // grid bound (partial slots per call: rows + CTAs)
+constexpr int kD4PartFloats = kHeadDim + 2;        // one head's partial: o[128], running max, sum
 constexpr uint32_t kD4Half = 128 * 128;            // [128 rows][64] bf16, swizzled: 16 KB
 constexpr uint32_t kD4QHalf = 16 * 128;            // [16 rows][64] bf16, swizzled: 2 KB
 constexpr uint32_t kD4OffK = 0;
@@ -467,34 +473,78 @@ constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
 
 __device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-// Log-sum-exp merge of one query head's split partials (unnormalised o, running max in
-// the exp2 domain, sum) for head dim d: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),
-// M = max_s m_s, splits in order. Written as bf16 or fp16, with an optional lo copy
-// o_lo elements after it (the hi/lo operand of the decode-sized o_proj).
+// Log-sum-exp merge of one query head's partials (unnormalised o, running max in the
+// exp2 domain, sum) for head dim d: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),
+// M = max_s m_s, partials in CTA order, read from L2 (other SMs wrote them). Written as
+// bf16 or fp16, with an optional lo copy o_lo elements after it (the hi/lo operand of
+// the decode-sized o_proj).
 struct DecodeMergeOut {
   uint16_t* out;
   long long ldo;
   int o_f16;
   long long o_lo;
 };
-__device__ __forceinline__ void merge_head_dim(const float* pp, int n_splits, int d, uint16_t* dst,
-                                               const DecodeMergeOut& mo) {
-  float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, pp[s * (kHeadDim + 2) + kHeadDim]);
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < n_splits; ++s) {
-    const float* q = pp + s * (kHeadDim + 2);
-    const float m = q[kHeadDim];
-    if (m == -INFINITY) continue;
-    const float w = exp2f(m - M);
-    L += q[kHeadDim + 1] * w;
-    acc += q[d] * w;
-  }
-  const float o = acc / L;
+__device__ __forceinline__ void store_head_dim(float o, int d, uint16_t* dst, const DecodeMergeOut& mo) {
   const uint16_t hi = to_op_bits(mo.o_f16 != 0, o);
   dst[d] = hi;
   if (mo.o_lo) dst[mo.o_lo + d] = to_op_bits(mo.o_f16 != 0, o - op_bits_to_f32(mo.o_f16 != 0, hi));
 }
+// CTA c's tile range [c T / n, (c + 1) T / n) is empty (only when T < n).
+__device__ __forceinline__ bool d4_cta_empty(int c, long long T, int n) {
+  return T * c / n == T * (c + 1) / n;
+}
+
+// Merge of one head's partials of a row: CTAs c_first..c_last with a non-empty range
+// wrote slot (row + c), `stride` floats apart from row_base's slot 0 numbering.
+__device__ __forceinline__ void merge_row_dim(const float* row_base, int c_first, int c_last, long long T, int n,
+                                              long long stride, int d, uint16_t* dst, const DecodeMergeOut& mo) {
+  float M = -INFINITY;
+  for (int c = c_first; c <= c_last; ++c)
+    if (!d4_cta_empty(c, T, n)) M = fmaxf(M, __ldcg(row_base + c * stride + kHeadDim));
+  float L = 0.f, acc = 0.f;
+  for (int c = c_first; c <= c_last; ++c) {
+    if (d4_cta_empty(c, T, n)) continue;
+    const float* q = row_base + c * stride;
+    const float m = __ldcg(q + kHeadDim);
+    if (m == -INFINITY) continue;
+    const float w = exp2f(m - M);
+    L += __ldcg(q + kHeadDim + 1) * w;
+    acc += __ldcg(q + d) * w;
+  }
+  store_head_dim(acc / L, d, dst, mo);
+}
+
+// CTA holding global tile t when T tiles are divided among n CTAs as [c T / n, (c+1) T / n).
+__device__ __forceinline__ int d4_cta_of(long long t, long long T, int n) { return (int)(((t + 1) * n - 1) / T); }
+
+// Walk over the (sequence, group) rows that meet this CTA's tile range. plan[b] is the
+// index of the first tile of sequence b's rows (Hkv rows of plan[b+1]-plan[b] tiles in
+// all); rows of an over-capacity sequence hold no tiles.
+struct D4Walk {
+  const int* plan;
+  int B, Hkv, b, g, nt;
+  long long rs, t_begin, t_end;  // rs: global index of the current row's first tile
+  __device__ D4Walk(const int* p, int B_, int Hkv_, int b0, long long tb, long long te)
+      : plan(p), B(B_), Hkv(Hkv_), b(b0), g(0), nt(0), rs(te), t_begin(tb), t_end(te) {
+    if (tb < te) {
+      nt = (plan[b + 1] - plan[b]) / Hkv;
+      g = (int)((tb - plan[b]) / nt);
+      rs = plan[b] + (long long)g * nt;
+    }
+  }
+  __device__ bool valid() const { return rs < t_end; }
+  __device__ int j0() const { return (int)((t_begin > rs ? t_begin : rs) - rs); }
+  __device__ int j1() const { return (int)((t_end < rs + nt ? t_end : rs + nt) - rs); }
+  __device__ void next() {
+    rs += nt;
+    if (++g == Hkv) {
+      g = 0;
+      do { ++b; } while (b < B && plan[b + 1] == plan[b]);
+      if (b < B) nt = (plan[b + 1] - plan[b]) / Hkv;
+      else rs = t_end;
+    }
+  }
+};
 
 // HILO (G <= 8): q arrives as 2G rows per group, q_hi = bf16(q) in rows 0..G-1 and
 // q_lo = bf16(q - q_hi) in rows G..2G-1, and P is written the same way, so the N = 16
@@ -505,8 +555,8 @@ template <int G, bool HILO>
 __global__ void __launch_bounds__(kD4Threads, 1)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, int B, int Hq, int Hkv,
-                          const int* __restrict__ cache_len, int s_max, int n_splits, float* __restrict__ part,
-                          int* err) {
+                          const int* __restrict__ cache_len, int s_max, const int* __restrict__ plan,
+                          float* __restrict__ part, int* __restrict__ counters, const DecodeMergeOut mo, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kD4OffBar);
@@ -519,11 +569,12 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   uint64_t* drain = bars + 14;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_b0 = s_abort + 1;   // sequence holding this CTA's first tile
+  volatile int* s_fix = s_abort + 2;  // 1 + first CTA of a row this CTA merges, else 0
   float* red_max = reinterpret_cast<float*>(smem + kD4OffRed);  // [2][4][16]
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_items = B * Hkv * n_splits;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kD4Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -531,6 +582,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
     for (int i = 0; i < 2; ++i) { mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1); }
     mbar_init(drain, 1);
     *s_abort = 0;
+    *s_b0 = 0;
     fence_barrier_init();
   }
   // Rows G..15 of the Q and P operand tiles are never written: clear all of them once.
@@ -549,20 +601,25 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
   pdl_trigger();
+  // this CTA's tiles [t_begin, t_end) of the T in the call; the sequence holding t_begin
+  const long long T = plan[B];
+  const int n_cta = (int)gridDim.x;
+  const long long t_begin = T * blockIdx.x / n_cta, t_end = T * (blockIdx.x + 1) / n_cta;
+  for (int b = threadIdx.x; b < B; b += blockDim.x)
+    if (plan[b] <= t_begin && t_begin < plan[b + 1]) *s_b0 = b;
+  __syncthreads();
+  const int b0 = *s_b0;
 
   if (warp == 4) {
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
       long long tc = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
-        const int n_total = cache_len[b] + 1;
-        if (n_total > s_max) continue;  // reported by the softmax warps
+      for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid() && ok; w.next()) {
+        const int b = w.b, g = w.g, bg = b * Hkv + g;
         const int row0 = bg * s_max;
-        for (int h = 0; h < 2; ++h) {
-          const int k0 = split * kD4Split + h * 128;
-          if (k0 >= n_total) break;
+        for (int j = w.j0(); j < w.j1(); ++j) {
+          const int k0 = j * 128;
           const int st = (int)(tc % kD4Stages);
           if (*s_abort || !mbar_wait(&empty[st], (uint32_t)((tc / kD4Stages) & 1) ^ 1u, err)) { ok = false; break; }
           uint8_t* base = smem + st * kD4StageBytes;
@@ -610,13 +667,9 @@ __global__ void __launch_bounds__(kD4Threads, 1)
       };
       long long tc = 0;
       bool ok = true, prev_first = false;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const int split = it % n_splits, b = (it / n_splits) / Hkv;
-        const int n_total = cache_len[b] + 1;
-        if (n_total > s_max) continue;
-        for (int h = 0; h < 2; ++h) {
-          const int k0 = split * kD4Split + h * 128;
-          if (k0 >= n_total) break;
+      for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid() && ok; w.next()) {
+        const int jb = w.j0(), je = w.j1();
+        for (int j = jb; j < je; ++j) {
           const int st = (int)(tc % kD4Stages), sb = (int)(tc & 1);
           if (*s_abort || !mbar_wait(&full[st], (uint32_t)((tc / kD4Stages) & 1), err)) { ok = false; break; }
           if (tc >= 2 && (*s_abort || !mbar_wait(&s_empty[sb], (uint32_t)(((tc - 2) >> 1) & 1), err))) {
@@ -634,7 +687,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           }
           mma_commit(&s_full[sb]);
           if (tc > 0 && !issue_pv(tc - 1, prev_first)) { ok = false; break; }
-          prev_first = (h == 0);
+          prev_first = (j == jb);
           ++tc;
         }
       }
@@ -650,18 +703,16 @@ __global__ void __launch_bounds__(kD4Threads, 1)
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     long long tc = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-      const int split = it % n_splits, bg = it / n_splits, b = bg / Hkv, g = bg % Hkv;
+    for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid(); w.next()) {
+      const int b = w.b, g = w.g, bg = b * Hkv + g;
       const int n_total = cache_len[b] + 1;
-      const bool over = n_total > s_max;
-      if (over && split == 0 && g == 0 && threadIdx.x == 0) record_error(err, kErrCapacity);
+      const int jb = w.j0(), je = w.j1();
       float m_run[G], l_part[G];
 #pragma unroll
       for (int j = 0; j < G; ++j) { m_run[j] = -INFINITY; l_part[j] = 0.f; }
       int n_tiles = 0;
-      for (int h = 0; h < 2 && !over; ++h) {
-        const int k0 = split * kD4Split + h * 128;
-        if (k0 >= n_total) break;
+      for (int j = jb; j < je; ++j) {
+        const int k0 = j * 128;
         const int nk = min(128, n_total - k0);
         const int sb = (int)(tc & 1);
         ok = ok && !*s_abort && mbar_wait(&s_full[sb], (uint32_t)((tc >> 1) & 1), err);
@@ -758,9 +809,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         ++n_tiles;
         ++tc;
       }
-      // this split's partial: unnormalised o, running maximum (log2 domain), sum
-      float* my_part = part + ((long long)(b * Hq + g * G) * n_splits + split) * (kHeadDim + 2);
-      const long long head_stride = (long long)n_splits * (kHeadDim + 2);
+      // end of the row's tiles in this CTA: O from tensor memory, the sums of the 4 warps
       uint32_t ov[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) ov[j] = 0u;
@@ -779,13 +828,48 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         }
         named_bar_softmax();
       }
+      uint16_t* out_row = mo.out + (long long)b * mo.ldo + (long long)g * G * kHeadDim;
+      if (jb == 0 && je == w.nt) {
+        // the whole row is here: normalise and write the output
 #pragma unroll
-      for (int j = 0; j < G; ++j) {
-        my_part[j * head_stride + t] = HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
-        if (t == j) {
-          const float L = n_tiles > 0 ? red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j] : 0.f;
-          my_part[j * head_stride + kHeadDim] = m_run[j];
-          my_part[j * head_stride + kHeadDim + 1] = L;
+        for (int j = 0; j < G; ++j) {
+          const float L = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
+          const float o = HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
+          store_head_dim(o / L, t, out_row + j * kHeadDim, mo);
+        }
+      } else {
+        // partial of the row in slot row + CTA (unique: the rows and the CTA ranges are
+        // both in tile order); the last CTA of the row to finish merges the slots
+        float* my_part = part + ((long long)bg + blockIdx.x) * G * kD4PartFloats;
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+          my_part[j * kD4PartFloats + t] =
+              HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
+          if (t == j) {
+            my_part[j * kD4PartFloats + kHeadDim] = m_run[j];
+            my_part[j * kD4PartFloats + kHeadDim + 1] = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
+          }
+        }
+        __threadfence();  // the partial, visible to the merging CTA before the ticket
+        named_bar_softmax();
+        const int c_first = d4_cta_of(w.rs, T, n_cta), c_last = d4_cta_of(w.rs + w.nt - 1, T, n_cta);
+        if (threadIdx.x == 0) {
+          // the row's CTAs: those of [c_first, c_last] whose range is not empty (fewer
+          // tiles than CTAs leaves some empty)
+          int n_seg = 0;
+          for (int c = c_first; c <= c_last; ++c) n_seg += d4_cta_empty(c, T, n_cta) ? 0 : 1;
+          const int prev = atomicAdd(&counters[bg], 1);
+          const bool last = prev == n_seg - 1;
+          if (last) counters[bg] = 0;  // ready for the next call
+          *s_fix = last ? 1 : 0;
+        }
+        named_bar_softmax();
+        if (*s_fix) {
+          __threadfence();  // the other CTAs' partials (their fences precede their tickets)
+#pragma unroll 1
+          for (int j = 0; j < G; ++j)
+            merge_row_dim(part + ((long long)bg * G + j) * kD4PartFloats, c_first, c_last, T, n_cta,
+                          (long long)G * kD4PartFloats, t, out_row + j * kHeadDim, mo);
         }
       }
     }
@@ -800,28 +884,75 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   }
 }
 
-__global__ void attn_decode_merge_kernel(const float* __restrict__ part, int Hq, int n_splits,
-                                         const DecodeMergeOut mo) {
+// Tile prefix of the decode call: plan[b] = index of the first tile of sequence b's rows
+// (Hkv rows of ceil((cache_len[b] + 1) / 128) tiles each; none for a sequence whose
+// new position is past the cache, which is reported), plan[B] = all tiles. Clears the
+// rows' merge tickets. One block.
+__global__ void __launch_bounds__(1024) attn_decode_plan_kernel(const int* __restrict__ cache_len, int B, int Hkv,
+                                                                int s_max, int* __restrict__ plan,
+                                                                int* __restrict__ counters, int* err) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
   pdl_wait();
   pdl_trigger();
-  const int bh = blockIdx.x;  // b * Hq + h
-  const int b = bh / Hq, h = bh % Hq;
-  merge_head_dim(part + (long long)bh * n_splits * (kHeadDim + 2), n_splits, threadIdx.x,
-                 mo.out + (long long)b * mo.ldo + (long long)h * kHeadDim, mo);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < B; base += blockDim.x) {
+    const int b = base + (int)threadIdx.x;
+    int v = 0;
+    if (b < B) {
+      const int len = cache_len[b];
+      if (len < 0) record_error(err, kErrInvalid);
+      else if (len >= s_max) record_error(err, kErrCapacity);
+      else v = Hkv * ((len + 1 + 127) / 128);
+    }
+    int x = v;  // inclusive scan within the warp, then over the warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+      int u = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, u, o);
+        if (lane >= o) u += y;
+      }
+      wsum[lane] = u;
+    }
+    __syncthreads();
+    if (b < B) plan[b] = carry + (wid > 0 ? wsum[wid - 1] : 0) + x - v;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += wsum[nw - 1];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) plan[B] = carry;
+  for (int i = threadIdx.x; i < B * Hkv; i += blockDim.x) counters[i] = 0;
 }
 
-int decode_splits(int s_max) { return (s_max + kD4Split - 1) / kD4Split; }
+// Scratch of one decode call: partial slots (rows + CTAs, G heads each), the tile plan,
+// the rows' merge tickets.
+static size_t d4_part_floats(int B, int Hq) { return ((size_t)B * Hq + (size_t)kD4MaxCtas * 16) * kD4PartFloats; }
+static size_t d4_plan_ints(int B) { return ((size_t)B + 1 + 3) & ~(size_t)3; }
 
-size_t decode_partial_bytes(int B, int Hq, int s_max) {
-  return (size_t)B * Hq * decode_splits(s_max) * (kHeadDim + 2) * sizeof(float);
+size_t decode_partial_bytes(int B, int Hq, int Hkv) {
+  return d4_part_floats(B, Hq) * sizeof(float) + (d4_plan_ints(B) + (size_t)B * Hkv) * sizeof(int) + 256;
 }
 
 // qkv: [B][ldqkv] with the Hq query heads at the start of each row; with q_hilo the row
 // holds 2 * Hq heads instead, for group g the G rows q_hi then the G rows q_lo
 // (G <= 8 only).
+// scratch: decode_partial_bytes(B, Hq, Hkv) bytes, 16-byte aligned. plan_ready: the
+// scratch already holds this call's tile plan (same cache_len, B, Hkv, s_max and scratch,
+// written by an earlier launch on the stream), so the plan kernel is skipped.
 int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv, const int* cache_len,
-                            const uint16_t* ck, const uint16_t* cv, int s_max, float* part, uint16_t* out,
-                            long long ldo, int* err, cudaStream_t s, bool o_f16, bool q_hilo, long long o_lo) {
+                            const uint16_t* ck, const uint16_t* cv, int s_max, float* scratch, uint16_t* out,
+                            long long ldo, int* err, cudaStream_t s, bool o_f16, bool q_hilo, long long o_lo,
+                            bool plan_ready) {
   if (B <= 0) return 0;
   const int G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) {
@@ -833,7 +964,6 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
                    (long long)B * Hkv * s_max);
     return -2;
   }
-  const int n_splits = decode_splits(s_max);
   if (q_hilo && G > 8) {
     set_last_error("attention decode: the hi/lo query layout needs at most 8 query heads per KV group");
     return -2;
@@ -851,8 +981,11 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     set_last_error("attention decode: cannot encode the KV-cache tensor maps");
     return -6;
   }
-  const long long items = (long long)B * Hkv * n_splits;
-  const int grid = (int)(items < num_sms() ? items : num_sms());
+  const int grid = num_sms() < kD4MaxCtas ? num_sms() : kD4MaxCtas;
+  float* part = scratch;
+  int* plan = reinterpret_cast<int*>(scratch + d4_part_floats(B, Hq));
+  int* counters = plan + d4_plan_ints(B);
+  if (!plan_ready) q3_launch(attn_decode_plan_kernel, 1, 1024, 0, s, cache_len, B, Hkv, s_max, plan, counters, err);
   DecodeMergeOut mo;
   mo.out = out;
   mo.ldo = ldo;
@@ -864,7 +997,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
   case GG * 2 + HL:                                                                                               \
     if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG, HL>), kD4Smem)) return -6;       \
     q3_launch(attn_decode_tc_kernel<GG, HL>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,  \
-              s_max, n_splits, part, err);                                                                        \
+              s_max, plan, part, counters, mo, err);                                                              \
     break;
     Q3_D4_CASE(1, false)
     Q3_D4_CASE(2, false)
@@ -877,7 +1010,6 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     Q3_D4_CASE(8, true)
 #undef Q3_D4_CASE
   }
-  q3_launch(attn_decode_merge_kernel, B * Hq, kHeadDim, 0, s, part, Hq, n_splits, mo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_last_error("attention decode launch failed: %s", cudaGetErrorString(e));
@@ -887,13 +1019,14 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
 }
 
 // ----------------------------------------------------------------------------
-// Decode attention without caller scratch. The split partials live in a fixed
-// device array of this library instead of a caller workspace, for callers that
-// cannot allocate device memory. Its capacity is kStaticDecodeFloats floats
-// (12 MiB): B * Hq * ceil(s_max / 256) * 130 floats must fit. The array's device
-// address is looked up on the host once per device (with that device current);
-// every call shares the array, so calls that overlap on the GPU race. Each call
-// rewrites every partial it reads, so nothing has to be cleared between calls.
+// Decode attention without caller scratch. The partials, the tile plan and the merge
+// tickets live in a fixed device array of this library instead of a caller workspace,
+// for callers that cannot allocate device memory. Its capacity is kStaticDecodeFloats
+// floats (12 MiB): decode_partial_bytes(B, Hq, Hkv) must fit (B * Hq up to about 20000).
+// The array's device address is looked up on the host once per device (with that device
+// current); every call shares the array, so calls that overlap on the GPU race. Each
+// call writes its plan and clears its tickets before use, and every partial it reads is
+// written by that same call, so nothing has to be cleared between calls.
 // ----------------------------------------------------------------------------
 constexpr size_t kStaticDecodeFloats = (size_t)3 << 20;
 static __device__ __align__(256) float g_decode_scratch[kStaticDecodeFloats];
@@ -906,11 +1039,10 @@ size_t static_decode_scratch_bytes() { return kStaticDecodeFloats * sizeof(float
 int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, int Hq, int Hkv,
                                    const int* cache_len, const uint16_t* ck, const uint16_t* cv, int s_max,
                                    uint16_t* out, long long ldo, int* err, cudaStream_t s, bool o_f16) {
-  const size_t need = decode_partial_bytes(B, Hq, s_max);
+  const size_t need = decode_partial_bytes(B, Hq, Hkv);
   if (need > kStaticDecodeFloats * sizeof(float)) {
-    set_last_error("attention_decode_noalloc: B=%d, Hq=%d, s_max=%d need %zu bytes of split scratch; the "
-                   "static scratch holds %zu bytes (B * Hq * ceil(s_max/256) must be <= %zu)",
-                   B, Hq, s_max, need, kStaticDecodeFloats * sizeof(float), kStaticDecodeFloats / (kHeadDim + 2));
+    set_last_error("attention_decode_noalloc: B=%d, Hq=%d, Hkv=%d need %zu bytes of scratch; the static scratch "
+                   "holds %zu bytes", B, Hq, Hkv, need, kStaticDecodeFloats * sizeof(float));
     return -5;
   }
   int dev = 0;
@@ -933,7 +1065,7 @@ int launch_attention_decode_static(const uint16_t* qkv, long long ldqkv, int B, 
     ptr = g_static_ptr[dev];
   }
   return launch_attention_decode(qkv, ldqkv, B, Hq, Hkv, cache_len, ck, cv, s_max, ptr, out, ldo, err, s, o_f16,
-                                 false, 0);
+                                 false, 0, false);
 }
 
 }  // namespace q3

@@ -9,8 +9,8 @@
 // on the MMA's 128-row side (swap form): tile = 128 output features x BN tokens.
 //
 // Design (sm_100a):
-//   * grid = feature tiles x S; the S CTAs of one feature tile form a cluster and each
-//     takes a contiguous range of the K blocks (64 wide);
+//   * grid = feature tiles x S; the S CTAs of one feature tile form a cluster (up to 16)
+//     and each takes a contiguous range of the K blocks (64 wide); two CTAs fit on an SM;
 //   * warp 0: TMA producer (weights 128 x 64 and tokens BN x 64 per K block, 128-byte
 //     swizzle; the weight loads of the first stages precede the grid-dependency
 //     wait, since no kernel of the call writes weights); warp 1: one thread issues
@@ -22,8 +22,10 @@
 //     ld.shared::cluster and applies the epilogue: plain store, residual add, SwiGLU, or
 //     per-head QK RMSNorm + rotate-half RoPE + KV-cache write;
 //   * residual projections can also produce the RMSNorm of their whole output (the
-//     norm that follows them in the block): every cluster stores its tile, takes a
-//     ticket, and the cluster holding the last ticket normalises all token rows;
+//     norm that follows them in the block): every warp writes the sum of squares of
+//     its token's 128 features, all CTAs (co-resident: one wave) meet at a grid-wide
+//     barrier, and each warp then adds the tiles' sums of its token in tile order and
+//     normalises the features it still holds in registers;
 //   * every mbarrier wait is bounded; cluster barriers are executed by every thread on
 //     every path, so an expired wait cannot leave a peer CTA waiting.
 #include <cstdio>
@@ -39,12 +41,14 @@ int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long c
 namespace {
 
 constexpr int kSkThreads = 192;
-constexpr int kSkMaxSplits = 8;
+constexpr int kSkMaxSplits = 16;  // cluster size: 16 is the non-portable maximum on sm_100
+constexpr int kSkPre = 4;        // tokens per epilogue warp whose side operands are prefetched
 constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 of K, bf16
 
 // HILO: the activation operand holds 2M rows, row t = hi(a_t) and row M + t = lo(a_t)
-// (a = hi + lo to about twice the type's precision); the MMA's N covers both and the
-// accumulator columns t and M + t are added before the split sum.
+// (a = hi + lo to about twice the type's precision). Two TMA boxes of BN rows put the hi
+// rows at tile rows [0, BN) and the lo rows at [BN, 2 BN), so the MMA's N = 2 BN covers
+// both and accumulator columns t and BN + t (32-aligned chunks) are added in registers.
 // The ring is sized so that two CTAs fit on an SM (at most ~110 KB each): a CTA keeps
 // its shared memory through the split reduction at its end, and the next projection's
 // CTAs, which prefetch their weights before the grid-dependency wait, can then start
@@ -81,13 +85,49 @@ struct SkParams {
   long long out_lo;   // SwiGLU: > 0: also write lo(out) this many elements after each hi value
   int N;
   float norm_eps;
-  int* ticket;
+  int* ticket;  // grid barrier of the fused norm: [0] arrivals (0 between launches), [1] generation
+  float* ssq;   // fused norm: per-tile sums of squares [N / 128][64]
   QKRopeArgs qk;
   int f16;  // operands fp16 (else bf16); the SwiGLU and fused-norm outputs are fp16 too
   int* err;
 };
 
 }  // namespace
+
+// Barrier of all n CTAs of the grid, called by one thread per CTA after a CTA-level
+// barrier (every CTA of the grid is resident: the launch is one wave). The arrival is a
+// release at GPU scope (cumulative over the writes the CTA barrier ordered before it),
+// the wait an acquire. bar[0] counts arrivals and is back at 0 after each use; bar[1] is
+// a generation that the last arrival advances. Bounded wait: false (and kErrTimeout).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ bool grid_barrier(int* bar, int n, int* err) {
+  const int g0 = ld_acquire_gpu(bar + 1);  // cannot advance before this CTA arrives
+  if (atom_add_acq_rel_gpu(bar, 1) == n - 1) {
+    bar[0] = 0;
+    atom_add_acq_rel_gpu(bar + 1, 1);  // releases the reset and everything before it
+    return true;
+  }
+  const unsigned long long t0 = global_ns();
+  while (ld_acquire_gpu(bar + 1) == g0) {
+    if (global_ns() - t0 > kWaitLimitNs) {
+      record_error(err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+// The 4 epilogue warps (2-5) only.
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 template <int BN, bool HILO>
 __global__ void __launch_bounds__(kSkThreads, 2)
@@ -102,7 +142,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   uint64_t* done = empty + kSkStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_last = s_abort + 1;
+  volatile int* s_last = s_abort + 1;  // the fused norm's grid barrier completed
   float* red = reinterpret_cast<float*>(smem);  // [BN][128] partial sums, over the stages once the MMAs are done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,6 +168,8 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       mbar_arrive_expect_tx(&full[i], C::STAGE);
       tma_load_2d(smem + i * C::STAGE, &tmP, &full[i], (kb0 + i) * 64, tile * 128);
     }
+    // the split's remaining weight blocks into L2, so that their ring loads hit L2
+    for (int i = p_pre; i < nkb; ++i) tma_prefetch_l2_2d(&tmP, (kb0 + i) * 64, tile * 128);
   }
   pdl_wait();
   pdl_trigger();
@@ -135,6 +177,34 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // epilogue warps 2-5 of every CTA: warp ew of the cluster finishes tokens ew + i enw
+  const int ew = (int)rank * 4 + (warp - 2);
+  const int enw = 4 * g.S;
+  float pre_a[kSkPre][4] = {};
+  float2 pre_c0[kSkPre] = {}, pre_c1[kSkPre] = {};
+  int pre_pos[kSkPre] = {};
+  float wn[4] = {0.f, 0.f, 0.f, 0.f};  // QK-norm weights (kEpiQKRope), fused-norm weights (norm_out)
+  float keep[kSkPre][4] = {};          // fused norm: the output values of the prefetched tokens
+  // residual values (kEpiResid), or position and rotary factors (kEpiQKRope) of token t
+  auto load_side = [&](int t, float(&a)[4], float2& c0, float2& c1, int& pos) {
+    if (g.epi == kEpiResid) {
+      const long long base = (long long)t * g.ldr + (long long)tile * 128 + lane;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        a[j] = g.resid_f32 ? static_cast<const float*>(g.resid)[base + 32 * j]
+                           : __uint_as_float((uint32_t)static_cast<const uint16_t*>(g.resid)[base + 32 * j] << 16);
+    } else if (g.epi == kEpiQKRope) {
+      const QKRopeArgs& q = g.qk;
+      const int b = t / q.T;
+      pos = q.pos_base[b] + (t - b * q.T);
+      c0 = c1 = make_float2(0.f, 0.f);
+      if (tile < q.Hq + q.Hkv && pos >= 0 && pos < q.s_max && pos < q.max_pos) {
+        c0 = *reinterpret_cast<const float2*>(q.rope + ((long long)pos * 64 + lane) * 2);
+        c1 = *reinterpret_cast<const float2*>(q.rope + ((long long)pos * 64 + 32 + lane) * 2);
+      }
+    }
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -145,15 +215,13 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const int st = i % kSkStages;
         const uint32_t ph = (uint32_t)(i / kSkStages) & 1u;
         uint8_t* sp = smem + st * C::STAGE;
-        if (i < p_pre) {  // weights already on their way; the stage expects both halves
-          tma_load_2d(sp + kSkPBytes, &tmQ, &full[st], (kb0 + i) * 64, 0);
-          ++issued;
-          continue;
+        if (i >= p_pre) {  // else the weights are on their way; the stage expects all boxes
+          if (*s_abort || !mbar_wait(&empty[st], ph ^ 1u, g.err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[st], C::STAGE);
+          tma_load_2d(sp, &tmP, &full[st], (kb0 + i) * 64, tile * 128);
         }
-        if (*s_abort || !mbar_wait(&empty[st], ph ^ 1u, g.err)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[st], C::STAGE);
-        tma_load_2d(sp, &tmP, &full[st], (kb0 + i) * 64, tile * 128);
         tma_load_2d(sp + kSkPBytes, &tmQ, &full[st], (kb0 + i) * 64, 0);
+        if (HILO) tma_load_2d(sp + kSkPBytes + BN * 128, &tmQ, &full[st], (kb0 + i) * 64, g.M);
         ++issued;
       }
       if (!ok) {
@@ -184,6 +252,22 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       mma_commit(done);
     }
   } else {
+    // epilogue operands that do not depend on the product (residual rows, positions,
+    // rotary factors, QK-norm weights), loaded while the weights stream and the MMAs run
+#pragma unroll
+    for (int i = 0; i < kSkPre; ++i) {
+      const int t = ew + i * enw;
+      if (t < g.M) load_side(t, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
+    }
+    if (g.epi == kEpiQKRope && tile < g.qk.Hq + g.qk.Hkv) {
+      const uint16_t* wsrc = tile < g.qk.Hq ? g.qk.q_norm : g.qk.k_norm;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)wsrc[32 * j + lane] << 16);
+    }
+    if (g.norm_out) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)g.norm_w[tile * 128 + 32 * j + lane] << 16);
+    }
     // ---------------------------------------------------------- accumulator -> smem
     const int quad = warp & 3;  // tensor-memory lanes [32 quad, 32 quad + 32)
     bool ok = mbar_wait(done, 0, g.err);
@@ -191,30 +275,33 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     tc_fence_after();
     const int f = quad * 32 + lane;
     const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16);
-    // column j < M: token j (its hi half with HILO); column M + t: token t's lo half,
-    // added after its hi value (columns are visited in increasing order)
+    // column j < M: token j (its hi half with HILO); with HILO, column BN + j: its lo half
     const int M = g.M;
-    auto put = [&](int j, uint32_t r) {
-      const float v = ok ? __uint_as_float(r) : 0.f;
-      if (j < M) red[j * 128 + f] = v;
-      else if (HILO && j < 2 * M) red[(j - M) * 128 + f] += v;
-    };
-    if constexpr (C::NQ == 16) {
-      uint32_t r[16];
+    if constexpr (BN == 16) {
+      uint32_t r[16], rl[16];
       tmem_ld16(taddr, r);
+      if constexpr (HILO) tmem_ld16(taddr + 16, rl);
       tmem_wait_ld_regs16(r);
+      if constexpr (HILO) tmem_wait_ld_regs16(rl);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) put(j, r[j]);
+      for (int j = 0; j < 16; ++j) {
+        const float v = HILO ? __uint_as_float(r[j]) + __uint_as_float(rl[j]) : __uint_as_float(r[j]);
+        if (j < M) red[j * 128 + f] = ok ? v : 0.f;
+      }
     } else {
-      const int used = HILO ? 2 * M : M;
 #pragma unroll 1
-      for (int c = 0; c < C::NQ / 32; ++c) {
-        if (c * 32 >= used) break;  // warp-uniform
-        uint32_t r[32];
+      for (int c = 0; c < BN / 32; ++c) {
+        if (c * 32 >= M) break;  // warp-uniform
+        uint32_t r[32], rl[32];
         tmem_ld32(taddr + c * 32, r);
+        if constexpr (HILO) tmem_ld32(taddr + BN + c * 32, rl);
         tmem_wait_ld_regs(r);
+        if constexpr (HILO) tmem_wait_ld_regs(rl);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) put(c * 32 + j, r[j]);
+        for (int j = 0; j < 32; ++j) {
+          const float v = HILO ? __uint_as_float(r[j]) + __uint_as_float(rl[j]) : __uint_as_float(r[j]);
+          if (c * 32 + j < M) red[(c * 32 + j) * 128 + f] = ok ? v : 0.f;
+        }
       }
     }
   }
@@ -224,54 +311,47 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 
   if (warp >= 2 && !*s_abort) {
     // -------------------------------------------------- split sum + epilogue, one warp per token
-    const int ew = (int)rank * 4 + (warp - 2);
-    uint32_t rbase[kSkMaxSplits];
+    // split s's partial of (token t, feature f) in CTA s: the mapa (a volatile asm after
+    // the barrier) keeps the loads, which no longer change, below the barrier
+    const uint32_t red0 = smem_u32(red);
+    auto sum_token = [&](int t, float(&v)[4]) {
 #pragma unroll
-    for (int s = 0; s < kSkMaxSplits; ++s) rbase[s] = s < g.S ? mapa_shared(red, (uint32_t)s) : 0u;
-    for (int t = ew; t < g.M; t += 4 * g.S) {
-      float part[kSkMaxSplits][4];
+      for (int j = 0; j < 4; ++j) v[j] = 0.f;
+#pragma unroll 4
+      for (int s = 0; s < g.S; ++s) {
+        const uint32_t base = mapa_shared_addr(red0 + (uint32_t)((t * 128 + lane) * 4), (uint32_t)s);
 #pragma unroll
-      for (int s = 0; s < kSkMaxSplits; ++s)
-        if (s < g.S)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) part[s][j] = ld_cluster_f32(rbase[s] + (uint32_t)((t * 128 + 32 * j + lane) * 4));
-      float v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < kSkMaxSplits; ++s)
-        if (s < g.S)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) v[j] += part[s][j];
+        for (int j = 0; j < 4; ++j) v[j] += ld_cluster_f32_ro(base + 128u * j);  // split order: deterministic
+      }
+    };
+    auto finish = [&](int i, int t, float(&v)[4], const float(&a)[4], float2 c0, float2 c1, int pos) {
       if (g.epi == kEpiQKRope) {
         // slot = head of the fused QKV row: q heads, then k heads, then v heads
-        const QKRopeArgs& a = g.qk;
+        const QKRopeArgs& q = g.qk;
         const int slot = tile;
-        const int b = t / a.T;
-        const int pos = a.pos_base[b] + (t - b * a.T);
-        if (pos < 0 || pos >= a.s_max || pos >= a.max_pos) {
+        const int b = t / q.T;
+        if (pos < 0 || pos >= q.s_max || pos >= q.max_pos) {
           if (lane == 0) record_error(g.err, kErrCapacity);
-          continue;
+          return;
         }
-        if (slot >= a.Hq + a.Hkv) {  // value head: straight to the cache
-          uint16_t* dst = a.cv + (((long long)b * a.Hkv + (slot - a.Hq - a.Hkv)) * a.s_max + pos) * 128;
+        if (slot >= q.Hq + q.Hkv) {  // value head: straight to the cache
+          uint16_t* dst = q.cv + (((long long)b * q.Hkv + (slot - q.Hq - q.Hkv)) * q.s_max + pos) * 128;
 #pragma unroll
           for (int j = 0; j < 4; ++j) dst[32 * j + lane] = to_bf16_bits(v[j]);
-          continue;
+          return;
         }
-        const bool is_q = slot < a.Hq;
-        const uint16_t* wn = is_q ? a.q_norm : a.k_norm;
+        const bool is_q = slot < q.Hq;
         const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
-        const float r = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
+        const float r = rsqrtf(ss * (1.0f / 128.0f) + q.eps);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] *= r * __uint_as_float((uint32_t)wn[32 * j + lane] << 16);
+        for (int j = 0; j < 4; ++j) v[j] *= r * wn[j];
         // rotation pairs (d, d + 64): d = lane (v[0], v[2]) and d = 32 + lane (v[1], v[3])
-        const float2 c0 = *reinterpret_cast<const float2*>(a.rope + ((long long)pos * 64 + lane) * 2);
-        const float2 c1 = *reinterpret_cast<const float2*>(a.rope + ((long long)pos * 64 + 32 + lane) * 2);
         const float o[4] = {v[0] * c0.x - v[2] * c0.y, v[1] * c1.x - v[3] * c1.y, v[0] * c0.y + v[2] * c0.x,
                             v[1] * c1.y + v[3] * c1.x};  // dims lane, 32 + lane, 64 + lane, 96 + lane
-        if (is_q && a.q2) {
+        if (is_q && q.q2) {
           // hi/lo rows of the decode attention: group grp, head j of the group
-          const int G = a.Hq / a.Hkv, grp = slot / G, j = slot - grp * G;
-          uint16_t* hi = a.q2 + (long long)t * a.ldq2 + ((long long)grp * 2 * G + j) * 128;
+          const int G = q.Hq / q.Hkv, grp = slot / G, jh = slot - grp * G;
+          uint16_t* hi = q.q2 + (long long)t * q.ldq2 + ((long long)grp * 2 * G + jh) * 128;
           uint16_t* lo = hi + (long long)G * 128;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -279,10 +359,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             hi[32 * i + lane] = h;
             lo[32 * i + lane] = to_bf16_bits(o[i] - __uint_as_float((uint32_t)h << 16));
           }
-          continue;
+          return;
         }
         uint16_t* dst = is_q ? static_cast<uint16_t*>(g.out) + (long long)t * g.ldo + (long long)slot * 128
-                             : a.ck + (((long long)b * a.Hkv + (slot - a.Hq)) * a.s_max + pos) * 128;
+                             : q.ck + (((long long)b * q.Hkv + (slot - q.Hq)) * q.s_max + pos) * 128;
 #pragma unroll
         for (int i = 0; i < 4; ++i) dst[32 * i + lane] = to_bf16_bits(o[i]);
       } else if (g.epi == kEpiSwiglu) {
@@ -293,96 +373,101 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         for (int j = 0; j < 4; ++j) {
           const float u = __shfl_down_sync(0xffffffffu, v[j], 16);
           if (lane < 16) {
-            const float a = silu_f(v[j]) * u;
-            const uint16_t hi = to_op_bits(f16, a);
+            const float h = silu_f(v[j]) * u;
+            const uint16_t hi = to_op_bits(f16, h);
             dst[16 * j + lane] = hi;
-            if (g.out_lo) dst[g.out_lo + 16 * j + lane] = to_op_bits(f16, a - op_bits_to_f32(f16, hi));
+            if (g.out_lo) dst[g.out_lo + 16 * j + lane] = to_op_bits(f16, h - op_bits_to_f32(f16, hi));
           }
         }
       } else {
         const long long col = (long long)tile * 128 + lane;
         if (g.epi == kEpiResid) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            v[j] += g.resid_f32 ? static_cast<const float*>(g.resid)[(long long)t * g.ldr + col + 32 * j]
-                                : __uint_as_float((uint32_t)static_cast<const uint16_t*>(
-                                                      g.resid)[(long long)t * g.ldr + col + 32 * j]
-                                                  << 16);
+          for (int j = 0; j < 4; ++j) v[j] += a[j];
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          if (g.out_f32) static_cast<float*>(g.out)[(long long)t * g.ldo + col + 32 * j] = v[j];
-          else static_cast<uint16_t*>(g.out)[(long long)t * g.ldo + col + 32 * j] = to_bf16_bits(v[j]);
+          if (g.out_f32) {
+            static_cast<float*>(g.out)[(long long)t * g.ldo + col + 32 * j] = v[j];
+          } else {
+            const uint16_t h = to_bf16_bits(v[j]);
+            static_cast<uint16_t*>(g.out)[(long long)t * g.ldo + col + 32 * j] = h;
+            v[j] = __uint_as_float((uint32_t)h << 16);  // the norm sees the stored value
+          }
+        }
+        if (g.norm_out) {
+          const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
+          if (lane == 0) g.ssq[tile * 64 + t] = ss;
+#pragma unroll
+          for (int k = 0; k < kSkPre; ++k)
+            if (k == i)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) keep[k][j] = v[j];
         }
       }
+    };
+#pragma unroll
+    for (int i = 0; i < kSkPre; ++i) {
+      const int t = ew + i * enw;
+      if (t < g.M) {
+        float v[4];
+        sum_token(t, v);
+        finish(i, t, v, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
+      }
+    }
+    for (int t = ew + kSkPre * enw; t < g.M; t += enw) {  // tokens beyond the prefetched ones
+      float a[4], v[4];
+      float2 c0, c1;
+      int pos = 0;
+      load_side(t, a, c0, c1, pos);
+      sum_token(t, v);
+      finish(kSkPre, t, v, a, c0, c1, pos);
     }
   }
 
-  if (g.norm_out) {
-    // ------------------------------------------ RMSNorm of the whole output, last cluster
-    __threadfence();  // this thread's output stores, visible to the whole GPU
-    __syncwarp();
-    cluster_sync();
-    if (rank == 0 && threadIdx.x == 0) {
-      const int prev = atomicAdd(g.ticket, 1);
-      const uint32_t last = prev == (int)(gridDim.x / (unsigned)g.S) - 1 ? 1u : 0u;
-      for (int s = 0; s < g.S; ++s) st_cluster_u32(mapa_shared((const void*)s_last, (uint32_t)s), last);
-    }
-    __syncwarp();
-    cluster_sync();
-    if (*s_last) {
-      __threadfence();  // the other clusters' stores (their fences precede their tickets)
-      const int gw = (int)rank * (kSkThreads / 32) + warp;
-      const int nw = g.S * (kSkThreads / 32);
-      const int N = g.N;
-      for (int t = gw; t < g.M; t += nw) {
+  if (g.norm_out && warp >= 2) {
+    // ------------------------------------------------ RMSNorm of the whole output rows
+    epi_bar_sync();  // the epilogue warps' output and sum-of-squares stores precede the arrival
+    if (threadIdx.x == 64) *s_last = grid_barrier(g.ticket, (int)gridDim.x, g.err) ? 1 : 0;
+    epi_bar_sync();
+    if (*s_last && !*s_abort) {
+      const int n_tiles = (int)(gridDim.x / (unsigned)g.S);
+      const bool f16 = g.f16 != 0;
+      const long long col = (long long)tile * 128 + lane;
+      // sum over the tiles in tile order (L2 reads: other SMs wrote them)
+      auto tiles_ss = [&](int t) {
         float ss = 0.f;
-        for (int col = lane * 8; col < N; col += 256) {
-          float x[8];
-          if (g.out_f32) {
-            const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(g.out) + (long long)t * g.ldo + col);
-            const float4 a = p[0], b = p[1];
-            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-          } else {
-            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.out) + (long long)t * g.ldo + col);
-            x[0] = bf16_lo(a.x); x[1] = bf16_hi(a.x); x[2] = bf16_lo(a.y); x[3] = bf16_hi(a.y);
-            x[4] = bf16_lo(a.z); x[5] = bf16_hi(a.z); x[6] = bf16_lo(a.w); x[7] = bf16_hi(a.w);
-          }
+#pragma unroll 8
+        for (int q = 0; q < n_tiles; ++q) ss += __ldcg(g.ssq + q * 64 + t);
+        return ss;
+      };
+      auto normalise = [&](int t, float ss, const float(&x)[4]) {
+        const float r = rsqrtf(ss / (float)g.N + g.norm_eps);
+        uint16_t* dst = g.norm_out + (long long)t * g.ld_norm + col;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) ss += x[j] * x[j];
+        for (int j = 0; j < 4; ++j) {
+          const float a = x[j] * r * wn[j];
+          const uint16_t hi = to_op_bits(f16, a);
+          dst[32 * j] = hi;
+          if (g.norm_lo) dst[g.norm_lo + 32 * j] = to_op_bits(f16, a - op_bits_to_f32(f16, hi));
         }
-        ss = warp_sum(ss);
-        const float r = rsqrtf(ss / (float)N + g.norm_eps);
-        for (int col = lane * 8; col < N; col += 256) {
-          float x[8];
-          if (g.out_f32) {
-            const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(g.out) + (long long)t * g.ldo + col);
-            const float4 a = p[0], b = p[1];
-            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-          } else {
-            const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(g.out) + (long long)t * g.ldo + col);
-            x[0] = bf16_lo(a.x); x[1] = bf16_hi(a.x); x[2] = bf16_lo(a.y); x[3] = bf16_hi(a.y);
-            x[4] = bf16_lo(a.z); x[5] = bf16_hi(a.z); x[6] = bf16_lo(a.w); x[7] = bf16_hi(a.w);
-          }
-          const uint4 w = *reinterpret_cast<const uint4*>(g.norm_w + col);
-          const bool f16 = g.f16 != 0;
-          const float wv[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                               bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-          uint32_t hi[4], lo[4];
+      };
+      float ssk[kSkPre];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float a0 = x[2 * j] * r * wv[2 * j], a1 = x[2 * j + 1] * r * wv[2 * j + 1];
-            hi[j] = pack_op_x2(f16, a0, a1);
-            lo[j] = pack_op_x2(f16, a0 - op_bits_to_f32(f16, (uint16_t)(hi[j] & 0xFFFFu)),
-                               a1 - op_bits_to_f32(f16, (uint16_t)(hi[j] >> 16)));
-          }
-          uint16_t* dst = g.norm_out + (long long)t * g.ld_norm + col;
-          *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          if (g.norm_lo) *reinterpret_cast<uint4*>(dst + g.norm_lo) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
+      for (int i = 0; i < kSkPre; ++i) ssk[i] = ew + i * enw < g.M ? tiles_ss(ew + i * enw) : 0.f;
+#pragma unroll
+      for (int i = 0; i < kSkPre; ++i) {
+        const int t = ew + i * enw;
+        if (t < g.M) normalise(t, ssk[i], keep[i]);
       }
-      // every cluster has taken its ticket: reset it for the next launch
-      if (rank == 0 && threadIdx.x == 0) atomicExch(g.ticket, 0);
+      for (int t = ew + kSkPre * enw; t < g.M; t += enw) {  // tokens past the kept ones: re-read
+        float x[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          x[j] = g.out_f32 ? static_cast<const float*>(g.out)[(long long)t * g.ldo + col + 32 * j]
+                           : __uint_as_float((uint32_t)static_cast<const uint16_t*>(g.out)[(long long)t * g.ldo + col + 32 * j] << 16);
+        normalise(t, tiles_ss(t), x);
+      }
     }
   }
   __syncwarp();
@@ -440,10 +525,29 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   using C = SkCfg<BN, HILO>;
   if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)C::SMEM)) return -6;
   const int n_tiles = d.N / 128, k_blocks = d.K / 64;
-  // splits: as many as fill the SMs in one wave of co-resident clusters
+  // splits: as many as fit in one wave of co-resident clusters (two CTAs per SM; clusters
+  // above 8 CTAs need the non-portable size, allowed once per kernel and device)
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> wide;  // (kernel, device) allowed 16-CTA clusters
+  int max_c = 8;
+  {
+    const void* func = reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(mu);
+    bool ok = false;
+    for (const auto& e : wide) ok = ok || (e.first == func && e.second == dev);
+    if (!ok && cudaFuncSetAttribute(gemm_skinny_kernel<BN, HILO>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                   cudaSuccess) {
+      wide.emplace_back(func, dev);
+      ok = true;
+    }
+    cudaGetLastError();
+    if (ok) max_c = kSkMaxSplits;
+  }
   int S = 1;
-  for (int c = kSkMaxSplits; c >= 1; --c) {
-    if ((long long)n_tiles * c > num_sms() || c > k_blocks) continue;
+  for (int c = max_c; c >= 1; --c) {
+    if ((long long)n_tiles * c > 2LL * num_sms() || c > k_blocks) continue;
     if (c > 1 && !clusters_fit<BN, HILO>(c, n_tiles)) continue;
     S = c;
     break;
@@ -452,7 +556,7 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   S = (k_blocks + kpb - 1) / kpb;  // every split gets at least one K block
   CUtensorMap tmP, tmQ;
   if (make_tmap_2d(&tmP, d.W, d.N, d.K, d.ldw, 128) != 0 ||
-      make_tmap_2d(&tmQ, d.A, HILO ? 2LL * d.M : d.M, d.K, d.lda, C::NQ) != 0) {
+      make_tmap_2d(&tmQ, d.A, HILO ? 2LL * d.M : d.M, d.K, d.lda, BN) != 0) {
     set_last_error("skinny gemm: cannot encode the operand tensor maps");
     return -6;
   }
@@ -477,6 +581,7 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   g.N = d.N;
   g.norm_eps = d.norm_eps;
   g.ticket = d.ticket;
+  g.ssq = d.ssq;
   g.qk = d.qk;
   g.f16 = d.f16 ? 1 : 0;
   g.err = err;
@@ -502,8 +607,9 @@ int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err) {
     set_last_error("skinny gemm: unsupported shape M %d N %d K %d", d.M, d.N, d.K);
     return -2;
   }
-  if (d.norm_out && (d.epi != kEpiResid || !d.norm_w || !d.ticket || d.N % 256 != 0)) {
-    set_last_error("skinny gemm: the fused RMSNorm needs the residual epilogue, weights, a ticket and N %% 256 == 0");
+  if (d.norm_out && (d.epi != kEpiResid || !d.norm_w || !d.ticket || !d.ssq || d.N / 128 > num_sms())) {
+    set_last_error("skinny gemm: the fused RMSNorm needs the residual epilogue, weights, a barrier word pair, the "
+                   "sum-of-squares scratch and at most one feature tile per SM");
     return -1;
   }
   if (d.epi == kEpiSwiglu ? false : d.out_lo != 0) {

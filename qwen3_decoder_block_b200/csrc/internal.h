@@ -101,11 +101,15 @@ struct SkinnyDesc {
   long long ldr = 0;
   bool resid_f32 = false;
   bool w_early = false;  // W is final before the previous kernel started (see GemmDesc::p_early)
+  // residual epilogue only: norm_out = RMSNorm(out rows) * norm_w (N features per row),
+  // through a grid-wide barrier on ticket[0..1] (ticket[0] zero before the launch) and
+  // per-tile sums of squares in ssq ([N / 128][64] floats)
   const uint16_t* norm_w = nullptr;
   uint16_t* norm_out = nullptr;
   long long ld_norm = 0;
   float norm_eps = 1e-6f;
   int* ticket = nullptr;
+  float* ssq = nullptr;
   QKRopeArgs qk;
   bool f16 = false;  // as GemmDesc::f16
   // a_hilo: A holds 2M rows, row t = hi(a_t), row M + t = lo(a_t) = round(a_t - hi), both in

@@ -2,7 +2,7 @@
 
 Some callers cannot allocate device memory (an application held to a fixed memory
 budget, a plugin handed tensors but no allocator or workspace). For them the
-library offers qwen3_op_attention_decode_noalloc, whose split scratch is a static
+library offers qwen3_op_attention_decode_noalloc, whose scratch is a static
 device array of the library. This test calls it through the C ABI twice in a row
 and checks each result against the workspace-taking qwen3_op_attention_decode, on
 the decode workload's shapes (B 64, 4097 visible positions). The file is named so
@@ -39,19 +39,21 @@ def test_noalloc_decode_matches_workspace_decode_twice():
         assert_device_ok()
         ref, got = from_gpu_bf16(o_ref), from_gpu_bf16(o_new)
         assert np.isfinite(got).all()
-        # the same kernels with the same split and merge order: only the scratch's
+        # the same kernels with the same tile ranges and merge order: only the scratch's
         # address differs, so the outputs are identical bit for bit
         np.testing.assert_array_equal(o_new.view(torch.int16).cpu().numpy(), o_ref.view(torch.int16).cpu().numpy())
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
-    """B 64, s_max 5889: 64 * 16 * ceil(5889 / 256) = 24576 split partials, above the
-    24197 the static array holds, so the call is refused before launch. The cache is
-    really allocated at that size (1.5 GB), so that the arguments describe valid memory
-    whatever the order of the checks."""
+    """The scratch of a call holds (B * Hkv + 256) partial slots of G heads x 130 floats,
+    the tile plan (B + 1 ints, padded to 4) and B * Hkv merge tickets. With 16 query
+    heads that is 12,583,536 bytes for B 1251, above the 12 MiB static array, so the call
+    is refused before launch; B 1250 (12,575,184 bytes) fits and runs. The cache is
+    really allocated (s_max 8), so that the arguments describe valid memory whatever the
+    order of the checks."""
     import qwen3_decoder_block_b200 as q3
     cfg = q3.config_qwen3_0_6b()
-    B, s_max = 64, 5889
+    B, s_max = 1251, 8
     k, v, kv = kv_cache(cfg, B, s_max)
     qkv = torch.zeros((B, 4096), dtype=torch.bfloat16, device="cuda")
     o = torch.zeros((B, 2048), dtype=torch.bfloat16, device="cuda")
@@ -60,12 +62,13 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
         q3.op_attention_decode_noalloc(cfg, qkv, B, cl, kv, o)
     assert e.value.status == q3.EWORKSPACE
     assert "static scratch" in str(e.value)
-    # one position less fits: 64 * 16 * 23 = 23552 partials
-    k2, v2, kv2 = kv_cache(cfg, B, s_max - 1)
-    k2.zero_()
-    v2.zero_()
+    # one sequence less fits
+    B2 = B - 1
+    k.zero_()
+    v.zero_()
     o.fill_(float("nan"))
-    q3.op_attention_decode_noalloc(cfg, qkv, B, cl, kv2, o)
+    q3.op_attention_decode_noalloc(cfg, qkv[:B2], B2, cl[:B2], kv, o[:B2])
     assert_device_ok()
-    assert bool((o == 0).all())  # one visible key whose value row is zero
-    del k, v, k2, v2
+    assert bool((o[:B2] == 0).all())  # one visible key whose value row is zero
+    assert bool(torch.isnan(o[B2:]).all())  # the refused row count is not exceeded
+    del k, v
