@@ -28,8 +28,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "Qwen3-0.6B prefill & decode tokens/s on 1 B200; % of BF16/HBM roofline"
-# measured DRAM bytes / algorithmic K/V bytes of one decode-attention launch (ncu)
-DECODE_ATTN_TRAFFIC_RATIO = 1.119217 / 1.074004
+# measured DRAM bytes / algorithmic K/V bytes of one decode-attention launch (ncu
+# dram__bytes_read.sum + dram__bytes_write.sum); None until captured for the current kernel
+DECODE_ATTN_TRAFFIC_RATIO = (1107874048 + 3586304) / 1074003968
+DECODE_ATTN_TRAFFIC_SOURCE = ("ncu capture of one attn_decode_tc_kernel launch at B64 x 4097 positions "
+                              "(profiles/attn_decode_B64_ctx4096_layer.md), scaled by positions")
+
 PREFILL_B, PREFILL_T = 4, 2048
 DECODE_B, DECODE_CTX, DECODE_STEPS = 64, 4096, 128
 SEED_PREFILL, SEED_DECODE = 1001, 1002
@@ -436,13 +440,12 @@ def run_decode(q3, torch, args, peaks, gemm_f16=1):
         "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes + w_bytes,
                           "achieved_gbs": (step_bytes + w_bytes) / (step_ms * 1e-3) / 1e9,
                           "frac": (step_bytes + w_bytes) / (step_ms * 1e-3) / 1e9 / hbm},
-        "roofline": {"bound": "hbm", "kernel": "attn_decode (split-KV + merge)", "achieved": achieved, "peak": hbm,
+        "roofline": {"bound": "hbm", "kernel": "attn_decode (plan + stream-K tiles, in-kernel merge)",
+                     "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} hbm copy",
-                     # DRAM bytes of one launch: ncu (dram__bytes_read.sum + dram__bytes_write.sum)
-                     # on attn_decode_tc_kernel at B64 x 4097 positions measured 1.119217 GB for
-                     # 1.074004 GB of K/V; scaled here to this launch's positions
-                     "traffic": kv_bytes / cfg.n_layers * DECODE_ATTN_TRAFFIC_RATIO,
-                     "traffic_source": "ncu capture of one B64 x 4097-position launch, scaled by positions"},
+                     "traffic": (kv_bytes / cfg.n_layers * DECODE_ATTN_TRAFFIC_RATIO
+                                 if DECODE_ATTN_TRAFFIC_RATIO else None),
+                     "traffic_source": DECODE_ATTN_TRAFFIC_SOURCE},
         "kernels": {k: {kk: round(vv, 5) for kk, vv in v.items()} for k, v in kernels.items()},
         "gpu_launches_per_step": len(records) / 8,
     }

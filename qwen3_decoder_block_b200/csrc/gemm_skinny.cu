@@ -10,7 +10,7 @@
 //
 // Design (sm_100a):
 //   * grid = feature tiles x S; the S CTAs of one feature tile form a cluster (up to 16)
-//     and each takes a contiguous range of the K blocks (64 wide); two CTAs fit on an SM;
+//     and each takes a contiguous range of the K blocks (64 wide); one CTA per SM;
 //   * warp 0: TMA producer (weights 128 x 64 and tokens BN x 64 per K block, 128-byte
 //     swizzle; the weight loads of the first stages precede the grid-dependency
 //     wait, since no kernel of the call writes weights); warp 1: one thread issues
@@ -49,16 +49,15 @@ constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 
 // (a = hi + lo to about twice the type's precision). Two TMA boxes of BN rows put the hi
 // rows at tile rows [0, BN) and the lo rows at [BN, 2 BN), so the MMA's N = 2 BN covers
 // both and accumulator columns t and BN + t (32-aligned chunks) are added in registers.
-// The ring is sized so that two CTAs fit on an SM (at most ~110 KB each): a CTA keeps
-// its shared memory through the split reduction at its end, and the next projection's
-// CTAs, which prefetch their weights before the grid-dependency wait, can then start
-// beside it instead of after it.
+// A kernel that allocates tensor memory runs one CTA per SM, so the ring takes up to
+// 200 KB: deep enough that a split's weight blocks (at most 8) are all requested before
+// the grid-dependency wait.
 template <int BN, bool HILO>
 struct SkCfg {
   static constexpr int NQ = HILO ? 2 * BN : BN;  // activation rows per tile = MMA N
   static constexpr uint32_t Q_BYTES = NQ * 64 * 2;
   static constexpr uint32_t STAGE = kSkPBytes + Q_BYTES;
-  static constexpr int STAGES = (int)(((110u << 10) - 1280u) / STAGE) > 8 ? 8 : (int)(((110u << 10) - 1280u) / STAGE);
+  static constexpr int STAGES = (int)(((200u << 10) - 1280u) / STAGE) > 8 ? 8 : (int)(((200u << 10) - 1280u) / STAGE);
   static constexpr uint32_t TMEM_COLS = NQ < 32 ? 32 : NQ;
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;  // + barriers and flags
   static_assert(STAGES >= 3, "ring too shallow");
@@ -130,7 +129,7 @@ __device__ __forceinline__ bool grid_barrier(int* bar, int n, int* err) {
 __device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 template <int BN, bool HILO>
-__global__ void __launch_bounds__(kSkThreads, 2)
+__global__ void __launch_bounds__(kSkThreads, 1)
     gemm_skinny_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                        const SkParams g) {
   using C = SkCfg<BN, HILO>;
@@ -525,7 +524,7 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   using C = SkCfg<BN, HILO>;
   if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)C::SMEM)) return -6;
   const int n_tiles = d.N / 128, k_blocks = d.K / 64;
-  // splits: as many as fit in one wave of co-resident clusters (two CTAs per SM; clusters
+  // splits: as many as fit in one wave of co-resident clusters (one CTA per SM; clusters
   // above 8 CTAs need the non-portable size, allowed once per kernel and device)
   static std::mutex mu;
   static std::vector<std::pair<const void*, int>> wide;  // (kernel, device) allowed 16-CTA clusters
@@ -547,7 +546,7 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   }
   int S = 1;
   for (int c = max_c; c >= 1; --c) {
-    if ((long long)n_tiles * c > 2LL * num_sms() || c > k_blocks) continue;
+    if ((long long)n_tiles * c > num_sms() || c > k_blocks) continue;
     if (c > 1 && !clusters_fit<BN, HILO>(c, n_tiles)) continue;
     S = c;
     break;
