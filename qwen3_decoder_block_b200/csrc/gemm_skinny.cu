@@ -15,7 +15,7 @@
 //     swizzle; the weight loads of the first stages precede the grid-dependency
 //     wait, since no kernel of the call writes weights); warp 1: one thread issues
 //     tcgen05.mma (M = 128, N = BN, K = 16) into one fp32 accumulator in tensor memory;
-//     warps 2-5: epilogue;
+//     warps 2-5 read the accumulator; all 8 warps then share the tokens' epilogues;
 //   * after the last MMA each CTA copies its accumulator to shared memory as
 //     [token][feature]; after a cluster barrier, token t is finished by one warp of the
 //     cluster, which adds the S partials in split order (deterministic) with
@@ -40,7 +40,7 @@ int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long c
 
 namespace {
 
-constexpr int kSkThreads = 192;
+constexpr int kSkThreads = 256;  // TMA warp, MMA warp, 4 accumulator warps, 2 more epilogue warps
 constexpr int kSkMaxSplits = 16;  // cluster size: 16 is the non-portable maximum on sm_100
 constexpr int kSkPre = 4;        // tokens per epilogue warp whose side operands are prefetched
 constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 of K, bf16
@@ -125,8 +125,8 @@ __device__ __forceinline__ bool grid_barrier(int* bar, int n, int* err) {
   return true;
 }
 
-// The 4 epilogue warps (2-5) only.
-__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+// All warps of the CTA, on the epilogue path.
+__device__ __forceinline__ void epi_bar_sync() { asm volatile("bar.sync 2, %0;" ::"n"(kSkThreads) : "memory"); }
 
 template <int BN, bool HILO>
 __global__ void __launch_bounds__(kSkThreads, 1)
@@ -177,9 +177,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // epilogue warps 2-5 of every CTA: warp ew of the cluster finishes tokens ew + i enw
-  const int ew = (int)rank * 4 + (warp - 2);
-  const int enw = 4 * g.S;
+  // warp ew = 8 rank + warp of the cluster finishes tokens ew + i enw; warps 2-7 load the
+  // side operands of their first kSkPre tokens while the MMAs run (npre), warps 0-1 (busy
+  // as producer and issuer then) load theirs when they get to them
+  const int ew = (int)rank * (kSkThreads / 32) + warp;
+  const int enw = (kSkThreads / 32) * g.S;
+  const int npre = warp >= 2 ? kSkPre : 0;
   float pre_a[kSkPre][4] = {};
   float2 pre_c0[kSkPre] = {}, pre_c1[kSkPre] = {};
   int pre_pos[kSkPre] = {};
@@ -258,15 +261,18 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       const int t = ew + i * enw;
       if (t < g.M) load_side(t, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
     }
-    if (g.epi == kEpiQKRope && tile < g.qk.Hq + g.qk.Hkv) {
-      const uint16_t* wsrc = tile < g.qk.Hq ? g.qk.q_norm : g.qk.k_norm;
+  }
+  // per-feature weights of the epilogue (QK-norm, or the fused RMSNorm), every warp
+  if (g.epi == kEpiQKRope && tile < g.qk.Hq + g.qk.Hkv) {
+    const uint16_t* wsrc = tile < g.qk.Hq ? g.qk.q_norm : g.qk.k_norm;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)wsrc[32 * j + lane] << 16);
-    }
-    if (g.norm_out) {
+    for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)wsrc[32 * j + lane] << 16);
+  }
+  if (g.norm_out) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)g.norm_w[tile * 128 + 32 * j + lane] << 16);
-    }
+    for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)g.norm_w[tile * 128 + 32 * j + lane] << 16);
+  }
+  if (warp >= 2 && warp < 6) {
     // ---------------------------------------------------------- accumulator -> smem
     const int quad = warp & 3;  // tensor-memory lanes [32 quad, 32 quad + 32)
     bool ok = mbar_wait(done, 0, g.err);
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   __syncwarp();
   cluster_sync();  // every split's partial is in its CTA's shared memory
 
-  if (warp >= 2 && !*s_abort) {
+  if (!*s_abort) {
     // -------------------------------------------------- split sum + epilogue, one warp per token
     // split s's partial of (token t, feature f) in CTA s: the mapa (a volatile asm after
     // the barrier) keeps the loads, which no longer change, below the barrier
@@ -408,13 +414,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
     for (int i = 0; i < kSkPre; ++i) {
       const int t = ew + i * enw;
-      if (t < g.M) {
+      if (i < npre && t < g.M) {
         float v[4];
         sum_token(t, v);
         finish(i, t, v, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
       }
     }
-    for (int t = ew + kSkPre * enw; t < g.M; t += enw) {  // tokens beyond the prefetched ones
+    for (int t = ew + npre * enw; t < g.M; t += enw) {  // tokens beyond the prefetched ones
       float a[4], v[4];
       float2 c0, c1;
       int pos = 0;
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
   }
 
-  if (g.norm_out && warp >= 2) {
+  if (g.norm_out) {
     // ------------------------------------------------ RMSNorm of the whole output rows
     epi_bar_sync();  // the epilogue warps' output and sum-of-squares stores precede the arrival
     if (threadIdx.x == 64) *s_last = grid_barrier(g.ticket, (int)gridDim.x, g.err) ? 1 : 0;
@@ -453,13 +459,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       };
       float ssk[kSkPre];
 #pragma unroll
-      for (int i = 0; i < kSkPre; ++i) ssk[i] = ew + i * enw < g.M ? tiles_ss(ew + i * enw) : 0.f;
+      for (int i = 0; i < kSkPre; ++i) ssk[i] = i < npre && ew + i * enw < g.M ? tiles_ss(ew + i * enw) : 0.f;
 #pragma unroll
       for (int i = 0; i < kSkPre; ++i) {
         const int t = ew + i * enw;
-        if (t < g.M) normalise(t, ssk[i], keep[i]);
+        if (i < npre && t < g.M) normalise(t, ssk[i], keep[i]);
       }
-      for (int t = ew + kSkPre * enw; t < g.M; t += enw) {  // tokens past the kept ones: re-read
+      for (int t = ew + npre * enw; t < g.M; t += enw) {  // tokens past the kept ones: re-read
         float x[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
