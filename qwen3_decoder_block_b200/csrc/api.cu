@@ -22,7 +22,7 @@ namespace q3 {
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
                    int rows, int n, float eps, cudaStream_t s, int* zero_word = nullptr, bool out_f16 = false,
-                   long long out_lo = 0);
+                   long long out_lo = 0, float* r_out = nullptr);
 int launch_qk_norm_rope(uint16_t* qkv, long long ldqkv, int B, int T, int Hq, int Hkv, const int* pos_base,
                         const uint16_t* qw, const uint16_t* kw, const float* rope, uint16_t* ck, uint16_t* cv,
                         int s_max, int max_pos, float eps, int* err, cudaStream_t s);
@@ -267,6 +267,13 @@ struct Buffers {
   // kernel of every call and left at zero by every launch that uses it, [1] a generation
   int* ticket = nullptr;
   float* ssq = nullptr;      // the fused RMSNorm's per-tile sums of squares [H / 128][64]
+  // decode-sized calls: 1/rms per token of the residual stream before (rs_x) and after
+  // (rs_x1) the attention sub-block, and whether b.h holds a deferred norm's output
+  // (y = x * w * s_t, to be rescaled by the projection that reads it)
+  float* rs_x = nullptr;     // [64]
+  float* rs_x1 = nullptr;    // [64]
+  bool h_deferred = false;   // b.h as the block's input norm (QKV side)
+  bool h2_deferred = false;  // b.h as the post-attention norm (gate/up side)
 };
 
 static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void* ws, Buffers* out) {
@@ -309,7 +316,11 @@ static size_t carve(const qwen3_config& c, int op, int B, int T, int s_max, void
     b.hf = cv.take<uint16_t>(M * H);
   }
   b.ticket = cv.take<int>(64);
-  if (M <= 64) b.ssq = cv.take<float>((size_t)(H / 128 + 1) * 64);
+  if (M <= 64) {
+    b.ssq = cv.take<float>((size_t)(H / 128 + 1) * 64);
+    b.rs_x = cv.take<float>(64);
+    b.rs_x1 = cv.take<float>(64);
+  }
   if (out) *out = b;
   return cv.used + 256;
 }
@@ -323,12 +334,22 @@ struct Ctx {
 
 static inline bool swap_for(long long M) { return M <= 256; }
 
+// Every projection of a dense block runs on the decode-sized cluster GEMM (at most 64
+// tokens): the RMSNorms after o_proj and down can then be deferred into the projection
+// that reads them.
+static bool decode_sized_block(const qwen3_config& c, long long M) {
+  const int H = c.hidden, I = c.intermediate, D = c.head_dim;
+  const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * D;
+  return skinny_supported((int)M, nqkv, H, kEpiQKRope) && skinny_supported((int)M, H, c.n_q_heads * D, kEpiResid) &&
+         skinny_supported((int)M, 2 * I, H, kEpiSwiglu) && skinny_supported((int)M, H, I, kEpiResid);
+}
+
 // x1 = x + o_proj(attn(norm1(x)))   ([P-Mini] section TransformerBlock, first half)
 // h_ready: b.h already holds norm1(x) (written by the previous layer's last GEMM).
 // *h2_ready is set when the o_proj GEMM also left norm2(x1) in b.h.
 static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void* x, bool x_f32, int B, int T,
                           bool decode, const int* pos, const qwen3_kv_layer& kv, const float* rope, Buffers& b,
-                          bool h_ready, bool* h2_ready) {
+                          bool h_ready, bool* h2_ready, bool defer2 = false) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, D = c.head_dim;
   const long long M = (long long)B * T;
@@ -346,7 +367,8 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
   if (!h_ready) {
     ProfScope ps("rmsnorm", k.s);
     rc = launch_rmsnorm(x, x_f32, H, w.in_norm, b.h, H, (int)M, H, c.rms_eps, k.s, b.ticket, f16,
-                        skinny ? M * H : 0);
+                        skinny ? M * H : 0, skinny ? b.rs_x : nullptr);
+    b.h_deferred = false;
   }
   if (rc) return rc;
   QKRopeArgs qa;
@@ -378,6 +400,10 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
       q.qk.ldq2 = 2LL * c.n_q_heads * D;
     }
     q.f16 = f16;
+    if (h_ready && b.h_deferred) {  // b.h = x * in_norm * s_t: scale by r_t / s_t, keep r_t
+      q.row_ssq = b.ssq; q.ssq_tiles = H / 128; q.ssq_n = H; q.ssq_eps = c.rms_eps;
+      q.row_s_in = b.rs_x1; q.row_r_out = b.rs_x;
+    }
     {
       ProfScope ps("gemm_qkv", k.s);
       rc = launch_gemm_skinny(q, k.s, k.err);
@@ -408,10 +434,17 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
     // the post-attention RMSNorm of x1 goes to b.h (hi/lo rows) in the same launch
     o.norm_w = w.post_norm; o.norm_out = b.h; o.ld_norm = H; o.norm_eps = c.rms_eps; o.ticket = b.ticket; o.ssq = b.ssq;
     o.norm_lo = M * H;
+    if (defer2) {  // the gate/up projection applies it: y = x1 * post_norm * r(x)_t
+      o.norm_deferred = true;
+      o.pre_scale = b.rs_x;
+    } else {
+      o.row_r_out = b.rs_x1;
+    }
     o.f16 = f16;
     ProfScope ps("gemm_o", k.s);
     rc = launch_gemm_skinny(o, k.s, k.err);
     *h2_ready = rc == 0;
+    b.h2_deferred = rc == 0 && defer2;
     return rc;
   }
   GemmDesc g;
@@ -508,7 +541,7 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
 // next_hilo: next_out feeds a decode-sized projection (it then also gets the lo rows).
 static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, void* out, bool out_f32, Buffers& b,
                      bool h2_ready, const uint16_t* next_norm = nullptr, uint16_t* next_out = nullptr,
-                     bool* next_ready = nullptr, bool next_hilo = false) {
+                     bool* next_ready = nullptr, bool next_hilo = false, bool next_defer = false) {
   const qwen3_config& c = k.c;
   const int H = c.hidden, I = c.intermediate;
   const bool f16 = c.gemm_f16 != 0;
@@ -517,7 +550,8 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
   if (!h2_ready) {
     ProfScope ps("rmsnorm", k.s);
     rc = launch_rmsnorm(b.x1, true, H, w.post_norm, b.h, H, (int)M, H, c.rms_eps, k.s, nullptr, f16,
-                        skinny ? M * H : 0);
+                        skinny ? M * H : 0, skinny ? b.rs_x1 : nullptr);
+    b.h2_deferred = false;
   }
   if (rc) return rc;
   if (skinny) {
@@ -530,6 +564,10 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
     g.out_lo = M * I;  // act as hi/lo rows for the down projection
     g.w_early = true;  // weights; a library kernel of this call runs before this GEMM
     g.f16 = f16;
+    if (h2_ready && b.h2_deferred) {  // b.h = x1 * post_norm * r(x)_t: scale by r(x1)_t / r(x)_t
+      g.row_ssq = b.ssq; g.ssq_tiles = H / 128; g.ssq_n = H; g.ssq_eps = c.rms_eps;
+      g.row_s_in = b.rs_x; g.row_r_out = b.rs_x1;
+    }
     {
       ProfScope ps("gemm_gate_up", k.s);
       rc = launch_gemm_skinny(g, k.s, k.err);
@@ -547,10 +585,17 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
     if (next_norm && next_out) {
       d.norm_w = next_norm; d.norm_out = next_out; d.ld_norm = H; d.norm_eps = c.rms_eps; d.ticket = b.ticket; d.ssq = b.ssq;
       d.norm_lo = next_hilo ? M * H : 0;
+      if (next_defer) {  // the next layer's QKV projection applies it: y = x * in_norm * r(x1)_t
+        d.norm_deferred = true;
+        d.pre_scale = b.rs_x1;
+      } else {
+        d.row_r_out = b.rs_x;
+      }
     }
     ProfScope ps("gemm_down", k.s);
     rc = launch_gemm_skinny(d, k.s, k.err);
     if (next_ready) *next_ready = rc == 0 && next_norm && next_out;
+    b.h_deferred = rc == 0 && next_norm && next_out && next_defer;
     return rc;
   }
   GemmDesc g;
@@ -985,7 +1030,9 @@ int qwen3_block_prefill(const qwen3_config* c, const qwen3_layer_weights* w, qwe
   carve(*c, QWEN3_OP_BLOCK_PREFILL, B, T, kv->s_max, ws, &b);
   Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
   bool h2 = false;
-  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b, false, &h2))) return finish(rc);
+  if ((rc = attention_half(k, *w, x, false, B, T, false, start_pos, *kv, rope, b, false, &h2,
+                           decode_sized_block(*c, (long long)B * T))))
+    return finish(rc);
   return finish(dense_ffn(k, *w, (long long)B * T, x, false, b, h2));
 }
 
@@ -999,7 +1046,9 @@ int qwen3_block_decode(const qwen3_config* c, const qwen3_layer_weights* w, qwen
   carve(*c, QWEN3_OP_BLOCK_DECODE, B, 1, kv->s_max, ws, &b);
   Ctx k{*c, static_cast<cudaStream_t>(stream), device_error_word()};
   bool h2 = false;
-  if ((rc = attention_half(k, *w, x, false, B, 1, true, cache_len, *kv, rope, b, false, &h2))) return finish(rc);
+  if ((rc = attention_half(k, *w, x, false, B, 1, true, cache_len, *kv, rope, b, false, &h2,
+                           decode_sized_block(*c, B))))
+    return finish(rc);
   return finish(dense_ffn(k, *w, B, x, false, b, h2));
 }
 
@@ -1075,13 +1124,16 @@ int qwen3_stack_forward(const qwen3_config* c, const qwen3_bf16* embed, const qw
   // kept) in b.h / b.hf, and the o_proj leaves norm2.
   bool h_ready = false;
   const bool fuse_final = !last_only || T == 1;
+  // decode-sized: the RMSNorms after o_proj and down are deferred into the next projection
+  const bool defer = decode_sized_block(*c, M);
   for (int l = 0; l < c->n_layers; ++l) {
     bool h2 = false;
-    if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b, h_ready, &h2)))
+    if ((rc = attention_half(k, layers[l], b.xs, true, B, T, decode, pos_or_len, kv[l], rope, b, h_ready, &h2,
+                             defer)))
       return finish(rc);
     const bool last = l + 1 == c->n_layers;
     const uint16_t* nn = last ? (fuse_final ? final_norm : nullptr) : layers[l + 1].in_norm;
-    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b, h2, nn, last ? b.hf : b.h, &h_ready, !last)))
+    if ((rc = dense_ffn(k, layers[l], M, b.xs, true, b, h2, nn, last ? b.hf : b.h, &h_ready, !last, defer && !last)))
       return finish(rc);
   }
   // final RMSNorm and tied LM head ([P-Mini] section 骨架; [P-SGL] section 一)

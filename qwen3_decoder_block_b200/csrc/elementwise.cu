@@ -38,11 +38,13 @@ __device__ __forceinline__ void rms_load8(const void* x, long long off, float (&
 // OUT_F16: the output feeds an fp16-operand projection (bf16 otherwise).
 // out_lo > 0: a lo copy lo = round(v - hi) of every output value, out_lo elements after it
 // (the hi/lo operand of a decode-sized projection).
+// r_out (optional): the row's 1/rms (the scale a deferred norm after the next projection
+// starts from).
 template <bool IN_F32, bool OUT_F16>
 __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
                                                          const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
                                                          long long ldo, int rows, int n, float eps, int* zero_word,
-                                                         long long out_lo) {
+                                                         long long out_lo, float* r_out) {
   pdl_wait();
   pdl_trigger();
   if (zero_word && blockIdx.x == 0 && threadIdx.x == 0) *zero_word = 0;
@@ -59,6 +61,7 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
     }
     ss = warp_sum(ss);
     const float r = rsqrtf(ss / (float)n + eps);
+    if (r_out && lane == 0) r_out[row] = r;
     for (int col = lane * 8; col < n; col += 256) {
       float v[8];
       rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
@@ -81,14 +84,15 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
 }
 
 int launch_rmsnorm(const void* x, bool x_f32, long long ldx, const uint16_t* w, uint16_t* out, long long ldo,
-                   int rows, int n, float eps, cudaStream_t s, int* zero_word, bool out_f16, long long out_lo) {
+                   int rows, int n, float eps, cudaStream_t s, int* zero_word, bool out_f16, long long out_lo,
+                   float* r_out) {
   if (rows <= 0) return 0;
   const int warps_per_block = 8;
   long long blocks = (rows + warps_per_block - 1) / warps_per_block;
   if (blocks > (long long)num_sms() * 16) blocks = (long long)num_sms() * 16;
   auto k = x_f32 ? (out_f16 ? rmsnorm_kernel<true, true> : rmsnorm_kernel<true, false>)
                  : (out_f16 ? rmsnorm_kernel<false, true> : rmsnorm_kernel<false, false>);
-  q3_launch(k, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps, zero_word, out_lo);
+  q3_launch(k, (int)blocks, 256, 0, s, x, ldx, w, out, ldo, rows, n, eps, zero_word, out_lo, r_out);
   return cudaGetLastError() == cudaSuccess ? 0 : -6;
 }
 

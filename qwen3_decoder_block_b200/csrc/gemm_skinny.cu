@@ -25,7 +25,13 @@
 //     norm that follows them in the block): every warp writes the sum of squares of
 //     its token's 128 features, all CTAs (co-resident: one wave) meet at a grid-wide
 //     barrier, and each warp then adds the tiles' sums of its token in tile order and
-//     normalises the features it still holds in registers;
+//     normalises the features it still holds in registers ("grid" mode); or, when the
+//     next projection is one of these kernels too, the norm is deferred: this kernel
+//     writes y = x * w * s_t (s_t = 1/rms of the residual stream before this projection,
+//     which keeps y at the normalised magnitude) and the sums of squares, and the next
+//     projection, which is linear in its input row, multiplies its accumulators of
+//     token t by r_t / s_t (r_t = 1/rms of x_t from the sums, in tile order) -- the same
+//     result as normalising first, without the barrier;
 //   * every mbarrier wait is bounded; cluster barriers are executed by every thread on
 //     every path, so an expired wait cannot leave a peer CTA waiting.
 #include <cstdio>
@@ -86,6 +92,15 @@ struct SkParams {
   float norm_eps;
   int* ticket;  // grid barrier of the fused norm: [0] arrivals (0 between launches), [1] generation
   float* ssq;   // fused norm: per-tile sums of squares [N / 128][64]
+  int norm_deferred;       // fused norm deferred to the next projection (no barrier)
+  const float* pre_scale;  // deferred norm: s_t, written as y = x * w * s_t ([64]; null: 1)
+  // this projection's input is a deferred norm's output: scale token t's accumulators by
+  // r_t / s_in[t], r_t = rsqrt(sum_q row_ssq[q * 64 + t] / ssq_n + eps) (q < ssq_tiles)
+  const float* row_ssq;
+  int ssq_tiles, ssq_n;
+  float ssq_eps;
+  const float* row_s_in;  // [64] (null: 1)
+  float* row_r_out;       // [64] r_t of the input rows (feature tile 0 writes it), or null
   QKRopeArgs qk;
   int f16;  // operands fp16 (else bf16); the SwiGLU and fused-norm outputs are fp16 too
   int* err;
@@ -177,15 +192,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // warp ew = 8 rank + warp of the cluster finishes tokens ew + i enw; warps 2-7 load the
-  // side operands of their first kSkPre tokens while the MMAs run (npre), warps 0-1 (busy
-  // as producer and issuer then) load theirs when they get to them
+  // warp ew = 8 rank + warp of the cluster finishes tokens ew + i enw; the side operands
+  // of its first kSkPre tokens are loaded ahead (npre)
   const int ew = (int)rank * (kSkThreads / 32) + warp;
   const int enw = (kSkThreads / 32) * g.S;
-  const int npre = warp >= 2 ? kSkPre : 0;
+  constexpr int npre = kSkPre;
   float pre_a[kSkPre][4] = {};
   float2 pre_c0[kSkPre] = {}, pre_c1[kSkPre] = {};
   int pre_pos[kSkPre] = {};
+  float pre_k[kSkPre], pre_r[kSkPre], pre_s[kSkPre];  // input-row scale, its r_t; deferred norm's s_t
   float wn[4] = {0.f, 0.f, 0.f, 0.f};  // QK-norm weights (kEpiQKRope), fused-norm weights (norm_out)
   float keep[kSkPre][4] = {};          // fused norm: the output values of the prefetched tokens
   // residual values (kEpiResid), or position and rotary factors (kEpiQKRope) of token t
@@ -207,6 +222,29 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       }
     }
   };
+
+  // the deferred-norm factors of token t: input-row scale k = r / s_in (and r), and the
+  // s_t this kernel's own deferred norm writes with
+  auto load_scales = [&](int t, float& k, float& r, float& sp) {
+    k = 1.f;
+    r = 1.f;
+    if (g.row_ssq) {
+      float ss = 0.f;
+#pragma unroll 8
+      for (int q = 0; q < g.ssq_tiles; ++q) ss += __ldcg(g.row_ssq + q * 64 + t);  // tile order
+      r = rsqrtf(ss / (float)g.ssq_n + g.ssq_eps);
+      k = r / (g.row_s_in ? g.row_s_in[t] : 1.f);
+    }
+    sp = g.pre_scale ? g.pre_scale[t] : 1.f;
+  };
+  // epilogue operands that do not depend on the product (residual rows, positions,
+  // rotary factors), requested by every warp before its role: the loads complete while
+  // the weights stream and the MMAs run
+#pragma unroll
+  for (int i = 0; i < kSkPre; ++i) {
+    const int t = ew + i * enw;
+    if (t < g.M) load_side(t, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -253,14 +291,6 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       // arrives once every MMA issued above has completed (at once if none was issued)
       mma_commit(done);
     }
-  } else {
-    // epilogue operands that do not depend on the product (residual rows, positions,
-    // rotary factors, QK-norm weights), loaded while the weights stream and the MMAs run
-#pragma unroll
-    for (int i = 0; i < kSkPre; ++i) {
-      const int t = ew + i * enw;
-      if (t < g.M) load_side(t, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
-    }
   }
   // per-feature weights of the epilogue (QK-norm, or the fused RMSNorm), every warp
   if (g.epi == kEpiQKRope && tile < g.qk.Hq + g.qk.Hkv) {
@@ -271,6 +301,16 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   if (g.norm_out) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)g.norm_w[tile * 128 + 32 * j + lane] << 16);
+  }
+  // the scales use their loads at once: the warps that wait for the MMAs compute them
+  // now, the TMA and MMA warps when they reach their tokens
+  const bool scales_ready = warp >= 2;
+  if (scales_ready) {
+#pragma unroll
+    for (int i = 0; i < kSkPre; ++i) {
+      const int t = ew + i * enw;
+      if (t < g.M) load_scales(t, pre_k[i], pre_r[i], pre_s[i]);
+    }
   }
   if (warp >= 2 && warp < 6) {
     // ---------------------------------------------------------- accumulator -> smem
@@ -329,7 +369,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         for (int j = 0; j < 4; ++j) v[j] += ld_cluster_f32_ro(base + 128u * j);  // split order: deterministic
       }
     };
-    auto finish = [&](int i, int t, float(&v)[4], const float(&a)[4], float2 c0, float2 c1, int pos) {
+    auto finish = [&](int i, int t, float(&v)[4], const float(&a)[4], float2 c0, float2 c1, int pos, float kin,
+                      float rin, float sp) {
+      if (g.row_ssq) {  // the input rows were a deferred norm's output
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] *= kin;
+        if (g.row_r_out && tile == 0 && lane == 0) g.row_r_out[t] = rin;
+      }
       if (g.epi == kEpiQKRope) {
         // slot = head of the fused QKV row: q heads, then k heads, then v heads
         const QKRopeArgs& q = g.qk;
@@ -403,11 +449,24 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         if (g.norm_out) {
           const float ss = warp_sum(v[0] * v[0] + v[1] * v[1] + v[2] * v[2] + v[3] * v[3]);
           if (lane == 0) g.ssq[tile * 64 + t] = ss;
+          if (g.norm_deferred) {
+            // y = x * w * s_t as hi/lo operand rows; the next projection applies r_t / s_t
+            uint16_t* dst = g.norm_out + (long long)t * g.ld_norm + col;
+            const bool f16 = g.f16 != 0;
 #pragma unroll
-          for (int k = 0; k < kSkPre; ++k)
-            if (k == i)
+            for (int j = 0; j < 4; ++j) {
+              const float y = v[j] * wn[j] * sp;
+              const uint16_t hi = to_op_bits(f16, y);
+              dst[32 * j] = hi;
+              if (g.norm_lo) dst[g.norm_lo + 32 * j] = to_op_bits(f16, y - op_bits_to_f32(f16, hi));
+            }
+          } else {
 #pragma unroll
-              for (int j = 0; j < 4; ++j) keep[k][j] = v[j];
+            for (int k = 0; k < kSkPre; ++k)
+              if (k == i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) keep[k][j] = v[j];
+          }
         }
       }
     };
@@ -416,21 +475,24 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       const int t = ew + i * enw;
       if (i < npre && t < g.M) {
         float v[4];
+        if (!scales_ready) load_scales(t, pre_k[i], pre_r[i], pre_s[i]);
         sum_token(t, v);
-        finish(i, t, v, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i]);
+        finish(i, t, v, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i], pre_k[i], pre_r[i], pre_s[i]);
       }
     }
     for (int t = ew + npre * enw; t < g.M; t += enw) {  // tokens beyond the prefetched ones
       float a[4], v[4];
       float2 c0, c1;
       int pos = 0;
+      float kin, rin, sp;
       load_side(t, a, c0, c1, pos);
+      load_scales(t, kin, rin, sp);
       sum_token(t, v);
-      finish(kSkPre, t, v, a, c0, c1, pos);
+      finish(kSkPre, t, v, a, c0, c1, pos, kin, rin, sp);
     }
   }
 
-  if (g.norm_out) {
+  if (g.norm_out && !g.norm_deferred) {
     // ------------------------------------------------ RMSNorm of the whole output rows
     epi_bar_sync();  // the epilogue warps' output and sum-of-squares stores precede the arrival
     if (threadIdx.x == 64) *s_last = grid_barrier(g.ticket, (int)gridDim.x, g.err) ? 1 : 0;
@@ -448,6 +510,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       };
       auto normalise = [&](int t, float ss, const float(&x)[4]) {
         const float r = rsqrtf(ss / (float)g.N + g.norm_eps);
+        if (g.row_r_out && tile == 0 && lane == 0) g.row_r_out[t] = r;  // the next stage's s_t
         uint16_t* dst = g.norm_out + (long long)t * g.ld_norm + col;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -587,6 +650,14 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
   g.norm_eps = d.norm_eps;
   g.ticket = d.ticket;
   g.ssq = d.ssq;
+  g.norm_deferred = d.norm_deferred ? 1 : 0;
+  g.pre_scale = d.pre_scale;
+  g.row_ssq = d.row_ssq;
+  g.ssq_tiles = d.ssq_tiles;
+  g.ssq_n = d.ssq_n;
+  g.ssq_eps = d.ssq_eps;
+  g.row_s_in = d.row_s_in;
+  g.row_r_out = d.row_r_out;
   g.qk = d.qk;
   g.f16 = d.f16 ? 1 : 0;
   g.err = err;
@@ -612,7 +683,13 @@ int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err) {
     set_last_error("skinny gemm: unsupported shape M %d N %d K %d", d.M, d.N, d.K);
     return -2;
   }
-  if (d.norm_out && (d.epi != kEpiResid || !d.norm_w || !d.ticket || !d.ssq || d.N / 128 > num_sms())) {
+  if (d.row_ssq && (d.ssq_tiles < 1 || d.ssq_tiles > 64 || d.ssq_n < 1)) {
+    set_last_error("skinny gemm: bad deferred-norm input (%d sum-of-squares tiles, row length %d)", d.ssq_tiles,
+                   d.ssq_n);
+    return -1;
+  }
+  if (d.norm_out && (d.epi != kEpiResid || !d.norm_w || !d.ssq || (!d.norm_deferred && !d.ticket) ||
+                     d.N / 128 > num_sms())) {
     set_last_error("skinny gemm: the fused RMSNorm needs the residual epilogue, weights, a barrier word pair, the "
                    "sum-of-squares scratch and at most one feature tile per SM");
     return -1;

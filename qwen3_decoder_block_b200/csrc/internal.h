@@ -110,6 +110,18 @@ struct SkinnyDesc {
   float norm_eps = 1e-6f;
   int* ticket = nullptr;
   float* ssq = nullptr;
+  // deferred norm (the next projection is one of these kernels): norm_out gets
+  // y = out * norm_w * pre_scale[t] and ssq the per-tile sums of squares; no barrier
+  bool norm_deferred = false;
+  const float* pre_scale = nullptr;
+  // the A rows are a deferred norm's y: scale token t's accumulators by r_t / row_s_in[t],
+  // r_t = rsqrt(sum over ssq_tiles tiles of row_ssq[q * 64 + t] / ssq_n + ssq_eps); r_t is
+  // written to row_r_out (also written by the grid-mode norm: r_t of its output rows)
+  const float* row_ssq = nullptr;
+  int ssq_tiles = 0, ssq_n = 0;
+  float ssq_eps = 1e-6f;
+  const float* row_s_in = nullptr;
+  float* row_r_out = nullptr;
   QKRopeArgs qk;
   bool f16 = false;  // as GemmDesc::f16
   // a_hilo: A holds 2M rows, row t = hi(a_t), row M + t = lo(a_t) = round(a_t - hi), both in
