@@ -17,9 +17,8 @@ namespace q3 {
 // One warp per row; each lane owns 8 consecutive elements of every 256-wide
 // slice (n <= 2048, n % 256 == 0).
 // ---------------------------------------------------------------------------
-// Two passes over the row: the sum of squares, then a second read (an L1 hit) to scale
-// and store, so that a thread holds no row values and 64 warps per SM keep rows in
-// flight.
+// A row of up to 1024 features is read once into registers (32 values per lane), then
+// scaled and stored; longer rows take two passes (the second read hits L1).
 template <bool IN_F32>
 __device__ __forceinline__ void rms_load8(const void* x, long long off, float (&v)[8]) {
   if (IN_F32) {
@@ -40,8 +39,10 @@ __device__ __forceinline__ void rms_load8(const void* x, long long off, float (&
 // (the hi/lo operand of a decode-sized projection).
 // r_out (optional): the row's 1/rms (the scale a deferred norm after the next projection
 // starts from).
+constexpr int kNormRegChunks = 4;  // rows of up to 4 x 256 features are read once, into registers
+
 template <bool IN_F32, bool OUT_F16>
-__global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
+__global__ void __launch_bounds__(256, 4) rmsnorm_kernel(const void* __restrict__ x, long long ldx,
                                                          const uint16_t* __restrict__ w, uint16_t* __restrict__ out,
                                                          long long ldo, int rows, int n, float eps, int* zero_word,
                                                          long long out_lo, float* r_out) {
@@ -51,7 +52,44 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
   const int lane = threadIdx.x & 31;
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int n_warps = (gridDim.x * blockDim.x) >> 5;
+  // the weighted, rounded output of 8 values at column col (hi, and lo when out_lo > 0)
+  auto emit8 = [&](int row, int col, const float(&v)[8], float r) {
+    const uint4 wv = *reinterpret_cast<const uint4*>(w + col);
+    const float wf[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
+                         bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a0 = v[2 * j] * r * wf[2 * j], a1 = v[2 * j + 1] * r * wf[2 * j + 1];
+      hi[j] = pack_op_x2(OUT_F16, a0, a1);
+      lo[j] = pack_op_x2(OUT_F16, a0 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] & 0xFFFFu)),
+                         a1 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] >> 16)));
+    }
+    uint16_t* dst = out + (long long)row * ldo + col;
+    *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    if (out_lo) *reinterpret_cast<uint4*>(dst + out_lo) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  };
   for (int row = warp_global; row < rows; row += n_warps) {
+    if (n <= 256 * kNormRegChunks) {
+      // the whole row in registers: one read of x
+      float v[kNormRegChunks][8];
+#pragma unroll
+      for (int c = 0; c < kNormRegChunks; ++c)
+        if (c * 256 + lane * 8 < n) rms_load8<IN_F32>(x, (long long)row * ldx + c * 256 + lane * 8, v[c]);
+      float ss = 0.f;
+#pragma unroll
+      for (int c = 0; c < kNormRegChunks; ++c)
+        if (c * 256 + lane * 8 < n)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss += v[c][j] * v[c][j];
+      ss = warp_sum(ss);
+      const float r = rsqrtf(ss / (float)n + eps);
+      if (r_out && lane == 0) r_out[row] = r;
+#pragma unroll
+      for (int c = 0; c < kNormRegChunks; ++c)
+        if (c * 256 + lane * 8 < n) emit8(row, c * 256 + lane * 8, v[c], r);
+      continue;
+    }
     float ss = 0.f;
     for (int col = lane * 8; col < n; col += 256) {
       float v[8];
@@ -65,20 +103,7 @@ __global__ void __launch_bounds__(256, 8) rmsnorm_kernel(const void* __restrict_
     for (int col = lane * 8; col < n; col += 256) {
       float v[8];
       rms_load8<IN_F32>(x, (long long)row * ldx + col, v);
-      const uint4 wv = *reinterpret_cast<const uint4*>(w + col);
-      const float wf[8] = {bf16_lo(wv.x), bf16_hi(wv.x), bf16_lo(wv.y), bf16_hi(wv.y),
-                           bf16_lo(wv.z), bf16_hi(wv.z), bf16_lo(wv.w), bf16_hi(wv.w)};
-      uint32_t hi[4], lo[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float a0 = v[2 * j] * r * wf[2 * j], a1 = v[2 * j + 1] * r * wf[2 * j + 1];
-        hi[j] = pack_op_x2(OUT_F16, a0, a1);
-        lo[j] = pack_op_x2(OUT_F16, a0 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] & 0xFFFFu)),
-                           a1 - op_bits_to_f32(OUT_F16, (uint16_t)(hi[j] >> 16)));
-      }
-      uint16_t* dst = out + (long long)row * ldo + col;
-      *reinterpret_cast<uint4*>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-      if (out_lo) *reinterpret_cast<uint4*>(dst + out_lo) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      emit8(row, col, v, r);
     }
   }
 }
