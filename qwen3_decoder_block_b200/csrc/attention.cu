@@ -554,7 +554,8 @@ struct D4Walk {
 template <int G, bool HILO>
 __global__ void __launch_bounds__(kD4Threads, 1)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                          const __grid_constant__ CUtensorMap tmV, int B, int Hq, int Hkv,
+                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
+                          const __grid_constant__ CUtensorMap tmV16, int B, int Hq, int Hkv,
                           const int* __restrict__ cache_len, int s_max, const int* __restrict__ plan,
                           float* __restrict__ part, int* __restrict__ counters, const DecodeMergeOut mo, int* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -593,7 +594,10 @@ __global__ void __launch_bounds__(kD4Threads, 1)
     reinterpret_cast<uint4*>(base)[off] = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
-  if (threadIdx.x == 128) { tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV); }
+  if (threadIdx.x == 128) {
+    tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmK16); tma_prefetch_desc(&tmV16);
+  }
   if (warp == 5) { tmem_alloc(tmem_slot, kD4TmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -618,19 +622,33 @@ __global__ void __launch_bounds__(kD4Threads, 1)
       for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid() && ok; w.next()) {
         const int b = w.b, g = w.g, bg = b * Hkv + g;
         const int row0 = bg * s_max;
+        const int n_total = cache_len[b] + 1;
         for (int j = w.j0(); j < w.j1(); ++j) {
           const int k0 = j * 128;
           const int st = (int)(tc % kD4Stages);
           if (*s_abort || !mbar_wait(&empty[st], (uint32_t)((tc / kD4Stages) & 1) ^ 1u, err)) { ok = false; break; }
           uint8_t* base = smem + st * kD4StageBytes;
           constexpr int QR = HILO ? 2 * G : G;  // query rows of a group in the tile
-          mbar_arrive_expect_tx(&full[st], 4 * kD4Half + 2 * QR * 128);
+          // a row's last tile: only the boxes of 16 keys that hold visible keys (the other
+          // rows keep stale data; their scores are masked and their V rows zeroed)
+          const int nb = n_total - k0 >= 128 ? 0 : (n_total - k0 + 15) / 16;
+          mbar_arrive_expect_tx(&full[st], (nb ? nb * 4 * 16 * 128 : 4 * kD4Half) + 2 * QR * 128);
           tma_load_3d(base + kD4OffQ, &tmQ, &full[st], 0, g * QR, b);
           tma_load_3d(base + kD4OffQ + kD4QHalf, &tmQ, &full[st], 64, g * QR, b);
-          tma_load_2d(base + kD4OffK, &tmK, &full[st], 0, row0 + k0);
-          tma_load_2d(base + kD4OffK + kD4Half, &tmK, &full[st], 64, row0 + k0);
-          tma_load_2d(base + kD4OffV, &tmV, &full[st], 0, row0 + k0);
-          tma_load_2d(base + kD4OffV + kD4Half, &tmV, &full[st], 64, row0 + k0);
+          if (nb == 0) {
+            tma_load_2d(base + kD4OffK, &tmK, &full[st], 0, row0 + k0);
+            tma_load_2d(base + kD4OffK + kD4Half, &tmK, &full[st], 64, row0 + k0);
+            tma_load_2d(base + kD4OffV, &tmV, &full[st], 0, row0 + k0);
+            tma_load_2d(base + kD4OffV + kD4Half, &tmV, &full[st], 64, row0 + k0);
+          } else {
+            for (int i = 0; i < nb; ++i) {  // 16 rows of 128 bytes per box: 2 KB, swizzle phase kept
+              const int r = row0 + k0 + 16 * i;
+              tma_load_2d(base + kD4OffK + i * 2048, &tmK16, &full[st], 0, r);
+              tma_load_2d(base + kD4OffK + kD4Half + i * 2048, &tmK16, &full[st], 64, r);
+              tma_load_2d(base + kD4OffV + i * 2048, &tmV16, &full[st], 0, r);
+              tma_load_2d(base + kD4OffV + kD4Half + i * 2048, &tmV16, &full[st], 64, r);
+            }
+          }
           ++tc;
         }
       }
@@ -976,8 +994,11 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
     return -6;
   }
   const long long kv_rows = (long long)B * Hkv * s_max;
+  CUtensorMap tmK16, tmV16;  // 16-row boxes for the last tile of a row
   if (make_tmap_2d(&tmK, ck, kv_rows, kHeadDim, kHeadDim, 128) != 0 ||
-      make_tmap_2d(&tmV, cv, kv_rows, kHeadDim, kHeadDim, 128) != 0) {
+      make_tmap_2d(&tmV, cv, kv_rows, kHeadDim, kHeadDim, 128) != 0 ||
+      make_tmap_2d(&tmK16, ck, kv_rows, kHeadDim, kHeadDim, 16) != 0 ||
+      make_tmap_2d(&tmV16, cv, kv_rows, kHeadDim, kHeadDim, 16) != 0) {
     set_last_error("attention decode: cannot encode the KV-cache tensor maps");
     return -6;
   }
@@ -996,8 +1017,8 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
 #define Q3_D4_CASE(GG, HL)                                                                                        \
   case GG * 2 + HL:                                                                                               \
     if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG, HL>), kD4Smem)) return -6;       \
-    q3_launch(attn_decode_tc_kernel<GG, HL>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, B, Hq, Hkv, cache_len,  \
-              s_max, plan, part, counters, mo, err);                                                              \
+    q3_launch(attn_decode_tc_kernel<GG, HL>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, tmK16, tmV16, B, Hq,    \
+              Hkv, cache_len, s_max, plan, part, counters, mo, err);                                              \
     break;
     Q3_D4_CASE(1, false)
     Q3_D4_CASE(2, false)
