@@ -514,6 +514,34 @@ __device__ __forceinline__ void merge_row_dim(const float* row_base, int c_first
   store_head_dim(acc / L, d, dst, mo);
 }
 
+// Maximum (MAX) or sum over the 32 lanes of each of G per-lane values, with log2(G) halving
+// exchanges (each leaves a lane the half of the heads its lane bit selects) and then a
+// plain butterfly over the remaining lane bits: G - 1 + 5 - log2(G) shuffles instead of
+// 5 G. Lane l ends with head hd = l >> (5 - log2 G).
+template <int G, bool MAX>
+__device__ __forceinline__ float warp_reduce_heads(const float (&x)[G], int lane) {
+  float a[G];
+#pragma unroll
+  for (int j = 0; j < G; ++j) a[j] = x[j];
+#pragma unroll
+  for (int half = G / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+    const bool upper = (lane & bit) != 0;
+#pragma unroll
+    for (int k = 0; k < half; ++k) {
+      const float send = upper ? a[k] : a[k + half];
+      const float keep = upper ? a[k + half] : a[k];
+      const float got = __shfl_xor_sync(0xffffffffu, send, bit);
+      a[k] = MAX ? fmaxf(keep, got) : keep + got;
+    }
+  }
+#pragma unroll
+  for (int o = 16 / G; o > 0; o >>= 1) {
+    const float got = __shfl_xor_sync(0xffffffffu, a[0], o);
+    a[0] = MAX ? fmaxf(a[0], got) : a[0] + got;
+  }
+  return a[0];
+}
+
 // CTA holding global tile t when T tiles are divided among n CTAs as [c T / n, (c+1) T / n).
 __device__ __forceinline__ int d4_cta_of(long long t, long long T, int n) { return (int)(((t + 1) * n - 1) / T); }
 
@@ -751,10 +779,9 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         }
         // tile maximum per head: the warp's 32 keys, then the 4 warps
         float* rm = red_max + (tc & 1) * 64;
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float wm = warp_max(s[j]);
-          if (lane == 0) rm[warp * 16 + j] = wm;
+        {
+          const float wm = warp_reduce_heads<G, true>(s, lane);
+          if ((lane & (32 / G - 1)) == 0) rm[warp * 16 + lane / (32 / G)] = wm;
         }
         named_bar_softmax();
         float alpha[G];
@@ -839,10 +866,9 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           tmem_ld16(tl + 32, ov);
           tmem_wait_ld_regs16(ov);
         }
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float ws = warp_sum(l_part[j]);
-          if (lane == 0) red_sum[warp * 16 + j] = ws;
+        {
+          const float ws = warp_reduce_heads<G, false>(l_part, lane);
+          if ((lane & (32 / G - 1)) == 0) red_sum[warp * 16 + lane / (32 / G)] = ws;
         }
         named_bar_softmax();
       }
