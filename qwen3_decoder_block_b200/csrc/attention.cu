@@ -468,10 +468,14 @@ constexpr uint32_t kD4OffP = kD4Stages * kD4StageBytes;         // P [2 buffers]
 constexpr uint32_t kD4OffRed = kD4OffP + 4 * kD4QHalf;          // maxima [2][4][16], sums [4][16]
 constexpr uint32_t kD4OffBar = kD4OffRed + (2 * 4 * 16 + 4 * 16) * 4;
 constexpr uint32_t kD4Smem = kD4OffBar + 16 * 8 + 16 + 1024;
-constexpr int kD4Threads = 192;  // softmax warps 0-3, TMA warp 4, MMA warp 5
+// softmax warps: two per tensor-memory lane quarter, each owning half of the group's
+// heads (G >= 2), or one per quarter (G = 1); then the TMA warp and the MMA warp
+__host__ __device__ constexpr int d4_softmax_warps(int G) { return G >= 2 ? 8 : 4; }
+__host__ __device__ constexpr int d4_threads(int G) { return 32 * (d4_softmax_warps(G) + 2); }
 constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
 
-__device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+template <int SW>
+__device__ __forceinline__ void named_bar_softmax() { asm volatile("bar.sync 1, %0;" ::"n"(32 * SW) : "memory"); }
 
 // Log-sum-exp merge of one query head's partials (unnormalised o, running max in the
 // exp2 domain, sum) for head dim d: o = sum_s o_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),
@@ -580,7 +584,7 @@ struct D4Walk {
 // O = V P_hi + V P_lo, summed in fp32 -- about 16 significant bits for q and P at no
 // extra MMA instruction (the kernel is bound by the K/V stream).
 template <int G, bool HILO>
-__global__ void __launch_bounds__(kD4Threads, 1)
+__global__ void __launch_bounds__(d4_threads(G), 1)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK16,
                           const __grid_constant__ CUtensorMap tmV16, int B, int Hq, int Hkv,
@@ -604,11 +608,13 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int SW = d4_softmax_warps(G);   // softmax warps; then the TMA warp SW, the MMA warp SW + 1
+  constexpr int GH = G >= 2 ? G / 2 : 1;    // heads per softmax warp
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kD4Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 128); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 32 * SW); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&p_full[i], 32 * SW); mbar_init(&pv_done[i], 1); }
     mbar_init(drain, 1);
     *s_abort = 0;
     *s_b0 = 0;
@@ -622,11 +628,11 @@ __global__ void __launch_bounds__(kD4Threads, 1)
     reinterpret_cast<uint4*>(base)[off] = make_uint4(0, 0, 0, 0);
   }
   fence_proxy_async_smem();
-  if (threadIdx.x == 128) {
+  if (threadIdx.x == 32 * SW) {
     tma_prefetch_desc(&tmQ); tma_prefetch_desc(&tmK); tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmK16); tma_prefetch_desc(&tmV16);
   }
-  if (warp == 5) { tmem_alloc(tmem_slot, kD4TmemCols); tmem_relinquish(); }
+  if (warp == SW + 1) { tmem_alloc(tmem_slot, kD4TmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -642,7 +648,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
   __syncthreads();
   const int b0 = *s_b0;
 
-  if (warp == 4) {
+  if (warp == SW) {
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
       long long tc = 0;
@@ -687,7 +693,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           mbar_wait(&full[i % kD4Stages], (uint32_t)((i / kD4Stages) & 1), err);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == SW + 1) {
     if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, 0, 0);
@@ -745,17 +751,20 @@ __global__ void __launch_bounds__(kD4Threads, 1)
     }
   } else {
     // -------------------------------------------------------------------- softmax
-    const int t = warp * 32 + lane;  // key of the tile (S) / head dim (O)
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    // warp (quarter q, half hh): key / head dim t of lanes [32 q, 32 q + 32), heads
+    // [j0, j0 + GH) of the group
+    const int q = warp & 3, hh = warp >> 2, j0 = hh * GH;
+    const int t = q * 32 + lane;  // key of the tile (S) / head dim (O)
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     long long tc = 0;
     bool ok = true;
     for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid(); w.next()) {
       const int b = w.b, g = w.g, bg = b * Hkv + g;
       const int n_total = cache_len[b] + 1;
       const int jb = w.j0(), je = w.j1();
-      float m_run[G], l_part[G];
+      float m_run[GH], l_part[GH];
 #pragma unroll
-      for (int j = 0; j < G; ++j) { m_run[j] = -INFINITY; l_part[j] = 0.f; }
+      for (int j = 0; j < GH; ++j) { m_run[j] = -INFINITY; l_part[j] = 0.f; }
       int n_tiles = 0;
       for (int j = jb; j < je; ++j) {
         const int k0 = j * 128;
@@ -771,36 +780,38 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         }
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        float s[G];
+        float s[GH];
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float sj = HILO ? __uint_as_float(sv[j]) + __uint_as_float(sv[G + j]) : __uint_as_float(sv[j]);
-          s[j] = (ok && t < nk) ? sj * kScaleLog2 : -INFINITY;
+        for (int jj = 0; jj < GH; ++jj) {
+          const int hd = j0 + jj;
+          const float sj = HILO ? __uint_as_float(hh ? sv[GH + jj] : sv[jj]) + __uint_as_float(hh ? sv[G + GH + jj] : sv[G + jj]) : __uint_as_float(hh ? sv[GH + jj] : sv[jj]);
+          s[jj] = (ok && t < nk) ? sj * kScaleLog2 : -INFINITY;
         }
-        // tile maximum per head: the warp's 32 keys, then the 4 warps
+        // tile maximum per head: the warp's 32 keys, then the 4 quarters
         float* rm = red_max + (tc & 1) * 64;
         {
-          const float wm = warp_reduce_heads<G, true>(s, lane);
-          if ((lane & (32 / G - 1)) == 0) rm[warp * 16 + lane / (32 / G)] = wm;
+          const float wm = warp_reduce_heads<GH, true>(s, lane);
+          if ((lane & (32 / GH - 1)) == 0) rm[q * 16 + j0 + lane / (32 / GH)] = wm;
         }
-        named_bar_softmax();
-        float alpha[G];
+        named_bar_softmax<SW>();
+        float alpha[GH];
         bool rescale = false;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float mt = fmaxf(fmaxf(rm[j], rm[16 + j]), fmaxf(rm[32 + j], rm[48 + j]));
-          alpha[j] = 1.f;
-          if (mt > m_run[j] + kRescaleThreshold || m_run[j] == -INFINITY) {
-            alpha[j] = (m_run[j] == -INFINITY) ? 0.f : ex2_approx(m_run[j] - mt);
-            m_run[j] = mt;
+        for (int jj = 0; jj < GH; ++jj) {
+          const int hd = j0 + jj;
+          const float mt = fmaxf(fmaxf(rm[hd], rm[16 + hd]), fmaxf(rm[32 + hd], rm[48 + hd]));
+          alpha[jj] = 1.f;
+          if (mt > m_run[jj] + kRescaleThreshold || m_run[jj] == -INFINITY) {
+            alpha[jj] = (m_run[jj] == -INFINITY) ? 0.f : ex2_approx(m_run[jj] - mt);
+            m_run[jj] = mt;
             rescale = true;
           }
         }
-        float p[G];
+        float p[GH];
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          p[j] = (t < nk && m_run[j] != -INFINITY) ? ex2_approx(s[j] - m_run[j]) : 0.f;
-          l_part[j] = l_part[j] * alpha[j] + p[j];
+        for (int jj = 0; jj < GH; ++jj) {
+          p[jj] = (t < nk && m_run[jj] != -INFINITY) ? ex2_approx(s[jj] - m_run[jj]) : 0.f;
+          l_part[jj] = l_part[jj] * alpha[jj] + p[jj];
         }
         // P is double-buffered: buffer tc & 1 was last read by the P.V of tile tc - 2. A
         // rescale of O (below) needs the P.V of tile tc - 1 complete as well.
@@ -809,39 +820,41 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           ok = ok && !*s_abort && mbar_wait(&pv_done[pbuf], (uint32_t)(((tc - 2) >> 1) & 1), err);
           ok = __all_sync(0xffffffffu, ok);
         }
-        if (n_tiles > 0 && rescale) {  // uniform: every thread holds the same maxima
+        if (n_tiles > 0 && rescale) {  // uniform within the warp: its lanes hold the same maxima
           ok = ok && !*s_abort && mbar_wait(&pv_done[pbuf ^ 1], (uint32_t)(((tc - 1) >> 1) & 1), err);
           ok = __all_sync(0xffffffffu, ok);
         }
         if (ok) {
           tc_fence_after();
-          if (n_tiles > 0 && rescale) {  // uniform: every thread holds the same maxima
+          if (n_tiles > 0 && rescale) {
+            // this warp's own O columns only (head hd: column hd, and G + hd for the lo half)
             uint32_t ov[16];
             tmem_ld16(tl + 32, ov);
             tmem_wait_ld_regs16(ov);
 #pragma unroll
-            for (int j = 0; j < G; ++j) {
-              ov[j] = __float_as_uint(__uint_as_float(ov[j]) * alpha[j]);
-              if (HILO) ov[G + j] = __float_as_uint(__uint_as_float(ov[G + j]) * alpha[j]);
+            for (int jj = 0; jj < GH; ++jj) {
+              const int hd = j0 + jj;
+              tmem_st1(tl + 32 + hd, __float_as_uint(__uint_as_float(hh ? ov[GH + jj] : ov[jj]) * alpha[jj]));
+              if (HILO) tmem_st1(tl + 32 + G + hd, __float_as_uint(__uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) * alpha[jj]));
             }
-            tmem_st16x(tl + 32, ov);
             tmem_wait_st();
           }
           // P[j][t] into the K-major B tile of buffer pbuf: row j, key t, 128-byte swizzle
           uint8_t* pb = smem + kD4OffP + pbuf * 2 * kD4QHalf + (t >> 6) * kD4QHalf + (t & 7) * 2;
           const int chunk = (t & 63) >> 3;
 #pragma unroll
-          for (int j = 0; j < G; ++j) {
-            const uint16_t hi = to_bf16_bits(p[j]);
-            *reinterpret_cast<uint16_t*>(pb + j * 128 + ((chunk ^ (j & 7)) << 4)) = hi;
+          for (int jj = 0; jj < GH; ++jj) {
+            const int hd = j0 + jj;
+            const uint16_t hi = to_bf16_bits(p[jj]);
+            *reinterpret_cast<uint16_t*>(pb + hd * 128 + ((chunk ^ (hd & 7)) << 4)) = hi;
             if (HILO) {
-              const int jl = G + j;
+              const int jl = G + hd;
               *reinterpret_cast<uint16_t*>(pb + jl * 128 + ((chunk ^ (jl & 7)) << 4)) =
-                  to_bf16_bits(p[j] - __uint_as_float((uint32_t)hi << 16));
+                  to_bf16_bits(p[jj] - __uint_as_float((uint32_t)hi << 16));
             }
           }
           // keys past the written cache: zero their V rows (0 * NaN would poison O)
-          if (t >= nk) {
+          if (hh == 0 && t >= nk) {
             uint4* v0 = reinterpret_cast<uint4*>(smem + (int)(tc % kD4Stages) * kD4StageBytes + kD4OffV + t * 128);
             uint4* v1 = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(v0) + kD4Half);
 #pragma unroll
@@ -854,7 +867,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
         ++n_tiles;
         ++tc;
       }
-      // end of the row's tiles in this CTA: O from tensor memory, the sums of the 4 warps
+      // end of the row's tiles in this CTA: O from tensor memory, the sums of the quarters
       uint32_t ov[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) ov[j] = 0u;
@@ -867,35 +880,38 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           tmem_wait_ld_regs16(ov);
         }
         {
-          const float ws = warp_reduce_heads<G, false>(l_part, lane);
-          if ((lane & (32 / G - 1)) == 0) red_sum[warp * 16 + lane / (32 / G)] = ws;
+          const float ws = warp_reduce_heads<GH, false>(l_part, lane);
+          if ((lane & (32 / GH - 1)) == 0) red_sum[q * 16 + j0 + lane / (32 / GH)] = ws;
         }
-        named_bar_softmax();
+        named_bar_softmax<SW>();
       }
       uint16_t* out_row = mo.out + (long long)b * mo.ldo + (long long)g * G * kHeadDim;
       if (jb == 0 && je == w.nt) {
         // the whole row is here: normalise and write the output
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          const float L = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
-          const float o = HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
-          store_head_dim(o / L, t, out_row + j * kHeadDim, mo);
+        for (int jj = 0; jj < GH; ++jj) {
+          const int hd = j0 + jj;
+          const float L = red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd];
+          const float o = HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+          store_head_dim(o / L, t, out_row + hd * kHeadDim, mo);
         }
       } else {
         // partial of the row in slot row + CTA (unique: the rows and the CTA ranges are
         // both in tile order); the last CTA of the row to finish merges the slots
         float* my_part = part + ((long long)bg + blockIdx.x) * G * kD4PartFloats;
 #pragma unroll
-        for (int j = 0; j < G; ++j) {
-          my_part[j * kD4PartFloats + t] =
-              HILO ? __uint_as_float(ov[j]) + __uint_as_float(ov[G + j]) : __uint_as_float(ov[j]);
-          if (t == j) {
-            my_part[j * kD4PartFloats + kHeadDim] = m_run[j];
-            my_part[j * kD4PartFloats + kHeadDim + 1] = red_sum[j] + red_sum[16 + j] + red_sum[32 + j] + red_sum[48 + j];
+        for (int jj = 0; jj < GH; ++jj) {
+          const int hd = j0 + jj;
+          my_part[hd * kD4PartFloats + t] =
+              HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+          if (t == hd) {
+            my_part[hd * kD4PartFloats + kHeadDim] = m_run[jj];
+            my_part[hd * kD4PartFloats + kHeadDim + 1] =
+                red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd];
           }
         }
         __threadfence();  // the partial, visible to the merging CTA before the ticket
-        named_bar_softmax();
+        named_bar_softmax<SW>();
         const int c_first = d4_cta_of(w.rs, T, n_cta), c_last = d4_cta_of(w.rs + w.nt - 1, T, n_cta);
         if (threadIdx.x == 0) {
           // the row's CTAs: those of [c_first, c_last] whose range is not empty (fewer
@@ -907,13 +923,13 @@ __global__ void __launch_bounds__(kD4Threads, 1)
           if (last) counters[bg] = 0;  // ready for the next call
           *s_fix = last ? 1 : 0;
         }
-        named_bar_softmax();
+        named_bar_softmax<SW>();
         if (*s_fix) {
           __threadfence();  // the other CTAs' partials (their fences precede their tickets)
 #pragma unroll 1
-          for (int j = 0; j < G; ++j)
-            merge_row_dim(part + ((long long)bg * G + j) * kD4PartFloats, c_first, c_last, T, n_cta,
-                          (long long)G * kD4PartFloats, t, out_row + j * kHeadDim, mo);
+          for (int jj = 0; jj < GH; ++jj)
+            merge_row_dim(part + ((long long)bg * G + j0 + jj) * kD4PartFloats, c_first, c_last, T, n_cta,
+                          (long long)G * kD4PartFloats, t, out_row + (j0 + jj) * kHeadDim, mo);
         }
       }
     }
@@ -922,7 +938,7 @@ __global__ void __launch_bounds__(kD4Threads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == SW + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kD4TmemCols);
   }
@@ -1043,7 +1059,7 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
 #define Q3_D4_CASE(GG, HL)                                                                                        \
   case GG * 2 + HL:                                                                                               \
     if (ensure_smem_attr(reinterpret_cast<const void*>(attn_decode_tc_kernel<GG, HL>), kD4Smem)) return -6;       \
-    q3_launch(attn_decode_tc_kernel<GG, HL>, grid, kD4Threads, kD4Smem, s, tmQ, tmK, tmV, tmK16, tmV16, B, Hq,    \
+    q3_launch(attn_decode_tc_kernel<GG, HL>, grid, d4_threads(GG), kD4Smem, s, tmQ, tmK, tmV, tmK16, tmV16, B, Hq, \
               Hkv, cache_len, s_max, plan, part, counters, mo, err);                                              \
     break;
     Q3_D4_CASE(1, false)

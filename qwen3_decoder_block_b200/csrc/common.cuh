@@ -405,6 +405,10 @@ __device__ __forceinline__ void tmem_wait_ld_regs16(uint32_t (&r)[16]) {
       :
       : "memory");
 }
+// One 32-bit column of 32 lanes.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
 __device__ __forceinline__ void tmem_st16x(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
