@@ -65,7 +65,9 @@ struct SkCfg {
   static constexpr uint32_t STAGE = kSkPBytes + Q_BYTES;
   static constexpr int STAGES = (int)(((200u << 10) - 1280u) / STAGE) > 8 ? 8 : (int)(((200u << 10) - 1280u) / STAGE);
   static constexpr uint32_t TMEM_COLS = NQ < 32 ? 32 : NQ;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;  // + barriers and flags
+  // + barriers, flags and the TMA and MMA warps' row scales
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 256;
+  static_assert((2 * STAGES + 1) * 8 + 16 + 2 * kSkPre * 3 * 4 <= 256, "barrier area too small");
   static_assert(STAGES >= 3, "ring too shallow");
   static_assert((size_t)BN * 128 * 4 <= (size_t)STAGES * STAGE, "the split partial must fit over the ring");
 };
@@ -157,6 +159,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_last = s_abort + 1;  // the fused norm's grid barrier completed
+  float* s_scale = reinterpret_cast<float*>(tmem_slot + 4);  // [2 warps][kSkPre tokens][k, r, s]
   float* red = reinterpret_cast<float*>(smem);  // [BN][128] partial sums, over the stages once the MMAs are done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -302,14 +305,27 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
     for (int j = 0; j < 4; ++j) wn[j] = __uint_as_float((uint32_t)g.norm_w[tile * 128 + 32 * j + lane] << 16);
   }
-  // the scales use their loads at once: the warps that wait for the MMAs compute them
-  // now, the TMA and MMA warps when they reach their tokens
-  const bool scales_ready = warp >= 2;
-  if (scales_ready) {
+  // the scales use their loads at once, so the warps that wait for the MMAs compute
+  // them: their own, and (warps 2 and 3) those of warps 0 and 1 into shared memory, read
+  // after the cluster barrier
+  if (warp >= 2) {
 #pragma unroll
     for (int i = 0; i < kSkPre; ++i) {
       const int t = ew + i * enw;
       if (t < g.M) load_scales(t, pre_k[i], pre_r[i], pre_s[i]);
+    }
+    if (warp < 4) {
+#pragma unroll
+      for (int i = 0; i < kSkPre; ++i) {
+        const int t = ew - 2 + i * enw;  // token i of warp (warp - 2)
+        float k = 1.f, r = 1.f, sp = 1.f;
+        if (t < g.M) load_scales(t, k, r, sp);
+        if (lane == 0) {
+          s_scale[((warp - 2) * kSkPre + i) * 3] = k;
+          s_scale[((warp - 2) * kSkPre + i) * 3 + 1] = r;
+          s_scale[((warp - 2) * kSkPre + i) * 3 + 2] = sp;
+        }
+      }
     }
   }
   if (warp >= 2 && warp < 6) {
@@ -369,8 +385,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         for (int j = 0; j < 4; ++j) v[j] += ld_cluster_f32_ro(base + 128u * j);  // split order: deterministic
       }
     };
-    auto finish = [&](int i, int t, float(&v)[4], const float(&a)[4], float2 c0, float2 c1, int pos, float kin,
-                      float rin, float sp) {
+    // v: the token's sums in, and (residual epilogue) the values the fused norm sees out
+    auto finish = [&](int t, float(&v)[4], const float(&a)[4], float2 c0, float2 c1, int pos, float kin, float rin,
+                      float sp) {
       if (g.row_ssq) {  // the input rows were a deferred norm's output
 #pragma unroll
         for (int j = 0; j < 4; ++j) v[j] *= kin;
@@ -460,25 +477,47 @@ __global__ void __launch_bounds__(kSkThreads, 1)
               dst[32 * j] = hi;
               if (g.norm_lo) dst[g.norm_lo + 32 * j] = to_op_bits(f16, y - op_bits_to_f32(f16, hi));
             }
-          } else {
-#pragma unroll
-            for (int k = 0; k < kSkPre; ++k)
-              if (k == i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) keep[k][j] = v[j];
           }
         }
       }
     };
+    // the TMA and MMA warps' scales, computed by warps 2 and 3 while the MMAs ran
+    if (warp < 2) {
 #pragma unroll
+      for (int i = 0; i < kSkPre; ++i) {
+        pre_k[i] = s_scale[(warp * kSkPre + i) * 3];
+        pre_r[i] = s_scale[(warp * kSkPre + i) * 3 + 1];
+        pre_s[i] = s_scale[(warp * kSkPre + i) * 3 + 2];
+      }
+    }
+    // one copy of the token code, run as a loop: a launch executes it from a cold
+    // instruction cache, so an unrolled copy per token would pay the fetches once per
+    // token. The prefetched operands rotate down to slot 0 (registers, fixed indices);
+    // the fused norm's values rotate in at the end of keep.
+#pragma unroll 1
     for (int i = 0; i < kSkPre; ++i) {
       const int t = ew + i * enw;
-      if (i < npre && t < g.M) {
-        float v[4];
-        if (!scales_ready) load_scales(t, pre_k[i], pre_r[i], pre_s[i]);
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (t < g.M) {
         sum_token(t, v);
-        finish(i, t, v, pre_a[i], pre_c0[i], pre_c1[i], pre_pos[i], pre_k[i], pre_r[i], pre_s[i]);
+        finish(t, v, pre_a[0], pre_c0[0], pre_c1[0], pre_pos[0], pre_k[0], pre_r[0], pre_s[0]);
       }
+#pragma unroll
+      for (int k = 0; k + 1 < kSkPre; ++k) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          pre_a[k][j] = pre_a[k + 1][j];
+          keep[k][j] = keep[k + 1][j];
+        }
+        pre_c0[k] = pre_c0[k + 1];
+        pre_c1[k] = pre_c1[k + 1];
+        pre_pos[k] = pre_pos[k + 1];
+        pre_k[k] = pre_k[k + 1];
+        pre_r[k] = pre_r[k + 1];
+        pre_s[k] = pre_s[k + 1];
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) keep[kSkPre - 1][j] = v[j];
     }
     for (int t = ew + npre * enw; t < g.M; t += enw) {  // tokens beyond the prefetched ones
       float a[4], v[4];
@@ -488,7 +527,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       load_side(t, a, c0, c1, pos);
       load_scales(t, kin, rin, sp);
       sum_token(t, v);
-      finish(kSkPre, t, v, a, c0, c1, pos, kin, rin, sp);
+      finish(t, v, a, c0, c1, pos, kin, rin, sp);
     }
   }
 
