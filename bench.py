@@ -300,28 +300,33 @@ def run_prefill(q3, torch, args, rank, world, dist, peaks, gemm_f16=1, light=Fal
     clk = clocks.stop() if rank == 0 else None
     assert q3.check_device_error() == 0
 
-    # per-kernel attribution: the same K steps again with CUDA events around every
-    # launch (kept out of the timed value above, which they would slow slightly)
-    q3.profile_begin(args.steps * 400 + 16)
-    for _ in range(args.steps):
-        step()
-    records = q3.profile_end(stream)
-
     # end to end through the public call with host buffers: ids H2D, logits of each
-    # sequence's last position D2H, inside the timed region
+    # sequence's last position D2H, inside the timed region (device events; the host's
+    # own time to issue the steps is reported beside it)
     ids_host = ids.cpu().pin_memory()
     out_host = torch.empty((B, cfg.vocab), dtype=torch.float32).pin_memory()
     last_rows = logits.view(B, T, cfg.vocab)[:, T - 1]
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
     f0.record(stream)
     for _ in range(args.steps):
         ids.copy_(ids_host, non_blocking=True)
         step()
         out_host.copy_(last_rows, non_blocking=True)
     f1.record(stream)
+    h1 = time.perf_counter()
     torch.cuda.synchronize()
+    h2 = time.perf_counter()
     e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), torch)
+    e2e_host = {"issue_ms_per_step": (h1 - h0) * 1e3 / args.steps, "wall_ms_per_step": (h2 - h0) * 1e3 / args.steps}
+
+    # per-kernel attribution: the same K steps again with CUDA events around every
+    # launch (kept out of the timed value above, which they would slow slightly)
+    q3.profile_begin(args.steps * 400 + 16)
+    for _ in range(args.steps):
+        step()
+    records = q3.profile_end(stream)
 
     kernels, prof_ms = summarize_profile(records, args.steps)
     g_tok, lm_tok = gemm_flops_per_token(cfg)
@@ -342,7 +347,7 @@ def run_prefill(q3, torch, args, rank, world, dist, peaks, gemm_f16=1, light=Fal
         "gemm_f16": gemm_f16,
         "ms_per_step": per_step_ms,
         "e2e": {"value": job_throughput(world, M, args.steps, e2e_ms), "unit": "tokens/s",
-                "h2d_bytes_per_step": M * 4, "d2h_bytes_per_step": B * cfg.vocab * 4},
+                "h2d_bytes_per_step": M * 4, "d2h_bytes_per_step": B * cfg.vocab * 4, "host": e2e_host},
         "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel (all projections + LM head)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{peaks['source']} bf16 burst (launches timed one by one)", "traffic": None,
@@ -514,12 +519,15 @@ def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
         call()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
     e0.record(stream)
     for _ in range(reps):
         call()
     e1.record(stream)
+    h1 = time.perf_counter()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / reps
+    host_issue_ms = (h1 - h0) * 1e3 / reps
     q3.profile_begin(400)
     call()
     recs = q3.profile_end(stream)
@@ -533,7 +541,7 @@ def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
         ffn = 2 * M * 3 * H * cfg.intermediate
     flops = lin + attn + ffn
     kern, _ = summarize_profile(recs, 1)
-    return {"workload": name, "tokens_per_s": M / (ms * 1e-3), "ms_per_call": ms,
+    return {"workload": name, "tokens_per_s": M / (ms * 1e-3), "ms_per_call": ms, "host_issue_ms_per_call": host_issue_ms,
             "tflops": flops / (ms * 1e-3) / 1e12, "algorithmic_tflop": flops / 1e12,
             "kernels_ms": {kk: round(vv["ms_per_step"], 4) for kk, vv in kern.items()}}
 

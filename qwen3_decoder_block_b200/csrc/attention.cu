@@ -783,7 +783,6 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
         float s[GH];
 #pragma unroll
         for (int jj = 0; jj < GH; ++jj) {
-          const int hd = j0 + jj;
           const float sj = HILO ? __uint_as_float(hh ? sv[GH + jj] : sv[jj]) + __uint_as_float(hh ? sv[G + GH + jj] : sv[G + jj]) : __uint_as_float(hh ? sv[GH + jj] : sv[jj]);
           s[jj] = (ok && t < nk) ? sj * kScaleLog2 : -INFINITY;
         }
