@@ -610,15 +610,25 @@ __global__ void __launch_bounds__(192, 1)
       }
       asm volatile("bar.sync 2, 128;" ::: "memory");  // the 4 epilogue warps only
     }
+    // residual epilogue with the TMA store: the residual (an input, final since the
+    // grid-dependency wait) is read two 32-column chunks ahead of the accumulator, the
+    // first two before the accumulator is waited for
+    const bool res_path = !ROPE && g.tma_store && g.epi == kEpiResid;
     for (int t = t_first; t < ntiles; t += t_step, ++local) {
       Tile tl = decode_tile<BN, BMT>(t, g, s_prefix, s_off);
       if (PAIR) tl.p0 += (int)rank * BM;
       const int buf = local & 1;
       const uint32_t use_par = (local >> 1) & 1;
+      const int row = quad * 32 + lane;
+      float res[32], nxt[32];
+      const int pr = tl.p0 + row < tl.p_end ? tl.p0 + row : -1;
+      if (res_path) {
+        load_resid_chunk(g, pr, tl.q0, res);
+        if (BN > 32 && tl.q0 + 32 < tl.q_end) load_resid_chunk(g, pr, tl.q0 + 32, nxt);
+      }
       bool ok = !*s_abort && mbar_wait(&tfull[buf], use_par, g.err);
       if (!__all_sync(0xffffffffu, ok)) { *s_abort = 1; break; }  // keep the warp converged
       tc_fence_after();
-      const int row = quad * 32 + lane;
       if constexpr (ROPE) {
         // non-swap only: the tile's BN columns are BN/128 whole heads
         const int p = tl.p0 + row;
@@ -626,20 +636,17 @@ __global__ void __launch_bounds__(192, 1)
         if (heads > 0)
           qk_rope_tile(g, tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN, tl.q0 / 128, heads, p,
                        p < tl.p_end, rope_lo);
-      } else if (g.tma_store && g.epi == kEpiResid) {
-        // residual epilogue, software-pipelined: the residual loads of chunk c + 1 are in
-        // flight while chunk c is read from tensor memory, added and staged
-        const int p = tl.p0 + row;
-        const int pr = p < tl.p_end ? p : -1;
-        float res[32];
-        load_resid_chunk(g, pr, tl.q0, res);
+      } else if (res_path) {
+        // software-pipelined: the residual loads of chunk c + 2 are in flight while chunk
+        // c is read from tensor memory, added and staged
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           const int q = tl.q0 + c * 32;
           if (q >= tl.q_end) break;  // warp-uniform
           const bool more = c + 1 < BN / 32 && q + 32 < tl.q_end;
-          float nxt[32];
-          if (more) load_resid_chunk(g, pr, q + 32, nxt);
+          const bool more2 = c + 2 < BN / 32 && q + 64 < tl.q_end;
+          float nxt2[32];
+          if (more2) load_resid_chunk(g, pr, q + 64, nxt2);
           uint32_t r[32];
           tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, r);
           tmem_wait_ld_regs(r);
@@ -657,6 +664,10 @@ __global__ void __launch_bounds__(192, 1)
           if (more) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) res[j] = nxt[j];
+          }
+          if (more2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) nxt[j] = nxt2[j];
           }
         }
       } else {
