@@ -330,12 +330,16 @@ __device__ __forceinline__ void qk_rope_tile(const GemmParams& g, uint32_t taddr
     if (hh >= n_heads || slot0 + hh >= a.Hq + a.Hkv) continue;  // warp-uniform
     float ss = 0.f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
+    for (int c = 0; c < 4; c += 2) {  // two loads in flight per wait
+      uint32_t v[32], w[32];
       tmem_ld32(taddr + hh * 128 + c * 32, v);
+      tmem_ld32(taddr + hh * 128 + c * 32 + 32, w);
       tmem_wait_ld_regs(v);
+      tmem_wait_ld_regs(w);
 #pragma unroll
       for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(v[i]), __uint_as_float(v[i]), ss);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(w[i]), __uint_as_float(w[i]), ss);
     }
     rinv[hh] = rsqrtf(ss * (1.0f / 128.0f) + a.eps);
   }
