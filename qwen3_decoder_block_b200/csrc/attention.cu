@@ -471,7 +471,8 @@ constexpr uint32_t kD4Smem = kD4OffBar + 16 * 8 + 16 + 1024;
 // softmax warps: two per tensor-memory lane quarter, each owning half of the group's
 // heads (G >= 2), or one per quarter (G = 1); then the TMA warp and the MMA warp
 __host__ __device__ constexpr int d4_softmax_warps(int G) { return G >= 2 ? 8 : 4; }
-__host__ __device__ constexpr int d4_threads(int G) { return 32 * (d4_softmax_warps(G) + 2); }
+// softmax warps, then the TMA warp, the S-issuing warp and the P.V-issuing warp
+__host__ __device__ constexpr int d4_threads(int G) { return 32 * (d4_softmax_warps(G) + 3); }
 constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
 
 template <int SW>
@@ -599,7 +600,8 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
   uint64_t* s_empty = bars + 8;  // [2] scores read
   uint64_t* p_full = bars + 10;  // [2] P buffer written (and O rescaled)
   uint64_t* pv_done = bars + 12; // [2] P.V of a tile using that buffer complete
-  uint64_t* drain = bars + 14;
+  uint64_t* drain = bars + 14;     // the S issuer's MMAs complete
+  uint64_t* drain_pv = bars + 15;  // the P.V issuer's MMAs complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* s_b0 = s_abort + 1;   // sequence holding this CTA's first tile
@@ -608,7 +610,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
   float* red_sum = red_max + 2 * 4 * 16;                         // [4][16]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int SW = d4_softmax_warps(G);   // softmax warps; then the TMA warp SW, the MMA warp SW + 1
+  constexpr int SW = d4_softmax_warps(G);   // softmax warps; then the TMA warp SW, the MMA warps SW + 1 (S), SW + 2 (P.V)
   constexpr int GH = G >= 2 ? G / 2 : 1;    // heads per softmax warp
 
   if (threadIdx.x == 0) {
@@ -616,6 +618,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
     for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 32 * SW); }
     for (int i = 0; i < 2; ++i) { mbar_init(&p_full[i], 32 * SW); mbar_init(&pv_done[i], 1); }
     mbar_init(drain, 1);
+    mbar_init(drain_pv, 1);
     *s_abort = 0;
     *s_b0 = 0;
     fence_barrier_init();
@@ -695,30 +698,10 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
     }
   } else if (warp == SW + 1) {
     if (lane == 0) {
-      // ------------------------------------------------------------------ MMA issuer
+      // ------------------------------------------------------------ S issuer: S = K q
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 16, 0, 0);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, 1, 0);  // V^T: MN-major A
-      const uint32_t sP = smem_u32(smem + kD4OffP);
-      // O^T += V^T P^T for tile u (the first tile of a split overwrites O); P of tile u is
-      // in buffer u & 1, whose barriers advance once every second tile
-      auto issue_pv = [&](long long u, bool first) -> bool {
-        const int pb = (int)(u & 1);
-        if (*s_abort || !mbar_wait(&p_full[pb], (uint32_t)((u >> 1) & 1), err)) return false;
-        tc_fence_after();
-        const uint32_t sV = smem_u32(smem + (int)(u % kD4Stages) * kD4StageBytes + kD4OffV);
-        const uint32_t sPb = sP + pb * 2 * kD4QHalf;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc_mnmajor_sw128(sV + kk * 16 * 128, kD4Half, 1024);
-          const uint64_t bp = sdesc_kmajor_sw128(sPb + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
-          mma_bf16_ss(tmem + 32, a, bp, idesc_o, (first && kk == 0) ? 0u : 1u);
-        }
-        mma_commit(&pv_done[pb]);
-        mma_commit(&empty[u % kD4Stages]);
-        return true;
-      };
       long long tc = 0;
-      bool ok = true, prev_first = false;
+      bool ok = true;
       for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid() && ok; w.next()) {
         const int jb = w.j0(), je = w.j1();
         for (int j = jb; j < je; ++j) {
@@ -738,16 +721,52 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
             mma_bf16_ss(tmem + 16 * sb, a, bq, idesc_s, kk ? 1u : 0u);
           }
           mma_commit(&s_full[sb]);
-          if (tc > 0 && !issue_pv(tc - 1, prev_first)) { ok = false; break; }
-          prev_first = (j == jb);
           ++tc;
         }
       }
-      if (ok && tc > 0) ok = issue_pv(tc - 1, prev_first);
       if (!ok) *s_abort = 1;
       // every MMA completes before the tensor memory is released
       mma_commit(drain);
       mbar_wait(drain, 0, err);
+    }
+  } else if (warp == SW + 2) {
+    if (lane == 0) {
+      // -------------------------------------------- P.V issuer: O^T += V^T P^T, stage release
+      // Its own warp, so that a stage is released as soon as its P is written, whether or
+      // not the next tile's data has landed. P of tile u is in buffer u & 1, whose barriers
+      // advance once every second tile; the first tile of a split overwrites O. S of tile u
+      // completed before its P was written, so this warp's commit also frees the stage's K.
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, 16, 1, 0);  // V^T: MN-major A
+      const uint32_t sP = smem_u32(smem + kD4OffP);
+      long long tc = 0;
+      bool ok = true;
+      for (D4Walk w(plan, B, Hkv, b0, t_begin, t_end); w.valid() && ok; w.next()) {
+        const int jb = w.j0(), je = w.j1();
+        for (int j = jb; j < je; ++j) {
+          const int st = (int)(tc % kD4Stages), pb = (int)(tc & 1);
+          // the stage's copies (V), observed here too, then the tile's P
+          if (*s_abort || !mbar_wait(&full[st], (uint32_t)((tc / kD4Stages) & 1), err) ||
+              !mbar_wait(&p_full[pb], (uint32_t)((tc >> 1) & 1), err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sV = smem_u32(smem + st * kD4StageBytes + kD4OffV);
+          const uint32_t sPb = sP + pb * 2 * kD4QHalf;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t a = sdesc_mnmajor_sw128(sV + kk * 16 * 128, kD4Half, 1024);
+            const uint64_t bp = sdesc_kmajor_sw128(sPb + (kk >> 2) * kD4QHalf) + 2 * (kk & 3);
+            mma_bf16_ss(tmem + 32, a, bp, idesc_o, (j == jb && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(&pv_done[pb]);
+          mma_commit(&empty[st]);
+          ++tc;
+        }
+      }
+      if (!ok) *s_abort = 1;
+      mma_commit(drain_pv);
+      mbar_wait(drain_pv, 0, err);
     }
   } else {
     // -------------------------------------------------------------------- softmax
