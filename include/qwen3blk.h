@@ -323,8 +323,8 @@ int qwen3_op_attention_prefill(const qwen3_config* cfg, const qwen3_bf16* qkv, l
  * prefill 与 decode). qkv: [B][ldqkv] bf16 with the Hq query heads (post-norm, post-RoPE)
  * at its start; ldqkv a multiple of 8 and >= Hq*128. The 128-key tiles of all (sequence,
  * KV group) rows are divided evenly among the SMs; a row shared by several SMs leaves
- * (max, sum, unnormalised output) partials in ws that the last of them merges with
- * log-sum-exp weights. ws also holds the call's tile plan and per-row tickets
+ * (max, sum, unnormalised output) partials in ws that the row's first SM merges with
+ * log-sum-exp weights. ws also holds the call's tile plan and per-row merge counters
  * (qwen3_workspace_size(cfg, QWEN3_OP_BLOCK_DECODE, B, 1, s_max) suffices; the size does
  * not depend on s_max). Hq / Hkv must be 1, 2, 4, 8 or 16. A position past the cache
  * (cache_len[b] >= s_max) is reported by the device as QWEN3_ECAPACITY, a negative one as
@@ -338,7 +338,7 @@ int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, lo
  * device memory (for example a host application given a fixed memory budget, or a plugin
  * that is handed tensors but no allocator or workspace). The pages have no counterpart:
  * this entry point exists for such callers only.
- * Instead of a caller workspace, the partials, tile plan and tickets live in a static
+ * Instead of a caller workspace, the partials, tile plan and merge counters live in a static
  * device array of this library, 12 MiB on every GPU that loads the library (held until
  * the process exits). Limit: (B * Hkv + 256) * G * 130 * 4 bytes of partials plus
  * (B + 4 + B * Hkv) * 4 bytes must fit (G = Hq / Hkv; B up to 1250 for 16 query heads in
@@ -349,7 +349,7 @@ int qwen3_op_attention_decode(const qwen3_config* cfg, const qwen3_bf16* qkv, lo
  * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
  * All calls share the one array: calls that overlap on the GPU (other streams, other
  * threads) race and must be serialised by the caller. Each call writes its plan and clears
- * its tickets before use, and every partial it reads is written by that same call, so
+ * its merge counters before use, and every partial it reads is written by that same call, so
  * nothing needs clearing between calls. */
 int qwen3_op_attention_decode_noalloc(const qwen3_config* cfg, const qwen3_bf16* qkv, long long ldqkv, int B,
                                       const int* cache_len, const qwen3_kv_layer* kv, qwen3_bf16* o, long long ldo,

@@ -245,7 +245,7 @@ struct Buffers {
   uint16_t* o = nullptr;     // [M, Hq*D]
   float* x1 = nullptr;       // [M, H] residual after attention (fp32)
   uint16_t* act = nullptr;   // [M, I] SwiGLU output
-  float* part = nullptr;     // decode attention scratch (partials, tile plan, merge tickets)
+  float* part = nullptr;     // decode attention scratch (partials, tile plan, merge counters)
   bool plan_ready = false;   // part holds this call's decode tile plan (same lengths for every layer)
   float* gpart = nullptr;    // split-K partials of small-M GEMMs
   // MoE

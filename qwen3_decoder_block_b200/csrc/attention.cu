@@ -445,15 +445,17 @@ int launch_attention_prefill(const uint16_t* qkv, long long ldqkv, int B, int T,
 //   S^T[key][j]  = sum_d K[key][d] q_j[d]      A = K tile (K-major), B = Q (K-major)
 //   O^T[d][j]   += sum_key V[key][d] P[j][key]  A = V tile (MN-major), B = P (K-major)
 // so the CUDA cores only run the softmax. A TMA warp streams Q, K and V of each tile
-// into a 3-stage shared-memory ring (128-byte swizzle, whole 256-byte rows); an MMA
-// warp issues the scores of tile i+1 before P.V of tile i (S double-buffered in
-// tensor memory); 4 softmax warps own one key each (S) and one head dim each (O):
-// the tile maximum per head is a warp reduction plus a 4-warp exchange, the online
-// softmax rescales O only when the running maximum grows by more than 2^8, and P is
-// written as bf16 into a swizzled K-major tile. A row that lies in one CTA is
-// normalised and written at once; otherwise each CTA writes its partial (unnormalised
-// O, running maximum, sum) to the scratch, takes the row's ticket, and the CTA with
-// the last ticket merges the row's partials in CTA order.
+// into a 3-stage shared-memory ring (128-byte swizzle, whole 256-byte rows); one warp
+// issues the scores of each tile as it lands (S double-buffered in tensor memory),
+// another P.V and the stage's release; 8 softmax warps (4 for G = 1), two per
+// tensor-memory lane quarter, own one key each (S) and one head dim each (O) for half
+// of the group's heads: the tile maximum per head is a warp reduction plus a 4-quarter
+// exchange, the online softmax rescales O only when the running maximum grows by more
+// than 2^8, and P is written as bf16 into a swizzled K-major tile. A row that lies in
+// one CTA is normalised and written at once; otherwise the CTAs after the row's first
+// write their partial (unnormalised O, running maximum, sum) to the scratch and count
+// it with a release add, and the row's first CTA, which reaches the row last, merges
+// its own values with theirs in CTA order.
 // ============================================================================
 constexpr int kD4Stages = 3;
 constexpr int kD4MaxCtas = 256;                    // grid bound (partial slots per call: rows + CTAs)
@@ -499,15 +501,23 @@ __device__ __forceinline__ bool d4_cta_empty(int c, long long T, int n) {
   return T * c / n == T * (c + 1) / n;
 }
 
-// Merge of one head's partials of a row: CTAs c_first..c_last with a non-empty range
-// wrote slot (row + c), `stride` floats apart from row_base's slot 0 numbering.
-__device__ __forceinline__ void merge_row_dim(const float* row_base, int c_first, int c_last, long long T, int n,
-                                              long long stride, int d, uint16_t* dst, const DecodeMergeOut& mo) {
-  float M = -INFINITY;
-  for (int c = c_first; c <= c_last; ++c)
+// Merge of one head's partials of a row, by the row's first CTA: its own (m, l, o_d) are
+// in registers and come first in the (deterministic) order; then the CTAs c_first + 1 ..
+// c_last with a non-empty range, which wrote slot (row + c), `stride` floats apart from
+// row_base's slot 0 numbering.
+__device__ __forceinline__ void merge_row_dim_own(const float* row_base, int c_first, int c_last, long long T, int n,
+                                                  long long stride, int d, float m_own, float l_own, float o_own,
+                                                  uint16_t* dst, const DecodeMergeOut& mo) {
+  float M = m_own;
+  for (int c = c_first + 1; c <= c_last; ++c)
     if (!d4_cta_empty(c, T, n)) M = fmaxf(M, __ldcg(row_base + c * stride + kHeadDim));
   float L = 0.f, acc = 0.f;
-  for (int c = c_first; c <= c_last; ++c) {
+  if (m_own != -INFINITY) {
+    const float w = exp2f(m_own - M);
+    L = l_own * w;
+    acc = o_own * w;
+  }
+  for (int c = c_first + 1; c <= c_last; ++c) {
     if (d4_cta_empty(c, T, n)) continue;
     const float* q = row_base + c * stride;
     const float m = __ldcg(q + kHeadDim);
@@ -914,40 +924,56 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
           store_head_dim(o / L, t, out_row + hd * kHeadDim, mo);
         }
       } else {
-        // partial of the row in slot row + CTA (unique: the rows and the CTA ranges are
-        // both in tile order); the last CTA of the row to finish merges the slots
-        float* my_part = part + ((long long)bg + blockIdx.x) * G * kD4PartFloats;
-#pragma unroll
-        for (int jj = 0; jj < GH; ++jj) {
-          const int hd = j0 + jj;
-          my_part[hd * kD4PartFloats + t] =
-              HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
-          if (t == hd) {
-            my_part[hd * kD4PartFloats + kHeadDim] = m_run[jj];
-            my_part[hd * kD4PartFloats + kHeadDim + 1] =
-                red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd];
-          }
-        }
-        __threadfence();  // the partial, visible to the merging CTA before the ticket
-        named_bar_softmax<SW>();
+        // a row shared by several CTAs: the row's first CTA merges, at the end of its range
+        // (where it reaches the row); the others leave a partial in slot row + CTA (unique:
+        // the rows and the CTA ranges are both in tile order) and publish it with one
+        // release add, without waiting
         const int c_first = d4_cta_of(w.rs, T, n_cta), c_last = d4_cta_of(w.rs + w.nt - 1, T, n_cta);
-        if (threadIdx.x == 0) {
-          // the row's CTAs: those of [c_first, c_last] whose range is not empty (fewer
-          // tiles than CTAs leaves some empty)
-          int n_seg = 0;
-          for (int c = c_first; c <= c_last; ++c) n_seg += d4_cta_empty(c, T, n_cta) ? 0 : 1;
-          const int prev = atomicAdd(&counters[bg], 1);
-          const bool last = prev == n_seg - 1;
-          if (last) counters[bg] = 0;  // ready for the next call
-          *s_fix = last ? 1 : 0;
-        }
-        named_bar_softmax<SW>();
-        if (*s_fix) {
-          __threadfence();  // the other CTAs' partials (their fences precede their tickets)
-#pragma unroll 1
-          for (int jj = 0; jj < GH; ++jj)
-            merge_row_dim(part + ((long long)bg * G + j0 + jj) * kD4PartFloats, c_first, c_last, T, n_cta,
-                          (long long)G * kD4PartFloats, t, out_row + (j0 + jj) * kHeadDim, mo);
+        if ((int)blockIdx.x != c_first) {
+          float* my_part = part + ((long long)bg + blockIdx.x) * G * kD4PartFloats;
+#pragma unroll
+          for (int jj = 0; jj < GH; ++jj) {
+            const int hd = j0 + jj;
+            my_part[hd * kD4PartFloats + t] =
+                HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+            if (t == hd) {
+              my_part[hd * kD4PartFloats + kHeadDim] = m_run[jj];
+              my_part[hd * kD4PartFloats + kHeadDim + 1] =
+                  red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd];
+            }
+          }
+          named_bar_softmax<SW>();  // every thread's partial stores precede the release
+          if (threadIdx.x == 0) red_release_gpu_add(&counters[bg], 1);
+        } else {
+          if (threadIdx.x == 0) {
+            // the row's other CTAs (those of (c_first, c_last] whose range is not empty:
+            // fewer tiles than CTAs leaves some empty) have all published (bounded wait)
+            int n_other = 0;
+            for (int c = c_first + 1; c <= c_last; ++c) n_other += d4_cta_empty(c, T, n_cta) ? 0 : 1;
+            bool done = true;
+            const unsigned long long t0 = global_ns();
+            while (ld_acquire_gpu_s32(&counters[bg]) < n_other) {
+              if (global_ns() - t0 > kWaitLimitNs) {
+                record_error(err, kErrTimeout);
+                done = false;
+                break;
+              }
+            }
+            counters[bg] = 0;  // ready for the next call
+            *s_fix = done ? 1 : 0;
+          }
+          named_bar_softmax<SW>();  // the acquire above precedes every thread's reads
+          if (*s_fix) {
+#pragma unroll
+            for (int jj = 0; jj < GH; ++jj) {
+              const int hd = j0 + jj;
+              const float o_own = HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+              merge_row_dim_own(part + ((long long)bg * G + hd) * kD4PartFloats, c_first, c_last, T, n_cta,
+                                (long long)G * kD4PartFloats, t, m_run[jj],
+                                red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd], o_own,
+                                out_row + hd * kHeadDim, mo);
+            }
+          }
         }
       }
     }
@@ -965,7 +991,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
 // Tile prefix of the decode call: plan[b] = index of the first tile of sequence b's rows
 // (Hkv rows of ceil((cache_len[b] + 1) / 128) tiles each; none for a sequence whose
 // new position is past the cache, which is reported), plan[B] = all tiles. Clears the
-// rows' merge tickets. One block.
+// rows' merge counters. One block.
 __global__ void __launch_bounds__(1024) attn_decode_plan_kernel(const int* __restrict__ cache_len, int B, int Hkv,
                                                                 int s_max, int* __restrict__ plan,
                                                                 int* __restrict__ counters, int* err) {
@@ -1013,7 +1039,7 @@ __global__ void __launch_bounds__(1024) attn_decode_plan_kernel(const int* __res
 }
 
 // Scratch of one decode call: partial slots (rows + CTAs, G heads each), the tile plan,
-// the rows' merge tickets.
+// the rows' merge counters.
 static size_t d4_part_floats(int B, int Hq) { return ((size_t)B * Hq + (size_t)kD4MaxCtas * 16) * kD4PartFloats; }
 static size_t d4_plan_ints(int B) { return ((size_t)B + 1 + 3) & ~(size_t)3; }
 
@@ -1101,12 +1127,12 @@ int launch_attention_decode(const uint16_t* qkv, long long ldqkv, int B, int Hq,
 
 // ----------------------------------------------------------------------------
 // Decode attention without caller scratch. The partials, the tile plan and the merge
-// tickets live in a fixed device array of this library instead of a caller workspace,
+// counters live in a fixed device array of this library instead of a caller workspace,
 // for callers that cannot allocate device memory. Its capacity is kStaticDecodeFloats
 // floats (12 MiB): decode_partial_bytes(B, Hq, Hkv) must fit (B * Hq up to about 20000).
 // The array's device address is looked up on the host once per device (with that device
 // current); every call shares the array, so calls that overlap on the GPU race. Each
-// call writes its plan and clears its tickets before use, and every partial it reads is
+// call writes its plan and clears its merge counters before use, and every partial it reads is
 // written by that same call, so nothing has to be cleared between calls.
 // ----------------------------------------------------------------------------
 constexpr size_t kStaticDecodeFloats = (size_t)3 << 20;
