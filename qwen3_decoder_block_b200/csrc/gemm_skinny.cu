@@ -46,9 +46,9 @@ int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long c
 
 namespace {
 
-constexpr int kSkThreads = 256;  // TMA warp, MMA warp, 4 accumulator warps, 2 more epilogue warps
+constexpr int kSkThreads = 512;  // TMA warp, MMA warp, 4 accumulator warps, 10 more epilogue warps
 constexpr int kSkMaxSplits = 16;  // cluster size: 16 is the non-portable maximum on sm_100
-constexpr int kSkPre = 4;        // tokens per epilogue warp whose side operands are prefetched
+constexpr int kSkPre = 2;        // tokens per epilogue warp whose side operands are prefetched
 constexpr uint32_t kSkPBytes = 128 * 64 * 2;  // weight tile: 128 features x 64 of K, bf16
 
 // HILO: the activation operand holds 2M rows, row t = hi(a_t) and row M + t = lo(a_t)
