@@ -441,6 +441,14 @@ static int attention_half(const Ctx& k, const qwen3_layer_weights& w, const void
       o.row_r_out = b.rs_x1;
     }
     o.f16 = f16;
+    if (defer2) {
+      // a dense FFN follows: leave the SMs of its gate/up projection free, so that all of
+      // its CTAs start beside this one and prefetch their weights
+      SkinnyDesc gu;
+      gu.M = (int)M; gu.N = 2 * c.intermediate; gu.K = H; gu.epi = kEpiSwiglu; gu.a_hilo = true;
+      const int n_gu = skinny_ctas(gu);
+      if (n_gu > 0 && n_gu < num_sms()) o.max_ctas = num_sms() - n_gu;
+    }
     ProfScope ps("gemm_o", k.s);
     rc = launch_gemm_skinny(o, k.s, k.err);
     *h2_ready = rc == 0;
@@ -591,6 +599,11 @@ static int dense_ffn(const Ctx& k, const qwen3_layer_weights& w, long long M, vo
       } else {
         d.row_r_out = b.rs_x;
       }
+    }
+    {
+      // fit beside the gate/up projection, so that all of this launch's CTAs start early
+      const int n_gu = skinny_ctas(g);
+      if (n_gu > 0 && n_gu < num_sms()) d.max_ctas = num_sms() - n_gu;
     }
     ProfScope ps("gemm_down", k.s);
     rc = launch_gemm_skinny(d, k.s, k.err);

@@ -627,13 +627,12 @@ bool clusters_fit(int S, int n_clusters) {
   return n >= n_clusters;
 }
 
+// K splits of d: as many as fit one wave of co-resident clusters (one CTA per SM;
+// clusters above 8 CTAs need the non-portable size, allowed once per kernel and device),
+// within d.max_ctas; every split gets at least one K block.
 template <int BN, bool HILO>
-int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
-  using C = SkCfg<BN, HILO>;
-  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)C::SMEM)) return -6;
+int choose_splits(const SkinnyDesc& d) {
   const int n_tiles = d.N / 128, k_blocks = d.K / 64;
-  // splits: as many as fit in one wave of co-resident clusters (one CTA per SM; clusters
-  // above 8 CTAs need the non-portable size, allowed once per kernel and device)
   static std::mutex mu;
   static std::vector<std::pair<const void*, int>> wide;  // (kernel, device) allowed 16-CTA clusters
   int max_c = 8;
@@ -653,6 +652,7 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
     if (ok) max_c = kSkMaxSplits;
   }
   int S = 1;
+  if (d.max_ctas > 0 && d.max_ctas / n_tiles < max_c) max_c = d.max_ctas / n_tiles > 1 ? d.max_ctas / n_tiles : 1;
   for (int c = max_c; c >= 1; --c) {
     if ((long long)n_tiles * c > num_sms() || c > k_blocks) continue;
     if (c > 1 && !clusters_fit<BN, HILO>(c, n_tiles)) continue;
@@ -660,7 +660,16 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
     break;
   }
   const int kpb = (k_blocks + S - 1) / S;
-  S = (k_blocks + kpb - 1) / kpb;  // every split gets at least one K block
+  return (k_blocks + kpb - 1) / kpb;
+}
+
+template <int BN, bool HILO>
+int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
+  using C = SkCfg<BN, HILO>;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)C::SMEM)) return -6;
+  const int n_tiles = d.N / 128, k_blocks = d.K / 64;
+  const int S = choose_splits<BN, HILO>(d);
+  const int kpb = (k_blocks + S - 1) / S;
   CUtensorMap tmP, tmQ;
   if (make_tmap_2d(&tmP, d.W, d.N, d.K, d.ldw, 128) != 0 ||
       make_tmap_2d(&tmQ, d.A, HILO ? 2LL * d.M : d.M, d.K, d.lda, BN) != 0) {
@@ -715,6 +724,19 @@ int launch_bn(const SkinnyDesc& d, cudaStream_t s, int* err) {
 bool skinny_supported(int M, int N, int K, int epi) {
   if (M < 1 || M > 64 || N % 128 != 0 || K % 64 != 0 || K < 64) return false;
   return epi == kEpiStore || epi == kEpiResid || epi == kEpiSwiglu || epi == kEpiQKRope;
+}
+
+int skinny_ctas(const SkinnyDesc& d) {
+  if (!skinny_supported(d.M, d.N, d.K, d.epi)) return 0;
+  const int n_tiles = d.N / 128;
+  if (d.a_hilo) {
+    if (d.M <= 16) return n_tiles * choose_splits<16, true>(d);
+    if (d.M <= 32) return n_tiles * choose_splits<32, true>(d);
+    return n_tiles * choose_splits<64, true>(d);
+  }
+  if (d.M <= 16) return n_tiles * choose_splits<16, false>(d);
+  if (d.M <= 32) return n_tiles * choose_splits<32, false>(d);
+  return n_tiles * choose_splits<64, false>(d);
 }
 
 int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err) {

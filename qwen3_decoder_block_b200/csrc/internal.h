@@ -131,10 +131,16 @@ struct SkinnyDesc {
   // each hi value: norm_lo for norm_out, out_lo for the SwiGLU output
   long long norm_lo = 0;
   long long out_lo = 0;
+  // at most this many CTAs (0: as many K splits as fit one wave), so that this launch and
+  // the next projection's fit the SMs together and the next one's CTAs all start early
+  int max_ctas = 0;
 };
 
 bool skinny_supported(int M, int N, int K, int epi);
 int launch_gemm_skinny(const SkinnyDesc& d, cudaStream_t s, int* err);
+// The CTAs launch_gemm_skinny would launch for d (feature tiles x K splits), 0 when the
+// shape is unsupported. Host only.
+int skinny_ctas(const SkinnyDesc& d);
 
 // Scratch the block calls reserve for split-K partials of small-M GEMMs.
 constexpr size_t kSplitKBytes = (size_t)2 * 148 * 128 * 256 * sizeof(float);
