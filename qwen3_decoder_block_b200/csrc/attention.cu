@@ -472,7 +472,9 @@ constexpr uint32_t kD4OffBar = kD4OffRed + (2 * 4 * 16 + 4 * 16) * 4;
 constexpr uint32_t kD4Smem = kD4OffBar + 16 * 8 + 16 + 1024;
 // softmax warps: two per tensor-memory lane quarter, each owning half of the group's
 // heads (G >= 2), or one per quarter (G = 1); then the TMA warp and the MMA warp
-__host__ __device__ constexpr int d4_softmax_warps(int G) { return G >= 2 ? 8 : 4; }
+// softmax warps per tensor-memory lane quarter, each owning G / that many of the heads
+__host__ __device__ constexpr int d4_head_warps(int G) { return G >= 8 ? 4 : (G >= 2 ? 2 : 1); }
+__host__ __device__ constexpr int d4_softmax_warps(int G) { return 4 * d4_head_warps(G); }
 // softmax warps, then the TMA warp, the S-issuing warp and the P.V-issuing warp
 __host__ __device__ constexpr int d4_threads(int G) { return 32 * (d4_softmax_warps(G) + 3); }
 constexpr uint32_t kD4TmemCols = 64;  // S0 [0,16), S1 [16,32), O [32,48)
@@ -594,6 +596,18 @@ struct D4Walk {
 // columns of both MMAs carry the hi and lo halves: S = K q_hi + K q_lo and
 // O = V P_hi + V P_lo, summed in fp32 -- about 16 significant bits for q and P at no
 // extra MMA instruction (the kernel is bound by the K/V stream).
+// Element base + hh * GH + jj of a register array for the warp's head group hh (run
+// time, < HW) and head jj (a constant after unrolling): only constant indices, so the
+// array stays in registers.
+template <int HW, int GH, int N>
+__device__ __forceinline__ uint32_t pick_head(const uint32_t (&a)[N], int base, int hh, int jj) {
+  uint32_t v = a[base + jj];
+#pragma unroll
+  for (int h = 1; h < HW; ++h)
+    if (hh == h) v = a[base + h * GH + jj];
+  return v;
+}
+
 template <int G, bool HILO>
 __global__ void __launch_bounds__(d4_threads(G), 1)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -621,7 +635,8 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int SW = d4_softmax_warps(G);   // softmax warps; then the TMA warp SW, the MMA warps SW + 1 (S), SW + 2 (P.V)
-  constexpr int GH = G >= 2 ? G / 2 : 1;    // heads per softmax warp
+  constexpr int HW = d4_head_warps(G);      // softmax warps per lane quarter
+  constexpr int GH = G / HW;                 // heads per softmax warp
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kD4Stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
@@ -812,7 +827,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
         float s[GH];
 #pragma unroll
         for (int jj = 0; jj < GH; ++jj) {
-          const float sj = HILO ? __uint_as_float(hh ? sv[GH + jj] : sv[jj]) + __uint_as_float(hh ? sv[G + GH + jj] : sv[G + jj]) : __uint_as_float(hh ? sv[GH + jj] : sv[jj]);
+          const float sj = HILO ? __uint_as_float(pick_head<HW, GH>(sv, 0, hh, jj)) + __uint_as_float(pick_head<HW, GH>(sv, G, hh, jj)) : __uint_as_float(pick_head<HW, GH>(sv, 0, hh, jj));
           s[jj] = (ok && t < nk) ? sj * kScaleLog2 : -INFINITY;
         }
         // tile maximum per head: the warp's 32 keys, then the 4 quarters
@@ -862,8 +877,8 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
 #pragma unroll
             for (int jj = 0; jj < GH; ++jj) {
               const int hd = j0 + jj;
-              tmem_st1(tl + 32 + hd, __float_as_uint(__uint_as_float(hh ? ov[GH + jj] : ov[jj]) * alpha[jj]));
-              if (HILO) tmem_st1(tl + 32 + G + hd, __float_as_uint(__uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) * alpha[jj]));
+              tmem_st1(tl + 32 + hd, __float_as_uint(__uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj)) * alpha[jj]));
+              if (HILO) tmem_st1(tl + 32 + G + hd, __float_as_uint(__uint_as_float(pick_head<HW, GH>(ov, G, hh, jj)) * alpha[jj]));
             }
             tmem_wait_st();
           }
@@ -920,7 +935,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
         for (int jj = 0; jj < GH; ++jj) {
           const int hd = j0 + jj;
           const float L = red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd];
-          const float o = HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+          const float o = HILO ? __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj)) + __uint_as_float(pick_head<HW, GH>(ov, G, hh, jj)) : __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj));
           store_head_dim(o / L, t, out_row + hd * kHeadDim, mo);
         }
       } else {
@@ -935,7 +950,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
           for (int jj = 0; jj < GH; ++jj) {
             const int hd = j0 + jj;
             my_part[hd * kD4PartFloats + t] =
-                HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+                HILO ? __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj)) + __uint_as_float(pick_head<HW, GH>(ov, G, hh, jj)) : __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj));
             if (t == hd) {
               my_part[hd * kD4PartFloats + kHeadDim] = m_run[jj];
               my_part[hd * kD4PartFloats + kHeadDim + 1] =
@@ -967,7 +982,7 @@ __global__ void __launch_bounds__(d4_threads(G), 1)
 #pragma unroll
             for (int jj = 0; jj < GH; ++jj) {
               const int hd = j0 + jj;
-              const float o_own = HILO ? __uint_as_float(hh ? ov[GH + jj] : ov[jj]) + __uint_as_float(hh ? ov[G + GH + jj] : ov[G + jj]) : __uint_as_float(hh ? ov[GH + jj] : ov[jj]);
+              const float o_own = HILO ? __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj)) + __uint_as_float(pick_head<HW, GH>(ov, G, hh, jj)) : __uint_as_float(pick_head<HW, GH>(ov, 0, hh, jj));
               merge_row_dim_own(part + ((long long)bg * G + hd) * kD4PartFloats, c_first, c_last, T, n_cta,
                                 (long long)G * kD4PartFloats, t, m_run[jj],
                                 red_sum[hd] + red_sum[16 + hd] + red_sum[32 + hd] + red_sum[48 + hd], o_own,
