@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 METRIC = "Qwen3-0.6B prefill & decode tokens/s on 1 B200; % of BF16/HBM roofline"
 # measured DRAM bytes / algorithmic K/V bytes of one decode-attention launch (ncu
 # dram__bytes_read.sum + dram__bytes_write.sum); None until captured for the current kernel
-DECODE_ATTN_TRAFFIC_RATIO = (1078513920 + 3666176) / 1074003968
+DECODE_ATTN_TRAFFIC_RATIO = (1078514176 + 7338240) / 1074003968
 DECODE_ATTN_TRAFFIC_SOURCE = ("ncu capture of one attn_decode_tc_kernel launch at B64 x 4097 positions "
                               "(profiles/attn_decode_B64_ctx4096_layer.md), scaled by positions")
 
