@@ -507,8 +507,9 @@ def run_single_layer(q3, torch, args, name, B, T, seed, moe=False, reps=None):
     ws = torch.empty(q3.workspace_size(cfg, op, B, T, T), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
+    # the block updates x in place, so successive calls chain the layer (each call's input
+    # is the previous call's output: the same work, no copy between calls)
     def call():
-        x.copy_(x0)
         if moe:
             q3.moe_block(cfg, w, x, B, T, pos, kv, rope, ws, stream=stream)
         else:

@@ -913,51 +913,136 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+// A tensor map is a function of its encode arguments only, and repeated calls (a decode
+// step, a small layer) encode the same maps every time: they come from a hash table keyed
+// by those arguments (open addressing over a short probe window, the window's first
+// slot replaced when it is full; under a lock).
+namespace {
+struct TmapKey {
+  int kind, rank;
+  const void* base;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+};
+constexpr int kTmapCache = 1024;  // a power of two
+constexpr int kTmapProbe = 8;
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool used;
+};
+std::mutex g_tmap_mu;
+TmapEntry g_tmap[kTmapCache];
+
+size_t key_hash(const TmapKey& k) {
+  size_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+  auto mix = [&](unsigned long long v) { h = (h ^ v) * 0x100000001B3ull; };
+  mix((unsigned long long)k.kind * 8 + (unsigned long long)k.rank);
+  for (int i = 0; i < k.rank; ++i) {
+    mix(k.dims[i]);
+    mix(k.box[i]);
+  }
+  for (int i = 0; i + 1 < k.rank; ++i) mix(k.strides[i]);
+  return h ^ (h >> 29);
+}
+
+bool same_key(const TmapKey& a, const TmapKey& b) {
+  if (a.kind != b.kind || a.rank != b.rank || a.base != b.base) return false;
+  for (int i = 0; i < a.rank; ++i)
+    if (a.dims[i] != b.dims[i] || a.box[i] != b.box[i]) return false;
+  for (int i = 0; i + 1 < a.rank; ++i)
+    if (a.strides[i] != b.strides[i]) return false;
+  return true;
+}
+
+// kind 0: bf16 operand, 128-byte swizzle, L2 256-byte promotion; 1: fp32 output, 128-byte
+// swizzle; 2: bf16 output, 64-byte swizzle (the epilogue staging layouts)
+int encode_cached(CUtensorMap* map, const TmapKey& k) {
+  const size_t h0 = key_hash(k);
+  {
+    std::lock_guard<std::mutex> lk(g_tmap_mu);
+    for (int i = 0; i < kTmapProbe; ++i) {
+      const TmapEntry& e = g_tmap[(h0 + i) & (kTmapCache - 1)];
+      if (!e.used) break;
+      if (same_key(e.key, k)) {
+        *map = e.map;
+        return 0;
+      }
+    }
+  }
+  auto enc = get_encode();
+  if (!enc) return -1;
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      enc(map, k.kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k.rank,
+          const_cast<void*>(k.base), k.dims, k.strides, k.box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          k.kind == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+          k.kind == 0 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_NONE,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return -2;
+  std::lock_guard<std::mutex> lk(g_tmap_mu);
+  int slot = (int)(h0 & (kTmapCache - 1));  // replaced when the window is full
+  for (int i = 0; i < kTmapProbe; ++i) {
+    const int j = (int)((h0 + i) & (kTmapCache - 1));
+    if (!g_tmap[j].used) {
+      slot = j;
+      break;
+    }
+  }
+  TmapEntry& e = g_tmap[slot];
+  e.key = k;
+  e.map = *map;
+  e.used = true;
+  return 0;
+}
+}  // namespace
+
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix with row stride ld
 // (elements), box = box_rows x 64 columns, 128-byte swizzle, zero fill out of bounds.
 int make_tmap_2d(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld, int box_rows) {
-  auto enc = get_encode();
-  if (!enc) return -1;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? 0 : -2;
+  TmapKey k = {};
+  k.kind = 0;
+  k.rank = 2;
+  k.base = base;
+  k.dims[0] = (cuuint64_t)cols;
+  k.dims[1] = (cuuint64_t)rows;
+  k.strides[0] = (cuuint64_t)(ld * 2);
+  k.box[0] = 64;
+  k.box[1] = (cuuint32_t)box_rows;
+  return encode_cached(map, k);
 }
 
 // 3-D bf16 tensor map: dims (inner, mid, outer) with byte strides for mid and outer.
 int make_tmap_3d(CUtensorMap* map, const void* base, long long inner, long long mid, long long outer,
                  long long mid_stride_bytes, long long outer_stride_bytes, int box_inner, int box_mid, int box_outer) {
-  auto enc = get_encode();
-  if (!enc) return -1;
-  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)mid, (cuuint64_t)outer};
-  cuuint64_t strides[2] = {(cuuint64_t)mid_stride_bytes, (cuuint64_t)outer_stride_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_mid, (cuuint32_t)box_outer};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? 0 : -2;
+  TmapKey k = {};
+  k.kind = 0;
+  k.rank = 3;
+  k.base = base;
+  k.dims[0] = (cuuint64_t)inner;
+  k.dims[1] = (cuuint64_t)mid;
+  k.dims[2] = (cuuint64_t)outer;
+  k.strides[0] = (cuuint64_t)mid_stride_bytes;
+  k.strides[1] = (cuuint64_t)outer_stride_bytes;
+  k.box[0] = (cuuint32_t)box_inner;
+  k.box[1] = (cuuint32_t)box_mid;
+  k.box[2] = (cuuint32_t)box_outer;
+  return encode_cached(map, k);
 }
 
 // Output tensor map for the TMA-store epilogue: [rows, cols] fp32 or bf16, box 32 x 32,
 // 128-byte (fp32) or 64-byte (bf16) swizzle matching stage_row_chunk.
 static int make_tmap_out(CUtensorMap* map, void* base, long long rows, long long cols, long long ld, bool f32) {
-  auto enc = get_encode();
-  if (!enc) return -1;
-  const int es = f32 ? 4 : 2;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
-  cuuint32_t box[2] = {32, 32};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? 0 : -2;
+  TmapKey k = {};
+  k.kind = f32 ? 1 : 2;
+  k.rank = 2;
+  k.base = base;
+  k.dims[0] = (cuuint64_t)cols;
+  k.dims[1] = (cuuint64_t)rows;
+  k.strides[0] = (cuuint64_t)(ld * (f32 ? 4 : 2));
+  k.box[0] = 32;
+  k.box[1] = 32;
+  return encode_cached(map, k);
 }
 
 // One kernel instantiation: shared-memory attribute (once per device), launch (CTA pairs as
