@@ -282,24 +282,15 @@ __device__ __forceinline__ uint32_t mapa_shared_addr(uint32_t addr, uint32_t ran
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
-// Distributed shared memory: 32-bit load and store at a shared::cluster address
-// (a peer CTA's shared memory, mapped with mapa_shared).
-__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
-// The same load for data that no thread changes any more, read after the cluster barrier
-// that published it: a pure asm (not volatile, no memory clobber), so the compiler may
-// schedule it freely. The address must come from mapa_shared issued after that barrier
-// (a volatile asm), which keeps the load from moving above it.
+// Distributed shared memory: 32-bit load at a shared::cluster address (a peer CTA's
+// shared memory, mapped with mapa_shared_addr), for data that no thread changes any more,
+// read after the cluster barrier that published it: a pure asm (not volatile, no memory
+// clobber), so the compiler may schedule it freely. The address must come from a mapa
+// issued after that barrier (a volatile asm), which keeps the load from moving above it.
 __device__ __forceinline__ float ld_cluster_f32_ro(uint32_t cluster_addr) {
   float v;
   asm("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr));
   return v;
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t cluster_nctarank() {
   uint32_t r;
@@ -421,14 +412,6 @@ __device__ __forceinline__ void tmem_wait_ld_regs16(uint32_t (&r)[16]) {
 // One 32-bit column of 32 lanes.
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
-}
-__device__ __forceinline__ void tmem_st16x(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
 }
 
 // ----------------------------------------------------------------------------
