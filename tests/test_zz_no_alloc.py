@@ -46,7 +46,7 @@ def test_noalloc_decode_matches_workspace_decode_twice():
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     """The scratch of a call holds (B * Hkv + 256) partial slots of G heads x 130 floats,
-    the tile plan (B + 1 ints, padded to 4) and B * Hkv merge tickets. With 16 query
+    the tile plan (B + 1 ints, padded to 4) and B * Hkv merge counters. With 16 query
     heads that is 12,583,536 bytes for B 1251, above the 12 MiB static array, so the call
     is refused before launch; B 1250 (12,575,184 bytes) fits and runs. The cache is
     really allocated (s_max 8), so that the arguments describe valid memory whatever the
