@@ -633,6 +633,10 @@ bool clusters_fit(int S, int n_clusters) {
 template <int BN, bool HILO>
 int choose_splits(const SkinnyDesc& d) {
   const int n_tiles = d.N / 128, k_blocks = d.K / 64;
+  // the occupancy answers below assume the kernel's shared-memory limit is raised (a
+  // grid computed before the first launch of this instantiation included)
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_skinny_kernel<BN, HILO>), (int)SkCfg<BN, HILO>::SMEM))
+    return 1;
   static std::mutex mu;
   static std::vector<std::pair<const void*, int>> wide;  // (kernel, device) allowed 16-CTA clusters
   int max_c = 8;
